@@ -1,0 +1,342 @@
+"""Pins for the CPU oracle: it is checked here against things other than
+itself -- brute force in 50-digit arithmetic without max-shift, closed forms,
+invariants the method fixes, exhaustive ranking, and library decoders.
+
+The method (HySparse2 announcement, "KV Reuse" section and the token-level
+selection / forced-window paragraphs): the full layer attends over all T
+positions and selects positions from its attention scores; the most recent
+W=128 tokens are always kept plus the top 1,024 of the rest; the sparse
+layers attend over exactly that list.
+"""
+import json
+import math
+import os
+
+import mpmath
+import numpy as np
+import pytest
+import torch
+
+from long_context_decode_full_b200 import synth
+
+mpmath.mp.dps = 50
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- helpers --
+
+def decode_bf16(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def decode_e4m3_torch(codes):
+    t = torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def dequant(w, which):
+    """Exact stored values of a workload's cache as float64 (library decoders)."""
+    t = getattr(w, which)
+    if w.spec.kv_dtype == "f32":
+        return t.double().numpy()
+    if w.spec.kv_dtype == "bf16":
+        return decode_bf16(synth.raw(t))
+    sc = getattr(w, which + "_scale").double().numpy()
+    return decode_e4m3_torch(synth.raw(t)) * sc[..., None]
+
+
+def qvals(q, dtype):
+    return q.double().numpy() if dtype == "f32" else decode_bf16(synth.raw(q))
+
+
+def dtype_code(s):
+    return {"f32": 0, "bf16": 1, "e4m3": 2}[s]
+
+
+def run_full(oracle, w, q=None, window=None, k_global=None):
+    s = w.spec
+    q = w.q_full if q is None else q
+    return oracle.full_attn_select(
+        synth.raw(q), dtype_code(s.q_dtype), synth.raw(w.k), synth.raw(w.v), dtype_code(s.kv_dtype),
+        synth.raw(w.seq_lens), synth.raw(w.page_table), w.page_size,
+        window=s.window if window is None else window,
+        k_global=s.k_global if k_global is None else k_global,
+        k_scale=synth.raw(w.k_scale), v_scale=synth.raw(w.v_scale))
+
+
+def run_sparse(oracle, w, q, idx):
+    s = w.spec
+    return oracle.sparse_attn(synth.raw(q), dtype_code(s.q_dtype), synth.raw(w.k), synth.raw(w.v),
+                              dtype_code(s.kv_dtype), idx, k_scale=synth.raw(w.k_scale),
+                              v_scale=synth.raw(w.v_scale))
+
+
+def brute_full(w, q=None):
+    """50-digit brute force: logits, softmax WITHOUT max-shift, out, lse,
+    group score; address rule applied by hand."""
+    s = w.spec
+    q = qvals(w.q_full if q is None else q, s.q_dtype)
+    K, V = dequant(w, "k"), dequant(w, "v")
+    B, Hq, d = q.shape
+    G = s.group
+    res = {"out": np.zeros((B, Hq, d)), "lse": np.zeros((B, Hq)), "score": {}}
+    pt = None if w.page_table is None else w.page_table.numpy()
+    for b in range(B):
+        T = int(w.seq_lens[b])
+        slots = [(b * w.page_size + t) if pt is None else
+                 (int(pt[b, t // w.page_size]) * w.page_size + t % w.page_size) for t in range(T)]
+        probs = {}
+        for h in range(Hq):
+            kvh = h // G
+            logits = [mpmath.fsum(mpmath.mpf(q[b, h, i]) * mpmath.mpf(K[sl, kvh, i]) for i in range(d))
+                      / mpmath.sqrt(d) for sl in slots]
+            e = [mpmath.exp(x) for x in logits]
+            Z = mpmath.fsum(e)
+            p = [x / Z for x in e]
+            probs[h] = p
+            res["lse"][b, h] = float(mpmath.log(Z))
+            for i in range(d):
+                res["out"][b, h, i] = float(mpmath.fsum(p[t] * mpmath.mpf(V[slots[t], kvh, i])
+                                                        for t in range(T)))
+        for kvh in range(s.num_kv_heads):
+            res["score"][(b, kvh)] = np.array(
+                [float(mpmath.fsum(probs[kvh * G + g][t] for g in range(G))) for t in range(T)])
+    return res
+
+
+def small_spec(**kw):
+    base = dict(name="pin", batch=2, num_kv_heads=2, group=2, head_dim=8, seq_len=37,
+                kv_dtype="bf16", q_dtype="bf16", page_size=4, sparse_layers=1, needles=3,
+                window=5, k_global=6)
+    base.update(kw)
+    return synth.WorkloadSpec(**base)
+
+
+# ---------------------------------------------------------------- pins ----
+
+def test_golden_hyperparameters_match_pages():
+    """window=128 and k_global=1024 are the numbers the pages state."""
+    with open(os.path.join(GOLDEN, "hybrid_block_params.json")) as f:
+        g = json.load(f)
+    for spec in synth.WORKLOADS.values():
+        assert spec.window == g["window"] and spec.k_global == g["k_global"]
+
+
+def test_e4m3_decode_matches_torch_for_all_codes(oracle):
+    codes = np.arange(256, dtype=np.uint8)
+    ref = decode_e4m3_torch(codes)
+    got = np.array([oracle.e4m3_value(int(c)) for c in codes])
+    nan = np.isnan(ref)
+    assert nan.sum() == 2 and np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+@pytest.mark.parametrize("kv_dtype,q_dtype,page", [("bf16", "bf16", 4), ("f32", "f32", None),
+                                                   ("e4m3", "bf16", 8)])
+def test_full_layer_matches_50_digit_brute_force(oracle, kv_dtype, q_dtype, page):
+    spec = small_spec(kv_dtype=kv_dtype, q_dtype=q_dtype, page_size=page, seq_len=(9, 23))
+    w = synth.generate(spec, seed=11)
+    got = run_full(oracle, w)
+    ref = brute_full(w)
+    np.testing.assert_allclose(got["out"], ref["out"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got["lse"], ref["lse"], rtol=0, atol=1e-12)
+    for (b, kvh), sc in ref["score"].items():
+        T = int(w.seq_lens[b])
+        np.testing.assert_allclose(got["score"][b, kvh, :T], sc, rtol=1e-12, atol=0)
+
+
+def test_two_position_closed_form(oracle):
+    """T=2, d=2: logits (x, 0) -> p0 = 1/(1+e^-x), out = p0 v0 + p1 v1."""
+    spec = synth.WorkloadSpec("cf", 1, 1, 1, 2, 2, "f32", "f32", None, 1, window=1, k_global=1)
+    w = synth.generate(spec, seed=0)
+    a, bk, c = 1.5, 2.0, -0.75
+    w.q_full[:] = torch.tensor([[[a, 0.0]]])
+    w.k[0, 0] = torch.tensor([bk, 0.0])
+    w.k[1, 0] = torch.tensor([0.0, c])
+    w.v[0, 0] = torch.tensor([1.0, -2.0])
+    w.v[1, 0] = torch.tensor([0.5, 4.0])
+    r = run_full(oracle, w)
+    x = a * bk / math.sqrt(2)
+    p0 = 1 / (1 + math.exp(-x))
+    np.testing.assert_allclose(r["out"][0, 0], [p0 * 1.0 + (1 - p0) * 0.5, p0 * -2.0 + (1 - p0) * 4.0],
+                               atol=1e-14)
+    np.testing.assert_allclose(r["lse"][0, 0], math.log(math.exp(x) + 1), atol=1e-14)
+    np.testing.assert_allclose(r["score"][0, 0, :2], [p0, 1 - p0], atol=1e-14)
+    # window = 1 keeps position 1; the single candidate (position 0) fits k_global = 1
+    assert list(r["idx"][0, 0]) == [0, 1]
+
+
+def test_zero_query_gives_uniform_mean_and_lowest_index_ties(oracle):
+    """q = 0: p = 1/T, out = mean of V, every score G/T, so the tie-break
+    (lower index first) decides the whole global selection."""
+    spec = small_spec(seq_len=40, page_size=8)
+    w = synth.generate(spec, seed=3)
+    w.q_full.zero_()
+    r = run_full(oracle, w)
+    V = dequant(w, "v")
+    for b in range(spec.batch):
+        T = int(w.seq_lens[b])
+        sl = synth.slots_of(w, b, torch.arange(T)).numpy()
+        for h in range(spec.num_q_heads):
+            np.testing.assert_allclose(r["out"][b, h], V[sl, h // spec.group].mean(0), atol=1e-14)
+        for kvh in range(spec.num_kv_heads):
+            np.testing.assert_allclose(r["score"][b, kvh, :T], spec.group / T, rtol=1e-14)
+            want = list(range(spec.k_global)) + list(range(T - spec.window, T))
+            assert list(r["idx"][b, kvh]) == [int(x) for x in sl[want]]
+
+
+def test_constant_values_give_that_value(oracle):
+    spec = small_spec(kv_dtype="f32", q_dtype="f32", page_size=None, seq_len=25)
+    w = synth.generate(spec, seed=5)
+    row = torch.linspace(-1, 1, spec.head_dim)
+    w.v[:] = row
+    r = run_full(oracle, w)
+    np.testing.assert_allclose(r["out"], np.broadcast_to(row.double().numpy(), r["out"].shape),
+                               atol=1e-14)
+
+
+def test_scores_sum_to_group_size_and_selection_invariants(oracle):
+    spec = small_spec(seq_len=(1, 60), batch=6, page_size=4)
+    w = synth.generate(spec, seed=7)
+    r = run_full(oracle, w)
+    W, K = spec.window, spec.k_global
+    for b in range(spec.batch):
+        T = int(w.seq_lens[b])
+        sl = synth.slots_of(w, b, torch.arange(T)).numpy()
+        pos_of = {int(s): t for t, s in enumerate(sl)}
+        for kvh in range(spec.num_kv_heads):
+            np.testing.assert_allclose(r["score"][b, kvh, :T].sum(), spec.group, rtol=1e-13)
+            n = int(r["n_sel"][b, kvh])
+            assert n == min(T, W + K)
+            idx = r["idx"][b, kvh]
+            assert all(x == -1 for x in idx[n:])
+            pos = [pos_of[int(x)] for x in idx[:n]]
+            assert pos == sorted(pos) and len(set(pos)) == n
+            assert set(range(max(0, T - W), T)) <= set(pos)
+
+
+def test_selection_matches_exhaustive_ranking(oracle):
+    """Each candidate's rank = #candidates with a higher score, or an equal
+    score at a lower index; the oracle must keep exactly the ranks < K."""
+    spec = small_spec(seq_len=(20, 60), batch=4, page_size=4, window=5, k_global=7)
+    for seed in range(4):
+        w = synth.generate(spec, seed=seed)
+        r = run_full(oracle, w)
+        for b in range(spec.batch):
+            T = int(w.seq_lens[b])
+            sl = synth.slots_of(w, b, torch.arange(T)).numpy()
+            C = max(0, T - spec.window)
+            for kvh in range(spec.num_kv_heads):
+                s = r["score"][b, kvh, :C]
+                keep = [t for t in range(C)
+                        if sum(1 for u in range(C) if s[u] > s[t] or (s[u] == s[t] and u < t))
+                        < spec.k_global]
+                want = sorted(set(keep) | set(range(C, T)))
+                n = int(r["n_sel"][b, kvh])
+                assert list(r["idx"][b, kvh, :n]) == [int(sl[t]) for t in want]
+
+
+def test_planted_key_order_and_ties_decide_selection(oracle):
+    """One head, q = e0: score order follows the planted first key component.
+    Three levels with ties: all of the top level, then the lowest indices of
+    the next level."""
+    T, W, K = 50, 4, 10
+    spec = synth.WorkloadSpec("plant", 1, 1, 1, 4, T, "f32", "f32", None, 1, window=W, k_global=K)
+    w = synth.generate(spec, seed=1)
+    w.q_full[:] = torch.tensor([[[1.0, 0, 0, 0]]])
+    rng = np.random.default_rng(0)
+    level = rng.choice([0, 1, 2], size=T, p=[0.5, 0.42, 0.08])
+    level[:6] = [2, 0, 1, 2, 1, 1]
+    w.k[:, 0, :] = 0.0
+    w.k[:T, 0, 0] = torch.tensor(level, dtype=torch.float32)
+    r = run_full(oracle, w)
+    C = T - W
+    top = [t for t in range(C) if level[t] == 2]
+    assert len(top) < K
+    nxt = [t for t in range(C) if level[t] == 1][:K - len(top)]
+    want = sorted(set(top) | set(nxt) | set(range(C, T)))
+    assert list(r["idx"][0, 0, :len(want)]) == want
+
+
+def test_short_sequences_take_everything(oracle):
+    spec = small_spec(window=8, k_global=5, page_size=4, batch=4)
+    w = synth.generate(spec, seed=2, seq_lens=[1, 8, 13, 14])
+    r = run_full(oracle, w)
+    for b, T in enumerate([1, 8, 13, 14]):
+        sl = synth.slots_of(w, b, torch.arange(T)).numpy()
+        n = min(T, 13)
+        for kvh in range(spec.num_kv_heads):
+            assert int(r["n_sel"][b, kvh]) == n
+            if T <= 13:
+                assert list(r["idx"][b, kvh, :n]) == [int(x) for x in sl]
+
+
+def test_paged_equals_contiguous(oracle):
+    spec = small_spec(page_size=4, seq_len=30, batch=2)
+    wp = synth.generate(spec, seed=9)
+    wc = synth.generate(spec.replace(page_size=None), seed=9)
+    for b in range(2):  # copy the paged data into the contiguous layout
+        sp = synth.slots_of(wp, b, torch.arange(30))
+        sc = synth.slots_of(wc, b, torch.arange(30))
+        wc.k[sc] = wp.k[sp]
+        wc.v[sc] = wp.v[sp]
+    wc.q_full.copy_(wp.q_full)
+    rp, rc = run_full(oracle, wp), run_full(oracle, wc)
+    assert np.array_equal(rp["out"], rc["out"]) and np.array_equal(rp["lse"], rc["lse"])
+    for b in range(2):
+        sp = synth.slots_of(wp, b, torch.arange(30)).numpy()
+        sc = synth.slots_of(wc, b, torch.arange(30)).numpy()
+        m = {int(c): int(p) for c, p in zip(sc, sp)}
+        for kvh in range(2):
+            n = int(rc["n_sel"][b, kvh])
+            assert [m[int(x)] for x in rc["idx"][b, kvh, :n]] == list(rp["idx"][b, kvh, :n])
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "e4m3", "f32"])
+def test_sparse_matches_brute_force_and_full_when_everything_fits(oracle, kv_dtype):
+    q_dtype = "f32" if kv_dtype == "f32" else "bf16"
+    spec = small_spec(kv_dtype=kv_dtype, q_dtype=q_dtype, seq_len=(5, 11), window=4, k_global=8)
+    w = synth.generate(spec, seed=4)
+    full = run_full(oracle, w)
+    # T <= W + K: the index list holds every position, so sparse == full
+    sp = run_sparse(oracle, w, w.q_full, full["idx"])
+    np.testing.assert_allclose(sp, full["out"], atol=1e-12, rtol=0)
+    # own query, shuffled list with holes: brute force over the listed rows
+    rng = np.random.default_rng(1)
+    idx = full["idx"].copy()
+    for b in range(spec.batch):
+        for kvh in range(spec.num_kv_heads):
+            n = int(full["n_sel"][b, kvh])
+            row = idx[b, kvh, :n].copy()
+            rng.shuffle(row)
+            row[::3] = -1
+            idx[b, kvh, :n] = row
+    q = w.q_sparse[0]
+    got = run_sparse(oracle, w, q, idx)
+    qv, K, V = qvals(q, q_dtype), dequant(w, "k"), dequant(w, "v")
+    for b in range(spec.batch):
+        for h in range(spec.num_q_heads):
+            kvh = h // spec.group
+            rows = [int(x) for x in idx[b, kvh] if x >= 0]
+            lg = [mpmath.fsum(mpmath.mpf(qv[b, h, i]) * mpmath.mpf(K[r, kvh, i])
+                              for i in range(spec.head_dim)) / mpmath.sqrt(spec.head_dim) for r in rows]
+            e = [mpmath.exp(x) for x in lg]
+            Z = mpmath.fsum(e)
+            ref = [float(mpmath.fsum(e[j] / Z * mpmath.mpf(V[rows[j], kvh, i]) for j in range(len(rows))))
+                   for i in range(spec.head_dim)]
+            np.testing.assert_allclose(got[b, h], ref, atol=1e-12, rtol=0)
+
+
+def test_sparse_single_row_and_order_independence(oracle):
+    spec = small_spec(seq_len=20)
+    w = synth.generate(spec, seed=6)
+    V = dequant(w, "v")
+    idx = np.full((spec.batch, spec.num_kv_heads, 6), -1, np.int32)
+    idx[:, :, 2] = 17
+    got = run_sparse(oracle, w, w.q_sparse[0], idx)
+    for h in range(spec.num_q_heads):
+        np.testing.assert_allclose(got[:, h], V[17, h // spec.group][None].repeat(2, 0), atol=1e-15)
+    idx2 = np.tile(np.array([3, 9, 4, 12, 0, 7], np.int32), (spec.batch, spec.num_kv_heads, 1))
+    a = run_sparse(oracle, w, w.q_sparse[0], idx2)
+    b = run_sparse(oracle, w, w.q_sparse[0], idx2[:, :, ::-1].copy())
+    np.testing.assert_allclose(a, b, atol=1e-15)
