@@ -1,0 +1,368 @@
+"""Hybrid-Block decode benchmark (HySparse2 Cross-Decoder block on B200).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one decode step of a Hybrid Block: the full-attention layer with
+token selection (hs2_full_attn_select) followed by three sparse-attention
+layers (hs2_sparse_attn), each with its own query, all reading the same
+shared KV cache and the same index list.  The default workload is 256K-token
+decode: batch 4, 4 KV heads, GQA 8, head_dim 128, bf16 paged KV (page 64).
+
+Prints one JSON line (rank 0).  Under torchrun every rank runs its own replica
+(weak scaling, no data-path collective); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_decode_full_b200 import synth  # noqa: E402
+
+METRIC = "Hybrid-Block decode steps/s at 256K ctx; achieved HBM GB/s vs B200 peak"
+DEFAULT_WORKLOAD = "ctx256k_b4_bf16_paged"
+ES = {"f32": 4, "bf16": 2, "e4m3": 1}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def algorithmic_bytes(w: synth.Workload):
+    """Compulsory bytes of one step: the full layer reads every K and V row
+    (+ per-token scales for E4M3) once and writes + reads one fp32 group score
+    per selectable position; each sparse layer reads its listed rows."""
+    s = w.spec
+    lens = [int(x) for x in w.seq_lens.cpu()]
+    row = 2 * s.head_dim * ES[s.kv_dtype] + (8 if s.kv_dtype == "e4m3" else 0)  # K+V (+2 scales)
+    kv = sum(lens) * s.num_kv_heads * row
+    scores = sum(max(0, T - s.window) for T in lens if T - s.window > s.k_global) * s.num_kv_heads * 8
+    rows = sum(min(T, s.window + s.k_global) for T in lens) * s.num_kv_heads * row
+    qo = s.batch * s.num_q_heads * s.head_dim * ES[s.q_dtype] * 2
+    return {"full_attention": kv, "full_layer": kv + scores + qo, "sparse_layer": rows + qo,
+            "step": kv + scores + qo + s.sparse_layers * (rows + qo)}
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def setup_dist(gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle
+def oracle_unit_seconds(w: synth.Workload, b: int, kvh: int):
+    """Time the CPU oracle on one (sequence, kv head) of the workload: the full
+    layer + selection, then every sparse layer.  Returns (seconds, threads)."""
+    import numpy as np
+
+    import oracle
+
+    oracle.build()
+    s = w.spec
+    T = int(w.seq_lens[b])
+    slots = synth.slots_of(w, b, torch.arange(T, device=w.k.device))
+    G = s.group
+    code = {"f32": 0, "bf16": 1, "e4m3": 2}
+    k = synth.raw(w.k[slots, kvh:kvh + 1])
+    v = synth.raw(w.v[slots, kvh:kvh + 1])
+    ks = synth.raw(None if w.k_scale is None else w.k_scale[slots, kvh:kvh + 1])
+    vs = synth.raw(None if w.v_scale is None else w.v_scale[slots, kvh:kvh + 1])
+    qf = synth.raw(w.q_full[b:b + 1, kvh * G:(kvh + 1) * G])
+    qs = [synth.raw(w.q_sparse[l, b:b + 1, kvh * G:(kvh + 1) * G]) for l in range(s.sparse_layers)]
+    t0 = time.perf_counter()
+    r = oracle.full_attn_select(qf, code[s.q_dtype], k, v, code[s.kv_dtype], np.array([T], np.int32), None, T,
+                                s.window, s.k_global, k_scale=ks, v_scale=vs)
+    for q in qs:
+        oracle.sparse_attn(q, code[s.q_dtype], k, v, code[s.kv_dtype], r["idx"], k_scale=ks, v_scale=vs)
+    return time.perf_counter() - t0, 1
+
+
+def cpu_baseline(w: synth.Workload, units: int = 1):
+    """Oracle steps/s estimated from `units` timed (sequence, kv head) units."""
+    s = w.spec
+    total_units = s.batch * s.num_kv_heads
+    secs = 0.0
+    for i in range(units):
+        b, kvh = divmod(i, s.num_kv_heads)
+        t, threads = oracle_unit_seconds(w, b % s.batch, kvh)
+        secs += t
+    per_step = secs / units * total_units
+    return {"value": 1.0 / per_step, "unit": "steps/s", "cores": threads, "kind": "oracle",
+            "sample": f"{units} of {total_units} (sequence, kv head) units of one step (full layer + selection + "
+                      f"{s.sparse_layers} sparse layers), fp64 single-threaded C; step time = unit time x "
+                      f"{total_units}", "seconds_measured": secs}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, rank, world, local):
+    from long_context_decode_full_b200 import hs2
+
+    spec = synth.WORKLOADS[args.workload]
+    w = synth.generate(spec, seed=args.seed + rank, device="cuda")
+    s = spec
+    dev = torch.device("cuda", local)
+    outs = [torch.empty_like(w.q_full) for _ in range(1 + s.sparse_layers)]
+    idx = torch.empty(s.batch, s.num_kv_heads, s.window + s.k_global, dtype=torch.int32, device=dev)
+    ws = hs2.alloc_workspace(s.batch, s.num_kv_heads, s.group, s.head_dim, w.t_cap, dev)
+    stream = torch.cuda.current_stream()
+    K, W = args.steps, args.warmup
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+
+    def step(e=None):
+        hs2.full_attn_select(w.q_full, w.k, w.v, w.seq_lens, w.page_table, w.page_size, s.window, s.k_global,
+                             w.k_scale, w.v_scale, out=outs[0], idx_out=idx, workspace=ws,
+                             mark_event=None if e is None else e[1])
+        if e is not None:
+            e[2].record(stream)
+        for l in range(s.sparse_layers):
+            hs2.sparse_attn(w.q_sparse[l], w.k, w.v, idx, w.k_scale, w.v_scale, w.page_size, out=outs[1 + l])
+
+    for e in ev:  # materialise the event handles before the first marked call
+        for x in e:
+            x.record(stream)
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    if hs2.workspace_status(ws) != 0:
+        raise RuntimeError("device-side wait expired during warm-up: " + hs2.last_error())
+
+    clocks = Clocks(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        step(ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms_total = t_start.elapsed_time(t_end)
+    ms_total = max_over_ranks(ms_total, world)
+    attn_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
+    sel_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(K))
+    ms_step = ms_total / K
+
+    # e2e: queries in from pinned host memory, outputs + index list back, every step
+    q_host = [w.q_full.cpu().pin_memory()] + [w.q_sparse[l].cpu().pin_memory() for l in range(s.sparse_layers)]
+    lens_host = w.seq_lens.cpu().pin_memory()
+    outs_host = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
+    idx_host = torch.empty_like(idx, device="cpu").pin_memory()
+    q_dev = [torch.empty_like(x, device=dev) for x in q_host]
+    lens_dev = torch.empty_like(lens_host, device=dev)
+    h2d = sum(x.numel() * x.element_size() for x in q_host) + lens_host.numel() * 4
+    d2h = sum(x.numel() * x.element_size() for x in outs_host) + idx_host.numel() * 4
+    K2 = max(3, min(K, args.e2e_steps))
+
+    def e2e_step():
+        for a, b in zip(q_dev, q_host):
+            a.copy_(b, non_blocking=True)
+        lens_dev.copy_(lens_host, non_blocking=True)
+        hs2.full_attn_select(q_dev[0], w.k, w.v, lens_dev, w.page_table, w.page_size, s.window, s.k_global,
+                             w.k_scale, w.v_scale, out=outs[0], idx_out=idx, workspace=ws)
+        for l in range(s.sparse_layers):
+            hs2.sparse_attn(q_dev[1 + l], w.k, w.v, idx, w.k_scale, w.v_scale, w.page_size, out=outs[1 + l])
+        for a, b in zip(outs_host, outs):
+            a.copy_(b, non_blocking=True)
+        idx_host.copy_(idx, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    barrier(world)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(K2):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1), world) / K2
+    status = hs2.workspace_status(ws)
+
+    ab = algorithmic_bytes(w)
+    peak, peak_kind = peaks()
+    attn_gbs = ab["full_attention"] / (attn_ms * 1e-3) / 1e9
+    step_gbs = ab["step"] / (ms_step * 1e-3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get(args.workload)
+    res = {
+        "metric": METRIC,
+        "value": world * 1000.0 / ms_step,
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": {"bf16": "bf16", "e4m3": "e4m3", "f32": "f32"}[s.kv_dtype],
+        "data": "synthetic",
+        "config": {"workload": s.name, "batch": s.batch, "seq_len": s.seq_len, "num_kv_heads": s.num_kv_heads,
+                   "gqa_group": s.group, "head_dim": s.head_dim, "kv_dtype": s.kv_dtype, "page_size": s.page_size,
+                   "sparse_layers": s.sparse_layers, "window": s.window, "k_global": s.k_global,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: %.2f GB of K/V read per step, no flush" % (ab["full_attention"] / 1e9)},
+        "roofline": {"bound": "hbm", "kernel": "full_attn_mma_kernel", "achieved": attn_gbs, "peak": peak,
+                     "unit": "GB/s", "frac": attn_gbs / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "algorithmic_bytes_per_launch": ab["full_attention"], "kernel_ms": attn_ms},
+        "step_roofline": {"achieved": step_gbs, "frac": step_gbs / peak, "compulsory_bytes": ab["step"],
+                          "roofline_steps_per_s": peak * 1e9 / ab["step"], "selection_ms": sel_ms,
+                          "sparse_and_rest_ms": ms_step - attn_ms - sel_ms},
+        "e2e": {"value": world * 1000.0 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": K2,
+                "what": "queries copied in from pinned host memory, outputs and index list copied out and synced, "
+                        "every step; the KV cache stays resident"},
+        "gpu_launches": K * (4 + s.sparse_layers),
+        "clocks": clk,
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, args.cpu_units)
+    return res
+
+
+def run_reference(args, rank, world, local):
+    """The oracle as it stands, timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    spec = synth.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = synth.generate(spec, seed=args.seed, device=dev)
+    times = []
+    for i in range(args.warmup + args.steps):
+        b, kvh = divmod(i % (spec.batch * spec.num_kv_heads), spec.num_kv_heads)
+        t, threads = oracle_unit_seconds(w, b, kvh)
+        if i >= args.warmup:
+            times.append(t * spec.batch * spec.num_kv_heads)
+    ms = statistics.mean(times) * 1000.0
+    v = 1000.0 / ms
+    return {"metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": spec.name, "batch": spec.batch, "seq_len": spec.seq_len,
+                       "parallelism": "oracle on host cores"},
+            "cpu_baseline": {"value": v, "unit": "steps/s", "cores": threads, "kind": "oracle",
+                             "sample": "each step = one (sequence, kv head) unit of the workload (full layer + "
+                                       "selection + sparse layers) timed and scaled by the unit count"},
+            "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(synth.WORKLOADS))
+    ap.add_argument("--impl", default="hs2", choices=["hs2", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=500)
+    ap.add_argument("--cpu-units", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        args.warmup = max(0, min(args.warmup, 1))
+        args.steps = max(1, min(args.steps, 3))
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")), 0)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    rank, world, local = setup_dist(args.gpus)
+    try:
+        res = run_gpu(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,171 @@
+/*
+ * hs2.h -- C ABI of libhs2: HySparse2 Cross-Decoder Hybrid-Block decode
+ * attention on NVIDIA B200 (sm_100a).
+ *
+ * The method (HySparse2 announcement for MiMo-V3, "KV Reuse" section and the
+ * two paragraphs after it on token-level selection and the forced window):
+ * a Hybrid Block is one full-attention layer followed by sparse-attention
+ * layers.  The full layer attends over the whole shared KV cache and, in the
+ * same computation, picks important positions from its attention scores; the
+ * sparse layers reuse that KV cache and that index list directly.  Selection
+ * is per token: the most recent 128 tokens are always kept, plus 1,024 global
+ * tokens from outside that window, and both parts are read from the one
+ * shared cache in a single sparse-attention computation.
+ *
+ * Readings fixed where the pages are silent:
+ *   score[t] of a KV head = sum over the query heads of its GQA group of the
+ *   full layer's softmax probability at t; the global part is the top
+ *   k_global of t < T - window by (score desc, position asc), or all such t
+ *   when there are no more than k_global; query head h uses KV head
+ *   floor(h / G); the softmax scale is 1/sqrt(head_dim); the current token's
+ *   K/V are already in the cache at position T-1.
+ *
+ * Conventions for every call:
+ *   - All pointers named "device" are CUDA device pointers on the current
+ *     device; the library never allocates, frees or keeps any of them.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream): no host synchronisation, no device-wide state.
+ *   - Return value: HS2_OK or an error code; on error nothing was launched
+ *     (except HS2_ERR_CUDA, where a launch itself failed) and
+ *     hs2_last_error() describes the problem.
+ *   - Device-side waits are bounded; an expired wait sets a sticky flag in the
+ *     workspace that hs2_workspace_status() reports as HS2_ERR_TIMEOUT.
+ */
+#ifndef HS2_H_
+#define HS2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HS2_OK 0
+#define HS2_ERR_INVALID_ARG 1  /* null pointer, bad shape, mismatched descriptors */
+#define HS2_ERR_UNSUPPORTED 2  /* dtype / head_dim / group / page size not built */
+#define HS2_ERR_WORKSPACE 3    /* workspace missing, too small or misaligned */
+#define HS2_ERR_CUDA 4         /* a CUDA runtime call or a launch failed */
+#define HS2_ERR_TIMEOUT 5      /* a bounded device-side wait expired */
+
+/* Element types. */
+#define HS2_F32 0  /* IEEE fp32 */
+#define HS2_BF16 1 /* bfloat16 */
+#define HS2_E4M3 2 /* OCP FP8 E4M3 ("fn": no inf, S.1111.111 = NaN), per-row fp32 scale */
+
+/*
+ * One K or V cache of the full layer (the cache every layer of the Hybrid
+ * Block reads).  Rows are [num_slots, num_kv_heads, head_dim], row-major,
+ * element type `dtype`.  Position t of sequence b lives in slot
+ *     page_table[b * max_pages + t / page_size] * page_size + t % page_size
+ * or, when the call's page_table is NULL (contiguous layout),
+ *     b * page_size + t         (page_size = per-sequence capacity).
+ * For HS2_E4M3 the stored value is decode(code) * scale[slot * num_kv_heads + h].
+ */
+typedef struct {
+  const void *data;    /* device; 16-byte aligned */
+  const float *scale;  /* device, [num_slots, num_kv_heads]; HS2_E4M3 only, else NULL */
+  int32_t dtype;       /* HS2_F32, HS2_BF16 or HS2_E4M3 */
+  int32_t num_kv_heads;
+  int32_t head_dim;    /* 64 or 128 */
+  int32_t page_size;   /* tokens per page (16, 32 or a multiple of 64 for
+                          HS2_BF16/HS2_E4M3; any >= 1 for HS2_F32) */
+  int64_t num_slots;   /* rows in the cache, < 2^31 */
+} hs2_cache;
+
+/* Per-head query or output vectors: [batch, num_heads, head_dim], row-major. */
+typedef struct {
+  void *data;          /* device; 16-byte aligned */
+  int32_t dtype;       /* HS2_F32 (with an HS2_F32 cache) or HS2_BF16 */
+  int32_t batch;
+  int32_t num_heads;   /* num_kv_heads * G, G in {1, 2, 4, 8} */
+  int32_t head_dim;
+} hs2_heads;
+
+/*
+ * Bytes of workspace hs2_full_attn_select() needs for this shape on the
+ * current device; t_cap = max_pages * page_size (paged) or page_size
+ * (contiguous).  Returns 0 for invalid shapes.
+ */
+size_t hs2_full_attn_select_workspace(int32_t batch, int32_t num_kv_heads, int32_t group,
+                                      int32_t head_dim, int64_t t_cap);
+
+/*
+ * Full-attention layer of a Hybrid Block, with token selection.
+ *
+ *   q          [B, Hq, d] device, the full layer's query of the new token.
+ *   k_cache,
+ *   v_cache    the shared cache (same dtype, heads, head_dim, page_size,
+ *              num_slots); the current token's K/V already at position T_b-1.
+ *   seq_lens   device int32 [B]: T_b, clamped to [0, t_cap] on the device.
+ *   page_table device int32 [B, max_pages], or NULL for the contiguous layout
+ *              (then max_pages must be 1).  Entries past ceil(T_b/page_size)
+ *              are never read.
+ *   window     W >= 0 (the pages use 128), k_global K >= 0 (the pages use
+ *              1,024), W + K >= 1.
+ *   out        [B, Hq, d] device, dtype of q: softmax(q k^T / sqrt(d)) v over
+ *              all T_b positions, per query head (zeros when T_b = 0).
+ *   idx_out    device int32 [B, Hkv, W + K]: for each (b, kv head) the
+ *              selected positions as SLOTS (page table applied), in
+ *              ascending position order, min(T_b, W + K) valid entries, the
+ *              rest -1.  This is the index list every sparse layer reuses.
+ *   workspace  device scratch of at least hs2_full_attn_select_workspace()
+ *              bytes, 256-byte aligned, owned by the caller; its contents
+ *              need no initialisation and are overwritten (except the sticky
+ *              error flag).  One workspace must not serve two calls that
+ *              run concurrently.
+ */
+int hs2_full_attn_select(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                         const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
+                         int32_t window, int32_t k_global, hs2_heads *out, int32_t *idx_out,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * hs2_full_attn_select() that also records `mark_event` (a cudaEvent_t, or
+ * NULL) on `stream` between the attention kernel and the selection kernels,
+ * so a caller can time the two parts with events.  Same arguments, same
+ * results.
+ */
+int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                                const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
+                                int32_t window, int32_t k_global, hs2_heads *out, int32_t *idx_out,
+                                void *workspace, size_t workspace_bytes, void *stream, void *mark_event);
+
+/*
+ * Sparse-attention layer of a Hybrid Block: for each (b, query head h) the
+ * softmax of q_l k^T / sqrt(d) over the rows idx[b, floor(h/G), :] (slots,
+ * -1 entries skipped), times those V rows.  It reads the same shared cache as
+ * the full layer and the index list that hs2_full_attn_select() wrote; its
+ * query q_l is the layer's own.  A (b, head) with no valid row gets zeros.
+ *
+ *   idx        device int32 [B, Hkv, idx_stride], idx_stride in [1, 4096].
+ *   out        [B, Hq, d] device, dtype of q_l.
+ * Needs no workspace.
+ */
+int hs2_sparse_attn(const hs2_heads *q_l, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                    const int32_t *idx, int32_t idx_stride, hs2_heads *out, void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the workspace's sticky
+ * device-error flag: HS2_OK, or HS2_ERR_TIMEOUT if a bounded device wait of
+ * an earlier call on this workspace expired.
+ */
+int hs2_workspace_status(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Device-to-device copy of `bytes` (a multiple of 16, both pointers 16-byte
+ * aligned) with a grid sized to the SM count: the HBM copy-bandwidth
+ * reference that the roofline is quoted against.
+ */
+int hs2_copy_peak(void *dst, const void *src, size_t bytes, void *stream);
+
+/* Thread-local text of the last non-zero status returned on this thread. */
+const char *hs2_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int hs2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HS2_H_ */

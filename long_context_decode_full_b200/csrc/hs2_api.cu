@@ -1,0 +1,412 @@
+// hs2_api.cu -- the C ABI of libhs2 (declared in include/hs2.h): argument
+// validation, workspace layout, TMA descriptors and the launch sequence of
+// the full-attention + selection call and of the sparse call.
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "hs2.h"
+#include "hs2_internal.h"
+
+using namespace hs2;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+  return fail(HS2_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxCtasPerSm = 4;  // bound used to size the per-unit record slots
+
+int sm_count() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// ---------------------------------------------------------------- TMA encode
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [num_slots, Hkv, D] cache -> 3-D map (D, Hkv, slots), box (128 bytes, 1, rows), 128-byte swizzle.
+int encode_cache_map(CUtensorMap *map, const hs2_cache *c, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int es = c->dtype == HS2_BF16 ? 2 : 1;
+  cuuint64_t dims[3] = {(cuuint64_t)c->head_dim, (cuuint64_t)c->num_kv_heads, (cuuint64_t)c->num_slots};
+  cuuint64_t strides[2] = {(cuuint64_t)c->head_dim * es, (cuuint64_t)c->head_dim * c->num_kv_heads * es};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / es), 1u, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, c->dtype == HS2_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                  const_cast<void *>(c->data), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return HS2_OK;
+}
+
+// ---------------------------------------------------------------- workspace
+struct Layout {
+  size_t err, prefix, records, logits, scores, cand, sel, tie, hist, thr, total;
+  int R;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Layout layout(int B, int Hkv, int G, int D, int64_t t_cap) {
+  Layout L;
+  const size_t U = (size_t)B * Hkv;
+  const size_t words = (size_t)((t_cap + 31) / 32);
+  L.R = sm_count() * kMaxCtasPerSm / Hkv + 2;
+  size_t o = 0;
+  L.err = o;
+  o += 256;
+  L.prefix = o;
+  o = align256(o + (size_t)(B + 1) * 4);
+  L.records = o;
+  o = align256(o + U * L.R * G * (D + 2) * 4);
+  L.logits = o;
+  o = align256(o + U * (size_t)t_cap * G * 4);
+  L.scores = o;
+  o = align256(o + U * (size_t)t_cap * 4);
+  L.cand = o;
+  o = align256(o + U * (size_t)t_cap * 8);
+  L.sel = o;
+  o = align256(o + U * words * 4);
+  L.tie = o;
+  o = align256(o + U * words * 4);
+  L.hist = o;  // hist [U][4096], ticket [U], cand_count [U] back to back
+  o = align256(o + U * (kHistBins + 2) * 4);
+  L.thr = o;
+  o = align256(o + U * 8);
+  L.total = o;
+  return L;
+}
+
+FullWs bind(const Layout &L, void *ws, int B, int Hkv) {
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  const size_t U = (size_t)B * Hkv;
+  FullWs f;
+  f.err = reinterpret_cast<uint32_t *>(w + L.err);
+  f.prefix = reinterpret_cast<int32_t *>(w + L.prefix);
+  f.records = reinterpret_cast<float *>(w + L.records);
+  f.logits = reinterpret_cast<float *>(w + L.logits);
+  f.scores = reinterpret_cast<float *>(w + L.scores);
+  f.cand = reinterpret_cast<uint2 *>(w + L.cand);
+  f.sel = reinterpret_cast<uint32_t *>(w + L.sel);
+  f.tie = reinterpret_cast<uint32_t *>(w + L.tie);
+  f.hist = reinterpret_cast<uint32_t *>(w + L.hist);
+  f.ticket = f.hist + U * kHistBins;
+  f.cand_count = f.ticket + U;
+  f.thr = reinterpret_cast<int2 *>(w + L.thr);
+  return f;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int group_ok(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
+
+// Checks a q/out descriptor against the cache; `what` names it in errors.
+int check_heads(const hs2_heads *h, const hs2_cache *k, const char *what) {
+  if (!h || !h->data) return fail(HS2_ERR_INVALID_ARG, "%s is NULL", what);
+  if (!aligned16(h->data)) return fail(HS2_ERR_INVALID_ARG, "%s data is not 16-byte aligned", what);
+  if (h->batch < 1 || h->batch > 65535) return fail(HS2_ERR_INVALID_ARG, "%s batch %d out of [1, 65535]", what, h->batch);
+  if (h->head_dim != k->head_dim)
+    return fail(HS2_ERR_INVALID_ARG, "%s head_dim %d != cache head_dim %d", what, h->head_dim, k->head_dim);
+  if (h->num_heads < 1 || h->num_heads % k->num_kv_heads)
+    return fail(HS2_ERR_INVALID_ARG, "%s num_heads %d is not a multiple of num_kv_heads %d", what, h->num_heads,
+                k->num_kv_heads);
+  if (!group_ok(h->num_heads / k->num_kv_heads))
+    return fail(HS2_ERR_UNSUPPORTED, "GQA group %d not built (1, 2, 4 or 8)", h->num_heads / k->num_kv_heads);
+  const int want = k->dtype == HS2_F32 ? HS2_F32 : HS2_BF16;
+  if (h->dtype != want)
+    return fail(HS2_ERR_UNSUPPORTED, "%s dtype %d with cache dtype %d (need %s)", what, h->dtype, k->dtype,
+                want == HS2_F32 ? "HS2_F32" : "HS2_BF16");
+  return HS2_OK;
+}
+
+int check_caches(const hs2_cache *k, const hs2_cache *v) {
+  if (!k || !v || !k->data || !v->data) return fail(HS2_ERR_INVALID_ARG, "k_cache / v_cache is NULL");
+  if (k->dtype != v->dtype || k->num_kv_heads != v->num_kv_heads || k->head_dim != v->head_dim ||
+      k->page_size != v->page_size || k->num_slots != v->num_slots)
+    return fail(HS2_ERR_INVALID_ARG, "k_cache and v_cache descriptors disagree");
+  if (k->dtype != HS2_F32 && k->dtype != HS2_BF16 && k->dtype != HS2_E4M3)
+    return fail(HS2_ERR_UNSUPPORTED, "cache dtype %d", k->dtype);
+  if (k->head_dim != 64 && k->head_dim != 128) return fail(HS2_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", k->head_dim);
+  if (k->dtype == HS2_E4M3 && k->head_dim != 128) return fail(HS2_ERR_UNSUPPORTED, "E4M3 caches need head_dim 128");
+  if (k->num_kv_heads < 1 || k->num_kv_heads > 65535) return fail(HS2_ERR_INVALID_ARG, "num_kv_heads %d", k->num_kv_heads);
+  if (k->num_slots < 1 || k->num_slots >= (int64_t(1) << 31))
+    return fail(HS2_ERR_INVALID_ARG, "num_slots %lld out of [1, 2^31)", (long long)k->num_slots);
+  if (k->page_size < 1) return fail(HS2_ERR_INVALID_ARG, "page_size %d", k->page_size);
+  if (!aligned16(k->data) || !aligned16(v->data)) return fail(HS2_ERR_INVALID_ARG, "cache data not 16-byte aligned");
+  if (k->dtype == HS2_E4M3) {
+    if (!k->scale || !v->scale) return fail(HS2_ERR_INVALID_ARG, "E4M3 caches need k and v scales");
+  } else if (k->scale || v->scale) {
+    return fail(HS2_ERR_INVALID_ARG, "scales are only used with HS2_E4M3 caches");
+  }
+  return HS2_OK;
+}
+
+FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged) {
+  FullMmaConfig c{4, 4};
+  (void)D;
+  (void)fp8;
+  if (const char *env = getenv("HS2_FULL_CFG")) {
+    int a = 0, b = 0;
+    if (sscanf(env, "%d,%d", &a, &b) == 2) c = FullMmaConfig{a, b};
+  }
+  const int tile = 16 * c.ncw;
+  if (paged && !(page_size % tile == 0 || tile % page_size == 0)) c = FullMmaConfig{4, 4};
+  return c;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *hs2_last_error(void) { return g_err; }
+
+int hs2_version(void) { return 100; }
+
+size_t hs2_full_attn_select_workspace(int32_t batch, int32_t num_kv_heads, int32_t group, int32_t head_dim,
+                                      int64_t t_cap) {
+  if (batch < 1 || num_kv_heads < 1 || !group_ok(group) || (head_dim != 64 && head_dim != 128) || t_cap < 1)
+    return 0;
+  return layout(batch, num_kv_heads, group, head_dim, t_cap).total;
+}
+
+int hs2_full_attn_select(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                         const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages, int32_t window,
+                         int32_t k_global, hs2_heads *out, int32_t *idx_out, void *workspace,
+                         size_t workspace_bytes, void *stream) {
+  return hs2_full_attn_select_marked(q, k_cache, v_cache, seq_lens, page_table, max_pages, window, k_global, out,
+                                     idx_out, workspace, workspace_bytes, stream, nullptr);
+}
+
+int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                                const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
+                                int32_t window, int32_t k_global, hs2_heads *out, int32_t *idx_out,
+                                void *workspace, size_t workspace_bytes, void *stream, void *mark_event) {
+  int rc;
+  if ((rc = check_caches(k_cache, v_cache))) return rc;
+  if ((rc = check_heads(q, k_cache, "q"))) return rc;
+  if ((rc = check_heads(out, k_cache, "out"))) return rc;
+  if (out->batch != q->batch || out->num_heads != q->num_heads || out->dtype != q->dtype)
+    return fail(HS2_ERR_INVALID_ARG, "out shape/dtype differs from q");
+  if (!seq_lens || !idx_out) return fail(HS2_ERR_INVALID_ARG, "seq_lens / idx_out is NULL");
+  if (window < 0 || k_global < 0 || (int64_t)window + k_global < 1 || (int64_t)window + k_global > (1 << 24))
+    return fail(HS2_ERR_INVALID_ARG, "window %d / k_global %d", window, k_global);
+  const int B = q->batch, Hkv = k_cache->num_kv_heads, G = q->num_heads / Hkv, D = k_cache->head_dim;
+  const int ps = k_cache->page_size;
+  const bool paged = page_table != nullptr;
+  int64_t t_cap;
+  if (paged) {
+    if (max_pages < 1) return fail(HS2_ERR_INVALID_ARG, "max_pages %d with a page table", max_pages);
+    t_cap = (int64_t)max_pages * ps;
+  } else {
+    if (max_pages != 1) return fail(HS2_ERR_INVALID_ARG, "contiguous layout (no page table) needs max_pages == 1");
+    t_cap = ps;
+    if ((int64_t)B * ps > k_cache->num_slots)
+      return fail(HS2_ERR_INVALID_ARG, "contiguous layout needs num_slots >= batch * page_size");
+  }
+  if (t_cap > (int64_t(1) << 30) || (int64_t)B * ((t_cap + 15) / 16) * Hkv >= (int64_t(1) << 31))
+    return fail(HS2_ERR_UNSUPPORTED, "context capacity too large");
+  if (B > kMaxBatchSmem) return fail(HS2_ERR_UNSUPPORTED, "batch %d > %d", B, kMaxBatchSmem);
+  const bool mma = k_cache->dtype != HS2_F32;
+  if (mma && paged && !(ps % 16 == 0 && (ps % 64 == 0 || 64 % ps == 0)))
+    return fail(HS2_ERR_UNSUPPORTED, "page_size %d (16, 32 or a multiple of 64)", ps);
+  const Layout L = layout(B, Hkv, G, D, t_cap);
+  if (!workspace) return fail(HS2_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return fail(HS2_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  if (workspace_bytes < L.total)
+    return fail(HS2_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, L.total);
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  FullParams p{};
+  p.q = q->data;
+  p.k = k_cache->data;
+  p.v = v_cache->data;
+  p.k_scale = k_cache->scale;
+  p.v_scale = v_cache->scale;
+  p.seq_lens = seq_lens;
+  p.page_table = page_table;
+  p.B = B;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.D = D;
+  p.page_size = ps;
+  p.max_pages = paged ? max_pages : 1;
+  p.t_cap = t_cap;
+  p.num_slots = k_cache->num_slots;
+  p.R = L.R;
+  p.c = 1.0f / sqrtf((float)D);
+  p.ws = bind(L, workspace, B, Hkv);
+  const int sms = sm_count();
+  cudaError_t e;
+  if (!mma) {
+    p.tile = full_f32_tile();
+    p.N = sms * full_f32_ctas_per_sm();
+    e = launch_full_f32(p, p.N, s);
+    if (e != cudaSuccess) return cuda_fail(e, "full-attention (fp32) launch");
+  } else {
+    const bool fp8 = k_cache->dtype == HS2_E4M3;
+    const FullMmaConfig cfg = pick_full_config(D, fp8, ps, paged);
+    p.tile = 16 * cfg.ncw;
+    p.N = sms;
+    const int box_rows = paged ? (ps < p.tile ? ps : p.tile) : p.tile;
+    CUtensorMap tmk, tmv;
+    if ((rc = encode_cache_map(&tmk, k_cache, box_rows))) return rc;
+    if ((rc = encode_cache_map(&tmv, v_cache, box_rows))) return rc;
+    e = launch_full_mma(p, tmk, tmv, fp8, cfg, p.N, s);
+    if (e == cudaErrorInvalidConfiguration)
+      return fail(HS2_ERR_UNSUPPORTED, "no full-attention kernel built for ncw=%d nstage=%d", cfg.ncw, cfg.nstage);
+    if (e != cudaSuccess) return cuda_fail(e, "full-attention launch");
+  }
+  if (mark_event) {
+    e = cudaEventRecord(static_cast<cudaEvent_t>(mark_event), s);
+    if (e != cudaSuccess) return cuda_fail(e, "recording the mark event");
+  }
+  ScoreParams sp{};
+  sp.seq_lens = seq_lens;
+  sp.page_table = page_table;
+  sp.out = out->data;
+  sp.out_dtype = out->dtype == HS2_F32 ? 0 : 1;
+  sp.idx_out = idx_out;
+  sp.B = B;
+  sp.Hkv = Hkv;
+  sp.G = G;
+  sp.D = D;
+  sp.page_size = ps;
+  sp.max_pages = p.max_pages;
+  sp.t_cap = t_cap;
+  sp.window = window;
+  sp.k_global = k_global;
+  sp.N = p.N;
+  sp.R = p.R;
+  sp.tile = p.tile;
+  sp.c = p.c;
+  sp.ws = p.ws;
+  e = launch_select(sp, s);
+  if (e != cudaSuccess) return cuda_fail(e, "selection launch");
+  return HS2_OK;
+}
+
+int hs2_sparse_attn(const hs2_heads *q_l, const hs2_cache *k_cache, const hs2_cache *v_cache, const int32_t *idx,
+                    int32_t idx_stride, hs2_heads *out, void *stream) {
+  int rc;
+  if ((rc = check_caches(k_cache, v_cache))) return rc;
+  if ((rc = check_heads(q_l, k_cache, "q_l"))) return rc;
+  if ((rc = check_heads(out, k_cache, "out"))) return rc;
+  if (out->batch != q_l->batch || out->num_heads != q_l->num_heads || out->dtype != q_l->dtype)
+    return fail(HS2_ERR_INVALID_ARG, "out shape/dtype differs from q_l");
+  if (!idx) return fail(HS2_ERR_INVALID_ARG, "idx is NULL");
+  if (idx_stride < 1 || idx_stride > 4096) return fail(HS2_ERR_UNSUPPORTED, "idx_stride %d out of [1, 4096]", idx_stride);
+  SparseParams p{};
+  p.q = q_l->data;
+  p.k = k_cache->data;
+  p.v = v_cache->data;
+  p.k_scale = k_cache->scale;
+  p.v_scale = v_cache->scale;
+  p.idx = idx;
+  p.out = out->data;
+  p.B = q_l->batch;
+  p.Hkv = k_cache->num_kv_heads;
+  p.G = q_l->num_heads / p.Hkv;
+  p.D = k_cache->head_dim;
+  p.L = idx_stride;
+  p.c = 1.0f / sqrtf((float)p.D);
+  // enough CTAs per unit to cover the SMs, at most 16 per cluster and 256 rows per CTA
+  const int units = p.B * p.Hkv, sms = sm_count();
+  const int want = (sms + units - 1) / units;
+  const int cap = units * 8 <= sms / 2 ? 16 : 8;  // 16-CTA clusters only when units are few
+  int S = want < 1 ? 1 : (want > cap ? cap : want);
+  const int min_s = (idx_stride + 255) / 256;
+  if (S < min_s) S = min_s;
+  int rows = ((idx_stride + S - 1) / S + 15) / 16 * 16;
+  S = (idx_stride + rows - 1) / rows;
+  p.rows_per_cta = rows;
+  p.splits = S;
+  cudaError_t e = launch_sparse_impl(p, k_cache->dtype, k_cache->num_slots, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "sparse-attention launch");
+  return HS2_OK;
+}
+
+int hs2_workspace_status(void *workspace, size_t workspace_bytes, void *stream) {
+  if (!workspace || workspace_bytes < 256) return fail(HS2_ERR_WORKSPACE, "workspace is NULL or too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t flag = 0;
+  cudaError_t e = cudaMemcpyAsync(&flag, workspace, 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, 4, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the workspace status");
+  if (flag) return fail(HS2_ERR_TIMEOUT, "device error flag 0x%x (1: consumer wait, 2: producer wait, 4: record)", flag);
+  return HS2_OK;
+}
+
+int hs2_copy_peak(void *dst, const void *src, size_t bytes, void *stream) {
+  if (!dst || !src || (bytes & 15) || !aligned16(dst) || !aligned16(src))
+    return fail(HS2_ERR_INVALID_ARG, "copy needs 16-byte aligned pointers and a multiple of 16 bytes");
+  cudaError_t e = launch_copy(dst, src, bytes, sm_count() * 4, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "copy launch");
+  return HS2_OK;
+}
+
+}  // extern "C"
+
+namespace hs2 {
+
+__global__ void __launch_bounds__(512) copy_kernel(uint4 *__restrict__ dst, const uint4 *__restrict__ src, size_t n) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n; i += 4 * stride) {
+    const uint4 a = __ldcs(src + i), b = __ldcs(src + i + stride), c = __ldcs(src + i + 2 * stride),
+                d = __ldcs(src + i + 3 * stride);
+    __stcs(dst + i, a);
+    __stcs(dst + i + stride, b);
+    __stcs(dst + i + 2 * stride, c);
+    __stcs(dst + i + 3 * stride, d);
+  }
+  for (; i < n; i += stride) __stcs(dst + i, __ldcs(src + i));
+}
+
+cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int grid, cudaStream_t s) {
+  if (bytes == 0) return cudaSuccess;
+  copy_kernel<<<grid, 512, 0, s>>>(static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), bytes / 16);
+  return cudaGetLastError();
+}
+
+}  // namespace hs2

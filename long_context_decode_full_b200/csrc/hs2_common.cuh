@@ -1,0 +1,209 @@
+// hs2_common.cuh -- shared device helpers of libhs2 (sm_100a).
+//
+// PTX wrappers (mbarrier, TMA bulk-tensor loads, cp.async, ldmatrix,
+// mma.sync), the workspace layout and the balanced tile partition that the
+// full-attention kernels and the score kernel agree on.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hs2 {
+
+// ---------------------------------------------------------------- constants
+constexpr int kHistBins = 4096;          // score histogram: float bits 30..19
+constexpr int kHistShift = 19;
+constexpr int kScoreChunk = 4096;        // positions per score / filter CTA
+constexpr int kScoreThreads = 256;
+constexpr int kFinalThreads = 1024;
+constexpr long long kSpinLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
+constexpr int kMaxBatchSmem = 4096;      // sequences whose tile prefix fits in smem
+
+// Error bits of the sticky workspace flag.
+constexpr uint32_t kErrFullWait = 1u;    // consumer timed out on a full barrier
+constexpr uint32_t kErrEmptyWait = 2u;   // producer timed out on an empty barrier
+constexpr uint32_t kErrRecord = 4u;      // record index outside its unit's slots
+
+// ---------------------------------------------------------------- workspace
+// Every array of the full-attention call lives in the caller's workspace.
+struct FullWs {
+  uint32_t *err;         // sticky error flag (offset 0 of the workspace)
+  int32_t *prefix;       // [B + 1] tiles before sequence b (tile = kernel's TILE positions)
+  float *logits;         // [U, t_cap, G] raw q.k per position and head (fp32, unscaled)
+  float *records;        // [U, R, G * (D + 2)]: m[G], l[G], o[G][D] of each segment
+  float *scores;         // [U, t_cap] group score of the selectable positions
+  uint2 *cand;           // [U, t_cap] (score bits, position) of the threshold bin
+  uint32_t *sel;         // [U, words] positions strictly above the threshold
+  uint32_t *tie;         // [U, words] positions equal to the threshold score
+  uint32_t *hist;        // [U, kHistBins]
+  uint32_t *ticket;      // [U]
+  uint32_t *cand_count;  // [U]
+  int2 *thr;             // [U] (threshold bin, count strictly above it)
+};
+
+// Balanced partition of the tile space over N persistent CTAs.  Tiles are
+// ordered by (sequence, kv head, tile); CTA c owns [c*total/N, (c+1)*total/N).
+// A unit (sequence, kv head) is cut into segments, one per CTA that touches
+// it; segment j of unit u writes record u*R + j, with j = c - cfirst(U_u).
+struct Partition {
+  int64_t total;  // Hkv * sum_b n_b
+  int32_t N;      // CTAs
+  __device__ __forceinline__ int64_t start(int64_t c) const { return c * total / N; }
+  // the CTA that owns tile x
+  __device__ __forceinline__ int64_t cfirst(int64_t x) const { return ((x + 1) * N - 1) / total; }
+};
+
+// ---------------------------------------------------------------- misc
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void set_error(uint32_t *err, uint32_t bit) {
+  if (err) atomicOr(err, bit);
+}
+
+__device__ __forceinline__ int clamp_len(int t, int t_cap) { return t < 0 ? 0 : (t > t_cap ? t_cap : t); }
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase with the given parity to complete; gives up after
+// kSpinLimitCycles and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(a, parity)) {
+    if (clock64() - t0 > kSpinLimitCycles) return false;
+  }
+  return true;
+}
+// cp.async completion of this thread's earlier copies arrives on `bar`
+// (the barrier's expected count must include this arrival).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// ---------------------------------------------------------------- TMA
+// 3-D tiled bulk-tensor load into this CTA's shared memory (no multicast).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint64_t *bar, int x,
+                                            int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------------------------- cp.async
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// ---------------------------------------------------------------- ldmatrix / mma
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void lds128(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// D(16x8, f32) += A(16x16) * B(16x8); A rows = M, B columns = N.
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                        uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+// two E4M3 codes (low byte first) -> two f16 (exact)
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes16) {
+  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes16 & 0xFFFFu), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// 128-byte swizzle of a [rows][128 B] panel (the TMA SWIZZLE_128B pattern):
+// 16-byte chunk c of row r lives at chunk c ^ (r & 7).
+__device__ __forceinline__ uint32_t swz(uint32_t panel, int row, int chunk) {
+  return panel + row * 128 + (((chunk ^ row) & 7) << 4);
+}
+
+// ---------------------------------------------------------------- warp reductions
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace hs2

@@ -1,0 +1,437 @@
+// hs2_full_attn.cu -- the full-attention layer of a Hybrid Block, split over
+// the context (HySparse2 announcement, "KV Reuse" section: the full layer
+// attends over the whole shared KV cache and its attention scores drive the
+// token selection).
+//
+// One persistent CTA per SM walks a balanced share of the (sequence, kv head,
+// tile) space.  A producer warp streams K and V tiles with TMA bulk-tensor
+// loads into a ring of shared-memory stages (mbarrier full/empty pairs, every
+// wait bounded); consumer warps each take 16 rows of a tile, run Q K^T and
+// V^T P^T on the tensor cores with an online softmax, and store the raw
+// logits that the score pass turns into group probabilities.  At the end of
+// each segment (a run of tiles of one unit inside one CTA) the consumer warps
+// merge their states into one (m, l, o) record.
+//
+// The fp32 cache variant runs the same partition on the CUDA cores (FFMA), so
+// fp32 logits keep full fp32 accuracy.
+#include "hs2_internal.h"
+#include "hs2_warp_attn.cuh"
+
+namespace hs2 {
+
+namespace {
+
+struct StageMeta {
+  int32_t b, kvh, tile, flags;
+  int32_t rec, T, pad0, pad1;
+};
+constexpr int kFirst = 1, kLast = 2, kDone = 4;
+
+template <int D, bool FP8, int NCW, int NSTAGE>
+struct Cfg {
+  static constexpr int TILE = 16 * NCW;
+  static constexpr int ES = FP8 ? 1 : 2;
+  static constexpr int ROWB = D * ES;
+  static constexpr int NPANEL = ROWB / 128;
+  static constexpr int PANEL = TILE * 128;
+  static constexpr int KVB = TILE * ROWB;
+  static constexpr int SCB = FP8 ? 2 * TILE * 4 : 0;
+  static constexpr int STAGE = 2 * KVB;
+  static constexpr int WSTRIDE = 16 + 8 * D;
+  static constexpr size_t OFF_SC = (size_t)NSTAGE * STAGE;
+  static constexpr size_t OFF_SCR = OFF_SC + (size_t)NSTAGE * SCB;
+  static constexpr size_t OFF_BAR = OFF_SCR + (size_t)NCW * WSTRIDE * 4;
+  static constexpr size_t OFF_META = OFF_BAR + (2 * NSTAGE + 1) * 8;
+  static constexpr size_t OFF_PREFIX = OFF_META + NSTAGE * sizeof(StageMeta);
+  static size_t bytes(int B) { return OFF_PREFIX + (size_t)(B + 1) * 4 + 1024; }
+  static_assert(ROWB % 128 == 0, "rows are whole 128-byte panels");
+};
+
+__device__ __forceinline__ int64_t slot_of(const int32_t *pt, int max_pages, int ps, int b, int64_t pos) {
+  if (pt == nullptr) return (int64_t)b * ps + pos;
+  return (int64_t)__ldg(pt + (int64_t)b * max_pages + pos / ps) * ps + pos % ps;
+}
+
+// Rendezvous of the consumer warps (bounded, unlike a named barrier, so a
+// warp that gave up on a wait cannot leave the others blocked forever).
+__device__ __forceinline__ bool consumer_sync(uint64_t *bar, uint32_t &phase) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase);
+  phase ^= 1u;
+  return ok;
+}
+
+// Tile prefix per sequence: prefix[b] = sum_{b' < b} ceil(T_b' / tile).
+__device__ void compute_prefix(const FullParams &p, int32_t *prefix, int tile) {
+  const int lane = threadIdx.x & 31;
+  int carry = 0;
+  for (int base = 0; base < p.B; base += 32) {
+    const int b = base + lane;
+    int n = 0;
+    if (b < p.B) {
+      const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
+      n = (T + tile - 1) / tile;
+    }
+    int x = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (b < p.B) prefix[b + 1] = carry + x;
+    carry += __shfl_sync(0xffffffffu, x, 31);
+  }
+  if (lane == 0) prefix[0] = 0;
+}
+
+// Zero the histogram / ticket / candidate counters of the selection pass.
+__device__ __forceinline__ void zero_counters(const FullParams &p, int tid, int nthreads) {
+  const int64_t U = (int64_t)p.B * p.Hkv;
+  const int64_t words = U * (kHistBins + 2);
+  for (int64_t i = (int64_t)blockIdx.x * nthreads + tid; i < words; i += (int64_t)gridDim.x * nthreads)
+    p.ws.hist[i] = 0u;
+}
+
+// Locate the sequence that owns linear tile x (prefix in shared memory).
+__device__ __forceinline__ int find_seq(const int32_t *prefix, int B, int Hkv, int64_t x) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {  // last b with Hkv * prefix[b] <= x
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int64_t)Hkv * prefix[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int D, bool FP8, int NCW, int NSTAGE>
+__global__ void __launch_bounds__(32 * (NCW + 1), 1)
+    full_attn_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                         const FullParams p) {
+  using C = Cfg<D, FP8, NCW, NSTAGE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float *scales = reinterpret_cast<float *>(smem + C::OFF_SC);
+  float *scratch = reinterpret_cast<float *>(smem + C::OFF_SCR);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+  uint64_t *empty = full + NSTAGE;
+  uint64_t *cbar = empty + NSTAGE;  // consumer-warp rendezvous at segment ends
+  StageMeta *meta = reinterpret_cast<StageMeta *>(smem + C::OFF_META);
+  int32_t *prefix = reinterpret_cast<int32_t *>(smem + C::OFF_PREFIX);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool producer = warp == NCW;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&full[s], FP8 ? 33u : 1u);
+      mbar_init(&empty[s], (uint32_t)NCW);
+    }
+    mbar_init(cbar, (uint32_t)NCW);
+    fence_mbar_init();
+  }
+  if (producer) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmk);
+      prefetch_tensormap(&tmv);
+    }
+    compute_prefix(p, prefix, C::TILE);
+  } else {
+    zero_counters(p, threadIdx.x, NCW * 32);
+  }
+  __syncthreads();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i <= p.B; i += blockDim.x) p.ws.prefix[i] = prefix[i];
+
+  const int64_t total = (int64_t)p.Hkv * prefix[p.B];
+  if (total == 0) return;
+  const Partition part{total, p.N};
+  const int64_t g0 = part.start(blockIdx.x), g1 = part.start(blockIdx.x + 1);
+
+  if (producer) {
+    // ------------------------------------------------------------ producer
+    const int RB = p.page_table ? min(C::TILE, p.page_size) : C::TILE;
+    int it = 0;
+    int b = g0 < g1 ? find_seq(prefix, p.B, p.Hkv, g0) : 0;
+    bool ok = true;
+    for (int64_t g = g0; g < g1; ++g, ++it) {
+      while ((int64_t)p.Hkv * prefix[b + 1] <= g) ++b;
+      const int nb = prefix[b + 1] - prefix[b];
+      const int64_t r = g - (int64_t)p.Hkv * prefix[b];
+      const int kvh = (int)(r / nb), i = (int)(r % nb);
+      const int64_t U = (int64_t)p.Hkv * prefix[b] + (int64_t)kvh * nb;
+      const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
+      const int stage = it % NSTAGE;
+      if (it >= NSTAGE && !mbar_wait(&empty[stage], ((it / NSTAGE) - 1) & 1)) {
+        set_error(p.ws.err, kErrEmptyWait);
+        ok = false;
+        break;
+      }
+      const int64_t j = blockIdx.x - part.cfirst(U);
+      const int64_t u = (int64_t)b * p.Hkv + kvh;
+      const int p0 = i * C::TILE;
+      if constexpr (FP8) {
+        float *ks = scales + stage * (2 * C::TILE);
+        for (int rr = lane; rr < C::TILE; rr += 32) {
+          const int pos = p0 + rr;
+          const int64_t slot = pos < T ? slot_of(p.page_table, p.max_pages, p.page_size, b, pos) : -1;
+          if (slot >= 0 && slot < p.num_slots) {
+            cp_async_4(smem_u32(ks + rr), p.k_scale + slot * p.Hkv + kvh);
+            cp_async_4(smem_u32(ks + C::TILE + rr), p.v_scale + slot * p.Hkv + kvh);
+          }
+        }
+        cp_async_mbar_arrive_noinc(&full[stage]);
+      }
+      if (lane == 0) {
+        StageMeta mt;
+        mt.b = b;
+        mt.kvh = kvh;
+        mt.tile = i;
+        mt.flags = ((i == 0 || g == g0) ? kFirst : 0) | ((i == nb - 1 || g == g1 - 1) ? kLast : 0);
+        mt.rec = (j >= 0 && j < p.R) ? (int)(u * p.R + j) : -1;
+        if (mt.rec < 0) set_error(p.ws.err, kErrRecord);
+        mt.T = T;
+        meta[stage] = mt;
+        uint32_t bytes = 0;
+        for (int rr = 0; rr < C::TILE && p0 + rr < T; rr += RB) bytes += 2u * RB * C::ROWB;
+        mbar_arrive_expect_tx(&full[stage], bytes);
+        const uint32_t kdst = sbase + stage * C::STAGE, vdst = kdst + C::KVB;
+        for (int rr = 0; rr < C::TILE && p0 + rr < T; rr += RB) {
+          const int slot = (int)slot_of(p.page_table, p.max_pages, p.page_size, b, p0 + rr);
+#pragma unroll
+          for (int pn = 0; pn < C::NPANEL; ++pn) {
+            tma_load_3d(kdst + pn * C::PANEL + rr * 128, &tmk, &full[stage], pn * (128 / C::ES), kvh, slot);
+            tma_load_3d(vdst + pn * C::PANEL + rr * 128, &tmv, &full[stage], pn * (128 / C::ES), kvh, slot);
+          }
+        }
+      }
+      __syncwarp();
+    }
+    if (ok) {  // end-of-work sentinel
+      const int stage = it % NSTAGE;
+      if (it >= NSTAGE && !mbar_wait(&empty[stage], ((it / NSTAGE) - 1) & 1)) {
+        set_error(p.ws.err, kErrEmptyWait);
+      } else {
+        if (lane == 0) {
+          meta[stage].flags = kDone;
+          mbar_arrive(&full[stage]);
+        }
+        if constexpr (FP8) mbar_arrive(&full[stage]);
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  WarpAttn<D, FP8> st;
+  st.reset();
+  uint32_t cphase = 0;
+  for (int it = 0;; ++it) {
+    const int stage = it % NSTAGE;
+    if (!mbar_wait(&full[stage], (it / NSTAGE) & 1)) {
+      set_error(p.ws.err, kErrFullWait);
+      break;
+    }
+    const StageMeta mt = meta[stage];
+    if (mt.flags & kDone) break;
+    const int64_t u = (int64_t)mt.b * p.Hkv + mt.kvh;
+    if (mt.flags & kFirst) {
+      st.reset();
+      st.load_q(reinterpret_cast<const __nv_bfloat16 *>(p.q) + ((int64_t)mt.b * p.Hkv * p.G + (int64_t)mt.kvh * p.G) * D,
+                p.G);
+    }
+    const int pos0 = mt.tile * C::TILE + 16 * warp;
+    const int nvalid = max(0, min(16, mt.T - pos0));
+    const uint32_t vmask = nvalid >= 16 ? 0xFFFFu : ((1u << nvalid) - 1u);
+    const uint32_t kp = sbase + stage * C::STAGE;
+    const float *ks = scales + stage * (2 * C::TILE) + 16 * warp;
+    if (nvalid > 0)
+      st.step(kp, kp + C::KVB, C::PANEL, 16 * warp, vmask, p.c, p.ws.logits + (u * p.t_cap + pos0) * p.G, p.G, ks,
+              ks + C::TILE);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+    if (mt.flags & kLast) {
+      float *scr = scratch + warp * C::WSTRIDE;
+      st.store(scr, scr + 8, scr + 16);
+      if (!consumer_sync(cbar, cphase)) {
+        set_error(p.ws.err, kErrFullWait);
+        break;
+      }
+      if (mt.rec >= 0)
+        merge_warp_states<D>(scratch, C::WSTRIDE, NCW, p.G, p.c, p.ws.records + (size_t)mt.rec * p.G * (D + 2),
+                             threadIdx.x, NCW * 32);
+      if (!consumer_sync(cbar, cphase)) {
+        set_error(p.ws.err, kErrFullWait);
+        break;
+      }
+      st.reset();
+    }
+  }
+}
+
+// ------------------------------------------------------------ fp32 caches
+constexpr int kF32Tile = 64;
+constexpr int kF32Warps = 4;
+
+template <int D>
+__global__ void __launch_bounds__(32 * kF32Warps) full_attn_f32_kernel(const FullParams p) {
+  extern __shared__ float fsm[];
+  float *Ks = fsm;                        // [64][D+1]
+  float *Vs = Ks + kF32Tile * (D + 1);    // [64][D+1]
+  float *Qs = Vs + kF32Tile * (D + 1);    // [8][D]
+  int32_t *prefix = reinterpret_cast<int32_t *>(Qs + 8 * D);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nthr = blockDim.x;
+
+  if (warp == 0) compute_prefix(p, prefix, kF32Tile);
+  zero_counters(p, threadIdx.x, nthr);
+  __syncthreads();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i <= p.B; i += nthr) p.ws.prefix[i] = prefix[i];
+  const int64_t total = (int64_t)p.Hkv * prefix[p.B];
+  if (total == 0) return;
+  const Partition part{total, p.N};
+  const int64_t g0 = part.start(blockIdx.x), g1 = part.start(blockIdx.x + 1);
+  const float *K = static_cast<const float *>(p.k), *V = static_cast<const float *>(p.v);
+
+  float m[2], l[2], o[2][D / 32];
+  int b = g0 < g1 ? find_seq(prefix, p.B, p.Hkv, g0) : 0;
+  for (int64_t g = g0; g < g1; ++g) {
+    while ((int64_t)p.Hkv * prefix[b + 1] <= g) ++b;
+    const int nb = prefix[b + 1] - prefix[b];
+    const int64_t r = g - (int64_t)p.Hkv * prefix[b];
+    const int kvh = (int)(r / nb), i = (int)(r % nb);
+    const int64_t U = (int64_t)p.Hkv * prefix[b] + (int64_t)kvh * nb;
+    const int64_t u = (int64_t)b * p.Hkv + kvh;
+    const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
+    const bool first = i == 0 || g == g0, last = i == nb - 1 || g == g1 - 1;
+    const int p0 = i * kF32Tile;
+    if (first) {
+      const float *q = static_cast<const float *>(p.q) + ((int64_t)b * p.Hkv * p.G + (int64_t)kvh * p.G) * D;
+      for (int e = threadIdx.x; e < p.G * D; e += nthr) Qs[e] = q[e];
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+        m[hs] = -INFINITY;
+        l[hs] = 0.f;
+        for (int j = 0; j < D / 32; ++j) o[hs][j] = 0.f;
+      }
+    }
+    for (int e = threadIdx.x; e < kF32Tile * D; e += nthr) {
+      const int rr = e / D, col = e % D, pos = p0 + rr;
+      float kv = 0.f, vv = 0.f;
+      const int64_t slot = pos < T ? slot_of(p.page_table, p.max_pages, p.page_size, b, pos) : -1;
+      if (slot >= 0 && slot < p.num_slots) {
+        kv = K[(slot * p.Hkv + kvh) * D + col];
+        vv = V[(slot * p.Hkv + kvh) * D + col];
+      }
+      Ks[rr * (D + 1) + col] = kv;
+      Vs[rr * (D + 1) + col] = vv;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int hs = 0; hs < 2; ++hs) {
+      const int h = warp + kF32Warps * hs;
+      if (h >= p.G) break;
+      float s[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int rr = lane + 32 * j;
+        float acc = 0.f;
+#pragma unroll 4
+        for (int e = 0; e < D; ++e) acc = fmaf(Qs[h * D + e], Ks[rr * (D + 1) + e], acc);
+        s[j] = p0 + rr < T ? acc : -INFINITY;
+        if (p0 + rr < T) p.ws.logits[(u * p.t_cap + p0 + rr) * p.G + h] = acc;
+      }
+      const float mx = warp_max(fmaxf(s[0], s[1]));
+      const float m_new = fmaxf(m[hs], mx);
+      const float alpha = expf(p.c * (m[hs] - m_new));
+      float pr[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) pr[j] = s[j] == -INFINITY ? 0.f : expf(p.c * (s[j] - m_new));
+      l[hs] = l[hs] * alpha + warp_sum(pr[0] + pr[1]);
+      m[hs] = m_new;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        float acc = o[hs][j] * alpha;
+#pragma unroll 4
+        for (int rr = 0; rr < kF32Tile; ++rr) {
+          const float pp = __shfl_sync(0xffffffffu, pr[rr >> 5], rr & 31);
+          acc = fmaf(pp, Vs[rr * (D + 1) + lane + 32 * j], acc);
+        }
+        o[hs][j] = acc;
+      }
+    }
+    __syncthreads();
+    if (last) {
+      const int64_t j = blockIdx.x - part.cfirst(U);
+      if (j < 0 || j >= p.R) {
+        if (threadIdx.x == 0) set_error(p.ws.err, kErrRecord);
+        continue;
+      }
+      float *rec = p.ws.records + (size_t)(u * p.R + j) * p.G * (D + 2);
+#pragma unroll
+      for (int hs = 0; hs < 2; ++hs) {
+        const int h = warp + kF32Warps * hs;
+        if (h >= p.G) break;
+        if (lane == 0) {
+          rec[h] = m[hs];
+          rec[p.G + h] = l[hs];
+        }
+        for (int jj = 0; jj < D / 32; ++jj) rec[2 * p.G + h * D + lane + 32 * jj] = o[hs][jj];
+      }
+    }
+  }
+}
+
+template <int D, bool FP8, int NCW, int NSTAGE>
+cudaError_t launch_mma_t(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, int grid,
+                         cudaStream_t s) {
+  using C = Cfg<D, FP8, NCW, NSTAGE>;
+  const size_t smem = C::bytes(p.B);
+  auto kern = full_attn_mma_kernel<D, FP8, NCW, NSTAGE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, 32 * (NCW + 1), smem, s>>>(tmk, tmv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, bool fp8,
+                            const FullMmaConfig &cfg, int grid, cudaStream_t s) {
+#define HS2_FULL_CASE(D_, F_, W_, S_)                                                   \
+  if (p.D == D_ && fp8 == F_ && cfg.ncw == W_ && cfg.nstage == S_)                      \
+    return launch_mma_t<D_, F_, W_, S_>(p, tmk, tmv, grid, s);
+  HS2_FULL_CASE(128, false, 4, 4)
+  HS2_FULL_CASE(128, false, 4, 3)
+  HS2_FULL_CASE(128, false, 8, 2)
+  HS2_FULL_CASE(128, false, 8, 3)
+  HS2_FULL_CASE(64, false, 4, 4)
+  HS2_FULL_CASE(64, false, 8, 3)
+  HS2_FULL_CASE(128, true, 4, 4)
+  HS2_FULL_CASE(128, true, 8, 3)
+  HS2_FULL_CASE(128, true, 8, 4)
+#undef HS2_FULL_CASE
+  return cudaErrorInvalidConfiguration;
+}
+
+int full_f32_tile() { return kF32Tile; }
+int full_f32_ctas_per_sm() { return 2; }
+
+cudaError_t launch_full_f32(const FullParams &p, int grid, cudaStream_t s) {
+  const size_t smem = (size_t)(2 * kF32Tile * (p.D + 1) + 8 * p.D) * 4 + (size_t)(p.B + 1) * 4;
+  cudaError_t e;
+  if (p.D == 64) {
+    e = cudaFuncSetAttribute(full_attn_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    full_attn_f32_kernel<64><<<grid, 32 * kF32Warps, smem, s>>>(p);
+  } else if (p.D == 128) {
+    e = cudaFuncSetAttribute(full_attn_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    full_attn_f32_kernel<128><<<grid, 32 * kF32Warps, smem, s>>>(p);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace hs2

@@ -1,0 +1,79 @@
+// hs2_internal.h -- host-side launchers shared between the C-ABI layer and
+// the kernel translation units (not part of the public ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hs2_common.cuh"
+
+namespace hs2 {
+
+// Parameters of the full-attention (split over the context) kernels.
+struct FullParams {
+  const void *q;             // [B, Hq, D] (bf16, or f32 for the f32 path)
+  const void *k, *v;         // caches (plain loads of the f32 path)
+  const float *k_scale;      // E4M3 only
+  const float *v_scale;
+  const int32_t *seq_lens;   // [B]
+  const int32_t *page_table; // [B, max_pages] or nullptr
+  int32_t B, Hkv, G, D;
+  int32_t page_size, max_pages;
+  int64_t t_cap;             // logical capacity per sequence
+  int64_t num_slots;
+  int32_t N;                 // persistent CTAs (grid size)
+  int32_t R;                 // record slots per unit
+  int32_t tile;              // positions per tile
+  float c;                   // 1/sqrt(D)
+  FullWs ws;
+};
+
+struct ScoreParams {
+  const int32_t *seq_lens;
+  const int32_t *page_table;
+  void *out;                 // [B, Hq, D] in out_dtype
+  int32_t out_dtype;         // 0 f32, 1 bf16
+  int32_t *idx_out;          // [B, Hkv, W + K]
+  int32_t B, Hkv, G, D;
+  int32_t page_size, max_pages;
+  int64_t t_cap;
+  int32_t window, k_global;
+  int32_t N, R, tile;
+  float c;
+  FullWs ws;
+};
+
+struct SparseParams {
+  const void *q;             // [B, Hq, D]
+  const void *k, *v;
+  const float *k_scale, *v_scale;
+  const int32_t *idx;        // [B, Hkv, L]
+  void *out;                 // [B, Hq, D]
+  int32_t B, Hkv, G, D;
+  int32_t L;                 // idx_stride
+  int32_t rows_per_cta;      // multiple of 16
+  int32_t splits;            // CTAs per unit (cluster size)
+  float c;
+};
+
+// Launch configuration chosen by the host for the tensor-core full kernel.
+struct FullMmaConfig {
+  int ncw;     // consumer warps (tile = 16 * ncw positions)
+  int nstage;  // pipeline stages
+};
+
+// ---- launchers (return cudaError_t of the launch) -------------------------
+cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, bool fp8,
+                            const FullMmaConfig &cfg, int grid, cudaStream_t s);
+cudaError_t launch_full_f32(const FullParams &p, int grid, cudaStream_t s);
+int full_f32_tile();
+int full_f32_ctas_per_sm();
+
+cudaError_t launch_select(const ScoreParams &p, cudaStream_t s);
+
+cudaError_t launch_sparse_impl(const SparseParams &p, int kv_dtype, int64_t num_slots, cudaStream_t s);
+
+cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int grid, cudaStream_t s);
+
+}  // namespace hs2

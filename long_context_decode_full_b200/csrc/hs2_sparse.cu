@@ -1,0 +1,213 @@
+// hs2_sparse.cu -- a sparse-attention layer of a Hybrid Block (HySparse2
+// announcement, "KV Reuse" section: the sparse layers reuse the full layer's
+// KV cache and its selection indices; the forced window and the global
+// tokens are read from that one cache in a single sparse computation, with
+// no separate sliding-window branch).
+//
+// Per (sequence, kv head) a thread-block cluster of `splits` CTAs shares the
+// index list: every warp gathers 16 listed rows of K and V (whole rows,
+// 16-byte cp.async into the swizzled tile layout), runs the tensor-core
+// attention step for the G query heads of the group, the CTA merges its
+// warps, and CTA 0 of the cluster merges the CTAs through distributed shared
+// memory and writes the output.  No workspace, no atomics, one launch.
+#include <cooperative_groups.h>
+
+#include "hs2_internal.h"
+#include "hs2_warp_attn.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace hs2 {
+
+namespace {
+
+template <int D, bool FP8>
+struct SCfg {
+  static constexpr int ES = FP8 ? 1 : 2;
+  static constexpr int ROWB = D * ES;
+  static constexpr int PANEL = 16 * 128;
+  static constexpr int KVB = 16 * ROWB;        // 16 rows of K (or V)
+  static constexpr int WARP_BYTES = 2 * KVB + (FP8 ? 2 * 16 * 4 : 0);
+  static constexpr int WSTRIDE = 16 + 8 * D;   // warp scratch floats
+  static size_t bytes(int nw, int G) {
+    return 128 + (size_t)nw * WARP_BYTES + (size_t)nw * WSTRIDE * 4 + (size_t)G * (D + 2) * 4;
+  }
+};
+
+template <int D, bool FP8>
+__global__ void __launch_bounds__(512, 1) sparse_mma_kernel(const SparseParams p, int64_t num_slots) {
+  using C = SCfg<D, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float *scratch = reinterpret_cast<float *>(smem + (size_t)nw * C::WARP_BYTES);
+  float *partial = scratch + (size_t)nw * C::WSTRIDE;  // m[G], l[G], o[G][D]
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int kvh = blockIdx.y, b = blockIdx.z, G = p.G;
+  const int64_t u = (int64_t)b * p.Hkv + kvh;
+
+  // ---- gather this warp's 16 rows
+  uint8_t *wb = smem + (size_t)warp * C::WARP_BYTES;
+  const uint32_t kp = smem_u32(wb), vp = kp + C::KVB;
+  float *ks = reinterpret_cast<float *>(wb + 2 * C::KVB), *vs = ks + 16;
+  const int r0 = rank * p.rows_per_cta + 16 * warp;
+  int slot = -1;
+  if (lane < 16 && r0 + lane < p.L) {
+    const int s = __ldg(p.idx + u * p.L + r0 + lane);
+    if (s >= 0 && s < num_slots) slot = s;
+  }
+  const uint32_t vmask = __ballot_sync(0xffffffffu, slot >= 0) & 0xFFFFu;
+  if constexpr (FP8) {
+    if (lane < 16) {
+      ks[lane] = slot >= 0 ? __ldg(p.k_scale + (int64_t)slot * p.Hkv + kvh) : 0.f;
+      vs[lane] = slot >= 0 ? __ldg(p.v_scale + (int64_t)slot * p.Hkv + kvh) : 0.f;
+    }
+  }
+  constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
+  const uint8_t *kg = static_cast<const uint8_t *>(p.k), *vg = static_cast<const uint8_t *>(p.v);
+#pragma unroll 4
+  for (int e = lane; e < 16 * CPR; e += 32) {
+    const int row = e / CPR, ch = e % CPR;
+    const int s = __shfl_sync(0xffffffffu, slot, row);
+    const uint32_t off = (ch >> 3) * C::PANEL;
+    const uint32_t dk = swz(kp + off, row, ch & 7), dv = swz(vp + off, row, ch & 7);
+    if (s >= 0) {
+      const int64_t src = ((int64_t)s * p.Hkv + kvh) * C::ROWB + ch * 16;
+      cp_async_16(dk, kg + src);
+      cp_async_16(dv, vg + src);
+    } else {
+      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dk), "r"(0u) : "memory");
+      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dv), "r"(0u) : "memory");
+    }
+  }
+  cp_async_commit();
+
+  WarpAttn<D, FP8> st;
+  st.reset();
+  st.load_q(static_cast<const __nv_bfloat16 *>(p.q) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D, G);
+  cp_async_wait_all();
+  __syncwarp();
+  if (vmask) st.step(kp, vp, C::PANEL, 0, vmask, p.c, nullptr, G, ks, vs);
+
+  // ---- merge the warps of this CTA, then the CTAs of the cluster
+  float *scr = scratch + warp * C::WSTRIDE;
+  st.store(scr, scr + 8, scr + 16);
+  __syncthreads();
+  merge_warp_states<D>(scratch, C::WSTRIDE, nw, G, p.c, partial, threadIdx.x, blockDim.x);
+  cluster.sync();
+  if (rank == 0) {
+    const int S = (int)cluster.num_blocks();
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+      const int h = e / D;
+      float M = -INFINITY;
+      for (int r = 0; r < S; ++r) M = fmaxf(M, cluster.map_shared_rank(partial, r)[h]);
+      float L = 0.f, acc = 0.f;
+      if (M != -INFINITY) {
+        for (int r = 0; r < S; ++r) {
+          const float *pr = cluster.map_shared_rank(partial, r);
+          if (pr[h] == -INFINITY) continue;
+          const float w = expf(p.c * (pr[h] - M));
+          L += w * pr[G + h];
+          acc += w * pr[2 * G + e];
+        }
+      }
+      const float val = L > 0.f ? acc / L : 0.f;
+      const int64_t oi = ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D + e;
+      static_cast<__nv_bfloat16 *>(p.out)[oi] = __float2bfloat16_rn(val);
+    }
+  }
+  cluster.sync();  // keep every CTA's shared memory alive until CTA 0 is done
+}
+
+// ------------------------------------------------------------ fp32 caches
+template <int D>
+__global__ void sparse_f32_kernel(const SparseParams p, int64_t num_slots) {
+  extern __shared__ float qs[];  // [G][D]
+  const int kvh = blockIdx.x, b = blockIdx.y, G = p.G;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float *q = static_cast<const float *>(p.q) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
+  for (int e = threadIdx.x; e < G * D; e += blockDim.x) qs[e] = q[e];
+  __syncthreads();
+  const int h = warp;
+  if (h >= G) return;
+  const float *K = static_cast<const float *>(p.k), *V = static_cast<const float *>(p.v);
+  const int32_t *idx = p.idx + ((int64_t)b * p.Hkv + kvh) * p.L;
+  float m = -INFINITY, l = 0.f, o[D / 32];
+#pragma unroll
+  for (int j = 0; j < D / 32; ++j) o[j] = 0.f;
+  for (int base = 0; base < p.L; base += 32) {
+    int slot = base + lane < p.L ? __ldg(idx + base + lane) : -1;
+    if (slot >= num_slots) slot = -1;
+    float s = -INFINITY;
+    if (slot >= 0) {
+      const float *kr = K + ((int64_t)slot * p.Hkv + kvh) * D;
+      float acc = 0.f;
+      for (int e = 0; e < D; ++e) acc = fmaf(qs[h * D + e], kr[e], acc);
+      s = acc;
+    }
+    const float mx = warp_max(s);
+    if (mx == -INFINITY) continue;
+    const float m_new = fmaxf(m, mx);
+    const float alpha = expf(p.c * (m - m_new));
+    const float pr = slot >= 0 ? expf(p.c * (s - m_new)) : 0.f;
+    l = l * alpha + warp_sum(pr);
+    m = m_new;
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) {
+      float acc = o[j] * alpha;
+      for (int r = 0; r < 32; ++r) {
+        const int sr = __shfl_sync(0xffffffffu, slot, r);
+        const float pp = __shfl_sync(0xffffffffu, pr, r);
+        if (sr >= 0) acc = fmaf(pp, V[((int64_t)sr * p.Hkv + kvh) * D + lane + 32 * j], acc);
+      }
+      o[j] = acc;
+    }
+  }
+  float *out = static_cast<float *>(p.out) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G + h) * D;
+#pragma unroll
+  for (int j = 0; j < D / 32; ++j) out[lane + 32 * j] = l > 0.f ? o[j] / l : 0.f;
+}
+
+template <int D, bool FP8>
+cudaError_t launch_mma_t(const SparseParams &p, int64_t num_slots, cudaStream_t s) {
+  using C = SCfg<D, FP8>;
+  const int nw = p.rows_per_cta / 16;
+  const size_t smem = C::bytes(nw, p.G);
+  auto kern = sparse_mma_kernel<D, FP8>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if (p.splits > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.splits, p.Hkv, p.B);
+  cfg.blockDim = dim3(32 * nw);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p, num_slots);
+}
+
+}  // namespace
+
+cudaError_t launch_sparse_impl(const SparseParams &p, int kv_dtype, int64_t num_slots, cudaStream_t s) {
+  if (kv_dtype == 0) {
+    const size_t smem = (size_t)p.G * p.D * 4;
+    if (p.D == 64) sparse_f32_kernel<64><<<dim3(p.Hkv, p.B), 32 * p.G, smem, s>>>(p, num_slots);
+    else sparse_f32_kernel<128><<<dim3(p.Hkv, p.B), 32 * p.G, smem, s>>>(p, num_slots);
+    return cudaGetLastError();
+  }
+  if (kv_dtype == 1) return p.D == 64 ? launch_mma_t<64, false>(p, num_slots, s) : launch_mma_t<128, false>(p, num_slots, s);
+  if (kv_dtype == 2 && p.D == 128) return launch_mma_t<128, true>(p, num_slots, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace hs2

@@ -1,0 +1,291 @@
+// hs2_warp_attn.cuh -- one warp's share of an attention tile: 16 K/V rows
+// against the G <= 8 query heads of one GQA group, on the tensor cores.
+//
+// Layout of the contraction (mma.sync m16n8k16, fp32 accumulate):
+//   S   = Q K^T   : A = Q (16 rows = the group's heads, rows >= G zero),
+//                   B = K^T (8 rows of the tile per n-tile), two n-tiles.
+//   O^T = V^T P^T : A = V^T (16 head dims per m-tile), B = P^T (16 rows x 8
+//                   heads).  The S accumulator of head g at rows 2t,2t+1 is
+//                   exactly the P^T fragment the second MMA needs, so P never
+//                   leaves registers, and no MMA row is padding.
+// The tile in shared memory is [panels][rows][128 B] with the 128-byte TMA
+// swizzle (16-byte chunk c of row r at chunk c ^ (r & 7)), written either by
+// TMA (full layer) or by cp.async (sparse layer).
+//
+// E4M3 caches: codes are widened to f16 in registers (exact); the query is
+// f16 with a per-head power-of-two prescale (exact for its bf16 values); the
+// K scale multiplies the logit and the V scale multiplies p, normalised by a
+// running maximum so that p stays inside f16's normal range.  The head-dim
+// order inside the MMAs is permuted consistently on both operands so every
+// shared-memory read is one conflict-free 16-byte load per row.
+#pragma once
+
+#include "hs2_common.cuh"
+
+namespace hs2 {
+
+template <int D, bool FP8>
+struct WarpAttn {
+  static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(!FP8 || D == 128, "E4M3 path is built for head_dim 128");
+  static constexpr int KS = D / 16;  // k-steps of Q K^T and m-tiles of V^T P^T
+
+  uint32_t qa[KS][2];  // A-fragments of Q (rows g; rows g+8 are zero)
+  float qscale;        // E4M3: 2^-e undoing the query prescale
+  float m;             // running max of raw logits of head g
+  float l;             // this lane's share of sum exp(c (s - m)) for head g
+  float sig;           // E4M3: running max of the V scale (warp uniform)
+  float o[KS][4];      // O^T accumulator: dims x heads (2t, 2t+1)
+
+  __device__ __forceinline__ void reset() {
+    m = -INFINITY;
+    l = 0.f;
+    sig = 0.f;
+#pragma unroll
+    for (int i = 0; i < KS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  }
+
+  // Query of the group (G consecutive heads, bf16 [G][D]) into A-fragments.
+  __device__ __forceinline__ void load_q(const __nv_bfloat16 *q, int G) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const uint32_t *q32 = reinterpret_cast<const uint32_t *>(q);
+    if constexpr (!FP8) {
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        qa[kk][0] = g < G ? __ldg(q32 + ((g * D + 16 * kk + 2 * t) >> 1)) : 0u;
+        qa[kk][1] = g < G ? __ldg(q32 + ((g * D + 16 * kk + 8 + 2 * t) >> 1)) : 0u;
+      }
+      qscale = 1.f;
+    } else {
+      // k-step kk of lane t covers dims 32t + 4kk + {0,1} (MMA k = 2t, 2t+1)
+      // and 32t + 4kk + {2,3} (MMA k = 2t+8, 2t+9).
+      float v[KS][4];
+      float amax = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        uint2 w = g < G ? __ldg(reinterpret_cast<const uint2 *>(q + g * D + 32 * t + 4 * kk)) : make_uint2(0, 0);
+        v[kk][0] = __uint_as_float(w.x << 16);
+        v[kk][1] = __uint_as_float(w.x & 0xFFFF0000u);
+        v[kk][2] = __uint_as_float(w.y << 16);
+        v[kk][3] = __uint_as_float(w.y & 0xFFFF0000u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(v[kk][e]));
+      }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      const int e = amax > 0.f ? 14 - ilogbf(amax) : 0;
+      const float up = ldexpf(1.f, e);
+      qscale = ldexpf(1.f, -e);
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        qa[kk][0] = pack_f16(v[kk][0] * up, v[kk][1] * up);
+        qa[kk][1] = pack_f16(v[kk][2] * up, v[kk][3] * up);
+      }
+    }
+  }
+
+  // One 16-row slice.  kp / vp: shared addresses of panel 0 of the K / V
+  // tile; pstride: bytes between panels; row0: first row of the slice inside
+  // the panel; vmask: bit r set when row r holds a real position; c: 1/sqrt(D)
+  // in the logit domain.  logit_dst (or nullptr): raw logits [16][G] of this
+  // slice.  ks / vs (E4M3): the slice's 16 K / V scales in shared memory.
+  __device__ __forceinline__ void step(uint32_t kp, uint32_t vp, uint32_t pstride, int row0, uint32_t vmask,
+                                       float c, float *logit_dst, int G, const float *ks, const float *vs) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    float s[2][4];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+
+    // ---- S = Q K^T
+    if constexpr (!FP8) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int row = row0 + 8 * j + (lane & 7);
+#pragma unroll
+        for (int kk = 0; kk < KS; kk += 2) {
+          const int cb = (16 * kk + 8 * (lane >> 3)) * 2;  // byte column
+          uint32_t r[4];
+          ldsm_x4(r, swz(kp + (cb >> 7) * pstride, row, (cb & 127) >> 4));
+          mma_bf16(s[j], qa[kk][0], 0u, qa[kk][1], 0u, r[0], r[1]);
+          mma_bf16(s[j], qa[kk + 1][0], 0u, qa[kk + 1][1], 0u, r[2], r[3]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int row = row0 + 8 * j + g;
+        uint32_t w0[4], w1[4];
+        lds128(w0, swz(kp, row, 2 * t));
+        lds128(w1, swz(kp, row, 2 * t + 1));
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          const uint32_t w = kk < 4 ? w0[kk & 3] : w1[kk & 3];
+          mma_f16(s[j], qa[kk][0], 0u, qa[kk][1], 0u, e4m3x2_to_f16x2(w), e4m3x2_to_f16x2(w >> 16));
+        }
+      }
+    }
+
+    // ---- logits, online softmax (head g; rows 2t, 2t+1, 8+2t, 9+2t)
+    const int rr[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
+    float x[4] = {s[0][0], s[0][1], s[1][0], s[1][1]};
+    bool ok[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ok[i] = (vmask >> rr[i]) & 1u;
+      if constexpr (FP8) x[i] *= (ok[i] ? ks[rr[i]] : 0.f) * qscale;
+    }
+    if (logit_dst != nullptr && g < G) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (ok[i]) logit_dst[rr[i] * G + g] = x[i];
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (ok[i]) mx = fmaxf(mx, x[i]);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m, mx);
+    float alpha = 1.f, p[4] = {0.f, 0.f, 0.f, 0.f};
+    if (m_new != -INFINITY) {
+      alpha = expf(c * (m - m_new));
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (ok[i]) p[i] = expf(c * (x[i] - m_new));
+    }
+    l = l * alpha + ((p[0] + p[1]) + (p[2] + p[3]));
+    m = m_new;
+
+    float pv[4] = {p[0], p[1], p[2], p[3]};
+    float beta = 1.f;
+    if constexpr (FP8) {
+      float sv[4], smax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        sv[i] = ok[i] ? vs[rr[i]] : 0.f;
+        smax = fmaxf(smax, sv[i]);
+      }
+      smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 1));
+      smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 2));
+      const float sig_new = fmaxf(sig, smax);
+      beta = sig_new > 0.f ? sig / sig_new : 1.f;
+      const float inv = sig_new > 0.f ? 1.f / sig_new : 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) pv[i] = p[i] * (sv[i] * inv);
+      sig = sig_new;
+    }
+
+    // ---- rescale O^T columns (heads 2t, 2t+1) by their heads' factors
+    const float f = alpha * beta;
+    const float f_lo = __shfl_sync(0xffffffffu, f, 8 * t);
+    const float f_hi = __shfl_sync(0xffffffffu, f, 8 * t + 4);
+    if (__any_sync(0xffffffffu, f_lo != 1.f || f_hi != 1.f)) {
+#pragma unroll
+      for (int i = 0; i < KS; ++i) {
+        o[i][0] *= f_lo;
+        o[i][1] *= f_hi;
+        o[i][2] *= f_lo;
+        o[i][3] *= f_hi;
+      }
+    }
+
+    // ---- O^T += V^T P^T
+    const bool full = vmask == 0xFFFFu;
+    const uint32_t m01 = (ok[0] ? 0x0000FFFFu : 0u) | (ok[1] ? 0xFFFF0000u : 0u);
+    const uint32_t m23 = (ok[2] ? 0x0000FFFFu : 0u) | (ok[3] ? 0xFFFF0000u : 0u);
+    if constexpr (!FP8) {
+      const uint32_t pb0 = pack_bf16(pv[0], pv[1]), pb1 = pack_bf16(pv[2], pv[3]);
+      const int row = row0 + (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        const int cb = (16 * mt + ((lane >> 3) & 1) * 8) * 2;
+        uint32_t a[4];
+        ldsm_x4_t(a, swz(vp + (cb >> 7) * pstride, row, (cb & 127) >> 4));
+        if (!full) {  // rows past the end may hold anything, NaN included
+          a[0] &= m01;
+          a[1] &= m01;
+          a[2] &= m23;
+          a[3] &= m23;
+        }
+        mma_bf16(o[mt], a[0], a[1], a[2], a[3], pb0, pb1);
+      }
+    } else {
+      const uint32_t pb0 = pack_f16(pv[0], pv[1]), pb1 = pack_f16(pv[2], pv[3]);
+      uint32_t w0[4], w1[4], w2[4], w3[4];
+      lds128(w0, swz(vp, row0 + rr[0], g));
+      lds128(w1, swz(vp, row0 + rr[1], g));
+      lds128(w2, swz(vp, row0 + rr[2], g));
+      lds128(w3, swz(vp, row0 + rr[3], g));
+      // byte masks: bytes 0,2 come from the even row, bytes 1,3 from the odd row
+      const uint32_t b01 = (ok[0] ? 0x00FF00FFu : 0u) | (ok[1] ? 0xFF00FF00u : 0u);
+      const uint32_t b23 = (ok[2] ? 0x00FF00FFu : 0u) | (ok[3] ? 0xFF00FF00u : 0u);
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+        uint32_t x01 = prmt(w0[mt >> 1], w1[mt >> 1], sel);
+        uint32_t x23 = prmt(w2[mt >> 1], w3[mt >> 1], sel);
+        if (!full) {
+          x01 &= b01;
+          x23 &= b23;
+        }
+        mma_f16(o[mt], e4m3x2_to_f16x2(x01), e4m3x2_to_f16x2(x01 >> 16), e4m3x2_to_f16x2(x23),
+                e4m3x2_to_f16x2(x23 >> 16), pb0, pb1);
+      }
+    }
+  }
+
+  // Writes this warp's state to shared scratch: m[8], l[8], o[8][D] (true
+  // scale, not yet normalised).  Heads >= G are written too and ignored.
+  __device__ __forceinline__ void store(float *sm, float *sl, float *so) const {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    float lt = l;
+    lt += __shfl_xor_sync(0xffffffffu, lt, 1);
+    lt += __shfl_xor_sync(0xffffffffu, lt, 2);
+    if (t == 0) {
+      sm[g] = m;
+      sl[g] = lt;
+    }
+    const float os = FP8 ? sig : 1.f;
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      const int d0 = FP8 ? 16 * g + 2 * mt : 16 * mt + g;
+      const int d1 = FP8 ? d0 + 1 : d0 + 8;
+      so[(2 * t) * D + d0] = o[mt][0] * os;
+      so[(2 * t + 1) * D + d0] = o[mt][1] * os;
+      so[(2 * t) * D + d1] = o[mt][2] * os;
+      so[(2 * t + 1) * D + d1] = o[mt][3] * os;
+    }
+  }
+};
+
+// Merges NW warp states in shared scratch (stride `wstride` floats per warp:
+// m[8], l[8], o[8][D]) into one record m[G], l[G], o[G][D] at `rec` (global or
+// shared).  Threads tid .. nthreads cooperate.
+template <int D>
+__device__ __forceinline__ void merge_warp_states(const float *scr, int wstride, int NW, int G, float c,
+                                                  float *rec, int tid, int nthreads) {
+  for (int h = tid; h < G; h += nthreads) {
+    float M = -INFINITY;
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, scr[w * wstride + h]);
+    float L = 0.f;
+    for (int w = 0; w < NW; ++w) {
+      const float mw = scr[w * wstride + h];
+      if (mw != -INFINITY) L += expf(c * (mw - M)) * scr[w * wstride + 8 + h];
+    }
+    rec[h] = M;
+    rec[G + h] = L;
+  }
+  for (int e = tid; e < G * D; e += nthreads) {
+    const int h = e / D;
+    float M = -INFINITY;
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, scr[w * wstride + h]);
+    float acc = 0.f;
+    for (int w = 0; w < NW; ++w) {
+      const float mw = scr[w * wstride + h];
+      if (mw != -INFINITY) acc += expf(c * (mw - M)) * scr[w * wstride + 16 + e];
+    }
+    rec[2 * G + e] = acc;
+  }
+}
+
+}  // namespace hs2

@@ -1,0 +1,187 @@
+"""Thin ctypes binding of ``libhs2.so`` (include/hs2.h) over torch tensors.
+
+Argument marshalling only: torch provides device memory and the current
+stream; every step of the Hybrid-Block path runs in the library's CUDA
+kernels.  If the library is missing or fails to load, every call raises --
+there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhs2.so")
+
+HS2_F32, HS2_BF16, HS2_E4M3 = 0, 1, 2
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+
+_DTYPE = {torch.float32: HS2_F32, torch.bfloat16: HS2_BF16, torch.uint8: HS2_E4M3,
+          torch.float8_e4m3fn: HS2_E4M3}
+
+
+class Cache(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("dtype", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("num_slots", ctypes.c_int64)]
+
+
+class Heads(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("batch", ctypes.c_int32),
+                ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+class HS2Error(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"hs2 error {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+EXPORTS = ["hs2_full_attn_select_workspace", "hs2_full_attn_select", "hs2_full_attn_select_marked",
+           "hs2_sparse_attn",
+           "hs2_workspace_status", "hs2_copy_peak", "hs2_last_error", "hs2_version"]
+
+
+def lib():
+    """The loaded library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m long_context_decode_full_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        L.hs2_full_attn_select_workspace.argtypes = [I32, I32, I32, I32, I64]
+        L.hs2_full_attn_select_workspace.restype = SZ
+        L.hs2_full_attn_select.argtypes = [ctypes.POINTER(Heads), ctypes.POINTER(Cache), ctypes.POINTER(Cache),
+                                           P, P, I32, I32, I32, ctypes.POINTER(Heads), P, P, SZ, P]
+        L.hs2_full_attn_select.restype = ctypes.c_int
+        L.hs2_full_attn_select_marked.argtypes = L.hs2_full_attn_select.argtypes + [P]
+        L.hs2_full_attn_select_marked.restype = ctypes.c_int
+        L.hs2_sparse_attn.argtypes = [ctypes.POINTER(Heads), ctypes.POINTER(Cache), ctypes.POINTER(Cache), P, I32,
+                                      ctypes.POINTER(Heads), P]
+        L.hs2_sparse_attn.restype = ctypes.c_int
+        L.hs2_workspace_status.argtypes = [P, SZ, P]
+        L.hs2_workspace_status.restype = ctypes.c_int
+        L.hs2_copy_peak.argtypes = [P, P, SZ, P]
+        L.hs2_copy_peak.restype = ctypes.c_int
+        L.hs2_last_error.argtypes = []
+        L.hs2_last_error.restype = ctypes.c_char_p
+        L.hs2_version.argtypes = []
+        L.hs2_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise HS2Error(rc, lib().hs2_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def cache_desc(kv: torch.Tensor, scale: Optional[torch.Tensor], page_size: int) -> Cache:
+    assert kv.dim() == 3 and kv.is_contiguous(), "cache must be a contiguous [num_slots, Hkv, d] tensor"
+    return Cache(kv.data_ptr(), None if scale is None else scale.data_ptr(), _DTYPE[kv.dtype], kv.shape[1],
+                 kv.shape[2], page_size, kv.shape[0])
+
+
+def heads_desc(x: torch.Tensor) -> Heads:
+    assert x.dim() == 3 and x.is_contiguous(), "q/out must be a contiguous [B, H, d] tensor"
+    return Heads(x.data_ptr(), _DTYPE[x.dtype], x.shape[0], x.shape[1], x.shape[2])
+
+
+def full_workspace_bytes(batch: int, num_kv_heads: int, group: int, head_dim: int, t_cap: int) -> int:
+    return int(lib().hs2_full_attn_select_workspace(batch, num_kv_heads, group, head_dim, t_cap))
+
+
+def alloc_workspace(batch, num_kv_heads, group, head_dim, t_cap, device="cuda") -> torch.Tensor:
+    n = full_workspace_bytes(batch, num_kv_heads, group, head_dim, t_cap)
+    if n == 0:
+        raise HS2Error(ERR_INVALID_ARG, "invalid workspace shape")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def full_attn_select(q, k, v, seq_lens, page_table=None, page_size=None, window=128, k_global=1024,
+                     k_scale=None, v_scale=None, out=None, idx_out=None, workspace=None, stream=None,
+                     mark_event=None):
+    """Full-attention layer + token selection.  Returns (out, idx) where idx
+    holds selected slots [B, Hkv, window + k_global], ascending, -1 padded.
+    ``mark_event`` (a recorded-once torch.cuda.Event) is recorded between the
+    attention kernel and the selection kernels."""
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if page_size is None:
+        assert page_table is None, "page_size is required with a page table"
+        page_size = k.shape[0] // B
+    max_pages = 1 if page_table is None else page_table.shape[1]
+    t_cap = page_size * max_pages
+    if out is None:
+        out = torch.empty_like(q)
+    if idx_out is None:
+        idx_out = torch.empty(B, Hkv, window + k_global, dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, Hkv, Hq // Hkv, d, t_cap, q.device)
+    kc, vc = cache_desc(k, k_scale, page_size), cache_desc(v, v_scale, page_size)
+    qd, od = heads_desc(q), heads_desc(out)
+    ev = None if mark_event is None else ctypes.c_void_p(mark_event.cuda_event)
+    _check(lib().hs2_full_attn_select_marked(ctypes.byref(qd), ctypes.byref(kc), ctypes.byref(vc),
+                                             _ptr(seq_lens), _ptr(page_table), max_pages, window, k_global,
+                                             ctypes.byref(od), _ptr(idx_out), _ptr(workspace), workspace.numel(),
+                                             _stream(stream), ev))
+    return out, idx_out
+
+
+def sparse_attn(q_l, k, v, idx, k_scale=None, v_scale=None, page_size=1, out=None, stream=None):
+    """Sparse-attention layer over the rows listed in ``idx`` (slots)."""
+    if out is None:
+        out = torch.empty_like(q_l)
+    kc, vc = cache_desc(k, k_scale, page_size), cache_desc(v, v_scale, page_size)
+    qd, od = heads_desc(q_l), heads_desc(out)
+    _check(lib().hs2_sparse_attn(ctypes.byref(qd), ctypes.byref(kc), ctypes.byref(vc), _ptr(idx), idx.shape[-1],
+                                 ctypes.byref(od), _stream(stream)))
+    return out
+
+
+def hybrid_block_step(q_full, q_sparse: Sequence[torch.Tensor], k, v, seq_lens, page_table=None, page_size=None,
+                      window=128, k_global=1024, k_scale=None, v_scale=None, outs=None, idx_out=None,
+                      workspace=None, stream=None):
+    """One decode step of a Hybrid Block: the full layer (attention + token
+    selection) then every sparse layer with its own query, all reusing the
+    same cache and the same index list.  Returns (outs, idx)."""
+    outs = outs if outs is not None else [None] * (1 + len(q_sparse))
+    o0, idx = full_attn_select(q_full, k, v, seq_lens, page_table, page_size, window, k_global, k_scale, v_scale,
+                               outs[0], idx_out, workspace, stream)
+    ps = page_size if page_size is not None else k.shape[0] // q_full.shape[0]
+    res = [o0]
+    for i, q in enumerate(q_sparse):
+        res.append(sparse_attn(q, k, v, idx, k_scale, v_scale, ps, outs[1 + i], stream))
+    return res, idx
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream, returns and clears the sticky device error flag."""
+    return int(lib().hs2_workspace_status(_ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def copy_peak(dst: torch.Tensor, src: torch.Tensor, stream=None):
+    _check(lib().hs2_copy_peak(_ptr(dst), _ptr(src), src.numel() * src.element_size(), _stream(stream)))
+
+
+def version() -> int:
+    return int(lib().hs2_version())
+
+
+def last_error() -> str:
+    return lib().hs2_last_error().decode()

@@ -19,3 +19,11 @@ def oracle():
 
     _oracle.build()
     return _oracle
+
+
+@pytest.fixture(scope="session")
+def libhs2():
+    from long_context_decode_full_b200 import build, hs2
+
+    build.build()
+    return hs2.lib()

@@ -1,0 +1,110 @@
+"""The C-ABI boundary without a GPU: the library builds for sm_100a, loads,
+exports every entry point that include/hs2.h declares, and rejects bad
+arguments on the host with the documented status codes (nothing launches)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_decode_full_b200 import hs2
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "hs2.h")
+FAKE = 0x10000  # 16-byte aligned, never dereferenced on the host
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(hs2_\w+)\s*\(", text, re.M)))
+
+
+def test_exports_every_declared_symbol(libhs2):
+    names = declared_functions()
+    assert "hs2_full_attn_select" in names and "hs2_sparse_attn" in names
+    for n in names:
+        assert hasattr(libhs2, n), n
+    assert set(hs2.EXPORTS) == set(names)
+    assert hs2.version() >= 100
+
+
+def cache(dtype=1, heads=2, dim=128, page=64, slots=1 << 16, scale=None, data=FAKE):
+    return hs2.Cache(data, scale, dtype, heads, dim, page, slots)
+
+
+def heads(dtype=1, b=2, h=16, dim=128, data=FAKE):
+    return hs2.Heads(data, dtype, b, h, dim)
+
+
+def full(q=None, k=None, v=None, seq=FAKE, pt=FAKE, max_pages=64, W=128, K=1024, out=None, idx=FAKE,
+         ws=FAKE * 16, ws_bytes=1 << 40):
+    q = q or heads()
+    k = k or cache()
+    v = v or cache()
+    out = out or heads()
+    return hs2.lib().hs2_full_attn_select(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), seq, pt, max_pages,
+                                          W, K, ctypes.byref(out), idx, ws, ws_bytes, None)
+
+
+def sparse(q=None, k=None, v=None, idx=FAKE, stride=1152, out=None):
+    q = q or heads()
+    k = k or cache()
+    v = v or cache()
+    out = out or heads()
+    return hs2.lib().hs2_sparse_attn(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), idx, stride,
+                                     ctypes.byref(out), None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=heads(data=0)), hs2.ERR_INVALID_ARG),
+    (dict(q=heads(data=FAKE + 8)), hs2.ERR_INVALID_ARG),
+    (dict(k=cache(dim=96), v=cache(dim=96)), hs2.ERR_UNSUPPORTED),
+    (dict(k=cache(heads=4)), hs2.ERR_INVALID_ARG),
+    (dict(q=heads(h=6), out=heads(h=6)), hs2.ERR_UNSUPPORTED),
+    (dict(q=heads(h=64), out=heads(h=64)), hs2.ERR_UNSUPPORTED),
+    (dict(q=heads(dtype=0), out=heads(dtype=0)), hs2.ERR_UNSUPPORTED),
+    (dict(out=heads(b=3)), hs2.ERR_INVALID_ARG),
+    (dict(seq=0), hs2.ERR_INVALID_ARG),
+    (dict(idx=0), hs2.ERR_INVALID_ARG),
+    (dict(W=-1), hs2.ERR_INVALID_ARG),
+    (dict(W=0, K=0), hs2.ERR_INVALID_ARG),
+    (dict(max_pages=0), hs2.ERR_INVALID_ARG),
+    (dict(pt=0, max_pages=4), hs2.ERR_INVALID_ARG),
+    (dict(k=cache(page=48), v=cache(page=48)), hs2.ERR_UNSUPPORTED),
+    (dict(k=cache(dtype=2), v=cache(dtype=2)), hs2.ERR_INVALID_ARG),
+    (dict(k=cache(dtype=2, dim=64, scale=FAKE), v=cache(dtype=2, dim=64, scale=FAKE),
+          q=heads(dim=64), out=heads(dim=64)), hs2.ERR_UNSUPPORTED),
+    (dict(k=cache(scale=FAKE), v=cache(scale=FAKE)), hs2.ERR_INVALID_ARG),
+    (dict(k=cache(slots=1 << 31), v=cache(slots=1 << 31)), hs2.ERR_INVALID_ARG),
+    (dict(ws=0), hs2.ERR_WORKSPACE),
+    (dict(ws=FAKE * 16 + 16), hs2.ERR_WORKSPACE),
+    (dict(ws_bytes=1024), hs2.ERR_WORKSPACE),
+])
+def test_full_call_rejects_bad_arguments(libhs2, kw, code):
+    assert full(**kw) == code
+    assert hs2.last_error()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(idx=0), hs2.ERR_INVALID_ARG),
+    (dict(stride=0), hs2.ERR_UNSUPPORTED),
+    (dict(stride=5000), hs2.ERR_UNSUPPORTED),
+    (dict(q=heads(dim=64)), hs2.ERR_INVALID_ARG),
+    (dict(out=heads(h=8)), hs2.ERR_INVALID_ARG),
+    (dict(k=cache(dtype=7), v=cache(dtype=7)), hs2.ERR_UNSUPPORTED),
+])
+def test_sparse_call_rejects_bad_arguments(libhs2, kw, code):
+    assert sparse(**kw) == code
+
+
+def test_workspace_size_rules(libhs2):
+    f = hs2.full_workspace_bytes
+    a = f(4, 4, 8, 128, 262144)
+    assert a > 4 * 4 * 262144 * (8 * 4 + 4)  # at least the logits and the scores
+    assert f(4, 4, 8, 128, 2 * 262144) > a
+    assert f(0, 4, 8, 128, 1024) == 0 and f(1, 4, 3, 128, 1024) == 0 and f(1, 4, 8, 96, 1024) == 0
+    assert a % 256 == 0
+
+
+def test_copy_rejects_misaligned(libhs2):
+    assert hs2.lib().hs2_copy_peak(FAKE, FAKE + 4, 64, None) == hs2.ERR_INVALID_ARG
+    assert hs2.lib().hs2_copy_peak(FAKE, FAKE, 60, None) == hs2.ERR_INVALID_ARG

@@ -1,0 +1,185 @@
+"""Parity of the CUDA path (through the C-ABI) with the CPU oracle on small
+seeded workloads that still span many tiles, several CTAs per sequence and
+ragged tails, plus the edge cases of the method.
+
+Full layer (attention + token selection) and sparse layers (attention over the
+selected rows) of the HySparse2 Hybrid Block; tolerances in hs2_testutil.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_decode_full_b200 import synth
+import hs2_testutil as U
+
+pytestmark = pytest.mark.gpu
+
+
+def spec(**kw):
+    base = dict(name="parity", batch=3, num_kv_heads=2, group=8, head_dim=128, seq_len=(1500, 5000),
+                kv_dtype="bf16", q_dtype="bf16", page_size=64, sparse_layers=2, needles=24)
+    base.update(kw)
+    return synth.WorkloadSpec(**base)
+
+
+CASES = {
+    "bf16_paged64": spec(),
+    "bf16_contiguous": spec(page_size=None),
+    "bf16_paged16_nanpad": spec(page_size=16, seq_len=(1100, 3000)),
+    "bf16_paged32": spec(page_size=32, batch=2),
+    "bf16_paged128": spec(page_size=128, batch=2),
+    "bf16_d64_g4": spec(head_dim=64, group=4, num_kv_heads=3),
+    "bf16_g1": spec(group=1, num_kv_heads=4, batch=2),
+    "bf16_g2": spec(group=2, num_kv_heads=2, batch=2),
+    "e4m3_paged64": spec(kv_dtype="e4m3", seq_len=(1500, 4000)),
+    "e4m3_paged32_nanpad": spec(kv_dtype="e4m3", page_size=32, batch=2, seq_len=(1200, 2600)),
+    "f32_tiny": synth.WORKLOADS["tiny_fp32_t2048"],
+    "f32_paged_ragged": spec(kv_dtype="f32", q_dtype="f32", head_dim=64, group=4, page_size=16,
+                             seq_len=(1200, 2500)),
+    "short_window_only": spec(seq_len=(1, 127), batch=4),
+    "exactly_window_plus_k": spec(batch=2, seq_len=1152),
+    "one_more_than_fits": spec(batch=2, seq_len=1153),
+}
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_decode_full_b200 import hs2
+    hs2.lib()
+    return hs2
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_full_and_sparse_match_oracle(oracle, lib, name):
+    sp = CASES[name]
+    pad = "nan" if "nanpad" in name else None
+    w = synth.generate(sp, seed=zlib.crc32(name.encode()) % 1000, pad_fill=pad)
+    ora = U.run_oracle(oracle, w)
+    wd = U.to_device(w)
+    out, idx = U.run_gpu(wd)
+    torch.cuda.synchronize()
+    err, ndiff = U.check_full(wd, out, idx, ora)
+    # sparse layers: oracle's index list into both sides, each layer's own query
+    ora_idx = torch.from_numpy(ora["idx"]).cuda()
+    for layer in range(sp.sparse_layers):
+        g = U.run_gpu_sparse(wd, wd.q_sparse[layer], ora_idx)
+        ref = U.run_oracle_sparse(oracle, w, w.q_sparse[layer], ora["idx"])
+        U.check_out(g, ref, sp.kv_dtype, f"sparse layer {layer}")
+    # and the GPU's own list drives the GPU sparse layer like the oracle's does
+    if ndiff == 0:
+        g2 = U.run_gpu_sparse(wd, wd.q_sparse[0], idx)
+        ref = U.run_oracle_sparse(oracle, w, w.q_sparse[0], ora["idx"])
+        U.check_out(g2, ref, sp.kv_dtype, "sparse layer with GPU indices")
+    lib_status = lib.workspace_status(torch.zeros(256, dtype=torch.uint8, device="cuda"))
+    assert lib_status == 0
+
+
+def test_sparse_equals_full_when_everything_fits(oracle, lib):
+    sp = spec(seq_len=(300, 1152), batch=3)
+    w = U.to_device(synth.generate(sp, seed=5))
+    out, idx = U.run_gpu(w)
+    s = U.run_gpu_sparse(w, w.q_full, idx)
+    torch.cuda.synchronize()
+    assert (out.float() - s.float()).abs().max().item() <= 2e-2
+
+
+def test_zero_query_ties_pick_lowest_positions(oracle, lib):
+    """q = 0: every score ties, so the global part is exactly the lowest
+    k_global positions (bit-exact), and out = mean of V."""
+    sp = spec(seq_len=3000, batch=2)
+    w = synth.generate(sp, seed=8)
+    w.q_full.zero_()
+    ora = U.run_oracle(oracle, w)
+    wd = U.to_device(w)
+    out, idx = U.run_gpu(wd)
+    gi = idx.cpu().numpy()
+    assert np.array_equal(gi, ora["idx"])
+    U.check_out(out, ora["out"], "bf16")
+
+
+def test_constant_keys_ties_and_planted_order(oracle, lib):
+    """All keys equal except a planted descending ladder: the ladder wins in
+    order, the rest tie and fall to the lowest positions."""
+    sp = spec(seq_len=2500, batch=1, num_kv_heads=1, page_size=None)
+    w = synth.generate(sp, seed=9)
+    w.k[:] = w.k[0:1].clone()
+    ladder = torch.arange(300, 100, -1)
+    base = w.k[0, 0].float()
+    for r, t in enumerate(ladder.tolist()):
+        w.k[t, 0] = (base * (1.0 + 0.02 * (300 - r) / 300.0)).to(w.k.dtype)
+    ora = U.run_oracle(oracle, w)
+    wd = U.to_device(w)
+    out, idx = U.run_gpu(wd)
+    err, ndiff = U.check_full(wd, out, idx, ora)
+    assert ndiff == 0
+
+
+def test_empty_sequence_gives_zeros_and_no_indices(lib):
+    sp = spec(batch=3)
+    w = U.to_device(synth.generate(sp, seed=2, seq_lens=[2000, 0, 700]))
+    out, idx = U.run_gpu(w)
+    torch.cuda.synchronize()
+    assert torch.all(out[1] == 0)
+    assert torch.all(idx[1] == -1)
+    assert torch.all(idx[0, :, :1152] >= 0)
+
+
+def test_window_and_budget_variants(oracle, lib):
+    sp = spec(batch=2, seq_len=(2000, 3000))
+    w = synth.generate(sp, seed=12)
+    wd = U.to_device(w)
+    for W, K in [(0, 1), (1, 0), (128, 1), (64, 2048), (512, 1024), (5, 7)]:
+        ora = U.run_oracle(oracle, w, window=W, k_global=K)
+        out, idx = U.run_gpu(wd, window=W, k_global=K)
+        U.check_full(wd, out, idx, ora, window=W, k_global=K)
+
+
+def test_repeatable_bitwise(lib):
+    sp = spec(kv_dtype="bf16")
+    w = U.to_device(synth.generate(sp, seed=4))
+    a = U.run_gpu(w)
+    b = U.run_gpu(w)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    s1 = U.run_gpu_sparse(w, w.q_sparse[0], a[1])
+    s2 = U.run_gpu_sparse(w, w.q_sparse[0], a[1])
+    assert torch.equal(s1, s2)
+
+
+def test_paged_and_contiguous_agree_bitwise(lib):
+    sp = spec(batch=2, seq_len=3000)
+    wp = U.to_device(synth.generate(sp, seed=6))
+    wc = U.to_device(synth.generate(sp.replace(page_size=None), seed=6))
+    for b in range(2):
+        T = int(wp.seq_lens[b])
+        spp = synth.slots_of(wp, b, torch.arange(T, device="cuda"))
+        scc = synth.slots_of(wc, b, torch.arange(T, device="cuda"))
+        wc.k[scc] = wp.k[spp]
+        wc.v[scc] = wp.v[spp]
+    wc.q_full.copy_(wp.q_full)
+    op, ip = U.run_gpu(wp)
+    oc, ic = U.run_gpu(wc)
+    torch.cuda.synchronize()
+    assert torch.equal(op, oc)
+    for b in range(2):
+        m = {int(c): int(p) for c, p in zip(
+            synth.slots_of(wc, b, torch.arange(3000)).tolist(),
+            synth.slots_of(wp, b, torch.arange(3000, device="cuda")).tolist())}
+        got = [[m[int(x)] for x in row] for row in ic[b].tolist()]
+        assert got == ip[b].tolist()
+
+
+def test_hybrid_block_step_runs_all_layers(oracle, lib):
+    from long_context_decode_full_b200 import hs2
+    sp = spec(batch=2, sparse_layers=3)
+    w = synth.generate(sp, seed=21)
+    wd = U.to_device(w)
+    outs, idx = hs2.hybrid_block_step(wd.q_full, list(wd.q_sparse), wd.k, wd.v, wd.seq_lens, wd.page_table,
+                                      wd.page_size)
+    ora = U.run_oracle(oracle, w)
+    U.check_full(wd, outs[0], idx, ora)
+    for layer in range(3):
+        ref = U.run_oracle_sparse(oracle, w, w.q_sparse[layer], ora["idx"])
+        U.check_out(outs[1 + layer], ref, "bf16", f"layer {layer}")
