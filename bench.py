@@ -176,6 +176,8 @@ def run_gpu(args, rank, world, local):
     from long_context_decode_full_b200 import hs2
 
     spec = synth.WORKLOADS[args.workload]
+    if args.seq_len:
+        spec = spec.replace(seq_len=args.seq_len)
     w = synth.generate(spec, seed=args.seed + rank, device="cuda")
     s = spec
     dev = torch.device("cuda", local)
@@ -345,6 +347,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=500)
     ap.add_argument("--cpu-units", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=0, help="override the workload's context (profiling runs)")
     args = ap.parse_args()
     if args.impl == "reference":
         args.warmup = max(0, min(args.warmup, 1))

@@ -38,7 +38,7 @@ __device__ __forceinline__ UnitInfo unit_info(const ScoreParams &p, int b, int k
   UnitInfo ui;
   ui.T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
   ui.nC = max(0, ui.T - p.window);
-  ui.select = ui.nC > p.k_global;
+  ui.select = ui.nC > p.k_global && p.k_global > 0;
   ui.nb = (ui.T + p.tile - 1) / p.tile;
   const int64_t total = (int64_t)p.Hkv * p.ws.prefix[p.B];
   ui.U = (int64_t)p.Hkv * p.ws.prefix[b] + (int64_t)kvh * ui.nb;
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
   const int nC = max(0, T - p.window);
-  if (nC <= p.k_global || chunk * kScoreChunk >= nC) return;
+  if (nC <= p.k_global || p.k_global == 0 || chunk * kScoreChunk >= nC) return;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
   const int2 thr = p.ws.thr[u];
   const uint32_t bin1 = (uint32_t)thr.x;
@@ -278,9 +278,10 @@ __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams 
   uint32_t *sel = p.ws.sel + (size_t)u * words;
   uint32_t *tie = p.ws.tie + (size_t)u * words;
   const bool all = nC <= p.k_global;
+  const bool none = !all && p.k_global == 0;  // window only
   int need_eq = 0;
 
-  if (!all) {
+  if (!all && !none) {
     const uint2 *cand = p.ws.cand + (size_t)u * p.t_cap;
     const uint32_t cc = p.ws.cand_count[u];
     const int n1 = cc < (uint32_t)nC ? (int)cc : nC;
@@ -330,7 +331,7 @@ __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams 
     return (1u << (T - lo)) - 1u;
   };
   int tie_before = 0;
-  if (!all) {
+  if (!all && !none) {
     int cnt = 0;
     for (int w = w0; w < w1; ++w) cnt += __popc(__ldcg(tie + w) & cmask(w));
     tie_before = block_exclusive_scan(cnt, sh_warp, &sh_tot);
@@ -338,6 +339,7 @@ __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams 
   auto word_sel = [&](int w, int &ties_seen) -> uint32_t {
     const uint32_t cm = cmask(w), tm = tmask(w);
     if (all) return tm;
+    if (none) return tm & ~cm;
     uint32_t x = (__ldcg(sel + w) & cm) | (tm & ~cm);
     uint32_t tw = __ldcg(tie + w) & cm;
     while (tw) {
