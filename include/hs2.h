@@ -132,6 +132,34 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
                                 void *workspace, size_t workspace_bytes, void *stream, void *mark_event);
 
 /*
+ * hs2_full_attn_select() for callers that cannot allocate device memory.
+ * The pages have no counterpart to this call; it exists for integration.
+ *
+ * Some callers only receive device pointers and a stream and are not allowed
+ * to call cudaMalloc: a plugin inside a serving engine that has already
+ * reserved nearly all HBM for its own KV-cache pool, or code whose launches
+ * are later recorded into a CUDA graph, where allocating is not permitted.
+ * They cannot provide the workspace hs2_full_attn_select() needs, so this
+ * call uses a scratch array that the library itself owns: a fixed 32 MiB
+ * device array that every GPU which loads the library keeps until the
+ * process exits.  The call allocates nothing.
+ *
+ *   Arguments and results are those of hs2_full_attn_select() without the
+ *   workspace.  Shapes whose workspace (hs2_full_attn_select_workspace())
+ *   exceeds 32 MiB are rejected with HS2_ERR_WORKSPACE and a message.
+ *   The first call on each device looks up the array's device address on
+ *   that device; make that first call before any stream capture begins.
+ *   All calls share the one array and it keeps the last call's contents (the
+ *   kernels clear what must start at zero themselves): calls that overlap on
+ *   the GPU -- on different streams, or from different threads -- race and
+ *   must be serialised by the caller.
+ */
+int hs2_full_attn_select_static(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                                const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
+                                int32_t window, int32_t k_global, hs2_heads *out, int32_t *idx_out,
+                                void *stream);
+
+/*
  * Sparse-attention layer of a Hybrid Block: for each (b, query head h) the
  * softmax of q_l k^T / sqrt(d) over the rows idx[b, floor(h/G), :] (slots,
  * -1 entries skipped), times those V rows.  It reads the same shared cache as

@@ -403,6 +403,8 @@ __global__ void __launch_bounds__(512) copy_kernel(uint4 *__restrict__ dst, cons
   for (; i < n; i += stride) __stcs(dst + i, __ldcs(src + i));
 }
 
+int set_last_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
 cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int grid, cudaStream_t s) {
   if (bytes == 0) return cudaSuccess;
   copy_kernel<<<grid, 512, 0, s>>>(static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), bytes / 16);

@@ -42,7 +42,7 @@ class HS2Error(RuntimeError):
 
 _lib = None
 EXPORTS = ["hs2_full_attn_select_workspace", "hs2_full_attn_select", "hs2_full_attn_select_marked",
-           "hs2_sparse_attn",
+           "hs2_full_attn_select_static", "hs2_sparse_attn",
            "hs2_workspace_status", "hs2_copy_peak", "hs2_last_error", "hs2_version"]
 
 
@@ -62,6 +62,10 @@ def lib():
         L.hs2_full_attn_select.restype = ctypes.c_int
         L.hs2_full_attn_select_marked.argtypes = L.hs2_full_attn_select.argtypes + [P]
         L.hs2_full_attn_select_marked.restype = ctypes.c_int
+        L.hs2_full_attn_select_static.argtypes = [ctypes.POINTER(Heads), ctypes.POINTER(Cache),
+                                                  ctypes.POINTER(Cache), P, P, I32, I32, I32,
+                                                  ctypes.POINTER(Heads), P, P]
+        L.hs2_full_attn_select_static.restype = ctypes.c_int
         L.hs2_sparse_attn.argtypes = [ctypes.POINTER(Heads), ctypes.POINTER(Cache), ctypes.POINTER(Cache), P, I32,
                                       ctypes.POINTER(Heads), P]
         L.hs2_sparse_attn.restype = ctypes.c_int
@@ -140,6 +144,29 @@ def full_attn_select(q, k, v, seq_lens, page_table=None, page_size=None, window=
                                              _ptr(seq_lens), _ptr(page_table), max_pages, window, k_global,
                                              ctypes.byref(od), _ptr(idx_out), _ptr(workspace), workspace.numel(),
                                              _stream(stream), ev))
+    return out, idx_out
+
+
+def full_attn_select_static(q, k, v, seq_lens, page_table=None, page_size=None, window=128, k_global=1024,
+                            k_scale=None, v_scale=None, out=None, idx_out=None, stream=None):
+    """full_attn_select() without a workspace: the library's own fixed 32 MiB
+    device scratch is used (for callers that may not allocate).  Calls that
+    overlap on the GPU race on that scratch."""
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if page_size is None:
+        assert page_table is None, "page_size is required with a page table"
+        page_size = k.shape[0] // B
+    max_pages = 1 if page_table is None else page_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if idx_out is None:
+        idx_out = torch.empty(B, Hkv, window + k_global, dtype=torch.int32, device=q.device)
+    kc, vc = cache_desc(k, k_scale, page_size), cache_desc(v, v_scale, page_size)
+    qd, od = heads_desc(q), heads_desc(out)
+    _check(lib().hs2_full_attn_select_static(ctypes.byref(qd), ctypes.byref(kc), ctypes.byref(vc),
+                                             _ptr(seq_lens), _ptr(page_table), max_pages, window, k_global,
+                                             ctypes.byref(od), _ptr(idx_out), _stream(stream)))
     return out, idx_out
 
 
