@@ -80,16 +80,19 @@ int encode_cache_map(CUtensorMap *map, const hs2_cache *c, int box_rows) {
 
 // ---------------------------------------------------------------- workspace
 struct Layout {
-  size_t err, prefix, records, logits, scores, cand, sel, tie, hist, thr, total;
-  int R;
+  size_t err, prefix, records, logits, scores, above, cand, subcnt, hist, thr, lse, total;
+  int R, nsub;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-Layout layout(int B, int Hkv, int G, int D, int64_t t_cap) {
+int64_t unit_stride(int64_t t_cap) { return (t_cap + 127) / 128 * 128; }
+
+Layout layout(int B, int Hkv, int G, int D, int64_t t_cap_in) {
   Layout L;
   const size_t U = (size_t)B * Hkv;
-  const size_t words = (size_t)((t_cap + 31) / 32);
+  const int64_t t_cap = unit_stride(t_cap_in);  // per-unit arrays keep 16-byte aligned rows
+  L.nsub = (int)((t_cap + kSubRange - 1) / kSubRange);
   L.R = sm_count() * kMaxCtasPerSm / Hkv + 2;
   size_t o = 0;
   L.err = o;
@@ -102,16 +105,18 @@ Layout layout(int B, int Hkv, int G, int D, int64_t t_cap) {
   o = align256(o + U * (size_t)t_cap * G * 4);
   L.scores = o;
   o = align256(o + U * (size_t)t_cap * 4);
+  L.above = o;
+  o = align256(o + U * (size_t)t_cap * 4);
   L.cand = o;
   o = align256(o + U * (size_t)t_cap * 8);
-  L.sel = o;
-  o = align256(o + U * words * 4);
-  L.tie = o;
-  o = align256(o + U * words * 4);
-  L.hist = o;  // hist [U][4096], ticket [U], cand_count [U] back to back
+  L.subcnt = o;
+  o = align256(o + U * (size_t)L.nsub * 8);
+  L.hist = o;  // hist [U][4096], ticket [U], spare [U] back to back
   o = align256(o + U * (kHistBins + 2) * 4);
   L.thr = o;
   o = align256(o + U * 8);
+  L.lse = o;
+  o = align256(o + U * 8 * sizeof(double));
   L.total = o;
   return L;
 }
@@ -125,13 +130,13 @@ FullWs bind(const Layout &L, void *ws, int B, int Hkv) {
   f.records = reinterpret_cast<float *>(w + L.records);
   f.logits = reinterpret_cast<float *>(w + L.logits);
   f.scores = reinterpret_cast<float *>(w + L.scores);
+  f.above = reinterpret_cast<int32_t *>(w + L.above);
   f.cand = reinterpret_cast<uint2 *>(w + L.cand);
-  f.sel = reinterpret_cast<uint32_t *>(w + L.sel);
-  f.tie = reinterpret_cast<uint32_t *>(w + L.tie);
+  f.subcnt = reinterpret_cast<int2 *>(w + L.subcnt);
   f.hist = reinterpret_cast<uint32_t *>(w + L.hist);
   f.ticket = f.hist + U * kHistBins;
-  f.cand_count = f.ticket + U;
   f.thr = reinterpret_cast<int2 *>(w + L.thr);
+  f.lse = reinterpret_cast<double *>(w + L.lse);
   return f;
 }
 
@@ -181,9 +186,9 @@ int check_caches(const hs2_cache *k, const hs2_cache *v) {
 }
 
 FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged) {
-  FullMmaConfig c{4, 4};
+  // 8 consumer warps (128-position tiles) keep two warps per SM sub-partition
+  FullMmaConfig c = fp8 ? FullMmaConfig{8, 4} : FullMmaConfig{8, 3};
   (void)D;
-  (void)fp8;
   if (const char *env = getenv("HS2_FULL_CFG")) {
     int a = 0, b = 0;
     if (sscanf(env, "%d,%d", &a, &b) == 2) c = FullMmaConfig{a, b};
@@ -203,7 +208,8 @@ int hs2_version(void) { return 100; }
 
 size_t hs2_full_attn_select_workspace(int32_t batch, int32_t num_kv_heads, int32_t group, int32_t head_dim,
                                       int64_t t_cap) {
-  if (batch < 1 || num_kv_heads < 1 || !group_ok(group) || (head_dim != 64 && head_dim != 128) || t_cap < 1)
+  if (batch < 1 || num_kv_heads < 1 || !group_ok(group) || (head_dim != 64 && head_dim != 128) || t_cap < 1 ||
+      t_cap > kMaxContext)
     return 0;
   return layout(batch, num_kv_heads, group, head_dim, t_cap).total;
 }
@@ -227,8 +233,9 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
   if (out->batch != q->batch || out->num_heads != q->num_heads || out->dtype != q->dtype)
     return fail(HS2_ERR_INVALID_ARG, "out shape/dtype differs from q");
   if (!seq_lens || !idx_out) return fail(HS2_ERR_INVALID_ARG, "seq_lens / idx_out is NULL");
-  if (window < 0 || k_global < 0 || (int64_t)window + k_global < 1 || (int64_t)window + k_global > (1 << 24))
-    return fail(HS2_ERR_INVALID_ARG, "window %d / k_global %d", window, k_global);
+  if (window < 0 || k_global < 0 || (int64_t)window + k_global < 1 || (int64_t)window + k_global > kMaxSelect)
+    return fail(HS2_ERR_INVALID_ARG, "window %d / k_global %d (need 1 <= window + k_global <= %d)", window,
+                k_global, kMaxSelect);
   const int B = q->batch, Hkv = k_cache->num_kv_heads, G = q->num_heads / Hkv, D = k_cache->head_dim;
   const int ps = k_cache->page_size;
   const bool paged = page_table != nullptr;
@@ -242,8 +249,9 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
     if ((int64_t)B * ps > k_cache->num_slots)
       return fail(HS2_ERR_INVALID_ARG, "contiguous layout needs num_slots >= batch * page_size");
   }
-  if (t_cap > (int64_t(1) << 30) || (int64_t)B * ((t_cap + 15) / 16) * Hkv >= (int64_t(1) << 31))
-    return fail(HS2_ERR_UNSUPPORTED, "context capacity too large");
+  if (t_cap > kMaxContext || (int64_t)B * ((t_cap + 15) / 16) * Hkv >= (int64_t(1) << 31))
+    return fail(HS2_ERR_UNSUPPORTED, "context capacity %lld too large (max %lld per sequence)", (long long)t_cap,
+                (long long)kMaxContext);
   if (B > kMaxBatchSmem) return fail(HS2_ERR_UNSUPPORTED, "batch %d > %d", B, kMaxBatchSmem);
   const bool mma = k_cache->dtype != HS2_F32;
   if (mma && paged && !(ps % 16 == 0 && (ps % 64 == 0 || 64 % ps == 0)))
@@ -270,6 +278,7 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
   p.page_size = ps;
   p.max_pages = paged ? max_pages : 1;
   p.t_cap = t_cap;
+  p.ustride = unit_stride(t_cap);
   p.num_slots = k_cache->num_slots;
   p.R = L.R;
   p.c = 1.0f / sqrtf((float)D);
@@ -312,11 +321,13 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
   sp.page_size = ps;
   sp.max_pages = p.max_pages;
   sp.t_cap = t_cap;
+  sp.ustride = p.ustride;
   sp.window = window;
   sp.k_global = k_global;
   sp.N = p.N;
   sp.R = p.R;
   sp.tile = p.tile;
+  sp.nsub = L.nsub;
   sp.c = p.c;
   sp.ws = p.ws;
   e = launch_select(sp, s);
@@ -349,10 +360,11 @@ int hs2_sparse_attn(const hs2_heads *q_l, const hs2_cache *k_cache, const hs2_ca
   p.L = idx_stride;
   p.c = 1.0f / sqrtf((float)p.D);
   // enough CTAs per unit to cover the SMs, at most 16 per cluster and 256 rows per CTA
-  const int units = p.B * p.Hkv, sms = sm_count();
-  const int want = (sms + units - 1) / units;
-  const int cap = units * 8 <= sms / 2 ? 16 : 8;  // 16-CTA clusters only when units are few
-  int S = want < 1 ? 1 : (want > cap ? cap : want);
+  // fewest CTAs per unit that keep a CTA at <= 256 rows (16 warps): fatter
+  // CTAs measured faster than more, smaller ones at the pages' 1152 rows
+  int want = 1;
+  if (const char *env = getenv("HS2_SPARSE_SPLITS")) want = atoi(env);  // tuning override
+  int S = want < 1 ? 1 : (want > 16 ? 16 : want);
   const int min_s = (idx_stride + 255) / 256;
   if (S < min_s) S = min_s;
   int rows = ((idx_stride + S - 1) / S + 15) / 16 * 16;

@@ -19,9 +19,12 @@ constexpr int kHistBins = 4096;          // score histogram: float bits 30..19
 constexpr int kHistShift = 19;
 constexpr int kScoreChunk = 4096;        // positions per score / filter CTA
 constexpr int kScoreThreads = 256;
-constexpr int kFinalThreads = 1024;
+constexpr int kFinalThreads = 512;
 constexpr long long kSpinLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
 constexpr int kMaxBatchSmem = 4096;      // sequences whose tile prefix fits in smem
+constexpr int kSubRange = 512;           // positions per filter-warp list
+constexpr int kMaxSelect = 4096;         // window + k_global upper bound
+constexpr int64_t kMaxContext = int64_t(1) << 23;  // positions per sequence
 
 // Error bits of the sticky workspace flag.
 constexpr uint32_t kErrFullWait = 1u;    // consumer timed out on a full barrier
@@ -36,13 +39,13 @@ struct FullWs {
   float *logits;         // [U, t_cap, G] raw q.k per position and head (fp32, unscaled)
   float *records;        // [U, R, G * (D + 2)]: m[G], l[G], o[G][D] of each segment
   float *scores;         // [U, t_cap] group score of the selectable positions
-  uint2 *cand;           // [U, t_cap] (score bits, position) of the threshold bin
-  uint32_t *sel;         // [U, words] positions strictly above the threshold
-  uint32_t *tie;         // [U, words] positions equal to the threshold score
-  uint32_t *hist;        // [U, kHistBins]
+  int32_t *above;        // [U, t_cap] positions above the threshold bin, per 512-position list
+  uint2 *cand;           // [U, t_cap] (score bits, position) inside the threshold bin, same lists
+  int2 *subcnt;          // [U, nsub] (above, in-bin) counts of each list
+  uint32_t *hist;        // [U, kHistBins], then ticket [U] and one spare word [U]
   uint32_t *ticket;      // [U]
-  uint32_t *cand_count;  // [U]
   int2 *thr;             // [U] (threshold bin, count strictly above it)
+  double *lse;           // [U, 8] per-head log-sum-exp of the scaled logits
 };
 
 // Balanced partition of the tile space over N persistent CTAs.  Tiles are
@@ -192,6 +195,13 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // 16-byte chunk c of row r lives at chunk c ^ (r & 7).
 __device__ __forceinline__ uint32_t swz(uint32_t panel, int row, int chunk) {
   return panel + row * 128 + (((chunk ^ row) & 7) << 4);
+}
+
+// 2^x by the MUFU approximation (flushes subnormal results to zero)
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ---------------------------------------------------------------- warp reductions

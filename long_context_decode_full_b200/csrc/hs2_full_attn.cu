@@ -150,7 +150,13 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
 
   if (producer) {
     // ------------------------------------------------------------ producer
+    // Boxes of RB rows (one page, or the whole tile when pages are larger).
+    // Lane L caches the first slot of CTA-local box cache_base + L, so page
+    // table reads are issued 32 at a time instead of one per box.
     const int RB = p.page_table ? min(C::TILE, p.page_size) : C::TILE;
+    const int BPT = C::TILE / RB;  // boxes per tile (<= 8)
+    int64_t cache_base = -(int64_t)64;
+    int my_slot = -1;
     int it = 0;
     int b = g0 < g1 ? find_seq(prefix, p.B, p.Hkv, g0) : 0;
     bool ok = true;
@@ -161,6 +167,23 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
       const int kvh = (int)(r / nb), i = (int)(r % nb);
       const int64_t U = (int64_t)p.Hkv * prefix[b] + (int64_t)kvh * nb;
       const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
+      const int64_t box0 = (g - g0) * BPT;
+      if (box0 + BPT > cache_base + 32) {  // refill: lane L -> box box0 + L
+        cache_base = box0;
+        const int64_t bx = box0 + lane, gl = g0 + bx / BPT;
+        my_slot = -1;
+        if (gl < g1) {
+          const int bl = find_seq(prefix, p.B, p.Hkv, gl);
+          const int nbl = prefix[bl + 1] - prefix[bl];
+          const int il = (int)((gl - (int64_t)p.Hkv * prefix[bl]) % nbl);
+          const int pos = il * C::TILE + (int)(bx % BPT) * RB;
+          const int Tl = clamp_len(__ldg(p.seq_lens + bl), (int)p.t_cap);
+          if (pos < Tl) {
+            const int64_t sl = slot_of(p.page_table, p.max_pages, p.page_size, bl, pos);
+            my_slot = (sl >= 0 && sl < p.num_slots) ? (int)sl : -1;
+          }
+        }
+      }
       const int stage = it % NSTAGE;
       if (it >= NSTAGE && !mbar_wait(&empty[stage], ((it / NSTAGE) - 1) & 1)) {
         set_error(p.ws.err, kErrEmptyWait);
@@ -170,18 +193,24 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
       const int64_t j = blockIdx.x - part.cfirst(U);
       const int64_t u = (int64_t)b * p.Hkv + kvh;
       const int p0 = i * C::TILE;
+      const int cl0 = (int)(box0 - cache_base);  // cache lane of this tile's first box
       if constexpr (FP8) {
         float *ks = scales + stage * (2 * C::TILE);
-        for (int rr = lane; rr < C::TILE; rr += 32) {
-          const int pos = p0 + rr;
-          const int64_t slot = pos < T ? slot_of(p.page_table, p.max_pages, p.page_size, b, pos) : -1;
-          if (slot >= 0 && slot < p.num_slots) {
+#pragma unroll
+        for (int k = 0; k < C::TILE / 32; ++k) {
+          const int rr = lane + 32 * k;
+          const int bs = __shfl_sync(0xffffffffu, my_slot, cl0 + rr / RB);
+          if (p0 + rr < T && bs >= 0) {
+            const int64_t slot = (int64_t)bs + rr % RB;
             cp_async_4(smem_u32(ks + rr), p.k_scale + slot * p.Hkv + kvh);
             cp_async_4(smem_u32(ks + C::TILE + rr), p.v_scale + slot * p.Hkv + kvh);
           }
         }
         cp_async_mbar_arrive_noinc(&full[stage]);
       }
+      int box_slot[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) box_slot[k] = __shfl_sync(0xffffffffu, my_slot, min(cl0 + k, 31));
       if (lane == 0) {
         StageMeta mt;
         mt.b = b;
@@ -193,15 +222,19 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
         mt.T = T;
         meta[stage] = mt;
         uint32_t bytes = 0;
-        for (int rr = 0; rr < C::TILE && p0 + rr < T; rr += RB) bytes += 2u * RB * C::ROWB;
+        for (int k = 0; k < BPT && p0 + k * RB < T; ++k) bytes += 2u * RB * C::ROWB;
         mbar_arrive_expect_tx(&full[stage], bytes);
         const uint32_t kdst = sbase + stage * C::STAGE, vdst = kdst + C::KVB;
-        for (int rr = 0; rr < C::TILE && p0 + rr < T; rr += RB) {
-          const int slot = (int)slot_of(p.page_table, p.max_pages, p.page_size, b, p0 + rr);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (k >= BPT || p0 + k * RB >= T) break;
+          // a slot outside the cache (bad page id) loads from row 2^31 - 1 .. : out of
+          // the tensor, so TMA fills zeros and the transfer still completes
+          const int slot = box_slot[k] >= 0 ? box_slot[k] : 0x7FFFFFFF - RB;
 #pragma unroll
           for (int pn = 0; pn < C::NPANEL; ++pn) {
-            tma_load_3d(kdst + pn * C::PANEL + rr * 128, &tmk, &full[stage], pn * (128 / C::ES), kvh, slot);
-            tma_load_3d(vdst + pn * C::PANEL + rr * 128, &tmv, &full[stage], pn * (128 / C::ES), kvh, slot);
+            tma_load_3d(kdst + pn * C::PANEL + k * RB * 128, &tmk, &full[stage], pn * (128 / C::ES), kvh, slot);
+            tma_load_3d(vdst + pn * C::PANEL + k * RB * 128, &tmv, &full[stage], pn * (128 / C::ES), kvh, slot);
           }
         }
       }
@@ -246,7 +279,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
     const uint32_t kp = sbase + stage * C::STAGE;
     const float *ks = scales + stage * (2 * C::TILE) + 16 * warp;
     if (nvalid > 0)
-      st.step(kp, kp + C::KVB, C::PANEL, 16 * warp, vmask, p.c, p.ws.logits + (u * p.t_cap + pos0) * p.G, p.G, ks,
+      st.step(kp, kp + C::KVB, C::PANEL, 16 * warp, vmask, p.c, p.ws.logits + (u * p.ustride + pos0) * p.G, p.G, ks,
               ks + C::TILE);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[stage]);
@@ -339,7 +372,7 @@ __global__ void __launch_bounds__(32 * kF32Warps) full_attn_f32_kernel(const Ful
 #pragma unroll 4
         for (int e = 0; e < D; ++e) acc = fmaf(Qs[h * D + e], Ks[rr * (D + 1) + e], acc);
         s[j] = p0 + rr < T ? acc : -INFINITY;
-        if (p0 + rr < T) p.ws.logits[(u * p.t_cap + p0 + rr) * p.G + h] = acc;
+        if (p0 + rr < T) p.ws.logits[(u * p.ustride + p0 + rr) * p.G + h] = acc;
       }
       const float mx = warp_max(fmaxf(s[0], s[1]));
       const float m_new = fmaxf(m[hs], mx);

@@ -21,6 +21,7 @@ struct FullParams {
   int32_t B, Hkv, G, D;
   int32_t page_size, max_pages;
   int64_t t_cap;             // logical capacity per sequence
+  int64_t ustride;           // positions per unit in the workspace arrays (t_cap rounded up to 128)
   int64_t num_slots;
   int32_t N;                 // persistent CTAs (grid size)
   int32_t R;                 // record slots per unit
@@ -38,8 +39,10 @@ struct ScoreParams {
   int32_t B, Hkv, G, D;
   int32_t page_size, max_pages;
   int64_t t_cap;
+  int64_t ustride;
   int32_t window, k_global;
   int32_t N, R, tile;
+  int32_t nsub;              // 512-position lists per unit: ceil(t_cap / 512)
   float c;
   FullWs ws;
 };

@@ -4,22 +4,28 @@
 // kept plus the top `k_global` tokens from outside that window).
 //
 // Score of position t for KV head j: sum over the query heads h of j's GQA
-// group of softmax probability p_{h,t} = exp(c * s_{h,t} - LSE_h).
+// group of the softmax probability p_{h,t} = exp(c * s_{h,t} - LSE_h).
 //
-// Three kernels, all on the CUDA cores:
-//   score  -- per (chunk, kv head, sequence): LSE of the group's heads from
-//             the segment records (fp64), the final attention output of the
-//             unit (chunk 0), the fp32 group score of every selectable
-//             position and a 4096-bin histogram of the score's top bits; the
-//             last chunk to finish (atomic ticket, no waiting) finds the bin
-//             that holds the k-th largest score.
-//   filter -- per chunk: positions above that bin go straight into a bitmap
-//             (one warp ballot per 32 positions); positions inside it are
-//             appended to a candidate list.
-//   final  -- per unit: radix refinement of the candidates to the exact k-th
-//             score, ties resolved to the lower position, then an ordered
-//             compaction (block scans over the bitmaps) that merges the forced
-//             window and writes slots in ascending position order.
+// Three kernels on the CUDA cores:
+//   score  -- grid (chunk, kv head, sequence) + one combine CTA per unit.
+//             Score CTAs rebuild each head's LSE from the segment records (a
+//             parallel fp64 reduction), turn the raw logits of 4096 positions
+//             into approximate group scores (one FMA and one ex2 per head,
+//             relative error below 1e-5) and a 4096-bin histogram of their top
+//             bits (16 bins per octave); the last chunk to finish (atomic
+//             ticket, no waiting) finds the bin b holding the k_global-th
+//             largest approximate score.  The combine CTA merges the records
+//             into the attention output.
+//   filter -- each warp owns 512 consecutive positions and writes, in
+//             position order, the positions whose approximate bin is >= b+2
+//             (certainly above the k-th exact score: a bin is 4.4% wide) and
+//             the positions in bins b-1 .. b+1 (the guard band that holds
+//             every position the exact k-th score can hinge on).
+//   final  -- one CTA per unit: exact scores of the guard-band positions
+//             (exponent formed in float-float, so only ex2's own rounding is
+//             left), radix select of the exact k-th score among them, ties to
+//             the lower position (the list is position-ordered), then a merge
+//             of the two sorted lists and the forced window into the index list.
 // Scores are >= 0, so their IEEE bit patterns order like the values.
 #include "hs2_internal.h"
 
@@ -27,11 +33,13 @@ namespace hs2 {
 
 namespace {
 
+constexpr double kLog2e = 1.4426950408889634074;
+
 struct UnitInfo {
   int T, nC, nb;
-  int64_t U;   // first linear tile of the unit
+  int64_t U;  // first linear tile of the unit
   int nseg;
-  bool select; // nC > k_global
+  bool select;  // nC > k_global > 0
 };
 
 __device__ __forceinline__ UnitInfo unit_info(const ScoreParams &p, int b, int kvh) {
@@ -57,7 +65,8 @@ __device__ __forceinline__ int64_t slot_of(const ScoreParams &p, int b, int64_t 
          pos % p.page_size;
 }
 
-// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024).
+// Block-wide exclusive scan of one int per thread; *total gets the sum.
+// sh_warp needs 33 ints.
 __device__ __forceinline__ int block_exclusive_scan(int x, int *sh_warp, int *total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
   int incl = x;
@@ -69,7 +78,7 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int *sh_warp, int *to
   if (lane == 31) sh_warp[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < nw ? sh_warp[lane] : 0;
+    const int w = lane < nw ? sh_warp[lane] : 0;
     int wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -77,27 +86,27 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int *sh_warp, int *to
       if (lane >= o) wi += y;
     }
     if (lane < nw) sh_warp[lane] = wi - w;
-    if (lane == 31) *total = wi;
+    if (lane == 31) sh_warp[32] = wi;
   }
   __syncthreads();
   const int r = sh_warp[warp] + incl - x;
+  *total = sh_warp[32];
   __syncthreads();
   return r;
 }
 
-// Finds, over a histogram in shared memory (nbins, bin index increasing with
-// score), the bin holding the need-th largest element: returns the bin and
-// writes the count strictly above it.  Called by the whole block.
+// Over a histogram in shared memory (bin index increasing with score), the
+// bin holding the need-th largest element and the count strictly above it.
+// Whole block.
 __device__ int find_threshold_bin(const uint32_t *hist, int nbins, int need, int *above_out, int *sh_warp,
                                   int *sh_res) {
   const int per = (nbins + blockDim.x - 1) / blockDim.x;
-  if (threadIdx.x == 0) {  // defaults if the histogram holds fewer than `need`
+  if (threadIdx.x == 0) {
     sh_res[0] = 0;
     sh_res[1] = 0;
   }
-  // thread i owns bins counted from the top: [i*per, (i+1)*per) in descending order
   int cnt = 0;
-  for (int k = 0; k < per; ++k) {
+  for (int k = 0; k < per; ++k) {  // thread i owns the i-th group of bins from the top
     const int bin = nbins - 1 - (threadIdx.x * per + k);
     if (bin >= 0) cnt += (int)hist[bin];
   }
@@ -123,64 +132,101 @@ __device__ int find_threshold_bin(const uint32_t *hist, int nbins, int need, int
   return bin;
 }
 
+// Per-head LSE (fp64), max and normaliser of a unit from its segment
+// records, as a block-wide reduction: thread t folds the pairs (segment j,
+// head h) with h = t % G.
+template <int G, int D>
+__device__ void unit_lse(const float *rec0, int nseg, float c, double *sh_lse, float *sh_M, float *sh_L,
+                         double *sh_red) {
+  constexpr int RS = G * (D + 2);
+  const int tid = threadIdx.x, nt = blockDim.x, h = tid % G;
+  float m = -INFINITY;
+  for (int i = tid; i < nseg * G; i += nt) m = fmaxf(m, rec0[(i / G) * RS + h]);
+  reinterpret_cast<float *>(sh_red)[tid] = m;
+  __syncthreads();
+  if (tid < G) {
+    float M = -INFINITY;
+    for (int t = tid; t < nt; t += G) M = fmaxf(M, reinterpret_cast<float *>(sh_red)[t]);
+    sh_M[tid] = M;
+  }
+  __syncthreads();
+  const float M = sh_M[h];
+  double L = 0.0;
+  for (int i = tid; i < nseg * G; i += nt) {
+    const int j = i / G;
+    const float mj = rec0[j * RS + h];
+    if (mj != -INFINITY) L += (double)rec0[j * RS + G + h] * exp((double)c * ((double)mj - (double)M));
+  }
+  sh_red[tid] = L;
+  __syncthreads();
+  if (tid < G) {
+    double S = 0.0;
+    for (int t = tid; t < nt; t += G) S += sh_red[t];
+    sh_lse[tid] = (double)c * (double)sh_M[tid] + log(S);
+    sh_L[tid] = (float)S;
+  }
+  __syncthreads();
+}
+
 // ------------------------------------------------------------------ score
 template <int G, int D>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams p) {
   __shared__ uint32_t sh_hist[kHistBins];
+  __shared__ double sh_red[kScoreThreads];
   __shared__ double sh_lse[G];
   __shared__ float sh_M[G], sh_L[G];
-  __shared__ int sh_warp[32], sh_res[2], sh_last;
+  __shared__ int sh_warp[33], sh_res[2], sh_last;
+  constexpr int RS = G * (D + 2);
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const bool combine = chunk == (int)gridDim.x - 1;  // the unit's combine CTA
   const UnitInfo ui = unit_info(p, b, kvh);
   const int n_chunks = ui.select ? (ui.nC + kScoreChunk - 1) / kScoreChunk : 0;
-  const bool do_out = chunk == 0;
-  if (!do_out && chunk >= n_chunks) return;
+  if (!combine && chunk >= n_chunks) return;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
-  const float *rec0 = p.ws.records + (size_t)u * p.R * G * (D + 2);
-  const int RS = G * (D + 2);
+  const float *rec0 = p.ws.records + (size_t)u * p.R * RS;
+  unit_lse<G, D>(rec0, ui.nseg, p.c, sh_lse, sh_M, sh_L, sh_red);
 
-  // LSE of each head from the segment records: c*M + log(sum_j l_j exp(c (m_j - M)))
-  if (threadIdx.x < G) {
-    const int h = threadIdx.x;
-    float M = -INFINITY;
-    for (int j = 0; j < ui.nseg; ++j) M = fmaxf(M, rec0[j * RS + h]);
-    double L = 0.0;
-    float Lf = 0.f;
-    for (int j = 0; j < ui.nseg; ++j) {
-      const float mj = rec0[j * RS + h];
-      if (mj == -INFINITY) continue;
-      const double w = exp((double)p.c * ((double)mj - (double)M));
-      L += (double)rec0[j * RS + G + h] * w;
-      Lf += rec0[j * RS + G + h] * expf(p.c * (mj - M));
-    }
-    sh_lse[h] = (double)p.c * (double)M + log(L);
-    sh_M[h] = M;
-    sh_L[h] = Lf;
-  }
-  __syncthreads();
-
-  if (do_out) {  // out = sum_j o_j exp(c (m_j - M)) / L
+  if (combine) {  // out = sum_j o_j exp(c (m_j - M)) / L
+    const int64_t ob = ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
     for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
       const int h = e / D;
+      const float M = sh_M[h];
       float acc = 0.f;
-      for (int j = 0; j < ui.nseg; ++j) {
+      int j = 0;
+      for (; j + 4 <= ui.nseg; j += 4) {  // four records in flight
+        float mv[4], ov[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          mv[q] = rec0[(j + q) * RS + h];
+          ov[q] = rec0[(j + q) * RS + 2 * G + e];
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (mv[q] != -INFINITY) acc += ov[q] * expf(p.c * (mv[q] - M));
+      }
+      for (; j < ui.nseg; ++j) {
         const float mj = rec0[j * RS + h];
-        if (mj == -INFINITY) continue;
-        acc += rec0[j * RS + 2 * G + e] * expf(p.c * (mj - sh_M[h]));
+        if (mj != -INFINITY) acc += rec0[j * RS + 2 * G + e] * expf(p.c * (mj - M));
       }
       const float val = ui.nseg > 0 && sh_L[h] > 0.f ? acc / sh_L[h] : 0.f;
-      const int64_t oi = ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D + e;
-      if (p.out_dtype == 0) static_cast<float *>(p.out)[oi] = val;
-      else static_cast<__nv_bfloat16 *>(p.out)[oi] = __float2bfloat16_rn(val);
+      if (p.out_dtype == 0) static_cast<float *>(p.out)[ob + e] = val;
+      else static_cast<__nv_bfloat16 *>(p.out)[ob + e] = __float2bfloat16_rn(val);
     }
+    return;
   }
-  if (chunk >= n_chunks) return;
 
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh_hist[i] = 0u;
   __syncthreads();
   const int t0 = chunk * kScoreChunk, t1 = min(ui.nC, t0 + kScoreChunk);
-  const float *lg = p.ws.logits + (size_t)u * p.t_cap * G;
-  float *sc = p.ws.scores + (size_t)u * p.t_cap;
+  const float *lg = p.ws.logits + (size_t)u * p.ustride * G;
+  float *sc = p.ws.scores + (size_t)u * p.ustride;
+  // approximate p_h = 2^(raw * a - b_h), a = c log2(e), b_h = LSE_h log2(e):
+  // the exponent rounds once in fp32 (|x| < 64: absolute error < 4e-6), so
+  // the score is within ~1e-5 relative -- only used to bin positions
+  const float a = (float)((double)p.c * kLog2e);
+  float bh[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) bh[h] = (float)(sh_lse[h] * kLog2e);
   for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
     float raw[G];
     if constexpr (G % 4 == 0) {
@@ -196,18 +242,15 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
 #pragma unroll
       for (int h = 0; h < G; ++h) raw[h] = __ldcs(lg + (size_t)t * G + h);
     }
-    // p_h = exp(c*raw - LSE_h): the argument in fp64, split hi + lo, so the
-    // only rounding left is expf's own
-    double acc = 0.0;
+    float pr[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const double x = (double)p.c * (double)raw[h] - sh_lse[h];
-      const float xh = (float)x;
-      const float xl = (float)(x - (double)xh);
-      const float e = expf(xh);
-      acc += (double)fmaf(e, xl, e);
-    }
-    const float s = acc >= 0.0 ? (float)acc : 0.f;  // NaN (bad inputs) ranks lowest
+    for (int h = 0; h < G; ++h) pr[h] = ex2_approx(fmaf(raw[h], a, -bh[h]));
+    // pairwise sum of the group's probabilities
+#pragma unroll
+    for (int w = 1; w < G; w <<= 1)
+#pragma unroll
+      for (int h = 0; h + w < G; h += 2 * w) pr[h] += pr[h + w];
+    const float s = pr[0] >= 0.f ? pr[0] : 0.f;  // NaN (bad inputs) ranks lowest
     sc[t] = s;
     atomicAdd(&sh_hist[__float_as_uint(s) >> kHistShift], 1u);
   }
@@ -226,6 +269,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   int above;
   const int bin = find_threshold_bin(sh_hist, kHistBins, p.k_global, &above, sh_warp, sh_res);
   if (threadIdx.x == 0) p.ws.thr[u] = make_int2(bin, above);
+  if (threadIdx.x < G) p.ws.lse[u * 8 + threadIdx.x] = sh_lse[threadIdx.x];
 }
 
 // ------------------------------------------------------------------ filter
@@ -235,140 +279,308 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
   const int nC = max(0, T - p.window);
   if (nC <= p.k_global || p.k_global == 0 || chunk * kScoreChunk >= nC) return;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
-  const int2 thr = p.ws.thr[u];
-  const uint32_t bin1 = (uint32_t)thr.x;
+  const int bin1 = p.ws.thr[u].x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t words = (p.t_cap + 31) / 32;
-  const float *sc = p.ws.scores + (size_t)u * p.t_cap;
-  uint32_t *sel = p.ws.sel + (size_t)u * words;
-  uint32_t *tie = p.ws.tie + (size_t)u * words;
-  uint2 *cand = p.ws.cand + (size_t)u * p.t_cap;
-  const int t0 = chunk * kScoreChunk, t1 = min(nC, t0 + kScoreChunk);
-  for (int base = t0 + 32 * warp; base < t1; base += 32 * (kScoreThreads / 32)) {
-    const int t = base + lane;
-    const bool valid = t < t1;
-    const uint32_t bits = valid ? __float_as_uint(__ldcs(sc + t)) : 0u;
-    const uint32_t bin = bits >> kHistShift;
-    const uint32_t above = __ballot_sync(0xffffffffu, valid && bin > bin1);
-    const uint32_t eq = __ballot_sync(0xffffffffu, valid && bin == bin1);
-    if (lane == 0) {
-      sel[base >> 5] = above;
-      tie[base >> 5] = 0u;
-    }
-    if (eq) {
-      uint32_t pos = 0;
-      if (lane == 0) pos = atomicAdd(p.ws.cand_count + u, (uint32_t)__popc(eq));
-      pos = __shfl_sync(0xffffffffu, pos, 0);
-      if (valid && bin == bin1) cand[pos + __popc(eq & ((1u << lane) - 1u))] = make_uint2(bits, (uint32_t)t);
-    }
+  const int sub = chunk * (kScoreChunk / kSubRange) + warp;  // this warp's sub-range
+  const int s0 = sub * kSubRange, s1 = min(nC, s0 + kSubRange);
+  if (s0 >= nC) return;
+  const float *sc = p.ws.scores + (size_t)u * p.ustride;
+  int32_t *above = p.ws.above + (size_t)u * p.ustride + s0;
+  uint2 *eqs = p.ws.cand + (size_t)u * p.ustride + s0;
+  // lane l of round r holds positions s0 + 128 r + 4 l .. +3 (one float4), so
+  // (round, lane, element) order is position order
+  constexpr int kRounds = kSubRange / 128;
+  float4 v[kRounds];
+#pragma unroll
+  for (int r = 0; r < kRounds; ++r) {
+    const int t = s0 + 128 * r + 4 * lane;
+    v[r] = t + 3 < s1 ? __ldcs(reinterpret_cast<const float4 *>(sc + t))
+                      : make_float4(t < s1 ? sc[t] : 0.f, t + 1 < s1 ? sc[t + 1] : 0.f,
+                                    t + 2 < s1 ? sc[t + 2] : 0.f, 0.f);
   }
+  int na = 0, ne = 0;
+#pragma unroll
+  for (int r = 0; r < kRounds; ++r) {
+    const int t = s0 + 128 * r + 4 * lane;
+    const float f[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+    int ca = 0, ce = 0;
+    uint32_t bits[4];
+    bool a[4], e[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      bits[k] = __float_as_uint(f[k]);
+      const int bin = (int)(bits[k] >> kHistShift);
+      const bool valid = t + k < s1;
+      a[k] = valid && bin >= bin1 + 2;                   // certainly above the k-th exact score
+      e[k] = valid && bin >= bin1 - 1 && bin <= bin1 + 1;  // guard band
+      ca += a[k];
+      ce += e[k];
+    }
+    // warp exclusive scans of the per-lane counts
+    int xa = ca, xe = ce;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ya = __shfl_up_sync(0xffffffffu, xa, o), ye = __shfl_up_sync(0xffffffffu, xe, o);
+      if (lane >= o) {
+        xa += ya;
+        xe += ye;
+      }
+    }
+    const int ta = __shfl_sync(0xffffffffu, xa, 31), te = __shfl_sync(0xffffffffu, xe, 31);
+    int oa = na + xa - ca, oe = ne + xe - ce;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (a[k]) above[oa++] = t + k;
+      if (e[k]) eqs[oe++] = make_uint2(bits[k], (uint32_t)(t + k));
+    }
+    na += ta;
+    ne += te;
+  }
+  if (lane == 0) p.ws.subcnt[(size_t)u * p.nsub + sub] = make_int2(na, ne);
 }
 
 // ------------------------------------------------------------------ final
+// Exact group score of one position: p_h = 2^(raw_h * a - b_h) with
+// a = c log2(e) and b_h = LSE_h log2(e) carried as float pairs, the exponent
+// formed with an exact product and a two-sum, so the only rounding of
+// consequence is the ex2 approximation (~2^-22 relative); pairwise sum.
+__device__ __forceinline__ float exact_score(const float *raw, int G, float c, const double *lse) {
+  const double ad = (double)c * kLog2e;
+  const float a_hi = (float)ad, a_lo = (float)(ad - (double)a_hi);
+  float pr[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    pr[h] = 0.f;
+    if (h >= G) continue;
+    const double bd = lse[h] * kLog2e;
+    const float b_hi = (float)bd, b_lo = (float)(bd - (double)b_hi);
+    const float x = __ldcg(raw + h);
+    const float ph = __fmul_rn(x, a_hi);
+    const float pl = fmaf(x, a_lo, fmaf(x, a_hi, -ph));  // x*a = ph + pl
+    const float sh = __fsub_rn(ph, b_hi);                // two-sum: sh + se = ph - b_hi exactly
+    const float z = __fsub_rn(sh, ph);
+    const float se = __fadd_rn(__fsub_rn(ph, __fsub_rn(sh, z)), __fsub_rn(-b_hi, z));
+    const float yl = (se + pl) - b_lo;
+    const float e = ex2_approx(sh);
+    pr[h] = fmaf(e, yl * 0.69314718055994531f, e);  // 2^(sh + yl) = 2^sh (1 + yl ln 2)
+  }
+#pragma unroll
+  for (int w = 1; w < 8; w <<= 1)
+#pragma unroll
+    for (int h = 0; h + w < 8; h += 2 * w) pr[h] += pr[h + w];
+  return pr[0] >= 0.f ? pr[0] : 0.f;  // NaN (bad inputs) ranks lowest
+}
+
+// Block-wide exclusive scan of two ints per thread at once.  sh needs 66 ints.
+__device__ __forceinline__ int2 block_exclusive_scan2(int2 x, int *sh, int2 *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  int ia = x.x, ie = x.y;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int ya = __shfl_up_sync(0xffffffffu, ia, o), ye = __shfl_up_sync(0xffffffffu, ie, o);
+    if (lane >= o) {
+      ia += ya;
+      ie += ye;
+    }
+  }
+  if (lane == 31) {
+    sh[warp] = ia;
+    sh[33 + warp] = ie;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int wa = lane < nw ? sh[lane] : 0, we = lane < nw ? sh[33 + lane] : 0;
+    int sa = wa, se = we;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ya = __shfl_up_sync(0xffffffffu, sa, o), ye = __shfl_up_sync(0xffffffffu, se, o);
+      if (lane >= o) {
+        sa += ya;
+        se += ye;
+      }
+    }
+    if (lane < nw) {
+      sh[lane] = sa - wa;
+      sh[33 + lane] = se - we;
+    }
+    if (lane == 31) {
+      sh[32] = sa;
+      sh[65] = se;
+    }
+  }
+  __syncthreads();
+  const int2 r = make_int2(sh[warp] + ia - x.x, sh[33 + warp] + ie - x.y);
+  *total = make_int2(sh[32], sh[65]);
+  __syncthreads();
+  return r;
+}
+
+// Exclusive offsets of the per-sub-range counts (above, in-bin) into shared
+// memory; off_x[nsub] holds the totals.
+__device__ void scan_subcounts(const int2 *cnt, int nsub, int *off_a, int *off_e, int *sh_scan) {
+  int carry_a = 0, carry_e = 0;
+  for (int base = 0; base < nsub; base += blockDim.x) {
+    const int s = base + threadIdx.x;
+    const int2 c = s < nsub ? __ldcg(cnt + s) : make_int2(0, 0);
+    int2 tot;
+    const int2 x = block_exclusive_scan2(c, sh_scan, &tot);
+    if (s < nsub) {
+      off_a[s] = carry_a + x.x;
+      off_e[s] = carry_e + x.y;
+    }
+    carry_a += tot.x;
+    carry_e += tot.y;
+  }
+  if (threadIdx.x == 0) {
+    off_a[nsub] = carry_a;
+    off_e[nsub] = carry_e;
+  }
+  __syncthreads();
+}
+
+// sub-range holding list element i (off ascending over [0, n], off[n] = total)
+__device__ __forceinline__ int find_sub(const int *off, int n, int i) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= i) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams p) {
+  extern __shared__ int fsm[];  // off_a[nsub+1], off_e[nsub+1], list_a[kMaxSelect], list_c[kMaxSelect],
+                                // then the in-bin list (bits, position) when it fits: list_e[kMaxSelect]
   __shared__ uint32_t sh_hist[2048];
-  __shared__ int sh_warp[32], sh_res[2], sh_tot;
+  __shared__ int sh_warp[66], sh_res[2], sh_ties;
   const int kvh = blockIdx.x, b = blockIdx.y;
   const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
   const int nC = max(0, T - p.window);
   const int L = p.window + p.k_global;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
   int32_t *idx = p.idx_out + (size_t)u * L;
-  const int64_t words = (p.t_cap + 31) / 32;
-  uint32_t *sel = p.ws.sel + (size_t)u * words;
-  uint32_t *tie = p.ws.tie + (size_t)u * words;
-  const bool all = nC <= p.k_global;
-  const bool none = !all && p.k_global == 0;  // window only
-  int need_eq = 0;
+  const bool select = nC > p.k_global && p.k_global > 0;
+  int *off_a = fsm, *off_e = fsm + p.nsub + 1;
+  int *list_a = fsm + 2 * (p.nsub + 1), *list_c = list_a + kMaxSelect;
+  uint2 *list_e = reinterpret_cast<uint2 *>(list_c + kMaxSelect);
 
-  if (!all && !none) {
-    const uint2 *cand = p.ws.cand + (size_t)u * p.t_cap;
-    const uint32_t cc = p.ws.cand_count[u];
-    const int n1 = cc < (uint32_t)nC ? (int)cc : nC;
-    const int2 thr = p.ws.thr[u];
-    int need = p.k_global - thr.y;  // >= 1
-    uint32_t prefix = (uint32_t)thr.x << kHistShift, mask = 0xFFFFFFFFu << kHistShift;
-    // two refinement rounds: bits 18..8 (2048 bins), then bits 7..0 (256 bins)
-    const int shifts[2] = {8, 0}, widths[2] = {11, 8};
-    for (int round = 0; round < 2; ++round) {
+  int n_sel = 0;  // selectable positions kept (all before the window)
+  if (select) {
+    const int nsub = (nC + kSubRange - 1) / kSubRange;
+    scan_subcounts(p.ws.subcnt + (size_t)u * p.nsub, nsub, off_a, off_e, sh_warp);
+    const int A = min(off_a[nsub], kMaxSelect), E = off_e[nsub];
+    const int32_t *above = p.ws.above + (size_t)u * p.ustride;
+    const uint2 *eqs_g = p.ws.cand + (size_t)u * p.ustride;
+    // the above-threshold positions (fewer than k_global), already in order,
+    // and the in-bin list when it fits, in one round of loads
+    const bool e_in_smem = E <= kMaxSelect;
+    for (int i = threadIdx.x; i < A; i += blockDim.x) {
+      const int s = find_sub(off_a, nsub, i);
+      list_a[i] = __ldcg(above + (size_t)s * kSubRange + (i - off_a[s]));
+    }
+    if (e_in_smem)
+      for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        const int s = find_sub(off_e, nsub, i);
+        list_e[i] = __ldcg(eqs_g + (size_t)s * kSubRange + (i - off_e[s]));
+      }
+    __syncthreads();
+    // exact scores of the guard band (replacing the approximate bits)
+    double lse[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.lse[u * 8 + h] : 0.0;
+    const float *lg = p.ws.logits + (size_t)u * p.ustride * p.G;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+      if (e_in_smem) {
+        list_e[i].x = __float_as_uint(exact_score(lg + (size_t)list_e[i].y * p.G, p.G, p.c, lse));
+      } else {
+        const int s = find_sub(off_e, nsub, i);
+        uint2 *ep = const_cast<uint2 *>(eqs_g) + (size_t)s * kSubRange + (i - off_e[s]);
+        ep->x = __float_as_uint(exact_score(lg + (size_t)__ldcg(&ep->y) * p.G, p.G, p.c, lse));
+      }
+    }
+    __threadfence_block();
+    __syncthreads();
+    auto in_bin = [&](int i) -> uint2 {  // i-th guard-band element in position order
+      if (e_in_smem) return list_e[i];
+      const int s = find_sub(off_e, nsub, i);
+      return __ldcg(eqs_g + (size_t)s * kSubRange + (i - off_e[s]));
+    };
+    // radix select of the need-th largest exact score: bits 31..21, 20..10, 9..0
+    int need = p.k_global - A;
+    uint32_t prefix = 0u, mask = 0u;
+    const int shifts[3] = {21, 10, 0}, widths[3] = {11, 11, 10};
+    for (int round = 0; round < 3; ++round) {
       const int sh = shifts[round], nb = 1 << widths[round];
       for (int i = threadIdx.x; i < nb; i += blockDim.x) sh_hist[i] = 0u;
       __syncthreads();
-      for (int i = threadIdx.x; i < n1; i += blockDim.x) {
-        const uint32_t bits = __ldcg(&cand[i].x);
+      for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        const uint32_t bits = in_bin(i).x;
         if ((bits & mask) == prefix) atomicAdd(&sh_hist[(bits >> sh) & (nb - 1)], 1u);
       }
       __syncthreads();
-      int above;
-      const int bin = find_threshold_bin(sh_hist, nb, need, &above, sh_warp, sh_res);
-      need -= above;
+      int ab;
+      const int bin = find_threshold_bin(sh_hist, nb, need, &ab, sh_warp, sh_res);
+      need -= ab;
       prefix |= (uint32_t)bin << sh;
       mask |= (uint32_t)(nb - 1) << sh;
-    }
-    need_eq = need;  // how many positions scoring exactly `prefix` are taken
-    const uint32_t kth = prefix;
-    for (int i = threadIdx.x; i < n1; i += blockDim.x) {
-      const uint2 cv = __ldcg(&cand[i]);
-      if (cv.x > kth) atomicOr(sel + (cv.y >> 5), 1u << (cv.y & 31));
-      else if (cv.x == kth) atomicOr(tie + (cv.y >> 5), 1u << (cv.y & 31));
+      if (round == 2 && threadIdx.x == 0) sh_ties = (int)sh_hist[bin];  // elements equal to the k-th score
     }
     __syncthreads();
-  }
-
-  // ordered compaction over the words of [0, T)
-  const int nw = (T + 31) / 32;
-  const int per = (nw + blockDim.x - 1) / blockDim.x;
-  const int w0 = min(nw, threadIdx.x * per), w1 = min(nw, w0 + per);
-  auto cmask = [&](int w) -> uint32_t {  // bits of selectable positions (< nC)
-    const int lo = w * 32;
-    if (lo + 32 <= nC) return 0xFFFFFFFFu;
-    if (lo >= nC) return 0u;
-    return (1u << (nC - lo)) - 1u;
-  };
-  auto tmask = [&](int w) -> uint32_t {  // bits of positions < T
-    const int lo = w * 32;
-    if (lo + 32 <= T) return 0xFFFFFFFFu;
-    return (1u << (T - lo)) - 1u;
-  };
-  int tie_before = 0;
-  if (!all && !none) {
-    int cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(__ldcg(tie + w) & cmask(w));
-    tie_before = block_exclusive_scan(cnt, sh_warp, &sh_tot);
-  }
-  auto word_sel = [&](int w, int &ties_seen) -> uint32_t {
-    const uint32_t cm = cmask(w), tm = tmask(w);
-    if (all) return tm;
-    if (none) return tm & ~cm;
-    uint32_t x = (__ldcg(sel + w) & cm) | (tm & ~cm);
-    uint32_t tw = __ldcg(tie + w) & cm;
-    while (tw) {
-      const uint32_t lowbit = tw & (0u - tw);
-      if (ties_seen < need_eq) x |= lowbit;
-      ++ties_seen;
-      tw ^= lowbit;
-    }
-    return x;
-  };
-  int cnt = 0;
-  {
-    int ts = tie_before;
-    for (int w = w0; w < w1; ++w) cnt += __popc(word_sel(w, ts));
-  }
-  const int out_before = block_exclusive_scan(cnt, sh_warp, &sh_tot);
-  const int n_total = sh_tot;
-  {
-    int ts = tie_before, o = out_before;
-    for (int w = w0; w < w1; ++w) {
-      uint32_t x = word_sel(w, ts);
-      while (x) {
-        const int bit = __ffs(x) - 1;
-        x &= x - 1;
-        if (o < L) idx[o] = (int32_t)slot_of(p, b, (int64_t)w * 32 + bit);
-        ++o;
+    const uint32_t kth = prefix;  // the exact k_global-th score; `need` of its ties are kept
+    const bool keep_all_ties = sh_ties <= need;
+    // walk the in-bin list in position order: keep scores above kth and the
+    // first `need` equal to it
+    int taken = 0, ties = 0;
+    for (int base = 0; base < E; base += blockDim.x) {
+      const int i = base + threadIdx.x;
+      const uint2 cv = i < E ? in_bin(i) : make_uint2(0u, 0u);
+      int take;
+      if (keep_all_ties) {
+        take = (i < E && cv.x >= kth) ? 1 : 0;
+      } else {
+        const int is_tie = (i < E && cv.x == kth) ? 1 : 0;
+        int tie_tot;
+        const int tie_rank = ties + block_exclusive_scan(is_tie, sh_warp, &tie_tot);
+        take = (i < E && (cv.x > kth || (is_tie && tie_rank < need))) ? 1 : 0;
+        ties += tie_tot;
       }
+      int take_tot;
+      const int pos = taken + block_exclusive_scan(take, sh_warp, &take_tot);
+      if (take && pos < kMaxSelect) list_c[pos] = (int)cv.y;
+      taken += take_tot;
     }
+    __syncthreads();
+    // merge two position-ordered lists: rank = own index + smaller elements of the other list
+    const int nc = min(taken, kMaxSelect);
+    n_sel = A + nc;
+    for (int i = threadIdx.x; i < A; i += blockDim.x) {
+      const int v = list_a[i];
+      int lo = 0, hi = nc;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (list_c[mid] < v) lo = mid + 1; else hi = mid;
+      }
+      if (i + lo < L) idx[i + lo] = (int32_t)slot_of(p, b, v);
+    }
+    for (int i = threadIdx.x; i < nc; i += blockDim.x) {
+      const int v = list_c[i];
+      int lo = 0, hi = A;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (list_a[mid] < v) lo = mid + 1; else hi = mid;
+      }
+      if (i + lo < L) idx[i + lo] = (int32_t)slot_of(p, b, v);
+    }
+  } else if (p.k_global > 0) {  // every selectable position is kept
+    n_sel = nC;
+    for (int t = threadIdx.x; t < nC && t < L; t += blockDim.x) idx[t] = (int32_t)slot_of(p, b, t);
   }
+  // the forced window follows every selectable position
+  for (int t = nC + threadIdx.x; t < T; t += blockDim.x) {
+    const int o = n_sel + (t - nC);
+    if (o < L) idx[o] = (int32_t)slot_of(p, b, t);
+  }
+  const int n_total = n_sel + (T - nC);
   for (int i = n_total + threadIdx.x; i < L; i += blockDim.x) idx[i] = -1;
 }
 
@@ -379,23 +591,28 @@ cudaError_t launch_score_g(const ScoreParams &p, dim3 grid, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+size_t final_smem_bytes(int nsub) { return (size_t)(2 * (nsub + 1) + 4 * kMaxSelect) * sizeof(int); }
+
 }  // namespace
 
 cudaError_t launch_select(const ScoreParams &p, cudaStream_t s) {
   const int chunks = (int)((p.t_cap + kScoreChunk - 1) / kScoreChunk);
-  const dim3 grid(max(chunks, 1), p.Hkv, p.B);
   cudaError_t e;
+  const dim3 sgrid(chunks + 1, p.Hkv, p.B);  // + the combine CTA of each unit
   switch (p.G) {
-    case 1: e = launch_score_g<1>(p, grid, s); break;
-    case 2: e = launch_score_g<2>(p, grid, s); break;
-    case 4: e = launch_score_g<4>(p, grid, s); break;
-    case 8: e = launch_score_g<8>(p, grid, s); break;
+    case 1: e = launch_score_g<1>(p, sgrid, s); break;
+    case 2: e = launch_score_g<2>(p, sgrid, s); break;
+    case 4: e = launch_score_g<4>(p, sgrid, s); break;
+    case 8: e = launch_score_g<8>(p, sgrid, s); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
-  filter_kernel<<<grid, kScoreThreads, 0, s>>>(p);
+  filter_kernel<<<dim3(chunks, p.Hkv, p.B), kScoreThreads, 0, s>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  final_kernel<<<dim3(p.Hkv, p.B), kFinalThreads, 0, s>>>(p);
+  const size_t smem = final_smem_bytes(p.nsub);
+  e = cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  final_kernel<<<dim3(p.Hkv, p.B), kFinalThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -29,8 +29,11 @@ struct SCfg {
   static constexpr int KVB = 16 * ROWB;        // 16 rows of K (or V)
   static constexpr int WARP_BYTES = 2 * KVB + (FP8 ? 2 * 16 * 4 : 0);
   static constexpr int WSTRIDE = 16 + 8 * D;   // warp scratch floats
-  static size_t bytes(int nw, int G) {
-    return 128 + (size_t)nw * WARP_BYTES + (size_t)nw * WSTRIDE * 4 + (size_t)G * (D + 2) * 4;
+  // one CTA's partial record m[G], l[G], o[G][D], padded to whole float4s
+  __host__ __device__ static int rec_floats(int G) { return (G * (D + 2) + 3) & ~3; }
+  static size_t bytes(int nw, int G, int S) {
+    return 128 + (size_t)nw * WARP_BYTES + (size_t)nw * WSTRIDE * 4 + (size_t)(1 + S) * rec_floats(G) * 4 +
+           (size_t)S * 8 * 4 * 2;
   }
 };
 
@@ -40,9 +43,14 @@ __global__ void __launch_bounds__(512, 1) sparse_mma_kernel(const SparseParams p
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float *scratch = reinterpret_cast<float *>(smem + (size_t)nw * C::WARP_BYTES);
-  float *partial = scratch + (size_t)nw * C::WSTRIDE;  // m[G], l[G], o[G][D]
   cg::cluster_group cluster = cg::this_cluster();
+  const int S = (int)cluster.num_blocks();
+  const int RSP = C::rec_floats(p.G);
+  float *scratch = reinterpret_cast<float *>(smem + (size_t)nw * C::WARP_BYTES);
+  float *partial = scratch + (size_t)nw * C::WSTRIDE;  // m[G], l[G], o[G][D] of this CTA
+  float *gathered = partial + RSP;                     // CTA 0: every CTA's partial
+  float *wts = gathered + (size_t)S * RSP;             // CTA 0: weight of (CTA, head)
+  float *inv_l = wts + S * 8;                          // CTA 0: 1 / normaliser per head
   const int rank = (int)cluster.block_rank();
   const int kvh = blockIdx.y, b = blockIdx.z, G = p.G;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
@@ -97,27 +105,36 @@ __global__ void __launch_bounds__(512, 1) sparse_mma_kernel(const SparseParams p
   merge_warp_states<D>(scratch, C::WSTRIDE, nw, G, p.c, partial, threadIdx.x, blockDim.x);
   cluster.sync();
   if (rank == 0) {
-    const int S = (int)cluster.num_blocks();
+    // one parallel copy of every CTA's partial into local shared memory
+    const int n4 = S * (RSP >> 2);
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+      const int r = i / (RSP >> 2), o = i - r * (RSP >> 2);
+      reinterpret_cast<float4 *>(gathered)[i] = reinterpret_cast<const float4 *>(cluster.map_shared_rank(partial, r))[o];
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+      const int h = threadIdx.x;
+      float M = -INFINITY;
+      for (int r = 0; r < S; ++r) M = fmaxf(M, gathered[r * RSP + h]);
+      float L = 0.f;
+      for (int r = 0; r < S; ++r) {
+        const float mr = gathered[r * RSP + h];
+        const float w = mr == -INFINITY ? 0.f : expf(p.c * (mr - M));
+        wts[r * 8 + h] = w;
+        L += w * gathered[r * RSP + G + h];
+      }
+      inv_l[h] = L > 0.f ? 1.f / L : 0.f;
+    }
+    __syncthreads();
+    const int64_t ob = ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
     for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
       const int h = e / D;
-      float M = -INFINITY;
-      for (int r = 0; r < S; ++r) M = fmaxf(M, cluster.map_shared_rank(partial, r)[h]);
-      float L = 0.f, acc = 0.f;
-      if (M != -INFINITY) {
-        for (int r = 0; r < S; ++r) {
-          const float *pr = cluster.map_shared_rank(partial, r);
-          if (pr[h] == -INFINITY) continue;
-          const float w = expf(p.c * (pr[h] - M));
-          L += w * pr[G + h];
-          acc += w * pr[2 * G + e];
-        }
-      }
-      const float val = L > 0.f ? acc / L : 0.f;
-      const int64_t oi = ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D + e;
-      static_cast<__nv_bfloat16 *>(p.out)[oi] = __float2bfloat16_rn(val);
+      float acc = 0.f;
+      for (int r = 0; r < S; ++r) acc += wts[r * 8 + h] * gathered[r * RSP + 2 * G + e];
+      static_cast<__nv_bfloat16 *>(p.out)[ob + e] = __float2bfloat16_rn(acc * inv_l[h]);
     }
   }
-  cluster.sync();  // keep every CTA's shared memory alive until CTA 0 is done
+  cluster.sync();  // keep every CTA's shared memory alive until CTA 0 has read it
 }
 
 // ------------------------------------------------------------ fp32 caches
@@ -173,7 +190,7 @@ template <int D, bool FP8>
 cudaError_t launch_mma_t(const SparseParams &p, int64_t num_slots, cudaStream_t s) {
   using C = SCfg<D, FP8>;
   const int nw = p.rows_per_cta / 16;
-  const size_t smem = C::bytes(nw, p.G);
+  const size_t smem = C::bytes(nw, p.G, p.splits);
   auto kern = sparse_mma_kernel<D, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

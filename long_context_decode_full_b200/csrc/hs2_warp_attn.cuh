@@ -275,16 +275,32 @@ __device__ __forceinline__ void merge_warp_states(const float *scr, int wstride,
     rec[h] = M;
     rec[G + h] = L;
   }
-  for (int e = tid; e < G * D; e += nthreads) {
-    const int h = e / D;
+  // thread -> (dim, first head); each head's warp weights computed once per thread
+  const int dim = tid % D, h0 = tid / D, hstep = nthreads / D;
+  if (hstep == 0) {  // fewer threads than head dims
+    for (int e = tid; e < G * D; e += nthreads) {
+      const int h = e / D;
+      float M = -INFINITY;
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, scr[w * wstride + h]);
+      float acc = 0.f;
+      for (int w = 0; w < NW; ++w) {
+        const float mw = scr[w * wstride + h];
+        if (mw != -INFINITY) acc += expf(c * (mw - M)) * scr[w * wstride + 16 + e];
+      }
+      rec[2 * G + e] = acc;
+    }
+    return;
+  }
+  if (h0 >= hstep * ((G + hstep - 1) / hstep)) return;
+  for (int h = h0; h < G; h += hstep) {
     float M = -INFINITY;
     for (int w = 0; w < NW; ++w) M = fmaxf(M, scr[w * wstride + h]);
     float acc = 0.f;
     for (int w = 0; w < NW; ++w) {
       const float mw = scr[w * wstride + h];
-      if (mw != -INFINITY) acc += expf(c * (mw - M)) * scr[w * wstride + 16 + e];
+      if (mw != -INFINITY) acc += expf(c * (mw - M)) * scr[w * wstride + 16 + h * D + dim];
     }
-    rec[2 * G + e] = acc;
+    rec[2 * G + h * D + dim] = acc;
   }
 }
 
