@@ -360,14 +360,13 @@ int hs2_sparse_attn(const hs2_heads *q_l, const hs2_cache *k_cache, const hs2_ca
   p.L = idx_stride;
   p.c = 1.0f / sqrtf((float)p.D);
   // enough CTAs per unit to cover the SMs, at most 16 per cluster and 256 rows per CTA
-  // fewest CTAs per unit that keep a CTA at <= 256 rows (16 warps): fatter
-  // CTAs measured faster than more, smaller ones at the pages' 1152 rows
-  int want = 1;
+  // 4 CTAs per unit (a 4-CTA cluster) measured best at the pages' 1152 rows
+  // for 16 and 32 units; rows per CTA in whole 64-row rounds (16 rows per
+  // warp per round)
+  int want = 4;
   if (const char *env = getenv("HS2_SPARSE_SPLITS")) want = atoi(env);  // tuning override
   int S = want < 1 ? 1 : (want > 16 ? 16 : want);
-  const int min_s = (idx_stride + 255) / 256;
-  if (S < min_s) S = min_s;
-  int rows = ((idx_stride + S - 1) / S + 15) / 16 * 16;
+  int rows = ((idx_stride + S - 1) / S + 63) / 64 * 64;
   S = (idx_stride + rows - 1) / rows;
   p.rows_per_cta = rows;
   p.splits = S;
@@ -416,6 +415,14 @@ __global__ void __launch_bounds__(512) copy_kernel(uint4 *__restrict__ dst, cons
 }
 
 int set_last_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char *env = getenv("HS2_PDL");
+    return !(env && env[0] == '0');
+  }();
+  return on;
+}
 
 cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int grid, cudaStream_t s) {
   if (bytes == 0) return cudaSuccess;

@@ -17,7 +17,8 @@ namespace hs2 {
 // ---------------------------------------------------------------- constants
 constexpr int kHistBins = 4096;          // score histogram: float bits 30..19
 constexpr int kHistShift = 19;
-constexpr int kScoreChunk = 4096;        // positions per score / filter CTA
+constexpr int kScoreChunk = 4096;        // positions per score CTA
+constexpr int kFilterChunk = 4096;       // positions per filter CTA (8 warps x 512)
 constexpr int kScoreThreads = 256;
 constexpr int kFinalThreads = 512;
 constexpr long long kSpinLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
@@ -195,6 +196,15 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // 16-byte chunk c of row r lives at chunk c ^ (r & 7).
 __device__ __forceinline__ uint32_t swz(uint32_t panel, int row, int chunk) {
   return panel + row * 128 + (((chunk ^ row) & 7) << 4);
+}
+
+// ---------------------------------------------------------------- PDL
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may be scheduled before its predecessor finishes; it must
+// wait before touching anything an earlier kernel produces or consumes.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // 2^x by the MUFU approximation (flushes subnormal results to zero)

@@ -130,11 +130,13 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
     mbar_init(cbar, (uint32_t)NCW);
     fence_mbar_init();
   }
+  if (producer && lane == 0) {
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+  }
+  griddep_wait();               // inputs and workspace are free from here on
+  griddep_launch_dependents();  // the score kernel may be scheduled as SMs free up
   if (producer) {
-    if (lane == 0) {
-      prefetch_tensormap(&tmk);
-      prefetch_tensormap(&tmv);
-    }
     compute_prefix(p, prefix, C::TILE);
   } else {
     zero_counters(p, threadIdx.x, NCW * 32);
@@ -314,7 +316,8 @@ __global__ void __launch_bounds__(32 * kF32Warps) full_attn_f32_kernel(const Ful
   float *Qs = Vs + kF32Tile * (D + 1);    // [8][D]
   int32_t *prefix = reinterpret_cast<int32_t *>(Qs + 8 * D);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nthr = blockDim.x;
-
+  griddep_wait();
+  griddep_launch_dependents();
   if (warp == 0) compute_prefix(p, prefix, kF32Tile);
   zero_counters(p, threadIdx.x, nthr);
   __syncthreads();
@@ -423,8 +426,7 @@ cudaError_t launch_mma_t(const FullParams &p, const CUtensorMap &tmk, const CUte
   auto kern = full_attn_mma_kernel<D, FP8, NCW, NSTAGE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, 32 * (NCW + 1), smem, s>>>(tmk, tmv, p);
-  return cudaGetLastError();
+  return launch_ex(kern, dim3(grid), dim3(32 * (NCW + 1)), smem, s, 0, tmk, tmv, p);
 }
 
 }  // namespace
@@ -456,15 +458,13 @@ cudaError_t launch_full_f32(const FullParams &p, int grid, cudaStream_t s) {
   if (p.D == 64) {
     e = cudaFuncSetAttribute(full_attn_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    full_attn_f32_kernel<64><<<grid, 32 * kF32Warps, smem, s>>>(p);
+    return launch_ex(full_attn_f32_kernel<64>, dim3(grid), dim3(32 * kF32Warps), smem, s, 0, p);
   } else if (p.D == 128) {
     e = cudaFuncSetAttribute(full_attn_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    full_attn_f32_kernel<128><<<grid, 32 * kF32Warps, smem, s>>>(p);
-  } else {
-    return cudaErrorInvalidValue;
+    return launch_ex(full_attn_f32_kernel<128>, dim3(grid), dim3(32 * kF32Warps), smem, s, 0, p);
   }
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace hs2

@@ -66,6 +66,36 @@ struct FullMmaConfig {
   int nstage;  // pipeline stages
 };
 
+// Launch with programmatic stream serialization (unless HS2_PDL=0) and an
+// optional 1-D cluster.
+bool pdl_enabled();
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster_x,
+                      Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // ---- launchers (return cudaError_t of the launch) -------------------------
 cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, bool fp8,
                             const FullMmaConfig &cfg, int grid, cudaStream_t s);

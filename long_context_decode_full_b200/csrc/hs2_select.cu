@@ -177,6 +177,8 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   __shared__ float sh_M[G], sh_L[G];
   __shared__ int sh_warp[33], sh_res[2], sh_last;
   constexpr int RS = G * (D + 2);
+  griddep_wait();
+  griddep_launch_dependents();
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const bool combine = chunk == (int)gridDim.x - 1;  // the unit's combine CTA
   const UnitInfo ui = unit_info(p, b, kvh);
@@ -227,24 +229,38 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   float bh[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) bh[h] = (float)(sh_lse[h] * kLog2e);
-  for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
-    float raw[G];
-    if constexpr (G % 4 == 0) {
+  constexpr int kUnroll = 2;  // positions per thread in flight
+  for (int t00 = t0 + threadIdx.x; t00 < t1; t00 += kUnroll * blockDim.x) {
+    float raw[kUnroll][G];
 #pragma unroll
-      for (int h4 = 0; h4 < G / 4; ++h4) {
-        const float4 v4 = __ldcs(reinterpret_cast<const float4 *>(lg + (size_t)t * G) + h4);
-        raw[4 * h4] = v4.x;
-        raw[4 * h4 + 1] = v4.y;
-        raw[4 * h4 + 2] = v4.z;
-        raw[4 * h4 + 3] = v4.w;
+    for (int q = 0; q < kUnroll; ++q) {
+      const int t = t00 + q * blockDim.x;
+      if (t >= t1) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) raw[q][h] = 0.f;
+        continue;
       }
-    } else {
+      if constexpr (G % 4 == 0) {
 #pragma unroll
-      for (int h = 0; h < G; ++h) raw[h] = __ldcs(lg + (size_t)t * G + h);
+        for (int h4 = 0; h4 < G / 4; ++h4) {
+          const float4 v4 = __ldcs(reinterpret_cast<const float4 *>(lg + (size_t)t * G) + h4);
+          raw[q][4 * h4] = v4.x;
+          raw[q][4 * h4 + 1] = v4.y;
+          raw[q][4 * h4 + 2] = v4.z;
+          raw[q][4 * h4 + 3] = v4.w;
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < G; ++h) raw[q][h] = __ldcs(lg + (size_t)t * G + h);
+      }
     }
+#pragma unroll
+    for (int q = 0; q < kUnroll; ++q) {
+    const int t = t00 + q * blockDim.x;
+    if (t >= t1) break;
     float pr[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) pr[h] = ex2_approx(fmaf(raw[h], a, -bh[h]));
+    for (int h = 0; h < G; ++h) pr[h] = ex2_approx(fmaf(raw[q][h], a, -bh[h]));
     // pairwise sum of the group's probabilities
 #pragma unroll
     for (int w = 1; w < G; w <<= 1)
@@ -253,6 +269,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
     const float s = pr[0] >= 0.f ? pr[0] : 0.f;  // NaN (bad inputs) ranks lowest
     sc[t] = s;
     atomicAdd(&sh_hist[__float_as_uint(s) >> kHistShift], 1u);
+    }
   }
   __syncthreads();
   uint32_t *gh = p.ws.hist + (size_t)u * kHistBins;
@@ -272,18 +289,54 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   if (threadIdx.x < G) p.ws.lse[u * 8 + threadIdx.x] = sh_lse[threadIdx.x];
 }
 
+// Exact group score of one position: p_h = 2^(raw_h * a - b_h) with
+// a = c log2(e) and b_h = LSE_h log2(e) carried as float pairs, the exponent
+// formed with an exact product and a two-sum, so the only rounding of
+// consequence is the ex2 approximation (~2^-22 relative); pairwise sum.
+__device__ __forceinline__ float exact_score(const float *raw, int G, float c, const double *lse) {
+  const double ad = (double)c * kLog2e;
+  const float a_hi = (float)ad, a_lo = (float)(ad - (double)a_hi);
+  float pr[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    pr[h] = 0.f;
+    if (h >= G) continue;
+    const double bd = lse[h] * kLog2e;
+    const float b_hi = (float)bd, b_lo = (float)(bd - (double)b_hi);
+    const float x = __ldcg(raw + h);
+    const float ph = __fmul_rn(x, a_hi);
+    const float pl = fmaf(x, a_lo, fmaf(x, a_hi, -ph));  // x*a = ph + pl
+    const float sh = __fsub_rn(ph, b_hi);                // two-sum: sh + se = ph - b_hi exactly
+    const float z = __fsub_rn(sh, ph);
+    const float se = __fadd_rn(__fsub_rn(ph, __fsub_rn(sh, z)), __fsub_rn(-b_hi, z));
+    const float yl = (se + pl) - b_lo;
+    const float e = ex2_approx(sh);
+    pr[h] = fmaf(e, yl * 0.69314718055994531f, e);  // 2^(sh + yl) = 2^sh (1 + yl ln 2)
+  }
+#pragma unroll
+  for (int w = 1; w < 8; w <<= 1)
+#pragma unroll
+    for (int h = 0; h + w < 8; h += 2 * w) pr[h] += pr[h + w];
+  return pr[0] >= 0.f ? pr[0] : 0.f;  // NaN (bad inputs) ranks lowest
+}
+
 // ------------------------------------------------------------------ filter
 __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
   const int nC = max(0, T - p.window);
-  if (nC <= p.k_global || p.k_global == 0 || chunk * kScoreChunk >= nC) return;
+  if (nC <= p.k_global || p.k_global == 0 || chunk * kFilterChunk >= nC) return;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
   const int bin1 = p.ws.thr[u].x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = chunk * (kScoreChunk / kSubRange) + warp;  // this warp's sub-range
+  const int sub = chunk * (kFilterChunk / kSubRange) + warp;  // this warp's sub-range
   const int s0 = sub * kSubRange, s1 = min(nC, s0 + kSubRange);
   if (s0 >= nC) return;
+  double lse[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.lse[u * 8 + h] : 0.0;
   const float *sc = p.ws.scores + (size_t)u * p.ustride;
   int32_t *above = p.ws.above + (size_t)u * p.ustride + s0;
   uint2 *eqs = p.ws.cand + (size_t)u * p.ustride + s0;
@@ -336,41 +389,17 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
     na += ta;
     ne += te;
   }
+  // guard band: the exact score replaces the approximate one (the whole warp
+  // works through this list's entries, all loads in flight together)
+  __syncwarp();
+  for (int i = lane; i < ne; i += 32) {
+    const uint32_t pos = eqs[i].y;
+    eqs[i].x = __float_as_uint(exact_score(p.ws.logits + ((size_t)u * p.ustride + pos) * p.G, p.G, p.c, lse));
+  }
   if (lane == 0) p.ws.subcnt[(size_t)u * p.nsub + sub] = make_int2(na, ne);
 }
 
 // ------------------------------------------------------------------ final
-// Exact group score of one position: p_h = 2^(raw_h * a - b_h) with
-// a = c log2(e) and b_h = LSE_h log2(e) carried as float pairs, the exponent
-// formed with an exact product and a two-sum, so the only rounding of
-// consequence is the ex2 approximation (~2^-22 relative); pairwise sum.
-__device__ __forceinline__ float exact_score(const float *raw, int G, float c, const double *lse) {
-  const double ad = (double)c * kLog2e;
-  const float a_hi = (float)ad, a_lo = (float)(ad - (double)a_hi);
-  float pr[8];
-#pragma unroll
-  for (int h = 0; h < 8; ++h) {
-    pr[h] = 0.f;
-    if (h >= G) continue;
-    const double bd = lse[h] * kLog2e;
-    const float b_hi = (float)bd, b_lo = (float)(bd - (double)b_hi);
-    const float x = __ldcg(raw + h);
-    const float ph = __fmul_rn(x, a_hi);
-    const float pl = fmaf(x, a_lo, fmaf(x, a_hi, -ph));  // x*a = ph + pl
-    const float sh = __fsub_rn(ph, b_hi);                // two-sum: sh + se = ph - b_hi exactly
-    const float z = __fsub_rn(sh, ph);
-    const float se = __fadd_rn(__fsub_rn(ph, __fsub_rn(sh, z)), __fsub_rn(-b_hi, z));
-    const float yl = (se + pl) - b_lo;
-    const float e = ex2_approx(sh);
-    pr[h] = fmaf(e, yl * 0.69314718055994531f, e);  // 2^(sh + yl) = 2^sh (1 + yl ln 2)
-  }
-#pragma unroll
-  for (int w = 1; w < 8; w <<= 1)
-#pragma unroll
-    for (int h = 0; h + w < 8; h += 2 * w) pr[h] += pr[h + w];
-  return pr[0] >= 0.f ? pr[0] : 0.f;  // NaN (bad inputs) ranks lowest
-}
-
 // Block-wide exclusive scan of two ints per thread at once.  sh needs 66 ints.
 __device__ __forceinline__ int2 block_exclusive_scan2(int2 x, int *sh, int2 *total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
@@ -453,6 +482,8 @@ __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams 
                                 // then the in-bin list (bits, position) when it fits: list_e[kMaxSelect]
   __shared__ uint32_t sh_hist[2048];
   __shared__ int sh_warp[66], sh_res[2], sh_ties;
+  griddep_wait();
+  griddep_launch_dependents();
   const int kvh = blockIdx.x, b = blockIdx.y;
   const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
   const int nC = max(0, T - p.window);
@@ -483,22 +514,6 @@ __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams 
         const int s = find_sub(off_e, nsub, i);
         list_e[i] = __ldcg(eqs_g + (size_t)s * kSubRange + (i - off_e[s]));
       }
-    __syncthreads();
-    // exact scores of the guard band (replacing the approximate bits)
-    double lse[8];
-#pragma unroll
-    for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.lse[u * 8 + h] : 0.0;
-    const float *lg = p.ws.logits + (size_t)u * p.ustride * p.G;
-    for (int i = threadIdx.x; i < E; i += blockDim.x) {
-      if (e_in_smem) {
-        list_e[i].x = __float_as_uint(exact_score(lg + (size_t)list_e[i].y * p.G, p.G, p.c, lse));
-      } else {
-        const int s = find_sub(off_e, nsub, i);
-        uint2 *ep = const_cast<uint2 *>(eqs_g) + (size_t)s * kSubRange + (i - off_e[s]);
-        ep->x = __float_as_uint(exact_score(lg + (size_t)__ldcg(&ep->y) * p.G, p.G, p.c, lse));
-      }
-    }
-    __threadfence_block();
     __syncthreads();
     auto in_bin = [&](int i) -> uint2 {  // i-th guard-band element in position order
       if (e_in_smem) return list_e[i];
@@ -586,9 +601,8 @@ __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams 
 
 template <int G>
 cudaError_t launch_score_g(const ScoreParams &p, dim3 grid, cudaStream_t s) {
-  if (p.D == 64) score_kernel<G, 64><<<grid, kScoreThreads, 0, s>>>(p);
-  else score_kernel<G, 128><<<grid, kScoreThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  if (p.D == 64) return launch_ex(score_kernel<G, 64>, grid, dim3(kScoreThreads), 0, s, 0, p);
+  return launch_ex(score_kernel<G, 128>, grid, dim3(kScoreThreads), 0, s, 0, p);
 }
 
 size_t final_smem_bytes(int nsub) { return (size_t)(2 * (nsub + 1) + 4 * kMaxSelect) * sizeof(int); }
@@ -607,13 +621,13 @@ cudaError_t launch_select(const ScoreParams &p, cudaStream_t s) {
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
-  filter_kernel<<<dim3(chunks, p.Hkv, p.B), kScoreThreads, 0, s>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int fchunks = (int)((p.t_cap + kFilterChunk - 1) / kFilterChunk);
+  e = launch_ex(filter_kernel, dim3(fchunks, p.Hkv, p.B), dim3(kScoreThreads), 0, s, 0, p);
+  if (e != cudaSuccess) return e;
   const size_t smem = final_smem_bytes(p.nsub);
   e = cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  final_kernel<<<dim3(p.Hkv, p.B), kFinalThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_ex(final_kernel, dim3(p.Hkv, p.B), dim3(kFinalThreads), smem, s, 0, p);
 }
 
 }  // namespace hs2

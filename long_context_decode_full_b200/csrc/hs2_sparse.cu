@@ -21,88 +21,133 @@ namespace hs2 {
 
 namespace {
 
+constexpr int kSparseWarps = 4;
+
 template <int D, bool FP8>
 struct SCfg {
   static constexpr int ES = FP8 ? 1 : 2;
   static constexpr int ROWB = D * ES;
   static constexpr int PANEL = 16 * 128;
-  static constexpr int KVB = 16 * ROWB;        // 16 rows of K (or V)
-  static constexpr int WARP_BYTES = 2 * KVB + (FP8 ? 2 * 16 * 4 : 0);
-  static constexpr int WSTRIDE = 16 + 8 * D;   // warp scratch floats
+  static constexpr int KVB = 16 * ROWB;                             // 16 rows of K (or V)
+  static constexpr int BUF_BYTES = 2 * KVB + (FP8 ? 2 * 16 * 4 : 0);  // one 16-row group
+  static constexpr int WARP_BYTES = 2 * BUF_BYTES;                  // double buffer
+  static constexpr int WSTRIDE = 16 + 8 * D;                        // warp scratch floats
   // one CTA's partial record m[G], l[G], o[G][D], padded to whole float4s
   __host__ __device__ static int rec_floats(int G) { return (G * (D + 2) + 3) & ~3; }
-  static size_t bytes(int nw, int G, int S) {
-    return 128 + (size_t)nw * WARP_BYTES + (size_t)nw * WSTRIDE * 4 + (size_t)(1 + S) * rec_floats(G) * 4 +
-           (size_t)S * 8 * 4 * 2;
+  // CTA 0 gathers the cluster's partials into the (then idle) staging buffers
+  // when they fit, else into a region of their own
+  __host__ __device__ static bool gather_in_staging(int G, int S) {
+    return (size_t)S * rec_floats(G) * 4 <= (size_t)kSparseWarps * WARP_BYTES;
+  }
+  static size_t bytes(int G, int S, int rows) {
+    return 128 + (size_t)kSparseWarps * WARP_BYTES + (size_t)kSparseWarps * WSTRIDE * 4 + (size_t)rec_floats(G) * 4 +
+           (size_t)(S + 1) * 8 * 4 + (size_t)rows * 4 +
+           (gather_in_staging(G, S) ? 0 : (size_t)S * rec_floats(G) * 4);
   }
 };
 
+// Grid (splits, Hkv, B), cluster (splits, 1, 1), 4 warps.  CTA `rank` of a
+// unit's cluster owns rows [rank * rows_per_cta, ...) of the index list; its
+// warps take 16-row groups round-robin, gathering the next group while the
+// current one is on the tensor cores.
 template <int D, bool FP8>
-__global__ void __launch_bounds__(512, 1) sparse_mma_kernel(const SparseParams p, int64_t num_slots) {
+__global__ void __launch_bounds__(32 * kSparseWarps) sparse_mma_kernel(const SparseParams p, int64_t num_slots) {
   using C = SCfg<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   cg::cluster_group cluster = cg::this_cluster();
   const int S = (int)cluster.num_blocks();
   const int RSP = C::rec_floats(p.G);
-  float *scratch = reinterpret_cast<float *>(smem + (size_t)nw * C::WARP_BYTES);
-  float *partial = scratch + (size_t)nw * C::WSTRIDE;  // m[G], l[G], o[G][D] of this CTA
-  float *gathered = partial + RSP;                     // CTA 0: every CTA's partial
-  float *wts = gathered + (size_t)S * RSP;             // CTA 0: weight of (CTA, head)
-  float *inv_l = wts + S * 8;                          // CTA 0: 1 / normaliser per head
+  float *scratch = reinterpret_cast<float *>(smem + (size_t)kSparseWarps * C::WARP_BYTES);
+  float *partial = scratch + (size_t)kSparseWarps * C::WSTRIDE;  // m[G], l[G], o[G][D] of this CTA
+  float *wts = partial + RSP;                                    // CTA 0: weight of (CTA, head)
+  float *inv_l = wts + S * 8;                                    // CTA 0: 1 / normaliser per head
+  int *slots = reinterpret_cast<int *>(inv_l + 8);               // this CTA's index entries
+  float *gathered = C::gather_in_staging(p.G, S) ? reinterpret_cast<float *>(smem)
+                                                     : reinterpret_cast<float *>(slots + p.rows_per_cta);
   const int rank = (int)cluster.block_rank();
   const int kvh = blockIdx.y, b = blockIdx.z, G = p.G;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
+  const int row_lo = rank * p.rows_per_cta, nrows = max(0, min(p.L, row_lo + p.rows_per_cta) - row_lo);
+  griddep_wait();  // the index list and the query come from earlier kernels
+  griddep_launch_dependents();
 
-  // ---- gather this warp's 16 rows
-  uint8_t *wb = smem + (size_t)warp * C::WARP_BYTES;
-  const uint32_t kp = smem_u32(wb), vp = kp + C::KVB;
-  float *ks = reinterpret_cast<float *>(wb + 2 * C::KVB), *vs = ks + 16;
-  const int r0 = rank * p.rows_per_cta + 16 * warp;
-  int slot = -1;
-  if (lane < 16 && r0 + lane < p.L) {
-    const int s = __ldg(p.idx + u * p.L + r0 + lane);
-    if (s >= 0 && s < num_slots) slot = s;
+  // the CTA's slice of the index list, validated (entries outside the cache are skipped)
+  for (int r = threadIdx.x; r < nrows; r += blockDim.x) {
+    const int sl = __ldg(p.idx + u * p.L + row_lo + r);
+    slots[r] = (sl >= 0 && sl < num_slots) ? sl : -1;
   }
-  const uint32_t vmask = __ballot_sync(0xffffffffu, slot >= 0) & 0xFFFFu;
-  if constexpr (FP8) {
-    if (lane < 16) {
-      ks[lane] = slot >= 0 ? __ldg(p.k_scale + (int64_t)slot * p.Hkv + kvh) : 0.f;
-      vs[lane] = slot >= 0 ? __ldg(p.v_scale + (int64_t)slot * p.Hkv + kvh) : 0.f;
-    }
-  }
-  constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
-  const uint8_t *kg = static_cast<const uint8_t *>(p.k), *vg = static_cast<const uint8_t *>(p.v);
-#pragma unroll 4
-  for (int e = lane; e < 16 * CPR; e += 32) {
-    const int row = e / CPR, ch = e % CPR;
-    const int s = __shfl_sync(0xffffffffu, slot, row);
-    const uint32_t off = (ch >> 3) * C::PANEL;
-    const uint32_t dk = swz(kp + off, row, ch & 7), dv = swz(vp + off, row, ch & 7);
-    if (s >= 0) {
-      const int64_t src = ((int64_t)s * p.Hkv + kvh) * C::ROWB + ch * 16;
-      cp_async_16(dk, kg + src);
-      cp_async_16(dv, vg + src);
-    } else {
-      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dk), "r"(0u) : "memory");
-      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dv), "r"(0u) : "memory");
-    }
-  }
-  cp_async_commit();
-
   WarpAttn<D, FP8> st;
   st.reset();
   st.load_q(static_cast<const __nv_bfloat16 *>(p.q) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D, G);
-  cp_async_wait_all();
-  __syncwarp();
-  if (vmask) st.step(kp, vp, C::PANEL, 0, vmask, p.c, nullptr, G, ks, vs);
+  __syncthreads();
+
+  constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
+  const uint8_t *kg = static_cast<const uint8_t *>(p.k), *vg = static_cast<const uint8_t *>(p.v);
+  uint8_t *wbase = smem + (size_t)warp * C::WARP_BYTES;
+  // issue the loads of 16-row group `grp` into buffer `buf`; returns its row mask
+  auto gather = [&](int grp, int buf) -> uint32_t {
+    uint8_t *wb = wbase + buf * C::BUF_BYTES;
+    const uint32_t kp = smem_u32(wb), vp = kp + C::KVB;
+    const int r = 16 * grp + (lane & 15);
+    const int slot = r < nrows ? slots[r] : -1;
+    const uint32_t vm = __ballot_sync(0xffffffffu, slot >= 0) & 0xFFFFu;
+    if constexpr (FP8) {
+      float *ks = reinterpret_cast<float *>(wb + 2 * C::KVB);
+      if (lane < 16) {
+        if (slot >= 0) {
+          cp_async_4(smem_u32(ks + lane), p.k_scale + (int64_t)slot * p.Hkv + kvh);
+          cp_async_4(smem_u32(ks + 16 + lane), p.v_scale + (int64_t)slot * p.Hkv + kvh);
+        } else {
+          ks[lane] = 0.f;
+          ks[16 + lane] = 0.f;
+        }
+      }
+    }
+#pragma unroll 4
+    for (int e = lane; e < 16 * CPR; e += 32) {
+      const int row = e / CPR, ch = e % CPR;
+      const int sr = __shfl_sync(0xffffffffu, slot, row);
+      const uint32_t off = (ch >> 3) * C::PANEL;
+      const uint32_t dk = swz(kp + off, row, ch & 7), dv = swz(vp + off, row, ch & 7);
+      if (sr >= 0) {
+        const int64_t src = ((int64_t)sr * p.Hkv + kvh) * C::ROWB + ch * 16;
+        cp_async_16(dk, kg + src);
+        cp_async_16(dv, vg + src);
+      } else {
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dk), "r"(0u) : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dv), "r"(0u) : "memory");
+      }
+    }
+    cp_async_commit();
+    return vm;
+  };
+
+  const int ngroups = (nrows + 15) / 16;
+  uint32_t vm[2] = {0u, 0u};
+  if (warp < ngroups) vm[0] = gather(warp, 0);
+  for (int k = 0, grp = warp; grp < ngroups; ++k, grp += kSparseWarps) {
+    const bool more = grp + kSparseWarps < ngroups;
+    if (more) {
+      vm[(k + 1) & 1] = gather(grp + kSparseWarps, (k + 1) & 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      cp_async_wait_all();
+    }
+    __syncwarp();
+    uint8_t *wb = wbase + (k & 1) * C::BUF_BYTES;
+    const uint32_t kp = smem_u32(wb);
+    const float *ks = reinterpret_cast<const float *>(wb + 2 * C::KVB);
+    if (vm[k & 1]) st.step(kp, kp + C::KVB, C::PANEL, 0, vm[k & 1], p.c, nullptr, G, ks, ks + 16);
+    __syncwarp();  // the buffer is refilled two groups later
+  }
 
   // ---- merge the warps of this CTA, then the CTAs of the cluster
   float *scr = scratch + warp * C::WSTRIDE;
   st.store(scr, scr + 8, scr + 16);
   __syncthreads();
-  merge_warp_states<D>(scratch, C::WSTRIDE, nw, G, p.c, partial, threadIdx.x, blockDim.x);
+  merge_warp_states<D>(scratch, C::WSTRIDE, kSparseWarps, G, p.c, partial, threadIdx.x, blockDim.x);
   cluster.sync();
   if (rank == 0) {
     // one parallel copy of every CTA's partial into local shared memory
@@ -143,6 +188,8 @@ __global__ void sparse_f32_kernel(const SparseParams p, int64_t num_slots) {
   extern __shared__ float qs[];  // [G][D]
   const int kvh = blockIdx.x, b = blockIdx.y, G = p.G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_wait();
+  griddep_launch_dependents();
   const float *q = static_cast<const float *>(p.q) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
   for (int e = threadIdx.x; e < G * D; e += blockDim.x) qs[e] = q[e];
   __syncthreads();
@@ -189,8 +236,7 @@ __global__ void sparse_f32_kernel(const SparseParams p, int64_t num_slots) {
 template <int D, bool FP8>
 cudaError_t launch_mma_t(const SparseParams &p, int64_t num_slots, cudaStream_t s) {
   using C = SCfg<D, FP8>;
-  const int nw = p.rows_per_cta / 16;
-  const size_t smem = C::bytes(nw, p.G, p.splits);
+  const size_t smem = C::bytes(p.G, p.splits, p.rows_per_cta);
   auto kern = sparse_mma_kernel<D, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -198,19 +244,7 @@ cudaError_t launch_mma_t(const SparseParams &p, int64_t num_slots, cudaStream_t 
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.splits, p.Hkv, p.B);
-  cfg.blockDim = dim3(32 * nw);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.splits;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p, num_slots);
+  return launch_ex(kern, dim3(p.splits, p.Hkv, p.B), dim3(32 * kSparseWarps), smem, s, p.splits, p, num_slots);
 }
 
 }  // namespace
@@ -218,9 +252,8 @@ cudaError_t launch_mma_t(const SparseParams &p, int64_t num_slots, cudaStream_t 
 cudaError_t launch_sparse_impl(const SparseParams &p, int kv_dtype, int64_t num_slots, cudaStream_t s) {
   if (kv_dtype == 0) {
     const size_t smem = (size_t)p.G * p.D * 4;
-    if (p.D == 64) sparse_f32_kernel<64><<<dim3(p.Hkv, p.B), 32 * p.G, smem, s>>>(p, num_slots);
-    else sparse_f32_kernel<128><<<dim3(p.Hkv, p.B), 32 * p.G, smem, s>>>(p, num_slots);
-    return cudaGetLastError();
+    if (p.D == 64) return launch_ex(sparse_f32_kernel<64>, dim3(p.Hkv, p.B), dim3(32 * p.G), smem, s, 0, p, num_slots);
+    return launch_ex(sparse_f32_kernel<128>, dim3(p.Hkv, p.B), dim3(32 * p.G), smem, s, 0, p, num_slots);
   }
   if (kv_dtype == 1) return p.D == 64 ? launch_mma_t<64, false>(p, num_slots, s) : launch_mma_t<128, false>(p, num_slots, s);
   if (kv_dtype == 2 && p.D == 128) return launch_mma_t<128, true>(p, num_slots, s);
