@@ -178,6 +178,10 @@ def run_gpu(args, rank, world, local):
     spec = synth.WORKLOADS[args.workload]
     if args.seq_len:
         spec = spec.replace(seq_len=args.seq_len)
+    if args.kv_heads:
+        spec = spec.replace(num_kv_heads=args.kv_heads)
+    if args.batch:
+        spec = spec.replace(batch=args.batch)
     w = synth.generate(spec, seed=args.seed + rank, device="cuda")
     s = spec
     dev = torch.device("cuda", local)
@@ -348,6 +352,8 @@ def main():
     ap.add_argument("--cpu-units", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's context (profiling runs)")
+    ap.add_argument("--kv-heads", type=int, default=0, help="override the workload's KV heads (experiments)")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (experiments)")
     args = ap.parse_args()
     if args.impl == "reference":
         args.warmup = max(0, min(args.warmup, 1))

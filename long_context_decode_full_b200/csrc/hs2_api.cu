@@ -185,17 +185,28 @@ int check_caches(const hs2_cache *k, const hs2_cache *v) {
   return HS2_OK;
 }
 
+// Consumer warps and pipeline stages of the attention kernel, most preferred
+// first: enough warps for two per SM sub-partition and enough stages that the
+// bytes in flight per SM cover the loaded HBM latency.  A tile (16 positions
+// per consumer warp) must fit the page size (one divides the other).
 FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged) {
-  // 8 consumer warps (128-position tiles) keep two warps per SM sub-partition
-  FullMmaConfig c = fp8 ? FullMmaConfig{8, 4} : FullMmaConfig{8, 3};
-  (void)D;
-  if (const char *env = getenv("HS2_FULL_CFG")) {
+  static const FullMmaConfig bf16_128[] = {{8, 3}, {4, 6}};
+  static const FullMmaConfig bf16_64[] = {{8, 6}, {4, 6}};
+  static const FullMmaConfig e4m3[] = {{12, 4}, {8, 6}, {4, 8}};
+  const FullMmaConfig *list = fp8 ? e4m3 : (D == 64 ? bf16_64 : bf16_128);
+  const int n = fp8 ? 3 : 2;
+  if (const char *env = getenv("HS2_FULL_CFG")) {  // tuning override
     int a = 0, b = 0;
-    if (sscanf(env, "%d,%d", &a, &b) == 2) c = FullMmaConfig{a, b};
+    if (sscanf(env, "%d,%d", &a, &b) == 2) {
+      const int tile = 16 * a;
+      if (!paged || page_size % tile == 0 || tile % page_size == 0) return FullMmaConfig{a, b};
+    }
   }
-  const int tile = 16 * c.ncw;
-  if (paged && !(page_size % tile == 0 || tile % page_size == 0)) c = FullMmaConfig{4, 4};
-  return c;
+  for (int i = 0; i < n; ++i) {
+    const int tile = 16 * list[i].ncw;
+    if (!paged || page_size % tile == 0 || tile % page_size == 0) return list[i];
+  }
+  return list[n - 1];
 }
 
 }  // namespace

@@ -59,6 +59,9 @@ struct Partition {
   __device__ __forceinline__ int64_t start(int64_t c) const { return c * total / N; }
   // the CTA that owns tile x
   __device__ __forceinline__ int64_t cfirst(int64_t x) const { return ((x + 1) * N - 1) / total; }
+  // whether CTA c owns any tile (with more CTAs than tiles some own none,
+  // and their record slots are never written)
+  __device__ __forceinline__ bool owns_tiles(int64_t c) const { return start(c + 1) > start(c); }
 };
 
 // ---------------------------------------------------------------- misc
@@ -124,6 +127,11 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
+// orders this thread's generic-proxy shared-memory accesses before later
+// async-proxy (TMA) accesses to the same memory
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -181,10 +189,15 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
 }
-// two E4M3 codes (low byte first) -> two f16 (exact)
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes16) {
-  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes16 & 0xFFFFu), __NV_E4M3);
-  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// four E4M3 codes (bytes 0..3 of w) -> two f16x2 (exact): lo = bytes 0,1,
+// hi = bytes 2,3, the lower byte of each pair in the lower half
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  asm("{\n\t.reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;

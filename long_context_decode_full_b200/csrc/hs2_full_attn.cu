@@ -35,16 +35,16 @@ struct Cfg {
   static constexpr int NPANEL = ROWB / 128;
   static constexpr int PANEL = TILE * 128;
   static constexpr int KVB = TILE * ROWB;
-  static constexpr int SCB = FP8 ? 2 * TILE * 4 : 0;
-  static constexpr int STAGE = 2 * KVB;
+  static constexpr int SCB = FP8 ? 2 * TILE * 4 : 0;                // K and V scales of a tile
+  static constexpr int STAGE = (2 * KVB + SCB + 1023) / 1024 * 1024;  // K, V, scales; 1 KB aligned for TMA
   static constexpr int WSTRIDE = 16 + 8 * D;
-  static constexpr size_t OFF_SC = (size_t)NSTAGE * STAGE;
-  static constexpr size_t OFF_SCR = OFF_SC + (size_t)NSTAGE * SCB;
-  static constexpr size_t OFF_BAR = OFF_SCR + (size_t)NCW * WSTRIDE * 4;
+  static constexpr size_t OFF_BAR = (size_t)NSTAGE * STAGE;
   static constexpr size_t OFF_META = OFF_BAR + (2 * NSTAGE + 1) * 8;
   static constexpr size_t OFF_PREFIX = OFF_META + NSTAGE * sizeof(StageMeta);
   static size_t bytes(int B) { return OFF_PREFIX + (size_t)(B + 1) * 4 + 1024; }
   static_assert(ROWB % 128 == 0, "rows are whole 128-byte panels");
+  // the warps merge a segment's states inside the stage they last read
+  static_assert((size_t)NCW * WSTRIDE * 4 <= (size_t)STAGE, "merge scratch must fit in one stage");
 };
 
 __device__ __forceinline__ int64_t slot_of(const int32_t *pt, int max_pages, int ps, int b, int64_t pos) {
@@ -111,8 +111,6 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  float *scales = reinterpret_cast<float *>(smem + C::OFF_SC);
-  float *scratch = reinterpret_cast<float *>(smem + C::OFF_SCR);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
   uint64_t *empty = full + NSTAGE;
   uint64_t *cbar = empty + NSTAGE;  // consumer-warp rendezvous at segment ends
@@ -197,7 +195,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
       const int p0 = i * C::TILE;
       const int cl0 = (int)(box0 - cache_base);  // cache lane of this tile's first box
       if constexpr (FP8) {
-        float *ks = scales + stage * (2 * C::TILE);
+        float *ks = reinterpret_cast<float *>(smem + (size_t)stage * C::STAGE + 2 * C::KVB);
 #pragma unroll
         for (int k = 0; k < C::TILE / 32; ++k) {
           const int rr = lane + 32 * k;
@@ -279,13 +277,17 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
     const int nvalid = max(0, min(16, mt.T - pos0));
     const uint32_t vmask = nvalid >= 16 ? 0xFFFFu : ((1u << nvalid) - 1u);
     const uint32_t kp = sbase + stage * C::STAGE;
-    const float *ks = scales + stage * (2 * C::TILE) + 16 * warp;
+    const float *ks = reinterpret_cast<const float *>(smem + (size_t)stage * C::STAGE + 2 * C::KVB) + 16 * warp;
     if (nvalid > 0)
       st.step(kp, kp + C::KVB, C::PANEL, 16 * warp, vmask, p.c, p.ws.logits + (u * p.ustride + pos0) * p.G, p.G, ks,
               ks + C::TILE);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
     if (mt.flags & kLast) {
+      // segment end: merge the warps' states inside this stage, then release it
+      if (!consumer_sync(cbar, cphase)) {  // every warp is done reading the tile
+        set_error(p.ws.err, kErrFullWait);
+        break;
+      }
+      float *scratch = reinterpret_cast<float *>(smem + (size_t)stage * C::STAGE);
       float *scr = scratch + warp * C::WSTRIDE;
       st.store(scr, scr + 8, scr + 16);
       if (!consumer_sync(cbar, cphase)) {
@@ -295,12 +297,15 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
       if (mt.rec >= 0)
         merge_warp_states<D>(scratch, C::WSTRIDE, NCW, p.G, p.c, p.ws.records + (size_t)mt.rec * p.G * (D + 2),
                              threadIdx.x, NCW * 32);
+      fence_proxy_async_smem();  // before TMA refills the stage
       if (!consumer_sync(cbar, cphase)) {
         set_error(p.ws.err, kErrFullWait);
         break;
       }
       st.reset();
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
   }
 }
 
@@ -436,15 +441,13 @@ cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const C
 #define HS2_FULL_CASE(D_, F_, W_, S_)                                                   \
   if (p.D == D_ && fp8 == F_ && cfg.ncw == W_ && cfg.nstage == S_)                      \
     return launch_mma_t<D_, F_, W_, S_>(p, tmk, tmv, grid, s);
-  HS2_FULL_CASE(128, false, 4, 4)
-  HS2_FULL_CASE(128, false, 4, 3)
-  HS2_FULL_CASE(128, false, 8, 2)
   HS2_FULL_CASE(128, false, 8, 3)
-  HS2_FULL_CASE(64, false, 4, 4)
-  HS2_FULL_CASE(64, false, 8, 3)
-  HS2_FULL_CASE(128, true, 4, 4)
-  HS2_FULL_CASE(128, true, 8, 3)
-  HS2_FULL_CASE(128, true, 8, 4)
+  HS2_FULL_CASE(128, false, 4, 6)
+  HS2_FULL_CASE(64, false, 8, 6)
+  HS2_FULL_CASE(64, false, 4, 6)
+  HS2_FULL_CASE(128, true, 12, 4)
+  HS2_FULL_CASE(128, true, 8, 6)
+  HS2_FULL_CASE(128, true, 4, 8)
 #undef HS2_FULL_CASE
   return cudaErrorInvalidConfiguration;
 }

@@ -37,9 +37,13 @@ constexpr double kLog2e = 1.4426950408889634074;
 
 struct UnitInfo {
   int T, nC, nb;
-  int64_t U;  // first linear tile of the unit
+  int64_t U;   // first linear tile of the unit
+  int64_t c0;  // CTA owning the unit's first tile: record j was written by CTA c0 + j
   int nseg;
   bool select;  // nC > k_global > 0
+  Partition part;
+  // record j holds a segment (its CTA owned tiles)
+  __device__ __forceinline__ bool rec_ok(int j) const { return part.owns_tiles(c0 + j); }
 };
 
 __device__ __forceinline__ UnitInfo unit_info(const ScoreParams &p, int b, int kvh) {
@@ -51,9 +55,11 @@ __device__ __forceinline__ UnitInfo unit_info(const ScoreParams &p, int b, int k
   const int64_t total = (int64_t)p.Hkv * p.ws.prefix[p.B];
   ui.U = (int64_t)p.Hkv * p.ws.prefix[b] + (int64_t)kvh * ui.nb;
   ui.nseg = 0;
+  ui.c0 = 0;
+  ui.part = Partition{total > 0 ? total : 1, p.N};
   if (ui.nb > 0 && total > 0) {
-    const Partition part{total, p.N};
-    ui.nseg = (int)(part.cfirst(ui.U + ui.nb - 1) - part.cfirst(ui.U) + 1);
+    ui.c0 = ui.part.cfirst(ui.U);
+    ui.nseg = (int)(ui.part.cfirst(ui.U + ui.nb - 1) - ui.c0 + 1);
     if (ui.nseg > p.R) ui.nseg = p.R;
   }
   return ui;
@@ -136,12 +142,14 @@ __device__ int find_threshold_bin(const uint32_t *hist, int nbins, int need, int
 // records, as a block-wide reduction: thread t folds the pairs (segment j,
 // head h) with h = t % G.
 template <int G, int D>
-__device__ void unit_lse(const float *rec0, int nseg, float c, double *sh_lse, float *sh_M, float *sh_L,
+__device__ void unit_lse(const float *rec0, const UnitInfo &ui, float c, double *sh_lse, float *sh_M, float *sh_L,
                          double *sh_red) {
   constexpr int RS = G * (D + 2);
+  const int nseg = ui.nseg;
   const int tid = threadIdx.x, nt = blockDim.x, h = tid % G;
   float m = -INFINITY;
-  for (int i = tid; i < nseg * G; i += nt) m = fmaxf(m, rec0[(i / G) * RS + h]);
+  for (int i = tid; i < nseg * G; i += nt)
+    if (ui.rec_ok(i / G)) m = fmaxf(m, rec0[(i / G) * RS + h]);
   reinterpret_cast<float *>(sh_red)[tid] = m;
   __syncthreads();
   if (tid < G) {
@@ -154,6 +162,7 @@ __device__ void unit_lse(const float *rec0, int nseg, float c, double *sh_lse, f
   double L = 0.0;
   for (int i = tid; i < nseg * G; i += nt) {
     const int j = i / G;
+    if (!ui.rec_ok(j)) continue;
     const float mj = rec0[j * RS + h];
     if (mj != -INFINITY) L += (double)rec0[j * RS + G + h] * exp((double)c * ((double)mj - (double)M));
   }
@@ -186,7 +195,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   if (!combine && chunk >= n_chunks) return;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
   const float *rec0 = p.ws.records + (size_t)u * p.R * RS;
-  unit_lse<G, D>(rec0, ui.nseg, p.c, sh_lse, sh_M, sh_L, sh_red);
+  unit_lse<G, D>(rec0, ui, p.c, sh_lse, sh_M, sh_L, sh_red);
 
   if (combine) {  // out = sum_j o_j exp(c (m_j - M)) / L
     const int64_t ob = ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
@@ -204,9 +213,10 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          if (mv[q] != -INFINITY) acc += ov[q] * expf(p.c * (mv[q] - M));
+          if (ui.rec_ok(j + q) && mv[q] != -INFINITY) acc += ov[q] * expf(p.c * (mv[q] - M));
       }
       for (; j < ui.nseg; ++j) {
+        if (!ui.rec_ok(j)) continue;
         const float mj = rec0[j * RS + h];
         if (mj != -INFINITY) acc += rec0[j * RS + 2 * G + e] * expf(p.c * (mj - M));
       }

@@ -119,8 +119,9 @@ struct WarpAttn {
         lds128(w1, swz(kp, row, 2 * t + 1));
 #pragma unroll
         for (int kk = 0; kk < KS; ++kk) {
-          const uint32_t w = kk < 4 ? w0[kk & 3] : w1[kk & 3];
-          mma_f16(s[j], qa[kk][0], 0u, qa[kk][1], 0u, e4m3x2_to_f16x2(w), e4m3x2_to_f16x2(w >> 16));
+          uint32_t b0, b1;
+          e4m3x4_to_f16x2x2(kk < 4 ? w0[kk & 3] : w1[kk & 3], b0, b1);
+          mma_f16(s[j], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
         }
       }
     }
@@ -148,10 +149,13 @@ struct WarpAttn {
     const float m_new = fmaxf(m, mx);
     float alpha = 1.f, p[4] = {0.f, 0.f, 0.f, 0.f};
     if (m_new != -INFINITY) {
-      alpha = expf(c * (m - m_new));
+      // exp(c (x - m)) as 2^((x - m) c log2 e): the difference first, so the
+      // dominant terms (x near m) carry no rounding of m into l
+      const float cl = c * 1.44269504088896341f;
+      alpha = ex2_approx((m - m_new) * cl);
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        if (ok[i]) p[i] = expf(c * (x[i] - m_new));
+        if (ok[i]) p[i] = ex2_approx((x[i] - m_new) * cl);
     }
     l = l * alpha + ((p[0] + p[1]) + (p[2] + p[3]));
     m = m_new;
@@ -168,8 +172,8 @@ struct WarpAttn {
       smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 1));
       smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 2));
       const float sig_new = fmaxf(sig, smax);
-      beta = sig_new > 0.f ? sig / sig_new : 1.f;
-      const float inv = sig_new > 0.f ? 1.f / sig_new : 0.f;
+      const float inv = sig_new > 0.f ? __frcp_rn(sig_new) : 0.f;
+      beta = sig_new > 0.f ? sig * inv : 1.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) pv[i] = p[i] * (sv[i] * inv);
       sig = sig_new;
@@ -228,8 +232,10 @@ struct WarpAttn {
           x01 &= b01;
           x23 &= b23;
         }
-        mma_f16(o[mt], e4m3x2_to_f16x2(x01), e4m3x2_to_f16x2(x01 >> 16), e4m3x2_to_f16x2(x23),
-                e4m3x2_to_f16x2(x23 >> 16), pb0, pb1);
+        uint32_t a0, a1, a2, a3;
+        e4m3x4_to_f16x2x2(x01, a0, a1);
+        e4m3x4_to_f16x2x2(x23, a2, a3);
+        mma_f16(o[mt], a0, a1, a2, a3, pb0, pb1);
       }
     }
   }

@@ -24,9 +24,24 @@ def to_device(w: synth.Workload, device="cuda") -> synth.Workload:
                           mv(w.seq_lens), mv(w.page_table), w.page_size, w.needle_pos)
 
 
+def garbage_workspace(w: synth.Workload, seed=0):
+    """A workspace full of random bytes: every result must be independent of
+    what an earlier call left behind."""
+    from long_context_decode_full_b200 import hs2
+    s = w.spec
+    n = hs2.full_workspace_bytes(s.batch, s.num_kv_heads, s.group, s.head_dim, w.t_cap)
+    g = torch.Generator(device=w.k.device)
+    g.manual_seed(seed)
+    ws = torch.randint(0, 256, (n,), dtype=torch.uint8, device=w.k.device, generator=g)
+    ws[:256] = 0  # the sticky error flag starts clear
+    return ws
+
+
 def run_gpu(w: synth.Workload, q=None, window=None, k_global=None, workspace=None):
     from long_context_decode_full_b200 import hs2
     s = w.spec
+    if workspace is None:
+        workspace = garbage_workspace(w)
     return hs2.full_attn_select(w.q_full if q is None else q, w.k, w.v, w.seq_lens, w.page_table, w.page_size,
                                 s.window if window is None else window, s.k_global if k_global is None else k_global,
                                 w.k_scale, w.v_scale, workspace=workspace)

@@ -36,7 +36,7 @@ def inverse_slots(w, b):
 def test_full_size_workload(oracle, name):
     spec = synth.WORKLOADS[name]
     w = synth.generate(spec, seed=0, device="cuda")
-    ws = hs2.alloc_workspace(spec.batch, spec.num_kv_heads, spec.group, spec.head_dim, w.t_cap)
+    ws = U.garbage_workspace(w)
     outs, idx = hs2.hybrid_block_step(w.q_full, list(w.q_sparse), w.k, w.v, w.seq_lens, w.page_table, w.page_size,
                                       spec.window, spec.k_global, w.k_scale, w.v_scale, workspace=ws)
     torch.cuda.synchronize()
