@@ -93,7 +93,7 @@ Layout layout(int B, int Hkv, int G, int D, int64_t t_cap_in) {
   const size_t U = (size_t)B * Hkv;
   const int64_t t_cap = unit_stride(t_cap_in);  // per-unit arrays keep 16-byte aligned rows
   L.nsub = (int)((t_cap + kSubRange - 1) / kSubRange);
-  L.R = sm_count() * kMaxCtasPerSm / Hkv + 2;
+  L.R = sm_count() * kMaxCtasPerSm / Hkv + 2;  // <= 1024 for up to 255 SMs
   size_t o = 0;
   L.err = o;
   o += 256;
@@ -371,16 +371,32 @@ int hs2_sparse_attn(const hs2_heads *q_l, const hs2_cache *k_cache, const hs2_ca
   p.L = idx_stride;
   p.c = 1.0f / sqrtf((float)p.D);
   // enough CTAs per unit to cover the SMs, at most 16 per cluster and 256 rows per CTA
-  // 4 CTAs per unit (a 4-CTA cluster) measured best at the pages' 1152 rows
-  // for 16 and 32 units; rows per CTA in whole 64-row rounds (16 rows per
-  // warp per round)
-  int want = 4;
-  if (const char *env = getenv("HS2_SPARSE_SPLITS")) want = atoi(env);  // tuning override
-  int S = want < 1 ? 1 : (want > 16 ? 16 : want);
-  int rows = ((idx_stride + S - 1) / S + 63) / 64 * 64;
-  S = (idx_stride + rows - 1) / rows;
+  // 8 warps per CTA take 16-row groups, each warp gathering up to `nbuf`
+  // groups at once: rows per CTA = 128 * nbuf.  One buffer per warp (a
+  // 9-CTA cluster at the pages' 1152 rows) unless that needs more than one
+  // CTA per SM (a CTA holds an SM's registers), then two, then four.
+  const int units = p.B * p.Hkv, sms = sm_count();
+  // a warp's gather buffers: 16 rows of K and V (+ scales); at most 192 KB per CTA
+  const int buf_bytes = 2 * 16 * p.D * (k_cache->dtype == HS2_E4M3 ? 1 : 2) + (k_cache->dtype == HS2_E4M3 ? 128 : 0);
+  int max_nbuf = (192 * 1024) / (8 * buf_bytes);
+  max_nbuf = max_nbuf < 1 ? 1 : (max_nbuf > 4 ? 4 : max_nbuf);
+  // two buffers per warp at least (one gather in flight while the other is
+  // consumed), more while the CTAs would not fit in one wave
+  int nbuf = max_nbuf < 2 ? max_nbuf : 2;
+  while (nbuf < max_nbuf && (units * ((idx_stride + 128 * nbuf - 1) / (128 * nbuf)) > sms ||
+                             (idx_stride + 128 * nbuf - 1) / (128 * nbuf) > 16))
+    ++nbuf;
+  if (const char *env = getenv("HS2_SPARSE_NBUF")) nbuf = atoi(env);  // tuning override
+  nbuf = nbuf < 1 ? 1 : (nbuf > max_nbuf ? max_nbuf : nbuf);
+  int rows = 128 * nbuf;
+  int S = (idx_stride + rows - 1) / rows;
+  while (S > 16) {  // larger lists: more rows per CTA, never more than 16 per cluster
+    rows += 128;
+    S = (idx_stride + rows - 1) / rows;
+  }
   p.rows_per_cta = rows;
   p.splits = S;
+  p.nbuf = nbuf;
   cudaError_t e = launch_sparse_impl(p, k_cache->dtype, k_cache->num_slots, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "sparse-attention launch");
   return HS2_OK;

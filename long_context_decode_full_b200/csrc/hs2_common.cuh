@@ -24,6 +24,7 @@ constexpr int kFinalThreads = 512;
 constexpr long long kSpinLimitCycles = 4000000000LL;  // ~2 s at 2 GHz
 constexpr int kMaxBatchSmem = 4096;      // sequences whose tile prefix fits in smem
 constexpr int kSubRange = 512;           // positions per filter-warp list
+constexpr float kBandMargin = 4e-4f;     // relative margin of the selection guard band
 constexpr int kMaxSelect = 4096;         // window + k_global upper bound
 constexpr int64_t kMaxContext = int64_t(1) << 23;  // positions per sequence
 

@@ -57,6 +57,7 @@ struct SparseParams {
   int32_t L;                 // idx_stride
   int32_t rows_per_cta;      // multiple of 16
   int32_t splits;            // CTAs per unit (cluster size)
+  int32_t nbuf;              // 16-row gather buffers per warp (1..4)
   float c;
 };
 

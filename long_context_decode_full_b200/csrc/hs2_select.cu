@@ -17,10 +17,11 @@
 //             largest approximate score.  The combine CTA merges the records
 //             into the attention output.
 //   filter -- each warp owns 512 consecutive positions and writes, in
-//             position order, the positions whose approximate bin is >= b+2
-//             (certainly above the k-th exact score: a bin is 4.4% wide) and
-//             the positions in bins b-1 .. b+1 (the guard band that holds
-//             every position the exact k-th score can hinge on).
+//             position order, the positions whose approximate score is above
+//             bin b widened by a 4e-4 margin (certainly above the k-th exact
+//             score) and, with exact scores, the positions inside that widened
+//             bin (the guard band that holds every position the exact k-th
+//             score can hinge on).
 //   final  -- one CTA per unit: exact scores of the guard-band positions
 //             (exponent formed in float-float, so only ex2's own rounding is
 //             left), radix select of the exact k-th score among them, ties to
@@ -35,6 +36,8 @@ namespace {
 
 constexpr double kLog2e = 1.4426950408889634074;
 
+constexpr int kMaxRecords = 1024;  // >= records per unit (4 * SMs / Hkv + 2)
+
 struct UnitInfo {
   int T, nC, nb;
   int64_t U;   // first linear tile of the unit
@@ -42,9 +45,16 @@ struct UnitInfo {
   int nseg;
   bool select;  // nC > k_global > 0
   Partition part;
-  // record j holds a segment (its CTA owned tiles)
-  __device__ __forceinline__ bool rec_ok(int j) const { return part.owns_tiles(c0 + j); }
+  const uint8_t *ok;  // shared: ok[j] = record j holds a segment (its CTA owned tiles)
+  __device__ __forceinline__ bool rec_ok(int j) const { return ok[j] != 0; }
 };
+
+// Marks which of the unit's record slots were written (whole block).
+__device__ __forceinline__ void mark_records(UnitInfo &ui, uint8_t *sh_ok) {
+  for (int j = threadIdx.x; j < ui.nseg; j += blockDim.x) sh_ok[j] = ui.part.owns_tiles(ui.c0 + j) ? 1 : 0;
+  ui.ok = sh_ok;
+  __syncthreads();
+}
 
 __device__ __forceinline__ UnitInfo unit_info(const ScoreParams &p, int b, int kvh) {
   UnitInfo ui;
@@ -61,7 +71,9 @@ __device__ __forceinline__ UnitInfo unit_info(const ScoreParams &p, int b, int k
     ui.c0 = ui.part.cfirst(ui.U);
     ui.nseg = (int)(ui.part.cfirst(ui.U + ui.nb - 1) - ui.c0 + 1);
     if (ui.nseg > p.R) ui.nseg = p.R;
+    if (ui.nseg > kMaxRecords) ui.nseg = kMaxRecords;
   }
+  ui.ok = nullptr;
   return ui;
 }
 
@@ -185,14 +197,16 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   __shared__ double sh_lse[G];
   __shared__ float sh_M[G], sh_L[G];
   __shared__ int sh_warp[33], sh_res[2], sh_last;
+  __shared__ uint8_t sh_ok[kMaxRecords];
   constexpr int RS = G * (D + 2);
   griddep_wait();
   griddep_launch_dependents();
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const bool combine = chunk == (int)gridDim.x - 1;  // the unit's combine CTA
-  const UnitInfo ui = unit_info(p, b, kvh);
+  UnitInfo ui = unit_info(p, b, kvh);
   const int n_chunks = ui.select ? (ui.nC + kScoreChunk - 1) / kScoreChunk : 0;
   if (!combine && chunk >= n_chunks) return;
+  mark_records(ui, sh_ok);
   const int64_t u = (int64_t)b * p.Hkv + kvh;
   const float *rec0 = p.ws.records + (size_t)u * p.R * RS;
   unit_lse<G, D>(rec0, ui, p.c, sh_lse, sh_M, sh_L, sh_red);
@@ -239,7 +253,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   float bh[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) bh[h] = (float)(sh_lse[h] * kLog2e);
-  constexpr int kUnroll = 2;  // positions per thread in flight
+  constexpr int kUnroll = 4;  // positions per thread in flight
   for (int t00 = t0 + threadIdx.x; t00 < t1; t00 += kUnroll * blockDim.x) {
     float raw[kUnroll][G];
 #pragma unroll
@@ -332,6 +346,7 @@ __device__ __forceinline__ float exact_score(const float *raw, int G, float c, c
 
 // ------------------------------------------------------------------ filter
 __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams p) {
+  __shared__ int sh_band[kScoreThreads / 32][kSubRange];  // each warp's guard-band positions
   griddep_wait();
   griddep_launch_dependents();
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -339,14 +354,10 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
   const int nC = max(0, T - p.window);
   if (nC <= p.k_global || p.k_global == 0 || chunk * kFilterChunk >= nC) return;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
-  const int bin1 = p.ws.thr[u].x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = chunk * (kFilterChunk / kSubRange) + warp;  // this warp's sub-range
   const int s0 = sub * kSubRange, s1 = min(nC, s0 + kSubRange);
   if (s0 >= nC) return;
-  double lse[8];
-#pragma unroll
-  for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.lse[u * 8 + h] : 0.0;
   const float *sc = p.ws.scores + (size_t)u * p.ustride;
   int32_t *above = p.ws.above + (size_t)u * p.ustride + s0;
   uint2 *eqs = p.ws.cand + (size_t)u * p.ustride + s0;
@@ -361,21 +372,24 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
                       : make_float4(t < s1 ? sc[t] : 0.f, t + 1 < s1 ? sc[t + 1] : 0.f,
                                     t + 2 < s1 ? sc[t + 2] : 0.f, 0.f);
   }
+  // The k-th exact score lies in the threshold bin [lo, hi) widened by the
+  // approximation error (< 2e-5 relative even for logits of several hundred);
+  // the band keeps a 4e-4 margin on both sides.
+  const int bin1 = p.ws.thr[u].x;
+  const float lo = __uint_as_float((uint32_t)bin1 << kHistShift) * (1.f - kBandMargin);
+  const float hi = bin1 >= 0x7F7 ? INFINITY : __uint_as_float((uint32_t)(bin1 + 1) << kHistShift) * (1.f + kBandMargin);
   int na = 0, ne = 0;
 #pragma unroll
   for (int r = 0; r < kRounds; ++r) {
     const int t = s0 + 128 * r + 4 * lane;
     const float f[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
     int ca = 0, ce = 0;
-    uint32_t bits[4];
     bool a[4], e[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      bits[k] = __float_as_uint(f[k]);
-      const int bin = (int)(bits[k] >> kHistShift);
       const bool valid = t + k < s1;
-      a[k] = valid && bin >= bin1 + 2;                   // certainly above the k-th exact score
-      e[k] = valid && bin >= bin1 - 1 && bin <= bin1 + 1;  // guard band
+      a[k] = valid && f[k] >= hi;                // certainly above the k-th exact score
+      e[k] = valid && f[k] >= lo && f[k] < hi;   // guard band
       ca += a[k];
       ce += e[k];
     }
@@ -394,17 +408,23 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       if (a[k]) above[oa++] = t + k;
-      if (e[k]) eqs[oe++] = make_uint2(bits[k], (uint32_t)(t + k));
+      if (e[k]) sh_band[warp][oe++] = t + k;
     }
     na += ta;
     ne += te;
   }
-  // guard band: the exact score replaces the approximate one (the whole warp
-  // works through this list's entries, all loads in flight together)
+  // guard band: exact scores, the whole warp working through the list with
+  // every load in flight together
   __syncwarp();
-  for (int i = lane; i < ne; i += 32) {
-    const uint32_t pos = eqs[i].y;
-    eqs[i].x = __float_as_uint(exact_score(p.ws.logits + ((size_t)u * p.ustride + pos) * p.G, p.G, p.c, lse));
+  if (ne > 0) {
+    double lse[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.lse[u * 8 + h] : 0.0;
+    for (int i = lane; i < ne; i += 32) {
+      const int pos = sh_band[warp][i];
+      const float ex = exact_score(p.ws.logits + ((size_t)u * p.ustride + pos) * p.G, p.G, p.c, lse);
+      eqs[i] = make_uint2(__float_as_uint(ex), (uint32_t)pos);
+    }
   }
   if (lane == 0) p.ws.subcnt[(size_t)u * p.nsub + sub] = make_int2(na, ne);
 }

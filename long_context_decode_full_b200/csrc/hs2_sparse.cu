@@ -21,7 +21,7 @@ namespace hs2 {
 
 namespace {
 
-constexpr int kSparseWarps = 4;
+constexpr int kSparseWarps = 8;
 
 template <int D, bool FP8>
 struct SCfg {
@@ -30,28 +30,39 @@ struct SCfg {
   static constexpr int PANEL = 16 * 128;
   static constexpr int KVB = 16 * ROWB;                             // 16 rows of K (or V)
   static constexpr int BUF_BYTES = 2 * KVB + (FP8 ? 2 * 16 * 4 : 0);  // one 16-row group
-  static constexpr int WARP_BYTES = 2 * BUF_BYTES;                  // double buffer
   static constexpr int WSTRIDE = 16 + 8 * D;                        // warp scratch floats
   // one CTA's partial record m[G], l[G], o[G][D], padded to whole float4s
   __host__ __device__ static int rec_floats(int G) { return (G * (D + 2) + 3) & ~3; }
-  // CTA 0 gathers the cluster's partials into the (then idle) staging buffers
-  // when they fit, else into a region of their own
-  __host__ __device__ static bool gather_in_staging(int G, int S) {
-    return (size_t)S * rec_floats(G) * 4 <= (size_t)kSparseWarps * WARP_BYTES;
+  __host__ __device__ static size_t staging(int nbuf) { return (size_t)kSparseWarps * nbuf * BUF_BYTES; }
+  // the warps' merge scratch and CTA 0's gathered partials reuse the staging
+  // buffers (idle by then) when they fit, else get a region of their own
+  __host__ __device__ static size_t scratch_bytes(int G, int S) {
+    const size_t a = (size_t)kSparseWarps * WSTRIDE * 4, b = (size_t)S * rec_floats(G) * 4;
+    return a > b ? a : b;
   }
-  static size_t bytes(int G, int S, int rows) {
-    return 128 + (size_t)kSparseWarps * WARP_BYTES + (size_t)kSparseWarps * WSTRIDE * 4 + (size_t)rec_floats(G) * 4 +
-           (size_t)(S + 1) * 8 * 4 + (size_t)rows * 4 +
-           (gather_in_staging(G, S) ? 0 : (size_t)S * rec_floats(G) * 4);
+  __host__ __device__ static bool scratch_in_staging(int G, int S, int nbuf) {
+    return scratch_bytes(G, S) <= staging(nbuf);
+  }
+  static size_t bytes(int G, int S, int rows, int nbuf) {
+    return 128 + staging(nbuf) + (scratch_in_staging(G, S, nbuf) ? 0 : scratch_bytes(G, S)) +
+           (size_t)rec_floats(G) * 4 + (size_t)(S + 1) * 8 * 4 + (size_t)rows * 4;
   }
 };
 
-// Grid (splits, Hkv, B), cluster (splits, 1, 1), 4 warps.  CTA `rank` of a
+__device__ __forceinline__ void cp_async_wait_n(int n) {  // n = groups allowed to stay pending (<= 3)
+  if (n <= 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
+  else if (n == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+  else if (n == 2) asm volatile("cp.async.wait_group 2;" ::: "memory");
+  else asm volatile("cp.async.wait_group 3;" ::: "memory");
+}
+
+// Grid (splits, Hkv, B), cluster (splits, 1, 1), 8 warps.  CTA `rank` of a
 // unit's cluster owns rows [rank * rows_per_cta, ...) of the index list; its
-// warps take 16-row groups round-robin, gathering the next group while the
-// current one is on the tensor cores.
+// warps take 16-row groups round-robin.  Each warp issues the gathers of up
+// to `nbuf` groups at once, so their latencies overlap, and computes each
+// group on the tensor cores as it lands.
 template <int D, bool FP8>
-__global__ void __launch_bounds__(32 * kSparseWarps) sparse_mma_kernel(const SparseParams p, int64_t num_slots) {
+__global__ void __launch_bounds__(32 * kSparseWarps, 1) sparse_mma_kernel(const SparseParams p, int64_t num_slots) {
   using C = SCfg<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -59,13 +70,15 @@ __global__ void __launch_bounds__(32 * kSparseWarps) sparse_mma_kernel(const Spa
   cg::cluster_group cluster = cg::this_cluster();
   const int S = (int)cluster.num_blocks();
   const int RSP = C::rec_floats(p.G);
-  float *scratch = reinterpret_cast<float *>(smem + (size_t)kSparseWarps * C::WARP_BYTES);
-  float *partial = scratch + (size_t)kSparseWarps * C::WSTRIDE;  // m[G], l[G], o[G][D] of this CTA
+  const int nbuf = p.nbuf;
+  const bool in_staging = C::scratch_in_staging(p.G, S, nbuf);
+  uint8_t *after = smem + C::staging(nbuf) + (in_staging ? 0 : C::scratch_bytes(p.G, S));
+  float *scratch = reinterpret_cast<float *>(in_staging ? smem : smem + C::staging(nbuf));
+  float *gathered = scratch;                                     // CTA 0, after the warp merge
+  float *partial = reinterpret_cast<float *>(after);             // m[G], l[G], o[G][D] of this CTA
   float *wts = partial + RSP;                                    // CTA 0: weight of (CTA, head)
   float *inv_l = wts + S * 8;                                    // CTA 0: 1 / normaliser per head
   int *slots = reinterpret_cast<int *>(inv_l + 8);               // this CTA's index entries
-  float *gathered = C::gather_in_staging(p.G, S) ? reinterpret_cast<float *>(smem)
-                                                     : reinterpret_cast<float *>(slots + p.rows_per_cta);
   const int rank = (int)cluster.block_rank();
   const int kvh = blockIdx.y, b = blockIdx.z, G = p.G;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
@@ -85,7 +98,7 @@ __global__ void __launch_bounds__(32 * kSparseWarps) sparse_mma_kernel(const Spa
 
   constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
   const uint8_t *kg = static_cast<const uint8_t *>(p.k), *vg = static_cast<const uint8_t *>(p.v);
-  uint8_t *wbase = smem + (size_t)warp * C::WARP_BYTES;
+  uint8_t *wbase = smem + (size_t)warp * nbuf * C::BUF_BYTES;
   // issue the loads of 16-row group `grp` into buffer `buf`; returns its row mask
   auto gather = [&](int grp, int buf) -> uint32_t {
     uint8_t *wb = wbase + buf * C::BUF_BYTES;
@@ -125,23 +138,26 @@ __global__ void __launch_bounds__(32 * kSparseWarps) sparse_mma_kernel(const Spa
   };
 
   const int ngroups = (nrows + 15) / 16;
-  uint32_t vm[2] = {0u, 0u};
-  if (warp < ngroups) vm[0] = gather(warp, 0);
-  for (int k = 0, grp = warp; grp < ngroups; ++k, grp += kSparseWarps) {
-    const bool more = grp + kSparseWarps < ngroups;
-    if (more) {
-      vm[(k + 1) & 1] = gather(grp + kSparseWarps, (k + 1) & 1);
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-    } else {
-      cp_async_wait_all();
-    }
+  const int mine = ngroups > warp ? (ngroups - warp + kSparseWarps - 1) / kSparseWarps : 0;  // groups of this warp
+  uint32_t vm[4] = {0u, 0u, 0u, 0u};
+  int issued = 0;
+  for (; issued < mine && issued < nbuf; ++issued) vm[issued & 3] = gather(warp + issued * kSparseWarps, issued % nbuf);
+  for (int k = 0; k < mine; ++k) {
+    cp_async_wait_n(issued - k - 1);
     __syncwarp();
-    uint8_t *wb = wbase + (k & 1) * C::BUF_BYTES;
+    uint8_t *wb = wbase + (k % nbuf) * C::BUF_BYTES;
     const uint32_t kp = smem_u32(wb);
     const float *ks = reinterpret_cast<const float *>(wb + 2 * C::KVB);
-    if (vm[k & 1]) st.step(kp, kp + C::KVB, C::PANEL, 0, vm[k & 1], p.c, nullptr, G, ks, ks + 16);
-    __syncwarp();  // the buffer is refilled two groups later
+    const uint32_t m = vm[k & 3];
+    if (m) st.step(kp, kp + C::KVB, C::PANEL, 0, m, p.c, nullptr, G, ks, ks + 16);
+    __syncwarp();  // the buffer is refilled by the next gather
+    if (issued < mine) {
+      vm[issued & 3] = gather(warp + issued * kSparseWarps, issued % nbuf);
+      ++issued;
+    }
   }
+  cp_async_wait_all();
+  __syncthreads();  // every warp is done with the staging buffers
 
   // ---- merge the warps of this CTA, then the CTAs of the cluster
   float *scr = scratch + warp * C::WSTRIDE;
@@ -236,7 +252,7 @@ __global__ void sparse_f32_kernel(const SparseParams p, int64_t num_slots) {
 template <int D, bool FP8>
 cudaError_t launch_mma_t(const SparseParams &p, int64_t num_slots, cudaStream_t s) {
   using C = SCfg<D, FP8>;
-  const size_t smem = C::bytes(p.G, p.splits, p.rows_per_cta);
+  const size_t smem = C::bytes(p.G, p.splits, p.rows_per_cta, p.nbuf);
   auto kern = sparse_mma_kernel<D, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -35,12 +35,14 @@ struct WarpAttn {
   float m;             // running max of raw logits of head g
   float l;             // this lane's share of sum exp(c (s - m)) for head g
   float sig;           // E4M3: running max of the V scale (warp uniform)
+  float inv_sig;       // E4M3: 1 / sig (0 while sig is 0)
   float o[KS][4];      // O^T accumulator: dims x heads (2t, 2t+1)
 
   __device__ __forceinline__ void reset() {
     m = -INFINITY;
     l = 0.f;
     sig = 0.f;
+    inv_sig = 0.f;
 #pragma unroll
     for (int i = 0; i < KS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   }
@@ -92,39 +94,51 @@ struct WarpAttn {
   __device__ __forceinline__ void step(uint32_t kp, uint32_t vp, uint32_t pstride, int row0, uint32_t vmask,
                                        float c, float *logit_dst, int G, const float *ks, const float *vs) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    float s[2][4];
+    // two accumulator chains per n-tile (even / odd k-steps) halve the
+    // dependent-MMA latency; their fp32 sum is the logit
+    float s[2][4], s2[2][4];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[j][e] = s2[j][e] = 0.f;
 
     // ---- S = Q K^T
     if constexpr (!FP8) {
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int row = row0 + 8 * j + (lane & 7);
+      for (int kk = 0; kk < KS; kk += 2) {
 #pragma unroll
-        for (int kk = 0; kk < KS; kk += 2) {
+        for (int j = 0; j < 2; ++j) {
+          const int row = row0 + 8 * j + (lane & 7);
           const int cb = (16 * kk + 8 * (lane >> 3)) * 2;  // byte column
           uint32_t r[4];
           ldsm_x4(r, swz(kp + (cb >> 7) * pstride, row, (cb & 127) >> 4));
           mma_bf16(s[j], qa[kk][0], 0u, qa[kk][1], 0u, r[0], r[1]);
-          mma_bf16(s[j], qa[kk + 1][0], 0u, qa[kk + 1][1], 0u, r[2], r[3]);
+          mma_bf16(s2[j], qa[kk + 1][0], 0u, qa[kk + 1][1], 0u, r[2], r[3]);
         }
       }
     } else {
+      uint32_t w[2][8];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int row = row0 + 8 * j + g;
-        uint32_t w0[4], w1[4];
-        lds128(w0, swz(kp, row, 2 * t));
-        lds128(w1, swz(kp, row, 2 * t + 1));
+        lds128(*reinterpret_cast<uint32_t(*)[4]>(&w[j][0]), swz(kp, row, 2 * t));
+        lds128(*reinterpret_cast<uint32_t(*)[4]>(&w[j][4]), swz(kp, row, 2 * t + 1));
+      }
 #pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
+      for (int kk = 0; kk < KS; ++kk) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
           uint32_t b0, b1;
-          e4m3x4_to_f16x2x2(kk < 4 ? w0[kk & 3] : w1[kk & 3], b0, b1);
-          mma_f16(s[j], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+          e4m3x4_to_f16x2x2(w[j][kk], b0, b1);
+          if (kk & 1) mma_f16(s2[j], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+          else mma_f16(s[j], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
         }
       }
     }
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[j][e] += s2[j][e];
 
     // ---- logits, online softmax (head g; rows 2t, 2t+1, 8+2t, 9+2t)
     const int rr[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
@@ -140,57 +154,64 @@ struct WarpAttn {
       for (int i = 0; i < 4; ++i)
         if (ok[i]) logit_dst[rr[i] * G + g] = x[i];
     }
-    float mx = -INFINITY;
+    // Lazy rescaling: the reference m only moves when a logit would lift
+    // exp(c (x - m)) above 2^8 (and sig when a V scale exceeds it); p <= 2^8
+    // is exact in the MMA's P operand, and (m, l, o) stay consistent, so the
+    // result equals an eager online softmax.  The common case costs one vote.
+    const float cl = c * 1.44269504088896341f;  // exp(c x) = 2^(x cl)
+    const float thr = 8.f / cl;
+    float sv[4] = {0.f, 0.f, 0.f, 0.f};
+    float mloc = -INFINITY, sloc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (ok[i]) mloc = fmaxf(mloc, x[i]);
+      if constexpr (FP8) {
+        sv[i] = ok[i] ? vs[rr[i]] : 0.f;
+        sloc = fmaxf(sloc, sv[i]);
+      }
+    }
+    const bool grow = mloc > m + thr || (FP8 && sloc > sig);
+    float alpha = 1.f;
+    if (__any_sync(0xffffffffu, grow)) {
+      float mx = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float m_new = fmaxf(m, mx);
+      if (m_new != m) alpha = ex2_approx((m - m_new) * cl);  // 0 when m was -inf
+      m = m_new;
+      float beta = 1.f;
+      if constexpr (FP8) {
+        float smax = fmaxf(sloc, __shfl_xor_sync(0xffffffffu, sloc, 1));
+        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 2));
+        const float sig_new = fmaxf(sig, smax);
+        if (sig_new > sig) {
+          inv_sig = __frcp_rn(sig_new);
+          beta = sig * inv_sig;
+          sig = sig_new;
+        }
+      }
+      // rescale O^T columns (heads 2t, 2t+1) by their heads' factors
+      const float f = alpha * beta;
+      const float f_lo = __shfl_sync(0xffffffffu, f, 8 * t);
+      const float f_hi = __shfl_sync(0xffffffffu, f, 8 * t + 4);
+      if (__any_sync(0xffffffffu, f_lo != 1.f || f_hi != 1.f)) {
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+          o[i][0] *= f_lo;
+          o[i][1] *= f_hi;
+          o[i][2] *= f_lo;
+          o[i][3] *= f_hi;
+        }
+      }
+    }
+    float p[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (ok[i]) mx = fmaxf(mx, x[i]);
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(m, mx);
-    float alpha = 1.f, p[4] = {0.f, 0.f, 0.f, 0.f};
-    if (m_new != -INFINITY) {
-      // exp(c (x - m)) as 2^((x - m) c log2 e): the difference first, so the
-      // dominant terms (x near m) carry no rounding of m into l
-      const float cl = c * 1.44269504088896341f;
-      alpha = ex2_approx((m - m_new) * cl);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (ok[i]) p[i] = ex2_approx((x[i] - m_new) * cl);
-    }
+      if (ok[i]) p[i] = ex2_approx((x[i] - m) * cl);  // the difference first: dominant terms exact
     l = l * alpha + ((p[0] + p[1]) + (p[2] + p[3]));
-    m = m_new;
-
     float pv[4] = {p[0], p[1], p[2], p[3]};
-    float beta = 1.f;
     if constexpr (FP8) {
-      float sv[4], smax = 0.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        sv[i] = ok[i] ? vs[rr[i]] : 0.f;
-        smax = fmaxf(smax, sv[i]);
-      }
-      smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 1));
-      smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 2));
-      const float sig_new = fmaxf(sig, smax);
-      const float inv = sig_new > 0.f ? __frcp_rn(sig_new) : 0.f;
-      beta = sig_new > 0.f ? sig * inv : 1.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) pv[i] = p[i] * (sv[i] * inv);
-      sig = sig_new;
-    }
-
-    // ---- rescale O^T columns (heads 2t, 2t+1) by their heads' factors
-    const float f = alpha * beta;
-    const float f_lo = __shfl_sync(0xffffffffu, f, 8 * t);
-    const float f_hi = __shfl_sync(0xffffffffu, f, 8 * t + 4);
-    if (__any_sync(0xffffffffu, f_lo != 1.f || f_hi != 1.f)) {
-#pragma unroll
-      for (int i = 0; i < KS; ++i) {
-        o[i][0] *= f_lo;
-        o[i][1] *= f_hi;
-        o[i][2] *= f_lo;
-        o[i][3] *= f_hi;
-      }
+      for (int i = 0; i < 4; ++i) pv[i] = p[i] * (sv[i] * inv_sig);
     }
 
     // ---- O^T += V^T P^T
