@@ -206,6 +206,14 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return r;
 }
 
+// Transpose of an 8x8 matrix of 16-bit values held as one fragment (lane
+// 4r + c holds row r, columns 2c and 2c+1) into the same fragment layout.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t r;
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
+
 // 128-byte swizzle of a [rows][128 B] panel (the TMA SWIZZLE_128B pattern):
 // 16-byte chunk c of row r lives at chunk c ^ (r & 7).
 __device__ __forceinline__ uint32_t swz(uint32_t panel, int row, int chunk) {

@@ -445,6 +445,7 @@ cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const C
   HS2_FULL_CASE(128, false, 4, 6)
   HS2_FULL_CASE(64, false, 8, 6)
   HS2_FULL_CASE(64, false, 4, 6)
+  HS2_FULL_CASE(128, true, 16, 3)
   HS2_FULL_CASE(128, true, 12, 4)
   HS2_FULL_CASE(128, true, 8, 6)
   HS2_FULL_CASE(128, true, 4, 8)

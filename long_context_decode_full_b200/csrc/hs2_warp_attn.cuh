@@ -2,12 +2,13 @@
 // against the G <= 8 query heads of one GQA group, on the tensor cores.
 //
 // Layout of the contraction (mma.sync m16n8k16, fp32 accumulate):
-//   S   = Q K^T   : A = Q (16 rows = the group's heads, rows >= G zero),
-//                   B = K^T (8 rows of the tile per n-tile), two n-tiles.
+//   S^T = K Q^T   : A = K (the 16 rows of the slice), B = Q^T (8 heads;
+//                   heads >= G zero), so no MMA row is padding.
 //   O^T = V^T P^T : A = V^T (16 head dims per m-tile), B = P^T (16 rows x 8
-//                   heads).  The S accumulator of head g at rows 2t,2t+1 is
-//                   exactly the P^T fragment the second MMA needs, so P never
-//                   leaves registers, and no MMA row is padding.
+//                   heads).  The S^T accumulator holds rows g, g+8 of heads
+//                   2t, 2t+1; one 8x8 register transpose (movmatrix) per half
+//                   turns it into the P^T fragment, so P never leaves
+//                   registers.
 // The tile in shared memory is [panels][rows][128 B] with the 128-byte TMA
 // swizzle (16-byte chunk c of row r at chunk c ^ (r & 7)), written either by
 // TMA (full layer) or by cp.async (sparse layer).
@@ -30,24 +31,24 @@ struct WarpAttn {
   static_assert(!FP8 || D == 128, "E4M3 path is built for head_dim 128");
   static constexpr int KS = D / 16;  // k-steps of Q K^T and m-tiles of V^T P^T
 
-  uint32_t qa[KS][2];  // A-fragments of Q (rows g; rows g+8 are zero)
-  float qscale;        // E4M3: 2^-e undoing the query prescale
-  float m;             // running max of raw logits of head g
-  float l;             // this lane's share of sum exp(c (s - m)) for head g
+  uint32_t qa[KS][2];  // B-fragments of Q^T (head g; zero for heads >= G)
+  float qscale[2];     // E4M3: 2^-e undoing the prescale of heads 2t, 2t+1
+  float m[2];          // running max of raw logits of heads 2t, 2t+1 (uniform over g)
+  float l[2];          // this lane's share of sum exp(c (s - m)) for heads 2t, 2t+1
   float sig;           // E4M3: running max of the V scale (warp uniform)
   float inv_sig;       // E4M3: 1 / sig (0 while sig is 0)
   float o[KS][4];      // O^T accumulator: dims x heads (2t, 2t+1)
 
   __device__ __forceinline__ void reset() {
-    m = -INFINITY;
-    l = 0.f;
+    m[0] = m[1] = -INFINITY;
+    l[0] = l[1] = 0.f;
     sig = 0.f;
     inv_sig = 0.f;
 #pragma unroll
     for (int i = 0; i < KS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   }
 
-  // Query of the group (G consecutive heads, bf16 [G][D]) into A-fragments.
+  // Query of the group (G consecutive heads, bf16 [G][D]) into B-fragments.
   __device__ __forceinline__ void load_q(const __nv_bfloat16 *q, int G) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const uint32_t *q32 = reinterpret_cast<const uint32_t *>(q);
@@ -57,7 +58,7 @@ struct WarpAttn {
         qa[kk][0] = g < G ? __ldg(q32 + ((g * D + 16 * kk + 2 * t) >> 1)) : 0u;
         qa[kk][1] = g < G ? __ldg(q32 + ((g * D + 16 * kk + 8 + 2 * t) >> 1)) : 0u;
       }
-      qscale = 1.f;
+      qscale[0] = qscale[1] = 1.f;
     } else {
       // k-step kk of lane t covers dims 32t + 4kk + {0,1} (MMA k = 2t, 2t+1)
       // and 32t + 4kk + {2,3} (MMA k = 2t+8, 2t+9).
@@ -77,7 +78,9 @@ struct WarpAttn {
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
       const int e = amax > 0.f ? 14 - ilogbf(amax) : 0;
       const float up = ldexpf(1.f, e);
-      qscale = ldexpf(1.f, -e);
+      // the logits of this lane belong to heads 2t, 2t+1 (lanes 8t, 8t + 4 hold their exponents)
+      qscale[0] = ldexpf(1.f, -__shfl_sync(0xffffffffu, e, 8 * t));
+      qscale[1] = ldexpf(1.f, -__shfl_sync(0xffffffffu, e, 8 * t + 4));
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
         qa[kk][0] = pack_f16(v[kk][0] * up, v[kk][1] * up);
@@ -94,27 +97,21 @@ struct WarpAttn {
   __device__ __forceinline__ void step(uint32_t kp, uint32_t vp, uint32_t pstride, int row0, uint32_t vmask,
                                        float c, float *logit_dst, int G, const float *ks, const float *vs) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    // two accumulator chains per n-tile (even / odd k-steps) halve the
-    // dependent-MMA latency; their fp32 sum is the logit
-    float s[2][4], s2[2][4];
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[j][e] = s2[j][e] = 0.f;
+    // two accumulator chains (even / odd k-steps) halve the dependent-MMA
+    // latency; their fp32 sum is the logit
+    float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
 
-    // ---- S = Q K^T
+    // ---- S^T = K Q^T
     if constexpr (!FP8) {
+      // matrices of one ldmatrix.x4: rows 0-7 / 8-15 x dims 0-7, then 8-15
+      const int row = row0 + (lane & 7) + (((lane >> 3) & 1) << 3);
 #pragma unroll
-      for (int kk = 0; kk < KS; kk += 2) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int row = row0 + 8 * j + (lane & 7);
-          const int cb = (16 * kk + 8 * (lane >> 3)) * 2;  // byte column
-          uint32_t r[4];
-          ldsm_x4(r, swz(kp + (cb >> 7) * pstride, row, (cb & 127) >> 4));
-          mma_bf16(s[j], qa[kk][0], 0u, qa[kk][1], 0u, r[0], r[1]);
-          mma_bf16(s2[j], qa[kk + 1][0], 0u, qa[kk + 1][1], 0u, r[2], r[3]);
-        }
+      for (int kk = 0; kk < KS; ++kk) {
+        const int cb = (16 * kk + 8 * (lane >> 4)) * 2;  // byte column
+        uint32_t r[4];
+        ldsm_x4(r, swz(kp + (cb >> 7) * pstride, row, (cb & 127) >> 4));
+        if (kk & 1) mma_bf16(s2, r[0], r[1], r[2], r[3], qa[kk][0], qa[kk][1]);
+        else mma_bf16(s, r[0], r[1], r[2], r[3], qa[kk][0], qa[kk][1]);
       }
     } else {
       uint32_t w[2][8];
@@ -126,33 +123,38 @@ struct WarpAttn {
       }
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          uint32_t b0, b1;
-          e4m3x4_to_f16x2x2(w[j][kk], b0, b1);
-          if (kk & 1) mma_f16(s2[j], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
-          else mma_f16(s[j], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
-        }
+        uint32_t lo0, hi0, lo1, hi1;
+        e4m3x4_to_f16x2x2(w[0][kk], lo0, hi0);
+        e4m3x4_to_f16x2x2(w[1][kk], lo1, hi1);
+        if (kk & 1) mma_f16(s2, lo0, lo1, hi0, hi1, qa[kk][0], qa[kk][1]);
+        else mma_f16(s, lo0, lo1, hi0, hi1, qa[kk][0], qa[kk][1]);
       }
     }
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[j][e] += s2[j][e];
 
-    // ---- logits, online softmax (head g; rows 2t, 2t+1, 8+2t, 9+2t)
-    const int rr[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
-    float x[4] = {s[0][0], s[0][1], s[1][0], s[1][1]};
-    bool ok[4];
+    // ---- logits, online softmax: x[j][h] = row g + 8j, head 2t + h
+    float x[2][2] = {{s[0] + s2[0], s[1] + s2[1]}, {s[2] + s2[2], s[3] + s2[3]}};
+    const bool ok[2] = {((vmask >> g) & 1u) != 0u, ((vmask >> (g + 8)) & 1u) != 0u};
+    float sv[2] = {0.f, 0.f};
+    if constexpr (FP8) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ok[i] = (vmask >> rr[i]) & 1u;
-      if constexpr (FP8) x[i] *= (ok[i] ? ks[rr[i]] : 0.f) * qscale;
+      for (int j = 0; j < 2; ++j) {
+        const float kj = ok[j] ? ks[g + 8 * j] : 0.f;
+        x[j][0] *= kj * qscale[0];
+        x[j][1] *= kj * qscale[1];
+        sv[j] = ok[j] ? vs[g + 8 * j] : 0.f;
+      }
     }
-    if (logit_dst != nullptr && g < G) {
+    if (logit_dst != nullptr && 2 * t < G) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (ok[i]) logit_dst[rr[i] * G + g] = x[i];
+      for (int j = 0; j < 2; ++j) {
+        if (!ok[j]) continue;
+        float *dst = logit_dst + (g + 8 * j) * G + 2 * t;
+        if ((G & 1) == 0) *reinterpret_cast<float2 *>(dst) = make_float2(x[j][0], x[j][1]);
+        else {
+          dst[0] = x[j][0];
+          if (2 * t + 1 < G) dst[1] = x[j][1];
+        }
+      }
     }
     // Lazy rescaling: the reference m only moves when a logit would lift
     // exp(c (x - m)) above 2^8 (and sig when a V scale exceeds it); p <= 2^8
@@ -160,28 +162,19 @@ struct WarpAttn {
     // result equals an eager online softmax.  The common case costs one vote.
     const float cl = c * 1.44269504088896341f;  // exp(c x) = 2^(x cl)
     const float thr = 8.f / cl;
-    float sv[4] = {0.f, 0.f, 0.f, 0.f};
-    float mloc = -INFINITY, sloc = 0.f;
+    float mloc[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (ok[i]) mloc = fmaxf(mloc, x[i]);
-      if constexpr (FP8) {
-        sv[i] = ok[i] ? vs[rr[i]] : 0.f;
-        sloc = fmaxf(sloc, sv[i]);
-      }
-    }
-    const bool grow = mloc > m + thr || (FP8 && sloc > sig);
-    float alpha = 1.f;
+    for (int h = 0; h < 2; ++h)
+      mloc[h] = fmaxf(ok[0] ? x[0][h] : -INFINITY, ok[1] ? x[1][h] : -INFINITY);
+    const float sloc = fmaxf(sv[0], sv[1]);
+    const bool grow = mloc[0] > m[0] + thr || mloc[1] > m[1] + thr || (FP8 && sloc > sig);
+    float alpha[2] = {1.f, 1.f};
     if (__any_sync(0xffffffffu, grow)) {
-      float mx = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float m_new = fmaxf(m, mx);
-      if (m_new != m) alpha = ex2_approx((m - m_new) * cl);  // 0 when m was -inf
-      m = m_new;
       float beta = 1.f;
       if constexpr (FP8) {
-        float smax = fmaxf(sloc, __shfl_xor_sync(0xffffffffu, sloc, 1));
-        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 2));
+        float smax = fmaxf(sloc, __shfl_xor_sync(0xffffffffu, sloc, 4));
+        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 8));
+        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
         const float sig_new = fmaxf(sig, smax);
         if (sig_new > sig) {
           inv_sig = __frcp_rn(sig_new);
@@ -189,37 +182,54 @@ struct WarpAttn {
           sig = sig_new;
         }
       }
-      // rescale O^T columns (heads 2t, 2t+1) by their heads' factors
-      const float f = alpha * beta;
-      const float f_lo = __shfl_sync(0xffffffffu, f, 8 * t);
-      const float f_hi = __shfl_sync(0xffffffffu, f, 8 * t + 4);
-      if (__any_sync(0xffffffffu, f_lo != 1.f || f_hi != 1.f)) {
+      float f[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // max over the rows: lanes of equal t
+        float mx = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float m_new = fmaxf(m[h], mx);
+        if (m_new != m[h]) alpha[h] = ex2_approx((m[h] - m_new) * cl);  // 0 when m was -inf
+        m[h] = m_new;
+        f[h] = alpha[h] * beta;
+      }
+      // rescale the O^T columns of heads 2t, 2t+1
+      if (__any_sync(0xffffffffu, f[0] != 1.f || f[1] != 1.f)) {
 #pragma unroll
         for (int i = 0; i < KS; ++i) {
-          o[i][0] *= f_lo;
-          o[i][1] *= f_hi;
-          o[i][2] *= f_lo;
-          o[i][3] *= f_hi;
+          o[i][0] *= f[0];
+          o[i][1] *= f[1];
+          o[i][2] *= f[0];
+          o[i][3] *= f[1];
         }
       }
     }
-    float p[4] = {0.f, 0.f, 0.f, 0.f};
+    float p[2][2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (ok[i]) p[i] = ex2_approx((x[i] - m) * cl);  // the difference first: dominant terms exact
-    l = l * alpha + ((p[0] + p[1]) + (p[2] + p[3]));
-    float pv[4] = {p[0], p[1], p[2], p[3]};
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)  // the difference first: dominant terms exact
+        p[j][h] = ok[j] ? ex2_approx((x[j][h] - m[h]) * cl) : 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) l[h] = l[h] * alpha[h] + (p[0][h] + p[1][h]);
     if constexpr (FP8) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) pv[i] = p[i] * (sv[i] * inv_sig);
+      for (int j = 0; j < 2; ++j) {
+        const float w8 = sv[j] * inv_sig;
+        p[j][0] *= w8;
+        p[j][1] *= w8;
+      }
     }
+    // P^T fragment: transpose the 8x8 halves (rows 0-7 and 8-15 x heads)
+    const uint32_t pb0 = movmatrix_t(FP8 ? pack_f16(p[0][0], p[0][1]) : pack_bf16(p[0][0], p[0][1]));
+    const uint32_t pb1 = movmatrix_t(FP8 ? pack_f16(p[1][0], p[1][1]) : pack_bf16(p[1][0], p[1][1]));
 
-    // ---- O^T += V^T P^T
+    // ---- O^T += V^T P^T (A rows 2t, 2t+1, 8+2t, 9+2t of the slice)
     const bool full = vmask == 0xFFFFu;
-    const uint32_t m01 = (ok[0] ? 0x0000FFFFu : 0u) | (ok[1] ? 0xFFFF0000u : 0u);
-    const uint32_t m23 = (ok[2] ? 0x0000FFFFu : 0u) | (ok[3] ? 0xFFFF0000u : 0u);
+    const uint32_t v0 = (vmask >> (2 * t)) & 3u, v1 = (vmask >> (2 * t + 8)) & 3u;
     if constexpr (!FP8) {
-      const uint32_t pb0 = pack_bf16(pv[0], pv[1]), pb1 = pack_bf16(pv[2], pv[3]);
+      const uint32_t m01 = ((v0 & 1u) ? 0x0000FFFFu : 0u) | ((v0 & 2u) ? 0xFFFF0000u : 0u);
+      const uint32_t m23 = ((v1 & 1u) ? 0x0000FFFFu : 0u) | ((v1 & 2u) ? 0xFFFF0000u : 0u);
       const int row = row0 + (lane & 7) + ((lane >> 4) << 3);
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
@@ -235,15 +245,14 @@ struct WarpAttn {
         mma_bf16(o[mt], a[0], a[1], a[2], a[3], pb0, pb1);
       }
     } else {
-      const uint32_t pb0 = pack_f16(pv[0], pv[1]), pb1 = pack_f16(pv[2], pv[3]);
       uint32_t w0[4], w1[4], w2[4], w3[4];
-      lds128(w0, swz(vp, row0 + rr[0], g));
-      lds128(w1, swz(vp, row0 + rr[1], g));
-      lds128(w2, swz(vp, row0 + rr[2], g));
-      lds128(w3, swz(vp, row0 + rr[3], g));
+      lds128(w0, swz(vp, row0 + 2 * t, g));
+      lds128(w1, swz(vp, row0 + 2 * t + 1, g));
+      lds128(w2, swz(vp, row0 + 2 * t + 8, g));
+      lds128(w3, swz(vp, row0 + 2 * t + 9, g));
       // byte masks: bytes 0,2 come from the even row, bytes 1,3 from the odd row
-      const uint32_t b01 = (ok[0] ? 0x00FF00FFu : 0u) | (ok[1] ? 0xFF00FF00u : 0u);
-      const uint32_t b23 = (ok[2] ? 0x00FF00FFu : 0u) | (ok[3] ? 0xFF00FF00u : 0u);
+      const uint32_t b01 = ((v0 & 1u) ? 0x00FF00FFu : 0u) | ((v0 & 2u) ? 0xFF00FF00u : 0u);
+      const uint32_t b23 = ((v1 & 1u) ? 0x00FF00FFu : 0u) | ((v1 & 2u) ? 0xFF00FF00u : 0u);
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
         const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
@@ -265,12 +274,16 @@ struct WarpAttn {
   // scale, not yet normalised).  Heads >= G are written too and ignored.
   __device__ __forceinline__ void store(float *sm, float *sl, float *so) const {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    float lt = l;
-    lt += __shfl_xor_sync(0xffffffffu, lt, 1);
-    lt += __shfl_xor_sync(0xffffffffu, lt, 2);
-    if (t == 0) {
-      sm[g] = m;
-      sl[g] = lt;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // sum over the rows: lanes of equal t
+      float lt = l[h];
+      lt += __shfl_xor_sync(0xffffffffu, lt, 4);
+      lt += __shfl_xor_sync(0xffffffffu, lt, 8);
+      lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+      if (g == 0) {
+        sm[2 * t + h] = m[h];
+        sl[2 * t + h] = lt;
+      }
     }
     const float os = FP8 ? sig : 1.f;
 #pragma unroll
