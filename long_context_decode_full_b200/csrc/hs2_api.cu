@@ -185,27 +185,30 @@ int check_caches(const hs2_cache *k, const hs2_cache *v) {
   return HS2_OK;
 }
 
-// Consumer warps and pipeline stages of the attention kernel, most preferred
-// first: enough warps for two per SM sub-partition and enough stages that the
-// bytes in flight per SM cover the loaded HBM latency.  A tile (16 positions
-// per consumer warp) must fit the page size (one divides the other).
+// Consumer warps, pipeline stages and slices per warp of the attention
+// kernel, most preferred first: enough independent work per SM sub-partition
+// to hide the MMA and conversion latencies, and enough stages that the bytes
+// in flight per SM cover the loaded HBM latency.  A tile must fit the page
+// size (one divides the other) in at most 8 page boxes.
+bool tile_fits_pages(int tile, int page_size, bool paged) {
+  if (!paged) return true;
+  if (page_size % tile == 0) return true;
+  return tile % page_size == 0 && tile / page_size <= 8;
+}
+
 FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged) {
-  static const FullMmaConfig bf16_128[] = {{8, 3}, {4, 6}};
-  static const FullMmaConfig bf16_64[] = {{8, 6}, {4, 6}};
-  static const FullMmaConfig e4m3[] = {{12, 4}, {8, 6}, {4, 8}};
+  static const FullMmaConfig bf16_128[] = {{4, 3, 2}, {8, 3, 1}, {4, 6, 1}};
+  static const FullMmaConfig bf16_64[] = {{8, 6, 1}, {4, 6, 1}};
+  static const FullMmaConfig e4m3[] = {{8, 3, 2}, {12, 4, 1}, {8, 6, 1}, {4, 8, 1}};
   const FullMmaConfig *list = fp8 ? e4m3 : (D == 64 ? bf16_64 : bf16_128);
-  const int n = fp8 ? 3 : 2;
-  if (const char *env = getenv("HS2_FULL_CFG")) {  // tuning override
-    int a = 0, b = 0;
-    if (sscanf(env, "%d,%d", &a, &b) == 2) {
-      const int tile = 16 * a;
-      if (!paged || page_size % tile == 0 || tile % page_size == 0) return FullMmaConfig{a, b};
-    }
+  const int n = fp8 ? 4 : (D == 64 ? 2 : 3);
+  if (const char *env = getenv("HS2_FULL_CFG")) {  // tuning override: "ncw,nstage[,nsl]"
+    int a = 0, b = 0, c = 1;
+    if (sscanf(env, "%d,%d,%d", &a, &b, &c) >= 2 && tile_fits_pages(16 * a * c, page_size, paged))
+      return FullMmaConfig{a, b, c};
   }
-  for (int i = 0; i < n; ++i) {
-    const int tile = 16 * list[i].ncw;
-    if (!paged || page_size % tile == 0 || tile % page_size == 0) return list[i];
-  }
+  for (int i = 0; i < n; ++i)
+    if (tile_fits_pages(16 * list[i].ncw * list[i].nsl, page_size, paged)) return list[i];
   return list[n - 1];
 }
 
@@ -304,7 +307,7 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
   } else {
     const bool fp8 = k_cache->dtype == HS2_E4M3;
     const FullMmaConfig cfg = pick_full_config(D, fp8, ps, paged);
-    p.tile = 16 * cfg.ncw;
+    p.tile = 16 * cfg.ncw * cfg.nsl;
     p.N = sms;
     const int box_rows = paged ? (ps < p.tile ? ps : p.tile) : p.tile;
     CUtensorMap tmk, tmv;
@@ -312,7 +315,8 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
     if ((rc = encode_cache_map(&tmv, v_cache, box_rows))) return rc;
     e = launch_full_mma(p, tmk, tmv, fp8, cfg, p.N, s);
     if (e == cudaErrorInvalidConfiguration)
-      return fail(HS2_ERR_UNSUPPORTED, "no full-attention kernel built for ncw=%d nstage=%d", cfg.ncw, cfg.nstage);
+      return fail(HS2_ERR_UNSUPPORTED, "no full-attention kernel built for ncw=%d nstage=%d nsl=%d", cfg.ncw, cfg.nstage,
+                  cfg.nsl);
     if (e != cudaSuccess) return cuda_fail(e, "full-attention launch");
   }
   if (mark_event) {

@@ -27,9 +27,10 @@ struct StageMeta {
 };
 constexpr int kFirst = 1, kLast = 2, kDone = 4;
 
-template <int D, bool FP8, int NCW, int NSTAGE>
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL>
 struct Cfg {
-  static constexpr int TILE = 16 * NCW;
+  static constexpr int RPW = 16 * NSL;  // rows per consumer warp
+  static constexpr int TILE = RPW * NCW;
   static constexpr int ES = FP8 ? 1 : 2;
   static constexpr int ROWB = D * ES;
   static constexpr int NPANEL = ROWB / 128;
@@ -103,11 +104,11 @@ __device__ __forceinline__ int find_seq(const int32_t *prefix, int B, int Hkv, i
   return lo;
 }
 
-template <int D, bool FP8, int NCW, int NSTAGE>
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL>
 __global__ void __launch_bounds__(32 * (NCW + 1), 1)
     full_attn_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                          const FullParams p) {
-  using C = Cfg<D, FP8, NCW, NSTAGE>;
+  using C = Cfg<D, FP8, NCW, NSTAGE, NSL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
   }
 
   // -------------------------------------------------------------- consumers
-  WarpAttn<D, FP8> st;
+  WarpAttn<D, FP8, NSL> st;
   st.reset();
   uint32_t cphase = 0;
   for (int it = 0;; ++it) {
@@ -273,14 +274,14 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
       st.load_q(reinterpret_cast<const __nv_bfloat16 *>(p.q) + ((int64_t)mt.b * p.Hkv * p.G + (int64_t)mt.kvh * p.G) * D,
                 p.G);
     }
-    const int pos0 = mt.tile * C::TILE + 16 * warp;
-    const int nvalid = max(0, min(16, mt.T - pos0));
-    const uint32_t vmask = nvalid >= 16 ? 0xFFFFu : ((1u << nvalid) - 1u);
+    const int pos0 = mt.tile * C::TILE + C::RPW * warp;
+    const int nvalid = max(0, min(C::RPW, mt.T - pos0));
+    const uint32_t vmask = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
     const uint32_t kp = sbase + stage * C::STAGE;
-    const float *ks = reinterpret_cast<const float *>(smem + (size_t)stage * C::STAGE + 2 * C::KVB) + 16 * warp;
+    const float *ks = reinterpret_cast<const float *>(smem + (size_t)stage * C::STAGE + 2 * C::KVB) + C::RPW * warp;
     if (nvalid > 0)
-      st.step(kp, kp + C::KVB, C::PANEL, 16 * warp, vmask, p.c, p.ws.logits + (u * p.ustride + pos0) * p.G, p.G, ks,
-              ks + C::TILE);
+      st.step(kp, kp + C::KVB, C::PANEL, C::RPW * warp, vmask, p.c, p.ws.logits + (u * p.ustride + pos0) * p.G, p.G,
+              ks, ks + C::TILE);
     if (mt.flags & kLast) {
       // segment end: merge the warps' states inside this stage, then release it
       if (!consumer_sync(cbar, cphase)) {  // every warp is done reading the tile
@@ -423,12 +424,12 @@ __global__ void __launch_bounds__(32 * kF32Warps) full_attn_f32_kernel(const Ful
   }
 }
 
-template <int D, bool FP8, int NCW, int NSTAGE>
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL>
 cudaError_t launch_mma_t(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, int grid,
                          cudaStream_t s) {
-  using C = Cfg<D, FP8, NCW, NSTAGE>;
+  using C = Cfg<D, FP8, NCW, NSTAGE, NSL>;
   const size_t smem = C::bytes(p.B);
-  auto kern = full_attn_mma_kernel<D, FP8, NCW, NSTAGE>;
+  auto kern = full_attn_mma_kernel<D, FP8, NCW, NSTAGE, NSL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_ex(kern, dim3(grid), dim3(32 * (NCW + 1)), smem, s, 0, tmk, tmv, p);
@@ -438,17 +439,20 @@ cudaError_t launch_mma_t(const FullParams &p, const CUtensorMap &tmk, const CUte
 
 cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, bool fp8,
                             const FullMmaConfig &cfg, int grid, cudaStream_t s) {
-#define HS2_FULL_CASE(D_, F_, W_, S_)                                                   \
-  if (p.D == D_ && fp8 == F_ && cfg.ncw == W_ && cfg.nstage == S_)                      \
-    return launch_mma_t<D_, F_, W_, S_>(p, tmk, tmv, grid, s);
-  HS2_FULL_CASE(128, false, 8, 3)
-  HS2_FULL_CASE(128, false, 4, 6)
-  HS2_FULL_CASE(64, false, 8, 6)
-  HS2_FULL_CASE(64, false, 4, 6)
-  HS2_FULL_CASE(128, true, 16, 3)
-  HS2_FULL_CASE(128, true, 12, 4)
-  HS2_FULL_CASE(128, true, 8, 6)
-  HS2_FULL_CASE(128, true, 4, 8)
+#define HS2_FULL_CASE(D_, F_, W_, S_, L_)                                               \
+  if (p.D == D_ && fp8 == F_ && cfg.ncw == W_ && cfg.nstage == S_ && cfg.nsl == L_)     \
+    return launch_mma_t<D_, F_, W_, S_, L_>(p, tmk, tmv, grid, s);
+  HS2_FULL_CASE(128, false, 8, 3, 1)
+  HS2_FULL_CASE(128, false, 4, 6, 1)
+  HS2_FULL_CASE(128, false, 4, 3, 2)
+  HS2_FULL_CASE(64, false, 8, 6, 1)
+  HS2_FULL_CASE(64, false, 4, 6, 1)
+  HS2_FULL_CASE(128, true, 8, 3, 2)
+  HS2_FULL_CASE(128, true, 4, 6, 2)
+  HS2_FULL_CASE(128, true, 16, 3, 1)
+  HS2_FULL_CASE(128, true, 12, 4, 1)
+  HS2_FULL_CASE(128, true, 8, 6, 1)
+  HS2_FULL_CASE(128, true, 4, 8, 1)
 #undef HS2_FULL_CASE
   return cudaErrorInvalidConfiguration;
 }

@@ -63,8 +63,9 @@ struct SparseParams {
 
 // Launch configuration chosen by the host for the tensor-core full kernel.
 struct FullMmaConfig {
-  int ncw;     // consumer warps (tile = 16 * ncw positions)
+  int ncw;     // consumer warps
   int nstage;  // pipeline stages
+  int nsl;     // 16-row slices per warp and tile (tile = 16 * ncw * nsl positions)
 };
 
 // Launch with programmatic stream serialization (unless HS2_PDL=0) and an

@@ -25,9 +25,12 @@
 
 namespace hs2 {
 
-template <int D, bool FP8>
+// NSL: 16-row slices per step.  Two slices give the warp two independent
+// instruction streams (MMA chains, conversions, exponentials) to interleave.
+template <int D, bool FP8, int NSL = 1>
 struct WarpAttn {
   static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(NSL == 1 || NSL == 2, "slices per step");
   static_assert(!FP8 || D == 128, "E4M3 path is built for head_dim 128");
   static constexpr int KS = D / 16;  // k-steps of Q K^T and m-tiles of V^T P^T
 
@@ -89,17 +92,22 @@ struct WarpAttn {
     }
   }
 
-  // One 16-row slice.  kp / vp: shared addresses of panel 0 of the K / V
-  // tile; pstride: bytes between panels; row0: first row of the slice inside
-  // the panel; vmask: bit r set when row r holds a real position; c: 1/sqrt(D)
-  // in the logit domain.  logit_dst (or nullptr): raw logits [16][G] of this
-  // slice.  ks / vs (E4M3): the slice's 16 K / V scales in shared memory.
+  // NSL 16-row slices.  kp / vp: shared addresses of panel 0 of the K / V
+  // tile; pstride: bytes between panels; row0: first row of the first slice
+  // inside the panel (slice sl starts at row0 + 16 sl); vmask: bit r set when
+  // row row0 + r holds a real position; c: 1/sqrt(D) in the logit domain.
+  // logit_dst (or nullptr): raw logits [16 NSL][G] of these rows.  ks / vs
+  // (E4M3): the rows' K / V scales in shared memory.
   __device__ __forceinline__ void step(uint32_t kp, uint32_t vp, uint32_t pstride, int row0, uint32_t vmask,
                                        float c, float *logit_dst, int G, const float *ks, const float *vs) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    // two accumulator chains (even / odd k-steps) halve the dependent-MMA
-    // latency; their fp32 sum is the logit
-    float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+    // two accumulator chains per slice (even / odd k-steps) halve the
+    // dependent-MMA latency; their fp32 sum is the logit
+    float s[NSL][4], s2[NSL][4];
+#pragma unroll
+    for (int sl = 0; sl < NSL; ++sl)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[sl][e] = s2[sl][e] = 0.f;
 
     // ---- S^T = K Q^T
     if constexpr (!FP8) {
@@ -108,53 +116,70 @@ struct WarpAttn {
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
         const int cb = (16 * kk + 8 * (lane >> 4)) * 2;  // byte column
-        uint32_t r[4];
-        ldsm_x4(r, swz(kp + (cb >> 7) * pstride, row, (cb & 127) >> 4));
-        if (kk & 1) mma_bf16(s2, r[0], r[1], r[2], r[3], qa[kk][0], qa[kk][1]);
-        else mma_bf16(s, r[0], r[1], r[2], r[3], qa[kk][0], qa[kk][1]);
+#pragma unroll
+        for (int sl = 0; sl < NSL; ++sl) {
+          uint32_t r[4];
+          ldsm_x4(r, swz(kp + (cb >> 7) * pstride, row + 16 * sl, (cb & 127) >> 4));
+          if (kk & 1) mma_bf16(s2[sl], r[0], r[1], r[2], r[3], qa[kk][0], qa[kk][1]);
+          else mma_bf16(s[sl], r[0], r[1], r[2], r[3], qa[kk][0], qa[kk][1]);
+        }
       }
     } else {
-      uint32_t w[2][8];
+      uint32_t w[NSL][2][8];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int row = row0 + 8 * j + g;
-        lds128(*reinterpret_cast<uint32_t(*)[4]>(&w[j][0]), swz(kp, row, 2 * t));
-        lds128(*reinterpret_cast<uint32_t(*)[4]>(&w[j][4]), swz(kp, row, 2 * t + 1));
-      }
+      for (int sl = 0; sl < NSL; ++sl)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int row = row0 + 16 * sl + 8 * j + g;
+          lds128(*reinterpret_cast<uint32_t(*)[4]>(&w[sl][j][0]), swz(kp, row, 2 * t));
+          lds128(*reinterpret_cast<uint32_t(*)[4]>(&w[sl][j][4]), swz(kp, row, 2 * t + 1));
+        }
 #pragma unroll
       for (int kk = 0; kk < KS; ++kk) {
-        uint32_t lo0, hi0, lo1, hi1;
-        e4m3x4_to_f16x2x2(w[0][kk], lo0, hi0);
-        e4m3x4_to_f16x2x2(w[1][kk], lo1, hi1);
-        if (kk & 1) mma_f16(s2, lo0, lo1, hi0, hi1, qa[kk][0], qa[kk][1]);
-        else mma_f16(s, lo0, lo1, hi0, hi1, qa[kk][0], qa[kk][1]);
+#pragma unroll
+        for (int sl = 0; sl < NSL; ++sl) {
+          uint32_t lo0, hi0, lo1, hi1;
+          e4m3x4_to_f16x2x2(w[sl][0][kk], lo0, hi0);
+          e4m3x4_to_f16x2x2(w[sl][1][kk], lo1, hi1);
+          if (kk & 1) mma_f16(s2[sl], lo0, lo1, hi0, hi1, qa[kk][0], qa[kk][1]);
+          else mma_f16(s[sl], lo0, lo1, hi0, hi1, qa[kk][0], qa[kk][1]);
+        }
       }
     }
 
-    // ---- logits, online softmax: x[j][h] = row g + 8j, head 2t + h
-    float x[2][2] = {{s[0] + s2[0], s[1] + s2[1]}, {s[2] + s2[2], s[3] + s2[3]}};
-    const bool ok[2] = {((vmask >> g) & 1u) != 0u, ((vmask >> (g + 8)) & 1u) != 0u};
-    float sv[2] = {0.f, 0.f};
-    if constexpr (FP8) {
+    // ---- logits, online softmax: x[sl][j][h] = row 16 sl + g + 8j, head 2t + h
+    float x[NSL][2][2];
+    bool ok[NSL][2];
+    float sv[NSL][2];
+#pragma unroll
+    for (int sl = 0; sl < NSL; ++sl)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        const float kj = ok[j] ? ks[g + 8 * j] : 0.f;
-        x[j][0] *= kj * qscale[0];
-        x[j][1] *= kj * qscale[1];
-        sv[j] = ok[j] ? vs[g + 8 * j] : 0.f;
-      }
-    }
-    if (logit_dst != nullptr && 2 * t < G) {
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        if (!ok[j]) continue;
-        float *dst = logit_dst + (g + 8 * j) * G + 2 * t;
-        if ((G & 1) == 0) *reinterpret_cast<float2 *>(dst) = make_float2(x[j][0], x[j][1]);
-        else {
-          dst[0] = x[j][0];
-          if (2 * t + 1 < G) dst[1] = x[j][1];
+        const int r = 16 * sl + 8 * j + g;
+        x[sl][j][0] = s[sl][2 * j] + s2[sl][2 * j];
+        x[sl][j][1] = s[sl][2 * j + 1] + s2[sl][2 * j + 1];
+        ok[sl][j] = ((vmask >> r) & 1u) != 0u;
+        sv[sl][j] = 0.f;
+        if constexpr (FP8) {
+          const float kj = ok[sl][j] ? ks[r] : 0.f;
+          x[sl][j][0] *= kj * qscale[0];
+          x[sl][j][1] *= kj * qscale[1];
+          sv[sl][j] = ok[sl][j] ? vs[r] : 0.f;
         }
       }
+    if (logit_dst != nullptr && 2 * t < G) {
+#pragma unroll
+      for (int sl = 0; sl < NSL; ++sl)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (!ok[sl][j]) continue;
+          float *dst = logit_dst + (16 * sl + 8 * j + g) * G + 2 * t;
+          if ((G & 1) == 0) *reinterpret_cast<float2 *>(dst) = make_float2(x[sl][j][0], x[sl][j][1]);
+          else {
+            dst[0] = x[sl][j][0];
+            if (2 * t + 1 < G) dst[1] = x[sl][j][1];
+          }
+        }
     }
     // Lazy rescaling: the reference m only moves when a logit would lift
     // exp(c (x - m)) above 2^8 (and sig when a V scale exceeds it); p <= 2^8
@@ -162,11 +187,15 @@ struct WarpAttn {
     // result equals an eager online softmax.  The common case costs one vote.
     const float cl = c * 1.44269504088896341f;  // exp(c x) = 2^(x cl)
     const float thr = 8.f / cl;
-    float mloc[2];
+    float mloc[2] = {-INFINITY, -INFINITY}, sloc = 0.f;
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
-      mloc[h] = fmaxf(ok[0] ? x[0][h] : -INFINITY, ok[1] ? x[1][h] : -INFINITY);
-    const float sloc = fmaxf(sv[0], sv[1]);
+    for (int sl = 0; sl < NSL; ++sl)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) mloc[h] = fmaxf(mloc[h], ok[sl][j] ? x[sl][j][h] : -INFINITY);
+        sloc = fmaxf(sloc, sv[sl][j]);
+      }
     const bool grow = mloc[0] > m[0] + thr || mloc[1] > m[1] + thr || (FP8 && sloc > sig);
     float alpha[2] = {1.f, 1.f};
     if (__any_sync(0xffffffffu, grow)) {
@@ -204,68 +233,86 @@ struct WarpAttn {
         }
       }
     }
-    float p[2][2];
+    uint32_t pb[NSL][2];  // P^T fragments: the transposed 8x8 halves (rows 0-7, 8-15 x heads)
+    float lsum[2] = {0.f, 0.f};
 #pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int h = 0; h < 2; ++h)  // the difference first: dominant terms exact
-        p[j][h] = ok[j] ? ex2_approx((x[j][h] - m[h]) * cl) : 0.f;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) l[h] = l[h] * alpha[h] + (p[0][h] + p[1][h]);
-    if constexpr (FP8) {
+    for (int sl = 0; sl < NSL; ++sl)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        const float w8 = sv[j] * inv_sig;
-        p[j][0] *= w8;
-        p[j][1] *= w8;
+        float p[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // the difference first: dominant terms exact
+          p[h] = ok[sl][j] ? ex2_approx((x[sl][j][h] - m[h]) * cl) : 0.f;
+          lsum[h] += p[h];
+        }
+        if constexpr (FP8) {
+          const float w8 = sv[sl][j] * inv_sig;
+          pb[sl][j] = movmatrix_t(pack_f16(p[0] * w8, p[1] * w8));
+        } else {
+          pb[sl][j] = movmatrix_t(pack_bf16(p[0], p[1]));
+        }
       }
-    }
-    // P^T fragment: transpose the 8x8 halves (rows 0-7 and 8-15 x heads)
-    const uint32_t pb0 = movmatrix_t(FP8 ? pack_f16(p[0][0], p[0][1]) : pack_bf16(p[0][0], p[0][1]));
-    const uint32_t pb1 = movmatrix_t(FP8 ? pack_f16(p[1][0], p[1][1]) : pack_bf16(p[1][0], p[1][1]));
+#pragma unroll
+    for (int h = 0; h < 2; ++h) l[h] = l[h] * alpha[h] + lsum[h];
 
-    // ---- O^T += V^T P^T (A rows 2t, 2t+1, 8+2t, 9+2t of the slice)
-    const bool full = vmask == 0xFFFFu;
-    const uint32_t v0 = (vmask >> (2 * t)) & 3u, v1 = (vmask >> (2 * t + 8)) & 3u;
+    // ---- O^T += V^T P^T (A rows 2t, 2t+1, 8+2t, 9+2t of each slice)
+    const bool full = vmask == (NSL == 2 ? 0xFFFFFFFFu : 0xFFFFu);
     if constexpr (!FP8) {
-      const uint32_t m01 = ((v0 & 1u) ? 0x0000FFFFu : 0u) | ((v0 & 2u) ? 0xFFFF0000u : 0u);
-      const uint32_t m23 = ((v1 & 1u) ? 0x0000FFFFu : 0u) | ((v1 & 2u) ? 0xFFFF0000u : 0u);
+      uint32_t m01[NSL], m23[NSL];
+#pragma unroll
+      for (int sl = 0; sl < NSL; ++sl) {
+        const uint32_t v0 = (vmask >> (16 * sl + 2 * t)) & 3u, v1 = (vmask >> (16 * sl + 2 * t + 8)) & 3u;
+        m01[sl] = ((v0 & 1u) ? 0x0000FFFFu : 0u) | ((v0 & 2u) ? 0xFFFF0000u : 0u);
+        m23[sl] = ((v1 & 1u) ? 0x0000FFFFu : 0u) | ((v1 & 2u) ? 0xFFFF0000u : 0u);
+      }
       const int row = row0 + (lane & 7) + ((lane >> 4) << 3);
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
         const int cb = (16 * mt + ((lane >> 3) & 1) * 8) * 2;
-        uint32_t a[4];
-        ldsm_x4_t(a, swz(vp + (cb >> 7) * pstride, row, (cb & 127) >> 4));
-        if (!full) {  // rows past the end may hold anything, NaN included
-          a[0] &= m01;
-          a[1] &= m01;
-          a[2] &= m23;
-          a[3] &= m23;
+#pragma unroll
+        for (int sl = 0; sl < NSL; ++sl) {
+          uint32_t a[4];
+          ldsm_x4_t(a, swz(vp + (cb >> 7) * pstride, row + 16 * sl, (cb & 127) >> 4));
+          if (!full) {  // rows past the end may hold anything, NaN included
+            a[0] &= m01[sl];
+            a[1] &= m01[sl];
+            a[2] &= m23[sl];
+            a[3] &= m23[sl];
+          }
+          mma_bf16(o[mt], a[0], a[1], a[2], a[3], pb[sl][0], pb[sl][1]);
         }
-        mma_bf16(o[mt], a[0], a[1], a[2], a[3], pb0, pb1);
       }
     } else {
-      uint32_t w0[4], w1[4], w2[4], w3[4];
-      lds128(w0, swz(vp, row0 + 2 * t, g));
-      lds128(w1, swz(vp, row0 + 2 * t + 1, g));
-      lds128(w2, swz(vp, row0 + 2 * t + 8, g));
-      lds128(w3, swz(vp, row0 + 2 * t + 9, g));
-      // byte masks: bytes 0,2 come from the even row, bytes 1,3 from the odd row
-      const uint32_t b01 = ((v0 & 1u) ? 0x00FF00FFu : 0u) | ((v0 & 2u) ? 0xFF00FF00u : 0u);
-      const uint32_t b23 = ((v1 & 1u) ? 0x00FF00FFu : 0u) | ((v1 & 2u) ? 0xFF00FF00u : 0u);
+      uint32_t vw[NSL][4][4];  // rows 2t, 2t+1, 2t+8, 2t+9 of each slice: chunk g
+      uint32_t b01[NSL], b23[NSL];
+#pragma unroll
+      for (int sl = 0; sl < NSL; ++sl) {
+        const int rb = row0 + 16 * sl + 2 * t;
+        lds128(vw[sl][0], swz(vp, rb, g));
+        lds128(vw[sl][1], swz(vp, rb + 1, g));
+        lds128(vw[sl][2], swz(vp, rb + 8, g));
+        lds128(vw[sl][3], swz(vp, rb + 9, g));
+        // byte masks: bytes 0,2 come from the even row, bytes 1,3 from the odd row
+        const uint32_t v0 = (vmask >> (16 * sl + 2 * t)) & 3u, v1 = (vmask >> (16 * sl + 2 * t + 8)) & 3u;
+        b01[sl] = ((v0 & 1u) ? 0x00FF00FFu : 0u) | ((v0 & 2u) ? 0xFF00FF00u : 0u);
+        b23[sl] = ((v1 & 1u) ? 0x00FF00FFu : 0u) | ((v1 & 2u) ? 0xFF00FF00u : 0u);
+      }
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
         const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
-        uint32_t x01 = prmt(w0[mt >> 1], w1[mt >> 1], sel);
-        uint32_t x23 = prmt(w2[mt >> 1], w3[mt >> 1], sel);
-        if (!full) {
-          x01 &= b01;
-          x23 &= b23;
+#pragma unroll
+        for (int sl = 0; sl < NSL; ++sl) {
+          uint32_t x01 = prmt(vw[sl][0][mt >> 1], vw[sl][1][mt >> 1], sel);
+          uint32_t x23 = prmt(vw[sl][2][mt >> 1], vw[sl][3][mt >> 1], sel);
+          if (!full) {
+            x01 &= b01[sl];
+            x23 &= b23[sl];
+          }
+          uint32_t a0, a1, a2, a3;
+          e4m3x4_to_f16x2x2(x01, a0, a1);
+          e4m3x4_to_f16x2x2(x23, a2, a3);
+          mma_f16(o[mt], a0, a1, a2, a3, pb[sl][0], pb[sl][1]);
         }
-        uint32_t a0, a1, a2, a3;
-        e4m3x4_to_f16x2x2(x01, a0, a1);
-        e4m3x4_to_f16x2x2(x23, a2, a3);
-        mma_f16(o[mt], a0, a1, a2, a3, pb0, pb1);
       }
     }
   }

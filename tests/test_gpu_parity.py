@@ -35,6 +35,8 @@ CASES = {
     "bf16_g2": spec(group=2, num_kv_heads=2, batch=2),
     "e4m3_paged64": spec(kv_dtype="e4m3", seq_len=(1500, 4000)),
     "e4m3_paged32_nanpad": spec(kv_dtype="e4m3", page_size=32, batch=2, seq_len=(1200, 2600)),
+    "e4m3_paged16": spec(kv_dtype="e4m3", page_size=16, batch=2, seq_len=(1100, 2700)),
+    "e4m3_contiguous_g4": spec(kv_dtype="e4m3", page_size=None, group=4, num_kv_heads=3, batch=2),
     "f32_tiny": synth.WORKLOADS["tiny_fp32_t2048"],
     "f32_paged_ragged": spec(kv_dtype="f32", q_dtype="f32", head_dim=64, group=4, page_size=16,
                              seq_len=(1200, 2500)),
@@ -183,3 +185,44 @@ def test_hybrid_block_step_runs_all_layers(oracle, lib):
     for layer in range(3):
         ref = U.run_oracle_sparse(oracle, w, w.q_sparse[layer], ora["idx"])
         U.check_out(outs[1 + layer], ref, "bf16", f"layer {layer}")
+
+
+def _scale_heads(q, G):
+    """Multiply query head h of every group by 2^(h - 3): exact in bf16, and the
+    heads of one group then need different power-of-two prescales."""
+    f = torch.tensor([2.0 ** (h % G - 3) for h in range(q.shape[-2])], dtype=torch.float32)
+    return (q.float() * f[:, None]).to(q.dtype)
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "e4m3"])
+def test_heads_of_unequal_magnitude(oracle, lib, kv_dtype):
+    sp = spec(kv_dtype=kv_dtype, batch=2, seq_len=(2000, 3000))
+    w = synth.generate(sp, seed=41)
+    w.q_full = _scale_heads(w.q_full, sp.group)
+    w.q_sparse = _scale_heads(w.q_sparse, sp.group)
+    ora = U.run_oracle(oracle, w)
+    wd = U.to_device(w)
+    out, idx = U.run_gpu(wd)
+    torch.cuda.synchronize()
+    U.check_full(wd, out, idx, ora)
+    g = U.run_gpu_sparse(wd, wd.q_sparse[0], torch.from_numpy(ora["idx"]).cuda())
+    U.check_out(g, U.run_oracle_sparse(oracle, w, w.q_sparse[0], ora["idx"]), kv_dtype, "sparse layer")
+
+
+# every built tensor-core configuration of the attention kernel: (ncw, nstage, nsl)
+FULL_CONFIGS = {
+    "bf16": ["8,3,1", "4,6,1", "4,3,2"],
+    "e4m3": ["8,3,2", "4,6,2", "16,3,1", "12,4,1", "8,6,1", "4,8,1"],
+}
+
+
+@pytest.mark.parametrize("kv_dtype,cfg", [(d, c) for d, cs in FULL_CONFIGS.items() for c in cs])
+def test_every_attention_config(oracle, lib, monkeypatch, kv_dtype, cfg):
+    sp = spec(kv_dtype=kv_dtype, batch=2, seq_len=(2500, 4100), page_size=None, sparse_layers=1)
+    w = synth.generate(sp, seed=7)
+    ora = U.run_oracle(oracle, w)
+    wd = U.to_device(w)
+    monkeypatch.setenv("HS2_FULL_CFG", cfg)
+    out, idx = U.run_gpu(wd)
+    torch.cuda.synchronize()
+    U.check_full(wd, out, idx, ora)
