@@ -6,7 +6,8 @@
 // One persistent CTA per SM walks a balanced share of the (sequence, kv head,
 // tile) space.  A producer warp streams K and V tiles with TMA bulk-tensor
 // loads into a ring of shared-memory stages (mbarrier full/empty pairs, every
-// wait bounded); consumer warps each take 16 rows of a tile, run Q K^T and
+// wait bounded); for E4M3 caches a second producer warp gathers the per-token
+// scales with cp.async at the same time; consumer warps each take 16 rows of a tile, run Q K^T and
 // V^T P^T on the tensor cores with an online softmax, and store the raw
 // logits that the score pass turns into group probabilities.  At the end of
 // each segment (a run of tiles of one unit inside one CTA) the consumer warps
@@ -104,8 +105,12 @@ __device__ __forceinline__ int find_seq(const int32_t *prefix, int B, int Hkv, i
   return lo;
 }
 
+// producer warps: TMA (+ stage metadata), and for E4M3 the scale gathers
+template <bool FP8>
+constexpr int kProducerWarps = FP8 ? 2 : 1;
+
 template <int D, bool FP8, int NCW, int NSTAGE, int NSL>
-__global__ void __launch_bounds__(32 * (NCW + 1), 1)
+__global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
     full_attn_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                          const FullParams p) {
   using C = Cfg<D, FP8, NCW, NSTAGE, NSL>;
@@ -119,7 +124,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
   int32_t *prefix = reinterpret_cast<int32_t *>(smem + C::OFF_PREFIX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool producer = warp == NCW;
+  const bool producer = warp >= NCW;
+  const bool tma_role = warp == NCW;  // the other producer warp (E4M3) gathers scales
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
@@ -129,15 +135,15 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
     mbar_init(cbar, (uint32_t)NCW);
     fence_mbar_init();
   }
-  if (producer && lane == 0) {
+  if (tma_role && lane == 0) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
   }
   griddep_wait();               // inputs and workspace are free from here on
   griddep_launch_dependents();  // the score kernel may be scheduled as SMs free up
-  if (producer) {
+  if (tma_role) {
     compute_prefix(p, prefix, C::TILE);
-  } else {
+  } else if (!producer) {
     zero_counters(p, threadIdx.x, NCW * 32);
   }
   __syncthreads();
@@ -150,24 +156,28 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
   const int64_t g0 = part.start(blockIdx.x), g1 = part.start(blockIdx.x + 1);
 
   if (producer) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producers
     // Boxes of RB rows (one page, or the whole tile when pages are larger).
     // Lane L caches the first slot of CTA-local box cache_base + L, so page
-    // table reads are issued 32 at a time instead of one per box.
+    // table reads are issued 32 at a time instead of one per box.  Both
+    // producer warps walk the same tiles; the (sequence, kv head, tile)
+    // coordinates advance incrementally.
     const int RB = p.page_table ? min(C::TILE, p.page_size) : C::TILE;
     const int BPT = C::TILE / RB;  // boxes per tile (<= 8)
     int64_t cache_base = -(int64_t)64;
     int my_slot = -1;
     int it = 0;
-    int b = g0 < g1 ? find_seq(prefix, p.B, p.Hkv, g0) : 0;
+    int b = 0, kvh = 0, i = 0, nb = 1, T = 0;
+    if (g0 < g1) {
+      b = find_seq(prefix, p.B, p.Hkv, g0);
+      nb = prefix[b + 1] - prefix[b];
+      const int64_t r = g0 - (int64_t)p.Hkv * prefix[b];
+      kvh = (int)(r / nb);
+      i = (int)(r % nb);
+      T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
+    }
     bool ok = true;
     for (int64_t g = g0; g < g1; ++g, ++it) {
-      while ((int64_t)p.Hkv * prefix[b + 1] <= g) ++b;
-      const int nb = prefix[b + 1] - prefix[b];
-      const int64_t r = g - (int64_t)p.Hkv * prefix[b];
-      const int kvh = (int)(r / nb), i = (int)(r % nb);
-      const int64_t U = (int64_t)p.Hkv * prefix[b] + (int64_t)kvh * nb;
-      const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
       const int64_t box0 = (g - g0) * BPT;
       if (box0 + BPT > cache_base + 32) {  // refill: lane L -> box box0 + L
         cache_base = box0;
@@ -191,66 +201,82 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
         ok = false;
         break;
       }
-      const int64_t j = blockIdx.x - part.cfirst(U);
-      const int64_t u = (int64_t)b * p.Hkv + kvh;
       const int p0 = i * C::TILE;
       const int cl0 = (int)(box0 - cache_base);  // cache lane of this tile's first box
-      if constexpr (FP8) {
-        float *ks = reinterpret_cast<float *>(smem + (size_t)stage * C::STAGE + 2 * C::KVB);
+      if (!tma_role) {
+        if constexpr (FP8) {  // per-token scales of the tile's rows
+          float *ks = reinterpret_cast<float *>(smem + (size_t)stage * C::STAGE + 2 * C::KVB);
 #pragma unroll
-        for (int k = 0; k < C::TILE / 32; ++k) {
-          const int rr = lane + 32 * k;
-          const int bs = __shfl_sync(0xffffffffu, my_slot, cl0 + rr / RB);
-          if (p0 + rr < T && bs >= 0) {
-            const int64_t slot = (int64_t)bs + rr % RB;
-            cp_async_4(smem_u32(ks + rr), p.k_scale + slot * p.Hkv + kvh);
-            cp_async_4(smem_u32(ks + C::TILE + rr), p.v_scale + slot * p.Hkv + kvh);
+          for (int k = 0; k < C::TILE / 32; ++k) {
+            const int rr = lane + 32 * k;
+            const int bs = __shfl_sync(0xffffffffu, my_slot, cl0 + rr / RB);
+            if (p0 + rr < T && bs >= 0) {
+              const int64_t slot = (int64_t)bs + rr % RB;
+              cp_async_4(smem_u32(ks + rr), p.k_scale + slot * p.Hkv + kvh);
+              cp_async_4(smem_u32(ks + C::TILE + rr), p.v_scale + slot * p.Hkv + kvh);
+            }
           }
+          cp_async_mbar_arrive_noinc(&full[stage]);
         }
-        cp_async_mbar_arrive_noinc(&full[stage]);
-      }
-      int box_slot[8];
+      } else {
+        int box_slot[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) box_slot[k] = __shfl_sync(0xffffffffu, my_slot, min(cl0 + k, 31));
-      if (lane == 0) {
-        StageMeta mt;
-        mt.b = b;
-        mt.kvh = kvh;
-        mt.tile = i;
-        mt.flags = ((i == 0 || g == g0) ? kFirst : 0) | ((i == nb - 1 || g == g1 - 1) ? kLast : 0);
-        mt.rec = (j >= 0 && j < p.R) ? (int)(u * p.R + j) : -1;
-        if (mt.rec < 0) set_error(p.ws.err, kErrRecord);
-        mt.T = T;
-        meta[stage] = mt;
-        uint32_t bytes = 0;
-        for (int k = 0; k < BPT && p0 + k * RB < T; ++k) bytes += 2u * RB * C::ROWB;
-        mbar_arrive_expect_tx(&full[stage], bytes);
-        const uint32_t kdst = sbase + stage * C::STAGE, vdst = kdst + C::KVB;
+        for (int k = 0; k < 8; ++k) box_slot[k] = __shfl_sync(0xffffffffu, my_slot, min(cl0 + k, 31));
+        if (lane == 0) {
+          const int64_t U = (int64_t)p.Hkv * prefix[b] + (int64_t)kvh * nb;  // first tile of the unit
+          const int64_t j = blockIdx.x - part.cfirst(U);
+          const int64_t u = (int64_t)b * p.Hkv + kvh;
+          StageMeta mt;
+          mt.b = b;
+          mt.kvh = kvh;
+          mt.tile = i;
+          mt.flags = ((i == 0 || g == g0) ? kFirst : 0) | ((i == nb - 1 || g == g1 - 1) ? kLast : 0);
+          mt.rec = (j >= 0 && j < p.R) ? (int)(u * p.R + j) : -1;
+          if (mt.rec < 0) set_error(p.ws.err, kErrRecord);
+          mt.T = T;
+          meta[stage] = mt;
+          const int nbox = min(BPT, (T - p0 + RB - 1) / RB);
+          mbar_arrive_expect_tx(&full[stage], (uint32_t)nbox * 2u * RB * C::ROWB);
+          const uint32_t kdst = sbase + stage * C::STAGE, vdst = kdst + C::KVB;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (k >= BPT || p0 + k * RB >= T) break;
-          // a slot outside the cache (bad page id) loads from row 2^31 - 1 .. : out of
-          // the tensor, so TMA fills zeros and the transfer still completes
-          const int slot = box_slot[k] >= 0 ? box_slot[k] : 0x7FFFFFFF - RB;
+          for (int k = 0; k < 8; ++k) {
+            if (k >= nbox) break;
+            // a slot outside the cache (bad page id) loads from row 2^31 - 1 .. : out of
+            // the tensor, so TMA fills zeros and the transfer still completes
+            const int slot = box_slot[k] >= 0 ? box_slot[k] : 0x7FFFFFFF - RB;
 #pragma unroll
-          for (int pn = 0; pn < C::NPANEL; ++pn) {
-            tma_load_3d(kdst + pn * C::PANEL + k * RB * 128, &tmk, &full[stage], pn * (128 / C::ES), kvh, slot);
-            tma_load_3d(vdst + pn * C::PANEL + k * RB * 128, &tmv, &full[stage], pn * (128 / C::ES), kvh, slot);
+            for (int pn = 0; pn < C::NPANEL; ++pn) {
+              tma_load_3d(kdst + pn * C::PANEL + k * RB * 128, &tmk, &full[stage], pn * (128 / C::ES), kvh, slot);
+              tma_load_3d(vdst + pn * C::PANEL + k * RB * 128, &tmv, &full[stage], pn * (128 / C::ES), kvh, slot);
+            }
           }
         }
       }
       __syncwarp();
+      // next tile: (b, kvh, i) in the order of the linear tile index
+      if (++i == nb) {
+        i = 0;
+        if (++kvh == p.Hkv) {
+          kvh = 0;
+          if (g + 1 < g1) {
+            do ++b; while (prefix[b + 1] == prefix[b]);  // sequences without tiles own none
+            nb = prefix[b + 1] - prefix[b];
+            T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
+          }
+        }
+      }
     }
     if (ok) {  // end-of-work sentinel
       const int stage = it % NSTAGE;
       if (it >= NSTAGE && !mbar_wait(&empty[stage], ((it / NSTAGE) - 1) & 1)) {
         set_error(p.ws.err, kErrEmptyWait);
-      } else {
+      } else if (tma_role) {
         if (lane == 0) {
           meta[stage].flags = kDone;
           mbar_arrive(&full[stage]);
         }
-        if constexpr (FP8) mbar_arrive(&full[stage]);
+      } else {
+        mbar_arrive(&full[stage]);  // the scale warp's 32 arrivals
       }
     }
     return;
@@ -432,7 +458,7 @@ cudaError_t launch_mma_t(const FullParams &p, const CUtensorMap &tmk, const CUte
   auto kern = full_attn_mma_kernel<D, FP8, NCW, NSTAGE, NSL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_ex(kern, dim3(grid), dim3(32 * (NCW + 1)), smem, s, 0, tmk, tmv, p);
+  return launch_ex(kern, dim3(grid), dim3(32 * (NCW + kProducerWarps<FP8>)), smem, s, 0, tmk, tmv, p);
 }
 
 }  // namespace
