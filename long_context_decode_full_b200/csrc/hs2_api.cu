@@ -297,6 +297,10 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
   p.R = L.R;
   p.c = 1.0f / sqrtf((float)D);
   p.ws = bind(L, workspace, B, Hkv);
+  {  // the logits this call writes, bounded by the sequence capacity: small next to the 126 MB L2?
+    const double logit_bytes = (double)B * Hkv * (double)t_cap * G * 4.0;
+    p.kv_evict_first = logit_bytes <= 48.0 * (1 << 20) ? 1 : 0;
+  }
   const int sms = sm_count();
   cudaError_t e;
   if (!mma) {

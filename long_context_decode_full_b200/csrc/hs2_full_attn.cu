@@ -238,6 +238,7 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
           const int nbox = min(BPT, (T - p0 + RB - 1) / RB);
           mbar_arrive_expect_tx(&full[stage], (uint32_t)nbox * 2u * RB * C::ROWB);
           const uint32_t kdst = sbase + stage * C::STAGE, vdst = kdst + C::KVB;
+          const uint64_t once = p.kv_evict_first ? l2_policy_evict_first() : l2_policy_evict_normal();
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             if (k >= nbox) break;
@@ -246,8 +247,10 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
             const int slot = box_slot[k] >= 0 ? box_slot[k] : 0x7FFFFFFF - RB;
 #pragma unroll
             for (int pn = 0; pn < C::NPANEL; ++pn) {
-              tma_load_3d(kdst + pn * C::PANEL + k * RB * 128, &tmk, &full[stage], pn * (128 / C::ES), kvh, slot);
-              tma_load_3d(vdst + pn * C::PANEL + k * RB * 128, &tmv, &full[stage], pn * (128 / C::ES), kvh, slot);
+              tma_load_3d_hint(kdst + pn * C::PANEL + k * RB * 128, &tmk, &full[stage], pn * (128 / C::ES), kvh,
+                               slot, once);
+              tma_load_3d_hint(vdst + pn * C::PANEL + k * RB * 128, &tmv, &full[stage], pn * (128 / C::ES), kvh,
+                               slot, once);
             }
           }
         }

@@ -26,6 +26,7 @@ struct FullParams {
   int32_t N;                 // persistent CTAs (grid size)
   int32_t R;                 // record slots per unit
   int32_t tile;              // positions per tile
+  int32_t kv_evict_first;    // K/V loads marked evict-first in L2 (when the logits fit in L2 beside them)
   float c;                   // 1/sqrt(D)
   FullWs ws;
 };

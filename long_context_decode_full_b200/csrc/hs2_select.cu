@@ -507,9 +507,15 @@ __device__ __forceinline__ int find_sub(const int *off, int n, int i) {
   return lo;
 }
 
+// Guard bands up to this size are ranked directly (each element against all
+// others, shared-memory broadcasts); larger ones take the radix select.
+constexpr int kRankSelectMax = 768;
+constexpr int kPerThread = kMaxSelect / kFinalThreads;  // list entries per thread, at most
+
 __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams p) {
   extern __shared__ int fsm[];  // off_a[nsub+1], off_e[nsub+1], list_a[kMaxSelect], list_c[kMaxSelect],
-                                // then the in-bin list (bits, position) when it fits: list_e[kMaxSelect]
+                                // slot_c[kMaxSelect], then the in-bin list (bits, position) when it
+                                // fits: list_e[kMaxSelect]
   __shared__ uint32_t sh_hist[2048];
   __shared__ int sh_warp[66], sh_res[2], sh_ties;
   griddep_wait();
@@ -522,8 +528,15 @@ __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams 
   int32_t *idx = p.idx_out + (size_t)u * L;
   const bool select = nC > p.k_global && p.k_global > 0;
   int *off_a = fsm, *off_e = fsm + p.nsub + 1;
-  int *list_a = fsm + 2 * (p.nsub + 1), *list_c = list_a + kMaxSelect;
-  uint2 *list_e = reinterpret_cast<uint2 *>(list_c + kMaxSelect);
+  int *list_a = fsm + 2 * (p.nsub + 1), *list_c = list_a + kMaxSelect, *slot_c = list_c + kMaxSelect;
+  uint2 *list_e = reinterpret_cast<uint2 *>(slot_c + kMaxSelect);
+  // the forced window's slots, looked up now and written last
+  int sw[kPerThread];
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    const int t = nC + threadIdx.x + k * kFinalThreads;
+    sw[k] = t < T ? (int)slot_of(p, b, t) : -1;
+  }
 
   int n_sel = 0;  // selectable positions kept (all before the window)
   if (select) {
@@ -535,6 +548,7 @@ __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams 
     // the above-threshold positions (fewer than k_global), already in order,
     // and the in-bin list when it fits, in one round of loads
     const bool e_in_smem = E <= kMaxSelect;
+    const bool rank_path = E <= kRankSelectMax;
     for (int i = threadIdx.x; i < A; i += blockDim.x) {
       const int s = find_sub(off_a, nsub, i);
       list_a[i] = __ldcg(above + (size_t)s * kSubRange + (i - off_a[s]));
@@ -545,67 +559,114 @@ __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams 
         list_e[i] = __ldcg(eqs_g + (size_t)s * kSubRange + (i - off_e[s]));
       }
     __syncthreads();
-    auto in_bin = [&](int i) -> uint2 {  // i-th guard-band element in position order
-      if (e_in_smem) return list_e[i];
-      const int s = find_sub(off_e, nsub, i);
-      return __ldcg(eqs_g + (size_t)s * kSubRange + (i - off_e[s]));
-    };
-    // radix select of the need-th largest exact score: bits 31..21, 20..10, 9..0
-    int need = p.k_global - A;
-    uint32_t prefix = 0u, mask = 0u;
-    const int shifts[3] = {21, 10, 0}, widths[3] = {11, 11, 10};
-    for (int round = 0; round < 3; ++round) {
-      const int sh = shifts[round], nb = 1 << widths[round];
-      for (int i = threadIdx.x; i < nb; i += blockDim.x) sh_hist[i] = 0u;
-      __syncthreads();
-      for (int i = threadIdx.x; i < E; i += blockDim.x) {
-        const uint32_t bits = in_bin(i).x;
-        if ((bits & mask) == prefix) atomicAdd(&sh_hist[(bits >> sh) & (nb - 1)], 1u);
-      }
-      __syncthreads();
-      int ab;
-      const int bin = find_threshold_bin(sh_hist, nb, need, &ab, sh_warp, sh_res);
-      need -= ab;
-      prefix |= (uint32_t)bin << sh;
-      mask |= (uint32_t)(nb - 1) << sh;
-      if (round == 2 && threadIdx.x == 0) sh_ties = (int)sh_hist[bin];  // elements equal to the k-th score
+    // output slots of the above list and of the guard band, in flight during the selection
+    int sa[kPerThread], se[2];
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int i = threadIdx.x + k * kFinalThreads;
+      sa[k] = i < A ? (int)slot_of(p, b, list_a[i]) : -1;
     }
-    __syncthreads();
-    const uint32_t kth = prefix;  // the exact k_global-th score; `need` of its ties are kept
-    const bool keep_all_ties = sh_ties <= need;
-    // walk the in-bin list in position order: keep scores above kth and the
-    // first `need` equal to it
-    int taken = 0, ties = 0;
-    for (int base = 0; base < E; base += blockDim.x) {
-      const int i = base + threadIdx.x;
-      const uint2 cv = i < E ? in_bin(i) : make_uint2(0u, 0u);
-      int take;
-      if (keep_all_ties) {
-        take = (i < E && cv.x >= kth) ? 1 : 0;
-      } else {
-        const int is_tie = (i < E && cv.x == kth) ? 1 : 0;
-        int tie_tot;
-        const int tie_rank = ties + block_exclusive_scan(is_tie, sh_warp, &tie_tot);
-        take = (i < E && (cv.x > kth || (is_tie && tie_rank < need))) ? 1 : 0;
-        ties += tie_tot;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int i = threadIdx.x + k * kFinalThreads;
+      se[k] = rank_path && i < E ? (int)slot_of(p, b, (int)list_e[i].y) : -1;
+    }
+    const int need = p.k_global - A;  // band elements to keep
+    int taken = 0;
+    if (rank_path) {
+      // element i (position order) is kept when fewer than `need` elements
+      // outrank it: a higher exact score, or an equal one at a lower position
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int i = threadIdx.x + k * kFinalThreads;
+        int take = 0;
+        if (i < E) {
+          const uint32_t si = list_e[i].x;
+          int r = 0;
+#pragma unroll 4
+          for (int j = 0; j < E; ++j) {
+            const uint32_t sj = list_e[j].x;
+            r += (sj > si) | ((sj == si) & (j < i));
+          }
+          take = r < need ? 1 : 0;
+        }
+        int tot;
+        const int pos = taken + block_exclusive_scan(take, sh_warp, &tot);
+        if (take) {
+          list_c[pos] = (int)list_e[i].y;
+          slot_c[pos] = se[k];
+        }
+        taken += tot;
       }
-      int take_tot;
-      const int pos = taken + block_exclusive_scan(take, sh_warp, &take_tot);
-      if (take && pos < kMaxSelect) list_c[pos] = (int)cv.y;
-      taken += take_tot;
+    } else {
+      auto in_bin = [&](int i) -> uint2 {  // i-th guard-band element in position order
+        if (e_in_smem) return list_e[i];
+        const int s = find_sub(off_e, nsub, i);
+        return __ldcg(eqs_g + (size_t)s * kSubRange + (i - off_e[s]));
+      };
+      // radix select of the need-th largest exact score: bits 31..21, 20..10, 9..0
+      int rem = need;
+      uint32_t prefix = 0u, mask = 0u;
+      const int shifts[3] = {21, 10, 0}, widths[3] = {11, 11, 10};
+      for (int round = 0; round < 3; ++round) {
+        const int sh = shifts[round], nb = 1 << widths[round];
+        for (int i = threadIdx.x; i < nb; i += blockDim.x) sh_hist[i] = 0u;
+        __syncthreads();
+        for (int i = threadIdx.x; i < E; i += blockDim.x) {
+          const uint32_t bits = in_bin(i).x;
+          if ((bits & mask) == prefix) atomicAdd(&sh_hist[(bits >> sh) & (nb - 1)], 1u);
+        }
+        __syncthreads();
+        int ab;
+        const int bin = find_threshold_bin(sh_hist, nb, rem, &ab, sh_warp, sh_res);
+        rem -= ab;
+        prefix |= (uint32_t)bin << sh;
+        mask |= (uint32_t)(nb - 1) << sh;
+        if (round == 2 && threadIdx.x == 0) sh_ties = (int)sh_hist[bin];  // elements equal to the k-th score
+      }
+      __syncthreads();
+      const uint32_t kth = prefix;  // the exact k_global-th score; `rem` of its ties are kept
+      const bool keep_all_ties = sh_ties <= rem;
+      // walk the in-bin list in position order: keep scores above kth and the
+      // first `rem` equal to it
+      int ties = 0;
+      for (int base = 0; base < E; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        const uint2 cv = i < E ? in_bin(i) : make_uint2(0u, 0u);
+        int take;
+        if (keep_all_ties) {
+          take = (i < E && cv.x >= kth) ? 1 : 0;
+        } else {
+          const int is_tie = (i < E && cv.x == kth) ? 1 : 0;
+          int tie_tot;
+          const int tie_rank = ties + block_exclusive_scan(is_tie, sh_warp, &tie_tot);
+          take = (i < E && (cv.x > kth || (is_tie && tie_rank < rem))) ? 1 : 0;
+          ties += tie_tot;
+        }
+        int take_tot;
+        const int pos = taken + block_exclusive_scan(take, sh_warp, &take_tot);
+        if (take && pos < kMaxSelect) {
+          list_c[pos] = (int)cv.y;
+          slot_c[pos] = (int)slot_of(p, b, cv.y);
+        }
+        taken += take_tot;
+      }
     }
     __syncthreads();
     // merge two position-ordered lists: rank = own index + smaller elements of the other list
     const int nc = min(taken, kMaxSelect);
     n_sel = A + nc;
-    for (int i = threadIdx.x; i < A; i += blockDim.x) {
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int i = threadIdx.x + k * kFinalThreads;
+      if (i >= A) break;
       const int v = list_a[i];
       int lo = 0, hi = nc;
       while (lo < hi) {
         const int mid = (lo + hi) >> 1;
         if (list_c[mid] < v) lo = mid + 1; else hi = mid;
       }
-      if (i + lo < L) idx[i + lo] = (int32_t)slot_of(p, b, v);
+      if (i + lo < L) idx[i + lo] = sa[k];
     }
     for (int i = threadIdx.x; i < nc; i += blockDim.x) {
       const int v = list_c[i];
@@ -614,16 +675,18 @@ __global__ void __launch_bounds__(kFinalThreads) final_kernel(const ScoreParams 
         const int mid = (lo + hi) >> 1;
         if (list_a[mid] < v) lo = mid + 1; else hi = mid;
       }
-      if (i + lo < L) idx[i + lo] = (int32_t)slot_of(p, b, v);
+      if (i + lo < L) idx[i + lo] = slot_c[i];
     }
   } else if (p.k_global > 0) {  // every selectable position is kept
     n_sel = nC;
     for (int t = threadIdx.x; t < nC && t < L; t += blockDim.x) idx[t] = (int32_t)slot_of(p, b, t);
   }
   // the forced window follows every selectable position
-  for (int t = nC + threadIdx.x; t < T; t += blockDim.x) {
+#pragma unroll
+  for (int k = 0; k < kPerThread; ++k) {
+    const int t = nC + threadIdx.x + k * kFinalThreads;
     const int o = n_sel + (t - nC);
-    if (o < L) idx[o] = (int32_t)slot_of(p, b, t);
+    if (t < T && o < L) idx[o] = sw[k];
   }
   const int n_total = n_sel + (T - nC);
   for (int i = n_total + threadIdx.x; i < L; i += blockDim.x) idx[i] = -1;
@@ -635,7 +698,7 @@ cudaError_t launch_score_g(const ScoreParams &p, dim3 grid, cudaStream_t s) {
   return launch_ex(score_kernel<G, 128>, grid, dim3(kScoreThreads), 0, s, 0, p);
 }
 
-size_t final_smem_bytes(int nsub) { return (size_t)(2 * (nsub + 1) + 4 * kMaxSelect) * sizeof(int); }
+size_t final_smem_bytes(int nsub) { return (size_t)(2 * (nsub + 1) + 5 * kMaxSelect) * sizeof(int); }
 
 }  // namespace
 

@@ -168,16 +168,17 @@ struct WarpAttn {
         }
       }
     if (logit_dst != nullptr && 2 * t < G) {
+      const uint64_t keep = l2_policy_evict_last();  // read back by the score pass
 #pragma unroll
       for (int sl = 0; sl < NSL; ++sl)
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           if (!ok[sl][j]) continue;
           float *dst = logit_dst + (16 * sl + 8 * j + g) * G + 2 * t;
-          if ((G & 1) == 0) *reinterpret_cast<float2 *>(dst) = make_float2(x[sl][j][0], x[sl][j][1]);
+          if ((G & 1) == 0) st_global_hint(dst, x[sl][j][0], x[sl][j][1], keep);
           else {
-            dst[0] = x[sl][j][0];
-            if (2 * t + 1 < G) dst[1] = x[sl][j][1];
+            st_global_hint(dst, x[sl][j][0], keep);
+            if (2 * t + 1 < G) st_global_hint(dst + 1, x[sl][j][1], keep);
           }
         }
     }
