@@ -190,6 +190,34 @@ __device__ void unit_lse(const float *rec0, const UnitInfo &ui, float c, double 
 }
 
 // ------------------------------------------------------------------ score
+// Loads the logits of positions tb + q * kScoreThreads (q < kScoreLoads) below t1.
+constexpr int kScoreLoads = 4;  // positions per thread in flight
+template <int G>
+__device__ __forceinline__ void load_logits(float (&raw)[kScoreLoads][G], const float *lg, int tb, int t1) {
+#pragma unroll
+  for (int q = 0; q < kScoreLoads; ++q) {
+    const int t = tb + q * kScoreThreads;
+    if (t >= t1) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) raw[q][h] = 0.f;
+      continue;
+    }
+    if constexpr (G % 4 == 0) {
+#pragma unroll
+      for (int h4 = 0; h4 < G / 4; ++h4) {
+        const float4 v4 = __ldcs(reinterpret_cast<const float4 *>(lg + (size_t)t * G) + h4);
+        raw[q][4 * h4] = v4.x;
+        raw[q][4 * h4 + 1] = v4.y;
+        raw[q][4 * h4 + 2] = v4.z;
+        raw[q][4 * h4 + 3] = v4.w;
+      }
+    } else {
+#pragma unroll
+      for (int h = 0; h < G; ++h) raw[q][h] = __ldcs(lg + (size_t)t * G + h);
+    }
+  }
+}
+
 template <int G, int D>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams p) {
   __shared__ uint32_t sh_hist[kHistBins];
@@ -206,8 +234,14 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   UnitInfo ui = unit_info(p, b, kvh);
   const int n_chunks = ui.select ? (ui.nC + kScoreChunk - 1) / kScoreChunk : 0;
   if (!combine && chunk >= n_chunks) return;
-  mark_records(ui, sh_ok);
   const int64_t u = (int64_t)b * p.Hkv + kvh;
+  const int t0 = chunk * kScoreChunk, t1 = min(ui.nC, t0 + kScoreChunk);
+  const float *lg = p.ws.logits + (size_t)u * p.ustride * G;
+  // the first batch of logits is in flight while the LSE is rebuilt
+  float raw[kScoreLoads][G];
+  if (!combine) load_logits<G>(raw, lg, t0 + threadIdx.x, t1);
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh_hist[i] = 0u;
+  mark_records(ui, sh_ok);
   const float *rec0 = p.ws.records + (size_t)u * p.R * RS;
   unit_lse<G, D>(rec0, ui, p.c, sh_lse, sh_M, sh_L, sh_red);
 
@@ -241,10 +275,6 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
     return;
   }
 
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh_hist[i] = 0u;
-  __syncthreads();
-  const int t0 = chunk * kScoreChunk, t1 = min(ui.nC, t0 + kScoreChunk);
-  const float *lg = p.ws.logits + (size_t)u * p.ustride * G;
   float *sc = p.ws.scores + (size_t)u * p.ustride;
   // approximate p_h = 2^(raw * a - b_h), a = c log2(e), b_h = LSE_h log2(e):
   // the exponent rounds once in fp32 (|x| < 64: absolute error < 4e-6), so
@@ -253,46 +283,23 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   float bh[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) bh[h] = (float)(sh_lse[h] * kLog2e);
-  constexpr int kUnroll = 4;  // positions per thread in flight
-  for (int t00 = t0 + threadIdx.x; t00 < t1; t00 += kUnroll * blockDim.x) {
-    float raw[kUnroll][G];
+  constexpr int kStep = kScoreLoads * kScoreThreads;
+  for (int tb = t0 + threadIdx.x; tb < t1; tb += kStep) {
+    if (tb > t0 + (int)threadIdx.x) load_logits<G>(raw, lg, tb, t1);  // (the first batch is loaded)
 #pragma unroll
-    for (int q = 0; q < kUnroll; ++q) {
-      const int t = t00 + q * blockDim.x;
-      if (t >= t1) {
+    for (int q = 0; q < kScoreLoads; ++q) {
+      const int t = tb + q * kScoreThreads;
+      if (t >= t1) break;
+      float pr[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) raw[q][h] = 0.f;
-        continue;
-      }
-      if constexpr (G % 4 == 0) {
+      for (int h = 0; h < G; ++h) pr[h] = ex2_approx(fmaf(raw[q][h], a, -bh[h]));
 #pragma unroll
-        for (int h4 = 0; h4 < G / 4; ++h4) {
-          const float4 v4 = __ldcs(reinterpret_cast<const float4 *>(lg + (size_t)t * G) + h4);
-          raw[q][4 * h4] = v4.x;
-          raw[q][4 * h4 + 1] = v4.y;
-          raw[q][4 * h4 + 2] = v4.z;
-          raw[q][4 * h4 + 3] = v4.w;
-        }
-      } else {
+      for (int w = 1; w < G; w <<= 1)  // pairwise sum of the group's probabilities
 #pragma unroll
-        for (int h = 0; h < G; ++h) raw[q][h] = __ldcs(lg + (size_t)t * G + h);
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < kUnroll; ++q) {
-    const int t = t00 + q * blockDim.x;
-    if (t >= t1) break;
-    float pr[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) pr[h] = ex2_approx(fmaf(raw[q][h], a, -bh[h]));
-    // pairwise sum of the group's probabilities
-#pragma unroll
-    for (int w = 1; w < G; w <<= 1)
-#pragma unroll
-      for (int h = 0; h + w < G; h += 2 * w) pr[h] += pr[h + w];
-    const float s = pr[0] >= 0.f ? pr[0] : 0.f;  // NaN (bad inputs) ranks lowest
-    sc[t] = s;
-    atomicAdd(&sh_hist[__float_as_uint(s) >> kHistShift], 1u);
+        for (int h = 0; h + w < G; h += 2 * w) pr[h] += pr[h + w];
+      const float s = pr[0] >= 0.f ? pr[0] : 0.f;  // NaN (bad inputs) ranks lowest
+      sc[t] = s;
+      atomicAdd(&sh_hist[__float_as_uint(s) >> kHistShift], 1u);
     }
   }
   __syncthreads();
@@ -345,42 +352,35 @@ __device__ __forceinline__ float exact_score(const float *raw, int G, float c, c
 }
 
 // ------------------------------------------------------------------ filter
-__global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams p) {
-  __shared__ int sh_band[kScoreThreads / 32][kSubRange];  // each warp's guard-band positions
-  griddep_wait();
-  griddep_launch_dependents();
-  const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
-  const int nC = max(0, T - p.window);
-  if (nC <= p.k_global || p.k_global == 0 || chunk * kFilterChunk >= nC) return;
-  const int64_t u = (int64_t)b * p.Hkv + kvh;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int sub = chunk * (kFilterChunk / kSubRange) + warp;  // this warp's sub-range
+constexpr int kFilterRounds = kSubRange / 128;
+constexpr int kFilterSubs = kFilterChunk / (kSubRange * (kScoreThreads / 32));  // sub-ranges per warp
+
+// Lane l of round r holds positions s0 + 128 r + 4 l .. +3 (one float4) of
+// sub-range `sub`, so (round, lane, element) order is position order.
+__device__ __forceinline__ void load_sub_scores(const float *sc, int sub, int nC, float4 (&v)[kFilterRounds]) {
+  const int lane = threadIdx.x & 31;
   const int s0 = sub * kSubRange, s1 = min(nC, s0 + kSubRange);
-  if (s0 >= nC) return;
-  const float *sc = p.ws.scores + (size_t)u * p.ustride;
-  int32_t *above = p.ws.above + (size_t)u * p.ustride + s0;
-  uint2 *eqs = p.ws.cand + (size_t)u * p.ustride + s0;
-  // lane l of round r holds positions s0 + 128 r + 4 l .. +3 (one float4), so
-  // (round, lane, element) order is position order
-  constexpr int kRounds = kSubRange / 128;
-  float4 v[kRounds];
 #pragma unroll
-  for (int r = 0; r < kRounds; ++r) {
+  for (int r = 0; r < kFilterRounds; ++r) {
     const int t = s0 + 128 * r + 4 * lane;
     v[r] = t + 3 < s1 ? __ldcs(reinterpret_cast<const float4 *>(sc + t))
                       : make_float4(t < s1 ? sc[t] : 0.f, t + 1 < s1 ? sc[t + 1] : 0.f,
                                     t + 2 < s1 ? sc[t + 2] : 0.f, 0.f);
   }
-  // The k-th exact score lies in the threshold bin [lo, hi) widened by the
-  // approximation error (< 2e-5 relative even for logits of several hundred);
-  // the band keeps a 4e-4 margin on both sides.
-  const int bin1 = p.ws.thr[u].x;
-  const float lo = __uint_as_float((uint32_t)bin1 << kHistShift) * (1.f - kBandMargin);
-  const float hi = bin1 >= 0x7F7 ? INFINITY : __uint_as_float((uint32_t)(bin1 + 1) << kHistShift) * (1.f + kBandMargin);
+}
+
+// One warp, one 512-position sub-range: writes, in position order, the
+// positions certainly above the k-th exact score and the guard band (with
+// exact scores), and the two counts.
+__device__ void filter_sub(const ScoreParams &p, int64_t u, int sub, int nC, float lo, float hi,
+                           const float4 (&v)[kFilterRounds], int *band, const double *lse) {
+  const int lane = threadIdx.x & 31;
+  const int s0 = sub * kSubRange, s1 = min(nC, s0 + kSubRange);
+  int32_t *above = p.ws.above + (size_t)u * p.ustride + s0;
+  uint2 *eqs = p.ws.cand + (size_t)u * p.ustride + s0;
   int na = 0, ne = 0;
 #pragma unroll
-  for (int r = 0; r < kRounds; ++r) {
+  for (int r = 0; r < kFilterRounds; ++r) {
     const int t = s0 + 128 * r + 4 * lane;
     const float f[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
     int ca = 0, ce = 0;
@@ -388,8 +388,8 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const bool valid = t + k < s1;
-      a[k] = valid && f[k] >= hi;                // certainly above the k-th exact score
-      e[k] = valid && f[k] >= lo && f[k] < hi;   // guard band
+      a[k] = valid && f[k] >= hi;               // certainly above the k-th exact score
+      e[k] = valid && f[k] >= lo && f[k] < hi;  // guard band
       ca += a[k];
       ce += e[k];
     }
@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       if (a[k]) above[oa++] = t + k;
-      if (e[k]) sh_band[warp][oe++] = t + k;
+      if (e[k]) band[oe++] = t + k;
     }
     na += ta;
     ne += te;
@@ -416,17 +416,49 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
   // guard band: exact scores, the whole warp working through the list with
   // every load in flight together
   __syncwarp();
-  if (ne > 0) {
-    double lse[8];
-#pragma unroll
-    for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.lse[u * 8 + h] : 0.0;
-    for (int i = lane; i < ne; i += 32) {
-      const int pos = sh_band[warp][i];
-      const float ex = exact_score(p.ws.logits + ((size_t)u * p.ustride + pos) * p.G, p.G, p.c, lse);
-      eqs[i] = make_uint2(__float_as_uint(ex), (uint32_t)pos);
-    }
+  for (int i = lane; i < ne; i += 32) {
+    const int pos = band[i];
+    const float ex = exact_score(p.ws.logits + ((size_t)u * p.ustride + pos) * p.G, p.G, p.c, lse);
+    eqs[i] = make_uint2(__float_as_uint(ex), (uint32_t)pos);
   }
+  __syncwarp();
   if (lane == 0) p.ws.subcnt[(size_t)u * p.nsub + sub] = make_int2(na, ne);
+}
+
+// Each warp owns kFilterSubs sub-ranges (strided by the CTA's warps), with
+// the scores of all of them loaded up front.
+__global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams p) {
+  __shared__ int sh_band[kScoreThreads / 32][kSubRange];  // each warp's guard-band positions
+  griddep_wait();
+  griddep_launch_dependents();
+  const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
+  const int nC = max(0, T - p.window);
+  if (nC <= p.k_global || p.k_global == 0 || chunk * kFilterChunk >= nC) return;
+  const int64_t u = (int64_t)b * p.Hkv + kvh;
+  const int warp = threadIdx.x >> 5;
+  constexpr int kWarps = kScoreThreads / 32;
+  const float *sc = p.ws.scores + (size_t)u * p.ustride;
+  const int sub0 = chunk * (kFilterChunk / kSubRange) + warp;
+  float4 v[kFilterSubs][kFilterRounds];
+#pragma unroll
+  for (int k = 0; k < kFilterSubs; ++k)
+    if ((sub0 + k * kWarps) * kSubRange < nC) load_sub_scores(sc, sub0 + k * kWarps, nC, v[k]);
+  // The k-th exact score lies in the threshold bin [lo, hi) widened by the
+  // approximation error (< 2e-5 relative even for logits of several hundred);
+  // the band keeps a 4e-4 margin on both sides.
+  const int bin1 = p.ws.thr[u].x;
+  const float lo = __uint_as_float((uint32_t)bin1 << kHistShift) * (1.f - kBandMargin);
+  const float hi = bin1 >= 0x7F7 ? INFINITY : __uint_as_float((uint32_t)(bin1 + 1) << kHistShift) * (1.f + kBandMargin);
+  double lse[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.lse[u * 8 + h] : 0.0;
+#pragma unroll
+  for (int k = 0; k < kFilterSubs; ++k) {
+    const int sub = sub0 + k * kWarps;
+    if (sub * kSubRange >= nC) break;
+    filter_sub(p, u, sub, nC, lo, hi, v[k], sh_band[warp], lse);
+  }
 }
 
 // ------------------------------------------------------------------ final
