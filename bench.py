@@ -14,6 +14,7 @@ Prints one JSON line (rank 0).  Under torchrun every rank runs its own replica
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -56,6 +57,31 @@ def algorithmic_bytes(w: synth.Workload):
     qo = s.batch * s.num_q_heads * s.head_dim * ES[s.q_dtype] * 2
     return {"full_attention": kv, "full_layer": kv + scores + qo, "sparse_layer": rows + qo,
             "step": kv + scores + qo + s.sparse_layers * (rows + qo)}
+
+
+ATTN_SOURCES = ("hs2_full_attn.cu", "hs2_warp_attn.cuh", "hs2_common.cuh")
+
+
+def attention_source_hash():
+    h = hashlib.sha256()
+    for name in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "long_context_decode_full_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload):
+    """DRAM bytes (read + write) of one attention launch from the committed ncu
+    capture, or None when there is none for this workload or the kernel's
+    sources changed since it was taken."""
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(tpath):
+        return None
+    with open(tpath) as f:
+        t = json.load(f)
+    if t.get("kernel_source_sha256") != attention_source_hash():
+        return None
+    return t.get("bytes_per_launch", {}).get(workload)
 
 
 class Clocks:
@@ -271,11 +297,7 @@ def run_gpu(args, rank, world, local):
     peak, peak_kind = peaks()
     attn_gbs = ab["full_attention"] / (attn_ms * 1e-3) / 1e9
     step_gbs = ab["step"] / (ms_step * 1e-3) / 1e9
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            traffic = json.load(f).get(args.workload)
+    traffic = measured_traffic(args.workload)
     res = {
         "metric": METRIC,
         "value": world * 1000.0 / ms_step,

@@ -347,6 +347,12 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
   sp.R = p.R;
   sp.tile = p.tile;
   sp.nsub = L.nsub;
+  {  // one wave of the selection kernels over the whole capacity
+    const double positions = (double)B * Hkv * (double)t_cap;
+    sp.score_chunk = 2048;  // about 4 score CTAs per SM (their register budget)
+    while (sp.score_chunk < 65536 && positions / sp.score_chunk > 4.0 * sms) sp.score_chunk *= 2;
+    sp.filter_subs = positions / 4096.0 > 5.0 * sms ? 2 : 1;  // 8 warps x 512 positions per sub-range
+  }
   sp.c = p.c;
   sp.ws = p.ws;
   e = launch_select(sp, s);

@@ -17,8 +17,6 @@ namespace hs2 {
 // ---------------------------------------------------------------- constants
 constexpr int kHistBins = 4096;          // score histogram: float bits 30..19
 constexpr int kHistShift = 19;
-constexpr int kScoreChunk = 8192;        // positions per score CTA
-constexpr int kFilterChunk = 8192;       // positions per filter CTA (8 warps x 2 x 512)
 constexpr int kScoreThreads = 256;
 constexpr int kFinalThreads = 512;
 constexpr long long kSpinLimitCycles = 4000000000LL;  // ~2 s at 2 GHz

@@ -44,6 +44,8 @@ struct ScoreParams {
   int32_t window, k_global;
   int32_t N, R, tile;
   int32_t nsub;              // 512-position lists per unit: ceil(t_cap / 512)
+  int32_t score_chunk;       // positions per score CTA (a power of two, 2048 .. 65536)
+  int32_t filter_subs;       // 512-position sub-ranges per filter warp (1 or 2)
   float c;
   FullWs ws;
 };

@@ -232,10 +232,10 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const bool combine = chunk == (int)gridDim.x - 1;  // the unit's combine CTA
   UnitInfo ui = unit_info(p, b, kvh);
-  const int n_chunks = ui.select ? (ui.nC + kScoreChunk - 1) / kScoreChunk : 0;
+  const int n_chunks = ui.select ? (ui.nC + p.score_chunk - 1) / p.score_chunk : 0;
   if (!combine && chunk >= n_chunks) return;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
-  const int t0 = chunk * kScoreChunk, t1 = min(ui.nC, t0 + kScoreChunk);
+  const int t0 = chunk * p.score_chunk, t1 = min(ui.nC, t0 + p.score_chunk);
   const float *lg = p.ws.logits + (size_t)u * p.ustride * G;
   // the first batch of logits is in flight while the LSE is rebuilt
   float raw[kScoreLoads][G];
@@ -353,7 +353,7 @@ __device__ __forceinline__ float exact_score(const float *raw, int G, float c, c
 
 // ------------------------------------------------------------------ filter
 constexpr int kFilterRounds = kSubRange / 128;
-constexpr int kFilterSubs = kFilterChunk / (kSubRange * (kScoreThreads / 32));  // sub-ranges per warp
+constexpr int kFilterSubsMax = 2;  // sub-ranges per warp (p.filter_subs <= this)
 
 // Lane l of round r holds positions s0 + 128 r + 4 l .. +3 (one float4) of
 // sub-range `sub`, so (round, lane, element) order is position order.
@@ -425,7 +425,7 @@ __device__ void filter_sub(const ScoreParams &p, int64_t u, int sub, int nC, flo
   if (lane == 0) p.ws.subcnt[(size_t)u * p.nsub + sub] = make_int2(na, ne);
 }
 
-// Each warp owns kFilterSubs sub-ranges (strided by the CTA's warps), with
+// Each warp owns p.filter_subs sub-ranges (strided by the CTA's warps), with
 // the scores of all of them loaded up front.
 __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams p) {
   __shared__ int sh_band[kScoreThreads / 32][kSubRange];  // each warp's guard-band positions
@@ -434,16 +434,17 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
   const int nC = max(0, T - p.window);
-  if (nC <= p.k_global || p.k_global == 0 || chunk * kFilterChunk >= nC) return;
+  const int fchunk = kSubRange * (kScoreThreads / 32) * p.filter_subs;  // positions per CTA
+  if (nC <= p.k_global || p.k_global == 0 || chunk * fchunk >= nC) return;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
   const int warp = threadIdx.x >> 5;
   constexpr int kWarps = kScoreThreads / 32;
   const float *sc = p.ws.scores + (size_t)u * p.ustride;
-  const int sub0 = chunk * (kFilterChunk / kSubRange) + warp;
-  float4 v[kFilterSubs][kFilterRounds];
+  const int sub0 = chunk * (fchunk / kSubRange) + warp;
+  float4 v[kFilterSubsMax][kFilterRounds];
 #pragma unroll
-  for (int k = 0; k < kFilterSubs; ++k)
-    if ((sub0 + k * kWarps) * kSubRange < nC) load_sub_scores(sc, sub0 + k * kWarps, nC, v[k]);
+  for (int k = 0; k < kFilterSubsMax; ++k)
+    if (k < p.filter_subs && (sub0 + k * kWarps) * kSubRange < nC) load_sub_scores(sc, sub0 + k * kWarps, nC, v[k]);
   // The k-th exact score lies in the threshold bin [lo, hi) widened by the
   // approximation error (< 2e-5 relative even for logits of several hundred);
   // the band keeps a 4e-4 margin on both sides.
@@ -454,9 +455,9 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
 #pragma unroll
   for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.lse[u * 8 + h] : 0.0;
 #pragma unroll
-  for (int k = 0; k < kFilterSubs; ++k) {
+  for (int k = 0; k < kFilterSubsMax; ++k) {
     const int sub = sub0 + k * kWarps;
-    if (sub * kSubRange >= nC) break;
+    if (k >= p.filter_subs || sub * kSubRange >= nC) break;
     filter_sub(p, u, sub, nC, lo, hi, v[k], sh_band[warp], lse);
   }
 }
@@ -735,7 +736,7 @@ size_t final_smem_bytes(int nsub) { return (size_t)(2 * (nsub + 1) + 5 * kMaxSel
 }  // namespace
 
 cudaError_t launch_select(const ScoreParams &p, cudaStream_t s) {
-  const int chunks = (int)((p.t_cap + kScoreChunk - 1) / kScoreChunk);
+  const int chunks = (int)((p.t_cap + p.score_chunk - 1) / p.score_chunk);
   cudaError_t e;
   const dim3 sgrid(chunks + 1, p.Hkv, p.B);  // + the combine CTA of each unit
   switch (p.G) {
@@ -746,7 +747,8 @@ cudaError_t launch_select(const ScoreParams &p, cudaStream_t s) {
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
-  const int fchunks = (int)((p.t_cap + kFilterChunk - 1) / kFilterChunk);
+  const int fchunk = kSubRange * (kScoreThreads / 32) * p.filter_subs;
+  const int fchunks = (int)((p.t_cap + fchunk - 1) / fchunk);
   e = launch_ex(filter_kernel, dim3(fchunks, p.Hkv, p.B), dim3(kScoreThreads), 0, s, 0, p);
   if (e != cudaSuccess) return e;
   const size_t smem = final_smem_bytes(p.nsub);
