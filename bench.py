@@ -181,20 +181,32 @@ def oracle_unit_seconds(w: synth.Workload, b: int, kvh: int):
     return time.perf_counter() - t0, 1
 
 
-def cpu_baseline(w: synth.Workload, units: int = 1):
-    """Oracle steps/s estimated from `units` timed (sequence, kv head) units."""
+def workload_config(w: synth.Workload, world: int):
+    s = w.spec
+    return {"workload": s.name, "batch": s.batch, "seq_len": s.seq_len, "num_kv_heads": s.num_kv_heads,
+            "gqa_group": s.group, "head_dim": s.head_dim, "kv_dtype": s.kv_dtype, "page_size": s.page_size,
+            "sparse_layers": s.sparse_layers, "window": s.window, "k_global": s.k_global,
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2: %.2f GB of K/V read per step, no flush"
+                  % (algorithmic_bytes(w)["full_attention"] / 1e9)}
+
+
+def cpu_baseline(w: synth.Workload, seconds: float = 10.0, max_units: int = 256):
+    """Oracle steps/s from timed (sequence, kv head) units, cycling over the
+    step's units until about `seconds` of oracle time has been measured."""
     s = w.spec
     total_units = s.batch * s.num_kv_heads
-    secs = 0.0
-    for i in range(units):
-        b, kvh = divmod(i, s.num_kv_heads)
-        t, threads = oracle_unit_seconds(w, b % s.batch, kvh)
+    secs, n, threads = 0.0, 0, 1
+    while n < max_units and (secs < seconds or n == 0):
+        b, kvh = divmod(n % total_units, s.num_kv_heads)
+        t, threads = oracle_unit_seconds(w, b, kvh)
         secs += t
-    per_step = secs / units * total_units
+        n += 1
+    per_step = secs / n * total_units
     return {"value": 1.0 / per_step, "unit": "steps/s", "cores": threads, "kind": "oracle",
-            "sample": f"{units} of {total_units} (sequence, kv head) units of one step (full layer + selection + "
-                      f"{s.sparse_layers} sparse layers), fp64 single-threaded C; step time = unit time x "
-                      f"{total_units}", "seconds_measured": secs}
+            "sample": f"{n} unit evaluations cycling over the {total_units} (sequence, kv head) units of one step "
+                      f"(full layer + selection + {s.sparse_layers} sparse layers), fp64 single-threaded C; "
+                      f"step time = mean unit time x {total_units}", "seconds_measured": secs}
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -311,11 +323,7 @@ def run_gpu(args, rank, world, local):
         "vs_baseline": None,
         "dtype": {"bf16": "bf16", "e4m3": "e4m3", "f32": "f32"}[s.kv_dtype],
         "data": "synthetic",
-        "config": {"workload": s.name, "batch": s.batch, "seq_len": s.seq_len, "num_kv_heads": s.num_kv_heads,
-                   "gqa_group": s.group, "head_dim": s.head_dim, "kv_dtype": s.kv_dtype, "page_size": s.page_size,
-                   "sparse_layers": s.sparse_layers, "window": s.window, "k_global": s.k_global,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2: %.2f GB of K/V read per step, no flush" % (ab["full_attention"] / 1e9)},
+        "config": workload_config(w, world),
         "roofline": {"bound": "hbm", "kernel": "full_attn_mma_kernel", "achieved": attn_gbs, "peak": peak,
                      "unit": "GB/s", "frac": attn_gbs / peak, "traffic": traffic,
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
@@ -332,7 +340,7 @@ def run_gpu(args, rank, world, local):
         "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(w, args.cpu_units)
+        res["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     return res
 
 
@@ -354,8 +362,7 @@ def run_reference(args, rank, world, local):
     return {"metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": spec.name, "batch": spec.batch, "seq_len": spec.seq_len,
-                       "parallelism": "oracle on host cores"},
+            "config": workload_config(w, world),
             "cpu_baseline": {"value": v, "unit": "steps/s", "cores": threads, "kind": "oracle",
                              "sample": "each step = one (sequence, kv head) unit of the workload (full layer + "
                                        "selection + sparse layers) timed and scaled by the unit count"},
@@ -371,7 +378,7 @@ def main():
     ap.add_argument("--impl", default="hs2", choices=["hs2", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=500)
-    ap.add_argument("--cpu-units", type=int, default=1)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for the CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's context (profiling runs)")
     ap.add_argument("--kv-heads", type=int, default=0, help="override the workload's KV heads (experiments)")
