@@ -8,8 +8,8 @@
 // index list: every warp gathers 16 listed rows of K and V (whole rows,
 // 16-byte cp.async into the swizzled tile layout), runs the tensor-core
 // attention step for the G query heads of the group, the CTA merges its
-// warps, and CTA 0 of the cluster merges the CTAs through distributed shared
-// memory and writes the output.  No workspace, no atomics, one launch.
+// warps, and the CTAs merge through distributed shared memory, each writing
+// its share of the output elements.  No workspace, no atomics, one launch.
 #include <cooperative_groups.h>
 
 #include "hs2_internal.h"
@@ -34,18 +34,15 @@ struct SCfg {
   // one CTA's partial record m[G], l[G], o[G][D], padded to whole float4s
   __host__ __device__ static int rec_floats(int G) { return (G * (D + 2) + 3) & ~3; }
   __host__ __device__ static size_t staging(int nbuf) { return (size_t)kSparseWarps * nbuf * BUF_BYTES; }
-  // the warps' merge scratch and CTA 0's gathered partials reuse the staging
-  // buffers (idle by then) when they fit, else get a region of their own
-  __host__ __device__ static size_t scratch_bytes(int G, int S) {
-    const size_t a = (size_t)kSparseWarps * WSTRIDE * 4, b = (size_t)S * rec_floats(G) * 4;
-    return a > b ? a : b;
-  }
+  // the warps' merge scratch reuses the staging buffers (idle by then) when
+  // it fits, else gets a region of their own
+  __host__ __device__ static size_t scratch_bytes(int, int) { return (size_t)kSparseWarps * WSTRIDE * 4; }
   __host__ __device__ static bool scratch_in_staging(int G, int S, int nbuf) {
     return scratch_bytes(G, S) <= staging(nbuf);
   }
   static size_t bytes(int G, int S, int rows, int nbuf) {
     return 128 + staging(nbuf) + (scratch_in_staging(G, S, nbuf) ? 0 : scratch_bytes(G, S)) +
-           (size_t)rec_floats(G) * 4 + (size_t)(S + 1) * 8 * 4 + (size_t)rows * 4;
+           (size_t)rec_floats(G) * 4 + (size_t)(3 * S + 1) * 8 * 4 + (size_t)rows * 4;
   }
 };
 
@@ -74,11 +71,11 @@ __global__ void __launch_bounds__(32 * kSparseWarps, 1) sparse_mma_kernel(const 
   const bool in_staging = C::scratch_in_staging(p.G, S, nbuf);
   uint8_t *after = smem + C::staging(nbuf) + (in_staging ? 0 : C::scratch_bytes(p.G, S));
   float *scratch = reinterpret_cast<float *>(in_staging ? smem : smem + C::staging(nbuf));
-  float *gathered = scratch;                                     // CTA 0, after the warp merge
   float *partial = reinterpret_cast<float *>(after);             // m[G], l[G], o[G][D] of this CTA
-  float *wts = partial + RSP;                                    // CTA 0: weight of (CTA, head)
-  float *inv_l = wts + S * 8;                                    // CTA 0: 1 / normaliser per head
-  int *slots = reinterpret_cast<int *>(inv_l + 8);               // this CTA's index entries
+  float *wts = partial + RSP;                                    // weight of (CTA, head)
+  float *inv_l = wts + S * 8;                                    // 1 / normaliser per head
+  float *ms_ = inv_l + 8, *ls_ = ms_ + S * 8;                    // (m, l) of (CTA, head)
+  int *slots = reinterpret_cast<int *>(ls_ + S * 8);             // this CTA's index entries
   const int rank = (int)cluster.block_rank();
   const int kvh = blockIdx.y, b = blockIdx.z, G = p.G;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
@@ -164,38 +161,42 @@ __global__ void __launch_bounds__(32 * kSparseWarps, 1) sparse_mma_kernel(const 
   st.store(scr, scr + 8, scr + 16);
   __syncthreads();
   merge_warp_states<D>(scratch, C::WSTRIDE, kSparseWarps, G, p.c, partial, threadIdx.x, blockDim.x);
-  cluster.sync();
-  if (rank == 0) {
-    // one parallel copy of every CTA's partial into local shared memory
-    const int n4 = S * (RSP >> 2);
-    for (int i = threadIdx.x; i < n4; i += blockDim.x) {
-      const int r = i / (RSP >> 2), o = i - r * (RSP >> 2);
-      reinterpret_cast<float4 *>(gathered)[i] = reinterpret_cast<const float4 *>(cluster.map_shared_rank(partial, r))[o];
+  cluster.sync();  // every CTA's partial is complete
+  // every CTA writes its share of the G x D outputs: the (m, l) pairs of all
+  // partials (one per thread), the heads' weights, then its elements with the
+  // partials' o read straight from the other CTAs' shared memory
+  if (threadIdx.x < S * 8) {
+    const int r = threadIdx.x >> 3, h = threadIdx.x & 7;
+    const float *pr = cluster.map_shared_rank(partial, r);
+    ms_[threadIdx.x] = h < G ? pr[h] : -INFINITY;
+    ls_[threadIdx.x] = h < G ? pr[G + h] : 0.f;
+  }
+  __syncthreads();
+  if (threadIdx.x < G) {
+    const int h = threadIdx.x;
+    float M = -INFINITY;
+    for (int r = 0; r < S; ++r) M = fmaxf(M, ms_[r * 8 + h]);
+    float L = 0.f;
+    for (int r = 0; r < S; ++r) {
+      const float mr = ms_[r * 8 + h];
+      const float w = mr == -INFINITY ? 0.f : expf(p.c * (mr - M));
+      wts[r * 8 + h] = w;
+      L += w * ls_[r * 8 + h];
     }
-    __syncthreads();
-    if (threadIdx.x < G) {
-      const int h = threadIdx.x;
-      float M = -INFINITY;
-      for (int r = 0; r < S; ++r) M = fmaxf(M, gathered[r * RSP + h]);
-      float L = 0.f;
-      for (int r = 0; r < S; ++r) {
-        const float mr = gathered[r * RSP + h];
-        const float w = mr == -INFINITY ? 0.f : expf(p.c * (mr - M));
-        wts[r * 8 + h] = w;
-        L += w * gathered[r * RSP + G + h];
-      }
-      inv_l[h] = L > 0.f ? 1.f / L : 0.f;
-    }
-    __syncthreads();
+    inv_l[h] = L > 0.f ? 1.f / L : 0.f;
+  }
+  __syncthreads();
+  {
+    const int per = (G * D + S - 1) / S, e0 = rank * per, e1 = min(G * D, e0 + per);
     const int64_t ob = ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
-    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+    for (int e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
       const int h = e / D;
       float acc = 0.f;
-      for (int r = 0; r < S; ++r) acc += wts[r * 8 + h] * gathered[r * RSP + 2 * G + e];
+      for (int r = 0; r < S; ++r) acc += wts[r * 8 + h] * cluster.map_shared_rank(partial, r)[2 * G + e];
       static_cast<__nv_bfloat16 *>(p.out)[ob + e] = __float2bfloat16_rn(acc * inv_l[h]);
     }
   }
-  cluster.sync();  // keep every CTA's shared memory alive until CTA 0 has read it
+  cluster.sync();  // keep every CTA's shared memory alive until all have read it
 }
 
 // ------------------------------------------------------------ fp32 caches
