@@ -181,6 +181,20 @@ def oracle_unit_seconds(w: synth.Workload, b: int, kvh: int):
     return time.perf_counter() - t0, 1
 
 
+def host_cpu():
+    """Model name and logical core count of the host running the oracle."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "nproc": os.cpu_count()}
+
+
 def workload_config(w: synth.Workload, world: int):
     s = w.spec
     return {"workload": s.name, "batch": s.batch, "seq_len": s.seq_len, "num_kv_heads": s.num_kv_heads,
@@ -204,6 +218,7 @@ def cpu_baseline(w: synth.Workload, seconds: float = 10.0, max_units: int = 256)
         n += 1
     per_step = secs / n * total_units
     return {"value": 1.0 / per_step, "unit": "steps/s", "cores": threads, "kind": "oracle",
+            "cpu": host_cpu(),
             "sample": f"{n} unit evaluations cycling over the {total_units} (sequence, kv head) units of one step "
                       f"(full layer + selection + {s.sparse_layers} sparse layers), fp64 single-threaded C; "
                       f"step time = mean unit time x {total_units}", "seconds_measured": secs}
@@ -363,7 +378,7 @@ def run_reference(args, rank, world, local):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": workload_config(w, world),
-            "cpu_baseline": {"value": v, "unit": "steps/s", "cores": threads, "kind": "oracle",
+            "cpu_baseline": {"value": v, "unit": "steps/s", "cores": threads, "kind": "oracle", "cpu": host_cpu(),
                              "sample": "each step = one (sequence, kv head) unit of the workload (full layer + "
                                        "selection + sparse layers) timed and scaled by the unit count"},
             "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -477,6 +477,7 @@ cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const C
   HS2_FULL_CASE(64, false, 8, 6, 1)
   HS2_FULL_CASE(64, false, 4, 6, 1)
   HS2_FULL_CASE(128, true, 8, 3, 2)
+  HS2_FULL_CASE(128, true, 6, 4, 2)
   HS2_FULL_CASE(128, true, 4, 6, 2)
   HS2_FULL_CASE(128, true, 16, 3, 1)
   HS2_FULL_CASE(128, true, 12, 4, 1)

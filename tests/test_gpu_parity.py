@@ -212,7 +212,7 @@ def test_heads_of_unequal_magnitude(oracle, lib, kv_dtype):
 # every built tensor-core configuration of the attention kernel: (ncw, nstage, nsl)
 FULL_CONFIGS = {
     "bf16": ["8,3,1", "4,6,1", "4,3,2"],
-    "e4m3": ["8,3,2", "4,6,2", "16,3,1", "12,4,1", "8,6,1", "4,8,1"],
+    "e4m3": ["8,3,2", "6,4,2", "4,6,2", "16,3,1", "12,4,1", "8,6,1", "4,8,1"],
 }
 
 
