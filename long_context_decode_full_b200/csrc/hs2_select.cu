@@ -237,13 +237,14 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   const int64_t u = (int64_t)b * p.Hkv + kvh;
   const int t0 = chunk * p.score_chunk, t1 = min(ui.nC, t0 + p.score_chunk);
   const float *lg = p.ws.logits + (size_t)u * p.ustride * G;
-  // the first batch of logits is in flight while the LSE is rebuilt
-  float raw[kScoreLoads][G];
-  if (!combine) load_logits<G>(raw, lg, t0 + threadIdx.x, t1);
+  // the LSE first: its dependent record loads would otherwise queue behind
+  // every CTA's first batch of logits
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh_hist[i] = 0u;
   mark_records(ui, sh_ok);
   const float *rec0 = p.ws.records + (size_t)u * p.R * RS;
   unit_lse<G, D>(rec0, ui, p.c, sh_lse, sh_M, sh_L, sh_red);
+  float raw[kScoreLoads][G];
+  if (!combine) load_logits<G>(raw, lg, t0 + threadIdx.x, t1);
 
   if (combine) {  // out = sum_j o_j exp(c (m_j - M)) / L
     const int64_t ob = ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
