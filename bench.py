@@ -127,15 +127,21 @@ class Clocks:
 
 
 def setup_dist(gpus: int):
+    """One process per GPU (torchrun environment); NCCL on GPUs, gloo on a
+    host without one (the CPU tests of the multi-process path)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    cuda = torch.cuda.is_available()
     if world > 1:
         import datetime
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
-    else:
+        timeout = datetime.timedelta(seconds=120)
+        if cuda:
+            torch.cuda.set_device(local)
+            torch.distributed.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            torch.distributed.init_process_group("gloo", timeout=timeout)
+    elif cuda:
         torch.cuda.set_device(0)
     return rank, world, local
 
@@ -148,7 +154,8 @@ def barrier(world):
 def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
