@@ -188,6 +188,17 @@ int hs2_workspace_status(void *workspace, size_t workspace_bytes, void *stream);
 int hs2_copy_peak(void *dst, const void *src, size_t bytes, void *stream);
 
 /* Thread-local text of the last non-zero status returned on this thread. */
+/*
+ * Self-test of the bounded device waits (no counterpart in the pages): one
+ * CTA waits on a barrier that nothing completes; the wait gives up after
+ * about 10 ms of clock cycles and sets the workspace's sticky flag, so a
+ * following hs2_workspace_status() returns HS2_ERR_TIMEOUT (and clears it)
+ * and the CUDA context stays usable.  No fault, trap or hang is involved.
+ *   workspace  device, >= 256 bytes, 256-byte aligned (only its flag word is used).
+ * Returns HS2_OK once launched (asynchronous on `stream`).
+ */
+int hs2_selftest_bounded_wait(void *workspace, size_t workspace_bytes, void *stream);
+
 const char *hs2_last_error(void);
 
 /* Library version, major * 10000 + minor * 100 + patch. */

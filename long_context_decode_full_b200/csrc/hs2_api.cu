@@ -429,6 +429,14 @@ int hs2_workspace_status(void *workspace, size_t workspace_bytes, void *stream) 
   return HS2_OK;
 }
 
+int hs2_selftest_bounded_wait(void *workspace, size_t workspace_bytes, void *stream) {
+  if (!workspace || workspace_bytes < 256) return fail(HS2_ERR_WORKSPACE, "workspace is NULL or too small");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return fail(HS2_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  cudaError_t e = launch_wait_selftest(static_cast<uint32_t *>(workspace), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return HS2_OK;
+}
+
 int hs2_copy_peak(void *dst, const void *src, size_t bytes, void *stream) {
   if (!dst || !src || (bytes & 15) || !aligned16(dst) || !aligned16(src))
     return fail(HS2_ERR_INVALID_ARG, "copy needs 16-byte aligned pointers and a multiple of 16 bytes");
@@ -440,6 +448,24 @@ int hs2_copy_peak(void *dst, const void *src, size_t bytes, void *stream) {
 }  // extern "C"
 
 namespace hs2 {
+
+// One CTA waits on an mbarrier that nothing ever arrives at: the bounded wait
+// must give up (after ~10 ms instead of the kernels' ~2 s) and set the
+// workspace's sticky flag, then the kernel returns normally.
+__global__ void wait_selftest_kernel(uint32_t *err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1u);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0u, 20000000LL)) set_error(err, kErrFullWait);
+}
+
+cudaError_t launch_wait_selftest(uint32_t *err, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(err);
+  return cudaGetLastError();
+}
 
 __global__ void __launch_bounds__(512) copy_kernel(uint4 *__restrict__ dst, const uint4 *__restrict__ src, size_t n) {
   const size_t stride = (size_t)gridDim.x * blockDim.x;

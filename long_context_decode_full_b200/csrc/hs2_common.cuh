@@ -100,13 +100,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Waits for the phase with the given parity to complete; gives up after
-// kSpinLimitCycles and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// `limit` cycles (kSpinLimitCycles by default) and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long long limit = kSpinLimitCycles) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(a, parity)) {
-    if (clock64() - t0 > kSpinLimitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
 }

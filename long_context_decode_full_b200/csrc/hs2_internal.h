@@ -114,6 +114,8 @@ cudaError_t launch_sparse_impl(const SparseParams &p, int kv_dtype, int64_t num_
 
 cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int grid, cudaStream_t s);
 
+cudaError_t launch_wait_selftest(uint32_t *err, cudaStream_t s);
+
 // Sets the thread's hs2_last_error() text and returns `code`.
 int set_last_error(int code, const char *msg);
 

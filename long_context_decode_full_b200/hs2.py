@@ -43,7 +43,7 @@ class HS2Error(RuntimeError):
 _lib = None
 EXPORTS = ["hs2_full_attn_select_workspace", "hs2_full_attn_select", "hs2_full_attn_select_marked",
            "hs2_full_attn_select_static", "hs2_sparse_attn",
-           "hs2_workspace_status", "hs2_copy_peak", "hs2_last_error", "hs2_version"]
+           "hs2_workspace_status", "hs2_selftest_bounded_wait", "hs2_copy_peak", "hs2_last_error", "hs2_version"]
 
 
 def lib():
@@ -71,6 +71,8 @@ def lib():
         L.hs2_sparse_attn.restype = ctypes.c_int
         L.hs2_workspace_status.argtypes = [P, SZ, P]
         L.hs2_workspace_status.restype = ctypes.c_int
+        L.hs2_selftest_bounded_wait.argtypes = [P, SZ, P]
+        L.hs2_selftest_bounded_wait.restype = ctypes.c_int
         L.hs2_copy_peak.argtypes = [P, P, SZ, P]
         L.hs2_copy_peak.restype = ctypes.c_int
         L.hs2_last_error.argtypes = []
@@ -200,6 +202,11 @@ def hybrid_block_step(q_full, q_sparse: Sequence[torch.Tensor], k, v, seq_lens, 
 def workspace_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronises the stream, returns and clears the sticky device error flag."""
     return int(lib().hs2_workspace_status(_ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def selftest_bounded_wait(workspace: torch.Tensor, stream=None):
+    """Makes one bounded device wait expire on purpose (it sets the sticky flag)."""
+    _check(lib().hs2_selftest_bounded_wait(_ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def copy_peak(dst: torch.Tensor, src: torch.Tensor, stream=None):

@@ -108,3 +108,9 @@ def test_workspace_size_rules(libhs2):
 def test_copy_rejects_misaligned(libhs2):
     assert hs2.lib().hs2_copy_peak(FAKE, FAKE + 4, 64, None) == hs2.ERR_INVALID_ARG
     assert hs2.lib().hs2_copy_peak(FAKE, FAKE, 60, None) == hs2.ERR_INVALID_ARG
+
+
+def test_selftest_rejects_bad_workspace(libhs2):
+    assert hs2.lib().hs2_selftest_bounded_wait(None, 256, None) == hs2.ERR_WORKSPACE
+    assert hs2.lib().hs2_selftest_bounded_wait(FAKE, 16, None) == hs2.ERR_WORKSPACE
+    assert hs2.lib().hs2_selftest_bounded_wait(FAKE + 8, 4096, None) == hs2.ERR_WORKSPACE

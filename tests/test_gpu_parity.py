@@ -226,3 +226,19 @@ def test_every_attention_config(oracle, lib, monkeypatch, kv_dtype, cfg):
     out, idx = U.run_gpu(wd)
     torch.cuda.synchronize()
     U.check_full(wd, out, idx, ora)
+
+
+def test_bounded_wait_expires_and_context_stays_usable(oracle, lib):
+    """A device wait that nothing completes gives up, flags the workspace,
+    and the next status read reports it once; the context keeps working."""
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    lib.selftest_bounded_wait(ws)
+    assert lib.workspace_status(ws) == lib.ERR_TIMEOUT
+    assert lib.workspace_status(ws) == 0  # the flag was cleared by the read
+    sp = spec(batch=1, seq_len=2000)
+    w = synth.generate(sp, seed=3)
+    ora = U.run_oracle(oracle, w)
+    wd = U.to_device(w)
+    out, idx = U.run_gpu(wd)
+    torch.cuda.synchronize()
+    U.check_full(wd, out, idx, ora)
