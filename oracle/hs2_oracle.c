@@ -18,7 +18,7 @@
  *   - the window and the global tokens are read from the same shared KV cache
  *     in one sparse-attention computation (no separate sliding-window branch).
  *
- * Readings fixed where the pages are silent (listed again in the design doc):
+ * Readings fixed where the pages are silent:
  *   - score[t] for a KV head = sum over the query heads of its GQA group of
  *     the full layer's softmax probability p_{h,t};
  *   - top-k over t < T-W by (score descending, index ascending); if there
