@@ -384,11 +384,12 @@ int hs2_sparse_attn(const hs2_heads *q_l, const hs2_cache *k_cache, const hs2_ca
   p.D = k_cache->head_dim;
   p.L = idx_stride;
   p.c = 1.0f / sqrtf((float)p.D);
-  // enough CTAs per unit to cover the SMs, at most 16 per cluster and 256 rows per CTA
   // 8 warps per CTA take 16-row groups, each warp gathering up to `nbuf`
-  // groups at once: rows per CTA = 128 * nbuf.  One buffer per warp (a
-  // 9-CTA cluster at the pages' 1152 rows) unless that needs more than one
-  // CTA per SM (a CTA holds an SM's registers), then two, then four.
+  // groups at once: rows per CTA = 128 * nbuf, one cluster of S CTAs per
+  // (sequence, kv head).  nbuf starts at 2 and grows (up to what shared
+  // memory holds) while the units' CTAs would not fit in one wave of one CTA
+  // per SM or a cluster would exceed 16 CTAs; very long lists then take more
+  // rows per CTA than buffers, walked as a rolling pipeline.
   const int units = p.B * p.Hkv, sms = sm_count();
   // a warp's gather buffers: 16 rows of K and V (+ scales); at most 192 KB per CTA
   const int buf_bytes = 2 * 16 * p.D * (k_cache->dtype == HS2_E4M3 ? 1 : 2) + (k_cache->dtype == HS2_E4M3 ? 128 : 0);
