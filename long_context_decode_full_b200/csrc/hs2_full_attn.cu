@@ -7,9 +7,10 @@
 // tile) space.  A producer warp streams K and V tiles with TMA bulk-tensor
 // loads into a ring of shared-memory stages (mbarrier full/empty pairs, every
 // wait bounded); for E4M3 caches a second producer warp gathers the per-token
-// scales with cp.async at the same time; consumer warps each take 16 rows of a tile, run Q K^T and
-// V^T P^T on the tensor cores with an online softmax, and store the raw
-// logits that the score pass turns into group probabilities.  At the end of
+// scales with cp.async at the same time.  Consumer warps each take one or two
+// 16-row slices of a tile, run K Q^T and V^T P^T on the tensor cores with an
+// online softmax, and store the raw logits (evict-last in L2) that the score
+// pass turns into group probabilities.  At the end of
 // each segment (a run of tiles of one unit inside one CTA) the consumer warps
 // merge their states into one (m, l, o) record.
 //

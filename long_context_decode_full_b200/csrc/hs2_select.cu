@@ -7,26 +7,28 @@
 // group of the softmax probability p_{h,t} = exp(c * s_{h,t} - LSE_h).
 //
 // Three kernels on the CUDA cores:
-//   score  -- grid (chunk, kv head, sequence) + one combine CTA per unit.
-//             Score CTAs rebuild each head's LSE from the segment records (a
-//             parallel fp64 reduction), turn the raw logits of 4096 positions
-//             into approximate group scores (one FMA and one ex2 per head,
-//             relative error below 1e-5) and a 4096-bin histogram of their top
-//             bits (16 bins per octave); the last chunk to finish (atomic
-//             ticket, no waiting) finds the bin b holding the k_global-th
-//             largest approximate score.  The combine CTA merges the records
-//             into the attention output.
-//   filter -- each warp owns 512 consecutive positions and writes, in
-//             position order, the positions whose approximate score is above
-//             bin b widened by a 4e-4 margin (certainly above the k-th exact
-//             score) and, with exact scores, the positions inside that widened
-//             bin (the guard band that holds every position the exact k-th
-//             score can hinge on).
-//   final  -- one CTA per unit: exact scores of the guard-band positions
-//             (exponent formed in float-float, so only ex2's own rounding is
-//             left), radix select of the exact k-th score among them, ties to
-//             the lower position (the list is position-ordered), then a merge
-//             of the two sorted lists and the forced window into the index list.
+//   score  -- grid (chunk, kv head, sequence) + one combine CTA per unit; a
+//             chunk (2048..65536 positions) is sized per call so the grid is
+//             one wave.  Score CTAs rebuild each head's LSE from the segment
+//             records (a parallel fp64 reduction), then turn the raw logits of
+//             their chunk into approximate group scores (one FMA and one ex2
+//             per head, relative error below 1e-5) and a 4096-bin histogram of
+//             their top bits (16 bins per octave); the last chunk to finish
+//             (atomic ticket, no waiting) finds the bin b holding the
+//             k_global-th largest approximate score.  The combine CTA merges
+//             the records into the attention output.
+//   filter -- each warp owns one or two 512-position sub-ranges and writes,
+//             in position order, the positions whose approximate score is
+//             above bin b widened by a 4e-4 margin (certainly above the k-th
+//             exact score) and, with exact scores (exponent formed in
+//             float-float, so only ex2's own rounding is left), the positions
+//             inside that widened bin: the guard band that holds every
+//             position the exact k-th score can hinge on.
+//   final  -- one CTA per unit: the need-th best guard-band entry by exact
+//             score, ties to the lower position (the lists are
+//             position-ordered), found by direct ranks for bands up to 768
+//             entries and by a radix select otherwise, then a merge of the two
+//             sorted lists and the forced window into the index list.
 // Scores are >= 0, so their IEEE bit patterns order like the values.
 #include "hs2_internal.h"
 
