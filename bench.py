@@ -62,11 +62,36 @@ def algorithmic_bytes(w: synth.Workload):
 ATTN_SOURCES = ("hs2_full_attn.cu", "hs2_warp_attn.cuh", "hs2_common.cuh")
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments and blank-space runs (a comment edit is
+    not a kernel change)."""
+    import re
+    out, i, n = [], 0, len(text)
+    while i < n:
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif text[i] == '"':  # string literal (inline PTX): kept verbatim
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(text[i])
+            i += 1
+    return re.sub(r"\s+", " ", "".join(out)).strip()
+
+
 def attention_source_hash():
+    """SHA-256 of the attention kernel's sources, comments and spacing removed."""
     h = hashlib.sha256()
     for name in ATTN_SOURCES:
-        with open(os.path.join(ROOT, "long_context_decode_full_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "long_context_decode_full_b200", "csrc", name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()
 
 

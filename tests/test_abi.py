@@ -114,3 +114,13 @@ def test_selftest_rejects_bad_workspace(libhs2):
     assert hs2.lib().hs2_selftest_bounded_wait(None, 256, None) == hs2.ERR_WORKSPACE
     assert hs2.lib().hs2_selftest_bounded_wait(FAKE, 16, None) == hs2.ERR_WORKSPACE
     assert hs2.lib().hs2_selftest_bounded_wait(FAKE + 8, 4096, None) == hs2.ERR_WORKSPACE
+
+
+def test_traffic_hash_ignores_comments_only():
+    import bench
+    a = 'int f() { // note\n  return 1; /* x */ }\nasm("mov.u64 %0, %%globaltimer; // kept");\n'
+    b = 'int f() {\n  return 1; }\nasm("mov.u64 %0, %%globaltimer; // kept");\n'
+    c = 'int f() {\n  return 2; }\nasm("mov.u64 %0, %%globaltimer; // kept");\n'
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(b) != bench._code_only(c)
+    assert "// kept" in bench._code_only(a)  # string literals (inline PTX) are code
