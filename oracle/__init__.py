@@ -46,6 +46,14 @@ def _load():
         lib.orc_full_attn_select.restype = I
         lib.orc_sparse_attn.argtypes = [P, I, I, I, P, P, P, P, I, I, I, P, I, P]
         lib.orc_sparse_attn.restype = I
+        lib.orc_e4m3_encode.argtypes = [ctypes.c_double]
+        lib.orc_e4m3_encode.restype = ctypes.c_uint8
+        lib.orc_bf16_encode.argtypes = [ctypes.c_double]
+        lib.orc_bf16_encode.restype = ctypes.c_uint16
+        lib.orc_e4m3_row.argtypes = [P, I, P, P]
+        lib.orc_e4m3_row.restype = None
+        lib.orc_kv_bridge.argtypes = [P, I, I, P, P, I, P, P]
+        lib.orc_kv_bridge.restype = I
         _lib = lib
     return _lib
 
@@ -131,3 +139,37 @@ def sparse_attn(q, q_dtype, k, v, kv_dtype, idx, k_scale=None, v_scale=None):
     if rc != 0:
         raise MemoryError("oracle allocation failed")
     return out
+
+
+def e4m3_encode(x: float) -> int:
+    """The E4M3 code nearest to x (ties to even), saturated at +-448."""
+    return int(_load().orc_e4m3_encode(float(x)))
+
+
+def bf16_encode(x: float) -> int:
+    """The bf16 bit pattern nearest to x (ties to even)."""
+    return int(_load().orc_bf16_encode(float(x)))
+
+
+def e4m3_row(x):
+    """One row of values -> (uint8 E4M3 codes, fp32 scale = max|x| / 448)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    codes = np.zeros(x.shape[-1], np.uint8)
+    scale = np.zeros(1, np.float32)
+    _load().orc_e4m3_row(_ptr(x), x.shape[-1], _ptr(codes), _ptr(scale))
+    return codes, float(scale[0])
+
+
+def kv_bridge(h, wk, wv):
+    """KV Bridging projections of one decode step: h [B, d_model] and
+    wk / wv [d_model, n] as bf16 bit patterns -> (k, v) float64 [B, n]."""
+    h = _c(h, np.uint16)
+    wk, wv = _c(wk, np.uint16), _c(wv, np.uint16)
+    B, dm = h.shape
+    n = wk.shape[1]
+    assert wk.shape == (dm, n) and wv.shape == (dm, n)
+    k = np.zeros((B, n), np.float64)
+    v = np.zeros((B, n), np.float64)
+    rc = _load().orc_kv_bridge(_ptr(h), B, dm, _ptr(wk), _ptr(wv), n, _ptr(k), _ptr(v))
+    assert rc == 0
+    return k, v

@@ -16,7 +16,11 @@
  *   - selection is per token (not per block): the most recent 128 tokens are
  *     always taken, plus 1,024 global tokens chosen from outside that window;
  *   - the window and the global tokens are read from the same shared KV cache
- *     in one sparse-attention computation (no separate sliding-window branch).
+ *     in one sparse-attention computation (no separate sliding-window branch);
+ *   - ("KV Bridging" paragraphs) each Cross-Decoder full-attention layer
+ *     builds its KV cache from the matching Self-Decoder layer's input hidden
+ *     state through its own K/V projections (orc_kv_bridge and the encoders
+ *     at the end of this file).
  *
  * Readings fixed where the pages are silent:
  *   - score[t] for a KV head = sum over the query heads of its GQA group of
@@ -300,6 +304,78 @@ int orc_sparse_attn(const void *q, int q_dtype, int B, int num_q_heads, const vo
                                idx + ((size_t)b * num_kv_heads + h) * idx_stride, idx_stride,
                                out + ((size_t)b * num_q_heads + (size_t)h * G) * d);
       if (rc < 0) return -1;
+    }
+  return 0;
+}
+
+/* ---- KV Bridging append ------------------------------------------------
+ * HySparse2 announcement, "KV Bridging" paragraphs: each Cross-Decoder
+ * full-attention layer builds its own KV cache from the input hidden state of
+ * the matching Self-Decoder full-attention layer, through its own K and V
+ * projections, so the cache exists before the Cross-Decoder runs.  For one
+ * decode step the new token's rows are
+ *     k = h W_k,   v = h W_v      (h [d_model], W [d_model, Hkv * d])
+ * in double.  Readings where the pages are silent: the projections are plain
+ * matrix products without bias; storage follows the cache type -- bf16
+ * rounded to nearest (ties to even), or E4M3 per (token, kv head) with
+ * scale = max|x| / 448 stored as fp32 (1 for an all-zero row) and each code
+ * the E4M3 value nearest to x / scale (ties to the even code), saturated at
+ * +-448. */
+
+/* The E4M3 code nearest to x, ties to the code with an even mantissa, |x| >=
+ * 448 saturating to +-448, NaN to 0x7F.  Plain definition: a scan of the 127
+ * finite non-negative codes, whose values increase with the code. */
+uint8_t orc_e4m3_encode(double x) {
+  if (x != x) return 0x7F;
+  const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  const double a = fabs(x);
+  if (a >= 448.0) return sign | 0x7E;
+  int lo = 0;
+  while (lo + 1 <= 0x7E && orc_e4m3_value((uint8_t)(lo + 1)) <= a) ++lo;
+  /* value(lo) <= a < value(lo + 1) */
+  const double vl = orc_e4m3_value((uint8_t)lo), vh = orc_e4m3_value((uint8_t)(lo + 1));
+  int c;
+  if (a - vl < vh - a) c = lo;
+  else if (a - vl > vh - a) c = lo + 1;
+  else c = (lo & 1) ? lo + 1 : lo;
+  return sign | (uint8_t)c;
+}
+
+/* bf16 bit pattern nearest to x (8 significant bits, ties to even), for
+ * values in the normal fp32 range. */
+uint16_t orc_bf16_encode(double x) {
+  if (x == 0.0) return signbit(x) ? 0x8000 : 0;
+  int e;
+  const double f = frexp(x, &e);          /* x = f 2^e, 0.5 <= |f| < 1 */
+  const double r = nearbyint(ldexp(f, 8)); /* 8 significant bits, ties to even */
+  const float y = (float)ldexp(r, e - 8);  /* exact */
+  uint32_t u;
+  memcpy(&u, &y, sizeof u);
+  return (uint16_t)(u >> 16);
+}
+
+/* One (token, kv head) row of d values into E4M3 codes and its fp32 scale. */
+void orc_e4m3_row(const double *x, int d, uint8_t *codes, float *scale) {
+  double amax = 0.0;
+  for (int i = 0; i < d; ++i) amax = fmax(amax, fabs(x[i]));
+  const float s = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;
+  for (int i = 0; i < d; ++i) codes[i] = orc_e4m3_encode(x[i] / (double)s);
+  *scale = s;
+}
+
+/* k[b][n] = sum_i h[b][i] wk[i][n], v likewise; h, w are bf16 bit patterns. */
+int orc_kv_bridge(const uint16_t *h, int B, int d_model, const uint16_t *wk, const uint16_t *wv, int n_out,
+                  double *k, double *v) {
+  for (int b = 0; b < B; ++b)
+    for (int n = 0; n < n_out; ++n) {
+      double sk = 0.0, sv = 0.0;
+      for (int i = 0; i < d_model; ++i) {
+        const double hi = bf16_value(h[(size_t)b * d_model + i]);
+        sk += hi * bf16_value(wk[(size_t)i * n_out + n]);
+        sv += hi * bf16_value(wv[(size_t)i * n_out + n]);
+      }
+      k[(size_t)b * n_out + n] = sk;
+      v[(size_t)b * n_out + n] = sv;
     }
   return 0;
 }

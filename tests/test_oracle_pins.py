@@ -340,3 +340,77 @@ def test_sparse_single_row_and_order_independence(oracle):
     a = run_sparse(oracle, w, w.q_sparse[0], idx2)
     b = run_sparse(oracle, w, w.q_sparse[0], idx2[:, :, ::-1].copy())
     np.testing.assert_allclose(a, b, atol=1e-15)
+
+
+# ---- KV Bridging append: encoders and projections --------------------------
+
+def test_e4m3_encode_round_trips_every_finite_code(oracle):
+    for c in list(range(0x00, 0x7F)) + list(range(0x80, 0xFF)):
+        assert oracle.e4m3_encode(oracle.e4m3_value(c)) == c or (c == 0x80 and oracle.e4m3_value(c) == 0.0)
+
+
+def test_e4m3_encode_midpoints_go_to_the_even_code_and_saturate(oracle):
+    for c in range(0x00, 0x7E):  # consecutive non-negative codes
+        mid = (oracle.e4m3_value(c) + oracle.e4m3_value(c + 1)) / 2
+        even = c if c % 2 == 0 else c + 1
+        assert oracle.e4m3_encode(mid) == even
+        assert oracle.e4m3_encode(-mid) == 0x80 | even
+    assert oracle.e4m3_encode(448.0) == 0x7E and oracle.e4m3_encode(1e9) == 0x7E
+    assert oracle.e4m3_encode(-464.0) == 0xFE
+    assert oracle.e4m3_encode(float("nan")) == 0x7F
+
+
+def test_e4m3_encode_matches_torch_cast_of_fp32_values(oracle):
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(20000, generator=g) * torch.exp2(torch.randint(-12, 9, (20000,), generator=g).float()))
+    x = x.clamp(-448, 448)
+    ref = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(v)) for v in x.numpy()], np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def test_bf16_encode_matches_torch_cast_of_fp32_values(oracle):
+    g = torch.Generator().manual_seed(6)
+    x = torch.randn(20000, generator=g) * torch.exp2(torch.randint(-30, 30, (20000,), generator=g).float())
+    ref = x.to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    got = np.array([oracle.bf16_encode(float(v)) for v in x.numpy()], np.uint16)
+    assert np.array_equal(got, ref)
+
+
+def test_e4m3_row_scale_and_extremes(oracle):
+    codes, s = oracle.e4m3_row(np.zeros(16))
+    assert s == 1.0 and not codes.any()
+    x = np.array([0.3, -2.5, 1.0, 2.5 - 1e-9])
+    codes, s = oracle.e4m3_row(x)
+    assert s == np.float32(2.5 / 448)
+    assert codes[1] == 0xFE  # -max|x| encodes -448
+    deq = np.array([oracle.e4m3_value(c) for c in codes]) * s
+    assert np.all(np.abs(deq - x) <= 2.5 / 16 + 1e-12)  # half an E4M3 step (2^-4 relative) at the top
+
+
+def _bf16_bits(a):
+    return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+
+
+def test_kv_bridge_closed_forms(oracle):
+    g = np.random.default_rng(7)
+    dm, n = 48, 24
+    wk = g.standard_normal((dm, n)).astype(np.float32)
+    wv = g.standard_normal((dm, n)).astype(np.float32)
+    wkb, wvb = _bf16_bits(wk), _bf16_bits(wv)
+    wk_exact = torch.from_numpy(wk).to(torch.bfloat16).double().numpy()
+    wv_exact = torch.from_numpy(wv).to(torch.bfloat16).double().numpy()
+    # unit hidden states pick rows of the weights
+    h = np.zeros((3, dm), np.float32)
+    h[0, 5] = 1.0
+    h[1, 17] = -2.0
+    k, v = oracle.kv_bridge(_bf16_bits(h), wkb, wvb)
+    assert np.array_equal(k[0], wk_exact[5]) and np.array_equal(v[1], -2.0 * wv_exact[17])
+    assert not k[2].any() and not v[2].any()
+    # general inputs: the fp64 matrix product of the stored values
+    h = g.standard_normal((4, dm)).astype(np.float32)
+    hb = _bf16_bits(h)
+    h_exact = torch.from_numpy(h).to(torch.bfloat16).double().numpy()
+    k, v = oracle.kv_bridge(hb, wkb, wvb)
+    np.testing.assert_allclose(k, h_exact @ wk_exact, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(v, h_exact @ wv_exact, rtol=0, atol=1e-12)
