@@ -256,6 +256,51 @@ def cpu_baseline(w: synth.Workload, seconds: float = 10.0, max_units: int = 256)
                       f"step time = mean unit time x {total_units}", "seconds_measured": secs}
 
 
+# ------------------------------------------------------------------ KV Bridging append
+BRIDGE_D_MODEL = 4096  # the pages give no hidden size; a synthetic stand-in
+
+
+def time_kv_bridge(w, dev, stream, peak, iters=20):
+    """The decode-time KV Bridging append on the workload's batch and cache:
+    each launch timed alone with CUDA events, L2 flushed before it so the
+    weights come from HBM as they do inside a real step.  It writes the rows
+    at position T_b - 1, so it runs after every other measurement."""
+    from long_context_decode_full_b200 import hs2
+
+    s = w.spec
+    N = s.num_kv_heads * s.head_dim
+    g = torch.Generator(device=dev).manual_seed(1234)
+    h = torch.randn(s.batch, BRIDGE_D_MODEL, device=dev, generator=g).to(torch.bfloat16)
+    wk = (torch.randn(BRIDGE_D_MODEL, N, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+    wv = (torch.randn(BRIDGE_D_MODEL, N, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+    ws = torch.empty(hs2.kv_bridge_workspace_bytes(s.batch, BRIDGE_D_MODEL, s.num_kv_heads, s.head_dim),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def call():
+        hs2.kv_bridge_append(h, wk, wv, w.k, w.v, w.seq_lens, w.page_table, w.page_size, w.k_scale, w.v_scale,
+                             workspace=ws)
+
+    for _ in range(3):
+        call()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    us = statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3
+    elt = w.k.element_size()
+    nbytes = (2 * BRIDGE_D_MODEL * N * 2 + s.batch * BRIDGE_D_MODEL * 2 + 2 * s.batch * N * elt
+              + (2 * s.batch * s.num_kv_heads * 4 if w.k_scale is not None else 0))
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"d_model": BRIDGE_D_MODEL, "us": us, "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
+            "frac": gbs / peak, "launches": 2, "l2": "flushed before each launch",
+            "what": "k = h W_k, v = h W_v for the new token of every sequence, stored at position T_b - 1 "
+                    "(E4M3: per-(token, kv head) scale); bytes = both weight matrices + hidden + stored rows"}
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_gpu(args, rank, world, local):
     from long_context_decode_full_b200 import hs2
@@ -386,6 +431,8 @@ def run_gpu(args, rank, world, local):
         "clocks": clk,
         "device_status": status,
     }
+    if not args.no_bridge:
+        res["kv_bridge_append"] = time_kv_bridge(w, dev, stream, peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     return res
@@ -422,6 +469,7 @@ def main():
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(synth.WORKLOADS))
+    ap.add_argument("--no-bridge", action="store_true", help="skip the KV Bridging append measurement")
     ap.add_argument("--impl", default="hs2", choices=["hs2", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=500)

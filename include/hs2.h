@@ -189,6 +189,45 @@ int hs2_copy_peak(void *dst, const void *src, size_t bytes, void *stream);
 
 /* Thread-local text of the last non-zero status returned on this thread. */
 /*
+ * Workspace bytes of hs2_kv_bridge_append() for this shape (0 if invalid).
+ */
+size_t hs2_kv_bridge_workspace(int32_t batch, int32_t d_model, int32_t num_kv_heads, int32_t head_dim);
+
+/*
+ * KV Bridging append of one decode step (HySparse2 announcement, "KV
+ * Bridging" paragraphs): each Cross-Decoder full-attention layer builds its
+ * own KV cache from the input hidden state of the matching Self-Decoder
+ * full-attention layer, through its own K and V projections.  For every
+ * sequence b the new token's rows
+ *     k_b = h_b W_k,   v_b = h_b W_v          (fp32 accumulation, no bias)
+ * are written at position T_b - 1 (the token being decoded, already counted in
+ * seq_lens, as hs2_full_attn_select() expects) of k_cache / v_cache through
+ * the page table: as computed for HS2_F32, rounded to nearest even for
+ * HS2_BF16, and for HS2_E4M3 with scale = max_i |x_i| / 448 per (token, kv
+ * head) (1 for an all-zero row) and codes the E4M3 values nearest x / scale
+ * (ties to even), saturated at +-448.
+ *
+ *   hidden     device bf16 [batch, d_model], 16-byte aligned; d_model a
+ *              positive multiple of 256.
+ *   w_k, w_v   device bf16 [d_model, num_kv_heads * head_dim], row-major,
+ *              16-byte aligned (the layer's own projections).
+ *   seq_lens   device int32 [batch]: T_b, clamped to [0, t_cap]; T_b = 0
+ *              writes nothing.
+ *   page_table device int32 [batch, max_pages], or NULL (contiguous layout,
+ *              max_pages = 1).  A page outside the cache writes nothing.
+ *   k_cache,
+ *   v_cache    the caches to write (descriptors as for hs2_full_attn_select;
+ *              this call writes one row per (sequence, kv head) and, for
+ *              E4M3, its scale).
+ *   workspace  device, >= hs2_kv_bridge_workspace() bytes, 256-byte aligned.
+ * Asynchronous on `stream`; rows of other positions are not touched.
+ */
+int hs2_kv_bridge_append(const void *hidden, int32_t batch, int32_t d_model, const void *w_k, const void *w_v,
+                         const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
+                         const hs2_cache *k_cache, const hs2_cache *v_cache, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/*
  * Self-test of the bounded device waits (no counterpart in the pages): one
  * CTA waits on a barrier that nothing completes; the wait gives up after
  * about 10 ms of clock cycles and sets the workspace's sticky flag, so a

@@ -430,6 +430,68 @@ int hs2_workspace_status(void *workspace, size_t workspace_bytes, void *stream) 
   return HS2_OK;
 }
 
+size_t hs2_kv_bridge_workspace(int32_t batch, int32_t d_model, int32_t num_kv_heads, int32_t head_dim) {
+  if (batch < 1 || batch > 65535 || d_model < 1 || d_model % bridge_row_multiple() || num_kv_heads < 1 ||
+      (head_dim != 64 && head_dim != 128))
+    return 0;
+  return align256((size_t)2 * bridge_splits(d_model) * batch * num_kv_heads * head_dim * 4);
+}
+
+int hs2_kv_bridge_append(const void *hidden, int32_t batch, int32_t d_model, const void *w_k, const void *w_v,
+                         const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
+                         const hs2_cache *k_cache, const hs2_cache *v_cache, void *workspace, size_t workspace_bytes,
+                         void *stream) {
+  int rc;
+  if ((rc = check_caches(k_cache, v_cache))) return rc;
+  if (!hidden || !w_k || !w_v || !seq_lens) return fail(HS2_ERR_INVALID_ARG, "hidden / w_k / w_v / seq_lens is NULL");
+  if (!aligned16(hidden) || !aligned16(w_k) || !aligned16(w_v))
+    return fail(HS2_ERR_INVALID_ARG, "hidden / weights not 16-byte aligned");
+  if (batch < 1 || batch > 65535) return fail(HS2_ERR_INVALID_ARG, "batch %d", batch);
+  if (d_model < 1 || d_model % bridge_row_multiple())
+    return fail(HS2_ERR_UNSUPPORTED, "d_model %d (a positive multiple of %d)", d_model, bridge_row_multiple());
+  const int ps = k_cache->page_size;
+  int64_t t_cap;
+  if (page_table) {
+    if (max_pages < 1) return fail(HS2_ERR_INVALID_ARG, "max_pages %d with a page table", max_pages);
+    t_cap = (int64_t)max_pages * ps;
+  } else {
+    if (max_pages != 1) return fail(HS2_ERR_INVALID_ARG, "contiguous layout (no page table) needs max_pages == 1");
+    t_cap = ps;
+    if ((int64_t)batch * ps > k_cache->num_slots)
+      return fail(HS2_ERR_INVALID_ARG, "contiguous layout needs num_slots >= batch * page_size");
+  }
+  const int Hkv = k_cache->num_kv_heads, D = k_cache->head_dim;
+  const size_t need = hs2_kv_bridge_workspace(batch, d_model, Hkv, D);
+  if (!workspace || workspace_bytes < need)
+    return fail(HS2_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return fail(HS2_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  BridgeParams p{};
+  p.h = static_cast<const __nv_bfloat16 *>(hidden);
+  p.wk = static_cast<const __nv_bfloat16 *>(w_k);
+  p.wv = static_cast<const __nv_bfloat16 *>(w_v);
+  p.seq_lens = seq_lens;
+  p.page_table = page_table;
+  p.k = const_cast<void *>(k_cache->data);  // this call writes the new rows
+  p.v = const_cast<void *>(v_cache->data);
+  p.k_scale = const_cast<float *>(k_cache->scale);
+  p.v_scale = const_cast<float *>(v_cache->scale);
+  p.kv_dtype = k_cache->dtype;
+  p.B = batch;
+  p.d_model = d_model;
+  p.Hkv = Hkv;
+  p.D = D;
+  p.N = Hkv * D;
+  p.page_size = ps;
+  p.max_pages = page_table ? max_pages : 1;
+  p.t_cap = t_cap;
+  p.num_slots = k_cache->num_slots;
+  p.nsplit = bridge_splits(d_model);
+  p.partial = static_cast<float *>(workspace);
+  cudaError_t e = launch_bridge(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "KV bridge launch");
+  return HS2_OK;
+}
+
 int hs2_selftest_bounded_wait(void *workspace, size_t workspace_bytes, void *stream) {
   if (!workspace || workspace_bytes < 256) return fail(HS2_ERR_WORKSPACE, "workspace is NULL or too small");
   if (reinterpret_cast<uintptr_t>(workspace) & 255) return fail(HS2_ERR_WORKSPACE, "workspace not 256-byte aligned");

@@ -116,6 +116,25 @@ cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int grid, cuda
 
 cudaError_t launch_wait_selftest(uint32_t *err, cudaStream_t s);
 
+// KV Bridging append of one decode step.
+struct BridgeParams {
+  const __nv_bfloat16 *h;            // [B, d_model]
+  const __nv_bfloat16 *wk, *wv;      // [d_model, N] row-major, N = Hkv * D
+  const int32_t *seq_lens;           // [B]
+  const int32_t *page_table;         // [B, max_pages] or nullptr
+  void *k, *v;                       // cache rows [num_slots, Hkv, D]
+  float *k_scale, *v_scale;          // E4M3 only
+  int32_t kv_dtype;
+  int32_t B, d_model, Hkv, D, N;
+  int32_t page_size, max_pages;
+  int64_t t_cap, num_slots;
+  int32_t nsplit;                    // d_model / 256 row splits
+  float *partial;                    // workspace [2][nsplit][B][N]
+};
+int bridge_splits(int d_model);
+int bridge_row_multiple();
+cudaError_t launch_bridge(const BridgeParams &p, cudaStream_t s);
+
 // Sets the thread's hs2_last_error() text and returns `code`.
 int set_last_error(int code, const char *msg);
 

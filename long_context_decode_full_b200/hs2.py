@@ -43,7 +43,8 @@ class HS2Error(RuntimeError):
 _lib = None
 EXPORTS = ["hs2_full_attn_select_workspace", "hs2_full_attn_select", "hs2_full_attn_select_marked",
            "hs2_full_attn_select_static", "hs2_sparse_attn",
-           "hs2_workspace_status", "hs2_selftest_bounded_wait", "hs2_copy_peak", "hs2_last_error", "hs2_version"]
+           "hs2_workspace_status", "hs2_selftest_bounded_wait", "hs2_kv_bridge_workspace", "hs2_kv_bridge_append",
+           "hs2_copy_peak", "hs2_last_error", "hs2_version"]
 
 
 def lib():
@@ -71,6 +72,11 @@ def lib():
         L.hs2_sparse_attn.restype = ctypes.c_int
         L.hs2_workspace_status.argtypes = [P, SZ, P]
         L.hs2_workspace_status.restype = ctypes.c_int
+        L.hs2_kv_bridge_workspace.argtypes = [I32, I32, I32, I32]
+        L.hs2_kv_bridge_workspace.restype = SZ
+        L.hs2_kv_bridge_append.argtypes = [P, I32, I32, P, P, P, P, I32, ctypes.POINTER(Cache),
+                                           ctypes.POINTER(Cache), P, SZ, P]
+        L.hs2_kv_bridge_append.restype = ctypes.c_int
         L.hs2_selftest_bounded_wait.argtypes = [P, SZ, P]
         L.hs2_selftest_bounded_wait.restype = ctypes.c_int
         L.hs2_copy_peak.argtypes = [P, P, SZ, P]
@@ -202,6 +208,32 @@ def hybrid_block_step(q_full, q_sparse: Sequence[torch.Tensor], k, v, seq_lens, 
 def workspace_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronises the stream, returns and clears the sticky device error flag."""
     return int(lib().hs2_workspace_status(_ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def kv_bridge_workspace_bytes(batch: int, d_model: int, num_kv_heads: int, head_dim: int) -> int:
+    return int(lib().hs2_kv_bridge_workspace(batch, d_model, num_kv_heads, head_dim))
+
+
+def kv_bridge_append(hidden, w_k, w_v, k, v, seq_lens, page_table=None, page_size=None, k_scale=None, v_scale=None,
+                     workspace=None, stream=None):
+    """KV Bridging append: writes the new token's K/V rows (hidden [B, d_model]
+    bf16 times w_k / w_v [d_model, Hkv * d] bf16) at position seq_lens[b] - 1
+    of the caches k / v (and the E4M3 scales)."""
+    assert hidden.dim() == 2 and hidden.is_contiguous() and w_k.is_contiguous() and w_v.is_contiguous()
+    B, dm = hidden.shape
+    if page_size is None:
+        assert page_table is None, "page_size is required with a page table"
+        page_size = k.shape[0] // B
+    max_pages = 1 if page_table is None else page_table.shape[1]
+    if workspace is None:
+        n = kv_bridge_workspace_bytes(B, dm, k.shape[1], k.shape[2])
+        if n == 0:
+            raise HS2Error(ERR_INVALID_ARG, "invalid KV bridge shape")
+        workspace = torch.empty(n, dtype=torch.uint8, device=hidden.device)
+    kc, vc = cache_desc(k, k_scale, page_size), cache_desc(v, v_scale, page_size)
+    _check(lib().hs2_kv_bridge_append(_ptr(hidden), B, dm, _ptr(w_k), _ptr(w_v), _ptr(seq_lens), _ptr(page_table),
+                                      max_pages, ctypes.byref(kc), ctypes.byref(vc), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)))
 
 
 def selftest_bounded_wait(workspace: torch.Tensor, stream=None):

@@ -124,3 +124,35 @@ def test_traffic_hash_ignores_comments_only():
     assert bench._code_only(a) == bench._code_only(b)
     assert bench._code_only(b) != bench._code_only(c)
     assert "// kept" in bench._code_only(a)  # string literals (inline PTX) are code
+
+
+def bridge(hidden=FAKE, B=4, dm=4096, wk=FAKE, wv=FAKE, seq=FAKE, pt=FAKE, max_pages=64, k=None, v=None,
+           ws=FAKE * 16, ws_bytes=1 << 40):
+    k = k or cache()
+    v = v or cache()
+    return hs2.lib().hs2_kv_bridge_append(hidden, B, dm, wk, wv, seq, pt, max_pages, ctypes.byref(k),
+                                          ctypes.byref(v), ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(hidden=0), hs2.ERR_INVALID_ARG),
+    (dict(wk=0), hs2.ERR_INVALID_ARG),
+    (dict(seq=0), hs2.ERR_INVALID_ARG),
+    (dict(wv=FAKE + 4), hs2.ERR_INVALID_ARG),
+    (dict(B=0), hs2.ERR_INVALID_ARG),
+    (dict(dm=1000), hs2.ERR_UNSUPPORTED),
+    (dict(pt=FAKE, max_pages=0), hs2.ERR_INVALID_ARG),
+    (dict(pt=0, max_pages=2), hs2.ERR_INVALID_ARG),
+    (dict(ws_bytes=1024), hs2.ERR_WORKSPACE),
+    (dict(ws=FAKE * 16 + 64), hs2.ERR_WORKSPACE),
+    (dict(k=cache(dtype=2), v=cache(dtype=2)), hs2.ERR_INVALID_ARG),  # E4M3 without scales
+    (dict(k=cache(heads=4), v=cache(heads=2)), hs2.ERR_INVALID_ARG),
+])
+def test_kv_bridge_rejects_bad_arguments(libhs2, kw, code):
+    assert bridge(**kw) == code
+
+
+def test_kv_bridge_workspace_size_rule(libhs2):
+    f = hs2.kv_bridge_workspace_bytes
+    assert f(4, 4096, 4, 128) == 2 * (4096 // 256) * 4 * 4 * 128 * 4
+    assert f(4, 4000, 4, 128) == 0 and f(0, 4096, 4, 128) == 0 and f(4, 4096, 4, 96) == 0
