@@ -208,7 +208,7 @@ size_t hs2_kv_bridge_workspace(int32_t batch, int32_t d_model, int32_t num_kv_he
  * (ties to even), saturated at +-448.
  *
  *   hidden     device bf16 [batch, d_model], 16-byte aligned; d_model a
- *              positive multiple of 256.
+ *              positive multiple of 128.
  *   w_k, w_v   device bf16 [d_model, num_kv_heads * head_dim], row-major,
  *              16-byte aligned (the layer's own projections).
  *   seq_lens   device int32 [batch]: T_b, clamped to [0, t_cap]; T_b = 0
@@ -219,8 +219,13 @@ size_t hs2_kv_bridge_workspace(int32_t batch, int32_t d_model, int32_t num_kv_he
  *   v_cache    the caches to write (descriptors as for hs2_full_attn_select;
  *              this call writes one row per (sequence, kv head) and, for
  *              E4M3, its scale).
- *   workspace  device, >= hs2_kv_bridge_workspace() bytes, 256-byte aligned.
- * Asynchronous on `stream`; rows of other positions are not touched.
+ *   workspace  device, >= hs2_kv_bridge_workspace() bytes, 256-byte aligned,
+ *              zero-filled before its first use: it starts with one counter
+ *              per (K or V, 128-column tile, group of 8 sequences) that the
+ *              call's last CTA of each returns to zero, so a workspace is
+ *              reused as is; calls sharing one must not overlap on the GPU.
+ * Asynchronous on `stream`; rows of other positions are not touched.  The
+ * result does not depend on the order in which CTAs finish.
  */
 int hs2_kv_bridge_append(const void *hidden, int32_t batch, int32_t d_model, const void *w_k, const void *w_v,
                          const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,

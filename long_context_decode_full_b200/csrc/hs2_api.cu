@@ -434,7 +434,7 @@ size_t hs2_kv_bridge_workspace(int32_t batch, int32_t d_model, int32_t num_kv_he
   if (batch < 1 || batch > 65535 || d_model < 1 || d_model % bridge_row_multiple() || num_kv_heads < 1 ||
       (head_dim != 64 && head_dim != 128))
     return 0;
-  return align256((size_t)2 * bridge_splits(d_model) * batch * num_kv_heads * head_dim * 4);
+  return bridge_workspace_bytes(batch, d_model, num_kv_heads * head_dim);
 }
 
 int hs2_kv_bridge_append(const void *hidden, int32_t batch, int32_t d_model, const void *w_k, const void *w_v,
@@ -486,8 +486,7 @@ int hs2_kv_bridge_append(const void *hidden, int32_t batch, int32_t d_model, con
   p.t_cap = t_cap;
   p.num_slots = k_cache->num_slots;
   p.nsplit = bridge_splits(d_model);
-  p.partial = static_cast<float *>(workspace);
-  cudaError_t e = launch_bridge(p, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_bridge(p, workspace, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "KV bridge launch");
   return HS2_OK;
 }

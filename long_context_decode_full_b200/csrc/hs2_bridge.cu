@@ -8,15 +8,18 @@
 // accumulation), written at position T_b - 1 of the paged cache: bf16 or fp32
 // as computed, or E4M3 with one fp32 scale per (token, kv head) = max|x| / 448.
 //
-// Two kernels, both memory- or latency-bound (the weights are read once):
-//   gemv  -- split-K over the hidden dimension: a CTA takes 64 output columns,
-//            256 rows of W and up to 8 tokens; each lane reads a bf16 pair of
-//            every row (128 B per warp, coalesced), the warps' partial sums
-//            meet in shared memory and land in the workspace;
-//   store -- one CTA per (sequence, kv head, K or V): the splits' partial
-//            sums in a fixed order (deterministic), then the row is stored
-//            (E4M3: block max, scale, codes rounded to nearest even with
-//            saturation).
+// One kernel, bound by reading the two weight matrices once.  A CTA takes 128
+// output columns, one split of 128 rows of W and up to 8 tokens:
+//   - each lane owns 4 columns and issues its warp's 16 row loads (8 bytes
+//     each, 256 bytes per warp and row) before any arithmetic, so about 32 KB
+//     per CTA is in flight;
+//   - the 8 warps' partial sums meet in shared memory and the CTA's tile of
+//     partial sums goes to the workspace;
+//   - the last CTA of each (K or V, column tile, token group) to finish -- a
+//     ticket counter in the workspace -- adds the splits' tiles in split order
+//     (so the result does not depend on which CTA came last), stores the rows
+//     (E4M3: one warp per token holds a whole head of 128 columns, so the
+//     row max is a warp reduction) and resets its ticket to zero.
 #include "hs2.h"
 #include "hs2_internal.h"
 
@@ -24,65 +27,102 @@ namespace hs2 {
 
 namespace {
 
-constexpr int kBridgeCols = 64;     // output columns per gemv CTA
-constexpr int kBridgeRows = 256;    // rows of W per gemv CTA (one split)
-constexpr int kBridgeTokens = 8;    // tokens per gemv CTA
+constexpr int kBridgeCols = 128;    // output columns per CTA, 4 per lane
+constexpr int kBridgeRows = 128;    // rows of W per CTA (one split)
+constexpr int kBridgeTokens = 8;    // tokens per CTA
 constexpr int kBridgeThreads = 256;
 constexpr int kBridgeWarps = kBridgeThreads / 32;
+constexpr int kRowsPerWarp = kBridgeRows / kBridgeWarps;
+static_assert(kBridgeTokens == kBridgeWarps, "the final sums give one warp to each token");
+static_assert(kBridgeCols == 4 * 32, "a lane owns 4 columns");
 
-__global__ void __launch_bounds__(kBridgeThreads) bridge_gemv_kernel(const BridgeParams p) {
-  __shared__ float sh_h[kBridgeTokens][kBridgeRows];                     // the tokens' hidden slice
-  __shared__ float sh_red[kBridgeWarps][kBridgeTokens][kBridgeCols];     // per-warp partial sums
+__device__ __forceinline__ float4 add4(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
+  __nv_bfloat162 v;
+  memcpy(&v, &u, 4);
+  return __bfloat1622float2(v);  // .x is the lower address
+}
+
+__global__ void __launch_bounds__(kBridgeThreads) bridge_kernel(const BridgeParams p) {
+  __shared__ float sh_h[kBridgeTokens][kBridgeRows];                                 // the tokens' hidden slice
+  __shared__ __align__(16) float sh_red[kBridgeWarps][kBridgeTokens][kBridgeCols];   // per-warp partial sums
+  __shared__ int sh_last;
   griddep_wait();
   griddep_launch_dependents();
   const int tile = blockIdx.x, split = blockIdx.y;
-  const int kv = blockIdx.z & 1, b0 = (blockIdx.z >> 1) * kBridgeTokens;
+  const int kv = blockIdx.z & 1, grp = blockIdx.z >> 1, b0 = grp * kBridgeTokens;
   const int nb = min(kBridgeTokens, p.B - b0);
   const int r0 = split * kBridgeRows;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = threadIdx.x; e < kBridgeTokens * kBridgeRows; e += blockDim.x) {
+  const int col = tile * kBridgeCols + 4 * lane;
+  const bool active = col < p.N;  // N is a multiple of 64: a lane's 4 columns are all in or all out
+
+  // the weight rows first (they are the traffic), then the hidden slice
+  const __nv_bfloat16 *w = kv ? p.wv : p.wk;
+  uint2 wr[kRowsPerWarp];
+#pragma unroll
+  for (int j = 0; j < kRowsPerWarp; ++j) {
+    const int r = r0 + warp + j * kBridgeWarps;
+    wr[j] = active ? __ldg(reinterpret_cast<const uint2 *>(w + (int64_t)r * p.N + col)) : make_uint2(0u, 0u);
+  }
+  for (int e = threadIdx.x; e < kBridgeTokens * kBridgeRows; e += kBridgeThreads) {
     const int t = e / kBridgeRows, r = e % kBridgeRows;
     sh_h[t][r] = t < nb ? __bfloat162float(p.h[(int64_t)(b0 + t) * p.d_model + r0 + r]) : 0.f;
   }
   __syncthreads();
-  const __nv_bfloat16 *w = kv ? p.wv : p.wk;
-  const int col = tile * kBridgeCols + 2 * lane;
-  float acc[kBridgeTokens][2];
+
+  float acc[kBridgeTokens][4];
 #pragma unroll
-  for (int t = 0; t < kBridgeTokens; ++t) acc[t][0] = acc[t][1] = 0.f;
-#pragma unroll 4
-  for (int r = warp; r < kBridgeRows; r += kBridgeWarps) {
-    const __nv_bfloat162 w2 =
-        __ldg(reinterpret_cast<const __nv_bfloat162 *>(w + (int64_t)(r0 + r) * p.N + col));
-    const float2 wf = __bfloat1622float2(w2);
+  for (int t = 0; t < kBridgeTokens; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+#pragma unroll
+  for (int j = 0; j < kRowsPerWarp; ++j) {
+    const int r = warp + j * kBridgeWarps;
+    const float2 w01 = bf16x2_to_float2(wr[j].x), w23 = bf16x2_to_float2(wr[j].y);
 #pragma unroll
     for (int t = 0; t < kBridgeTokens; ++t) {
       const float hv = sh_h[t][r];
-      acc[t][0] = fmaf(hv, wf.x, acc[t][0]);
-      acc[t][1] = fmaf(hv, wf.y, acc[t][1]);
+      acc[t][0] = fmaf(hv, w01.x, acc[t][0]);
+      acc[t][1] = fmaf(hv, w01.y, acc[t][1]);
+      acc[t][2] = fmaf(hv, w23.x, acc[t][2]);
+      acc[t][3] = fmaf(hv, w23.y, acc[t][3]);
     }
   }
 #pragma unroll
-  for (int t = 0; t < kBridgeTokens; ++t) {
-    sh_red[warp][t][2 * lane] = acc[t][0];
-    sh_red[warp][t][2 * lane + 1] = acc[t][1];
+  for (int t = 0; t < kBridgeTokens; ++t)
+    *reinterpret_cast<float4 *>(&sh_red[warp][t][4 * lane]) = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
+  __syncthreads();
+
+  // this split's tile: warp `tok` sums the 8 warps' rows of token tok in warp order
+  const int tok = warp;
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int w8 = 0; w8 < kBridgeWarps; ++w8) s = add4(s, *reinterpret_cast<const float4 *>(&sh_red[w8][tok][4 * lane]));
+  if (tok < nb && active)
+    __stcg(reinterpret_cast<float4 *>(p.partial + (((int64_t)kv * p.nsplit + split) * p.B + b0 + tok) * p.N + col), s);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int *ticket = p.tickets + ((int64_t)kv * p.ntiles + tile) * p.ngroups + grp;
+    const int last = atomicAdd(ticket, 1) == p.nsplit - 1;
+    if (last) *ticket = 0;  // every split has counted: ready for the next call
+    sh_last = last;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kBridgeTokens * kBridgeCols; e += blockDim.x) {
-    const int t = e / kBridgeCols, c = e % kBridgeCols;
-    if (t >= nb) continue;
-    float s = 0.f;
-#pragma unroll
-    for (int w8 = 0; w8 < kBridgeWarps; ++w8) s += sh_red[w8][t][c];  // fixed order
-    p.partial[(((int64_t)kv * p.nsplit + split) * p.B + b0 + t) * p.N + tile * kBridgeCols + c] = s;
-  }
-}
+  if (!sh_last || tok >= nb) return;
+  __threadfence();
 
-__global__ void bridge_store_kernel(const BridgeParams p) {
-  __shared__ float sh_max[32];
-  griddep_wait();
-  griddep_launch_dependents();
-  const int b = blockIdx.x, kvh = blockIdx.y, kv = blockIdx.z;
+  // last CTA: the splits in order, then the store (warp-uniform from here on)
+  const int b = b0 + tok;
+  float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (active) {
+    const float *src = p.partial + ((int64_t)kv * p.nsplit * p.B + b) * p.N + col;
+    const int64_t step = (int64_t)p.B * p.N;
+#pragma unroll 8
+    for (int sp = 0; sp < p.nsplit; ++sp) x = add4(x, __ldcg(reinterpret_cast<const float4 *>(src + sp * step)));
+  }
   const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
   if (T < 1) return;  // no token to append
   const int64_t pos = T - 1;
@@ -91,38 +131,56 @@ __global__ void bridge_store_kernel(const BridgeParams p) {
                            : (int64_t)__ldg(p.page_table + (int64_t)b * p.max_pages + pos / p.page_size) *
                                      p.page_size + pos % p.page_size;
   if (slot < 0 || slot >= p.num_slots) return;  // a page outside the cache: nothing is written
-  const int d = threadIdx.x;                     // blockDim.x = head_dim
-  const int n = kvh * p.D + d;
-  float x = 0.f;
-  for (int s = 0; s < p.nsplit; ++s) x += __ldcg(p.partial + (((int64_t)kv * p.nsplit + s) * p.B + b) * p.N + n);
+  const int kvh = col / p.D, d = col % p.D;      // a lane's 4 columns share one head
   const int64_t e = (slot * p.Hkv + kvh) * p.D + d;
   void *cache = kv ? p.v : p.k;
   if (p.kv_dtype == HS2_BF16) {
-    static_cast<__nv_bfloat16 *>(cache)[e] = __float2bfloat16_rn(x);
+    if (!active) return;
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(x.x, x.y), hi = __floats2bfloat162_rn(x.z, x.w);
+    uint2 u;
+    memcpy(&u.x, &lo, 4);
+    memcpy(&u.y, &hi, 4);
+    *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(cache) + e) = u;
   } else if (p.kv_dtype == HS2_F32) {
-    static_cast<float *>(cache)[e] = x;
-  } else {  // E4M3: scale = max|x| / 448 over the row, codes nearest-even, saturated
-    float m = warp_max(fabsf(x));
-    if ((threadIdx.x & 31) == 0) sh_max[threadIdx.x >> 5] = m;
-    __syncthreads();
-    float amax = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) amax = fmaxf(amax, sh_max[w]);
+    if (!active) return;
+    *reinterpret_cast<float4 *>(static_cast<float *>(cache) + e) = x;
+  } else {
+    // E4M3 caches have D = 128 = kBridgeCols: the warp holds head kvh of token
+    // b whole, every lane active.  scale = max|x| / 448, codes nearest-even,
+    // saturated.
+    const float amax = warp_max(fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w))));
     const float scale = amax > 0.f ? amax / 448.f : 1.f;
-    static_cast<__nv_fp8_e4m3 *>(cache)[e] = __nv_fp8_e4m3(x / scale);
-    if (d == 0) (kv ? p.v_scale : p.k_scale)[slot * p.Hkv + kvh] = scale;
+    const __nv_fp8_e4m3 c0(x.x / scale), c1(x.y / scale), c2(x.z / scale), c3(x.w / scale);
+    const uint32_t packed = (uint32_t)c0.__x | ((uint32_t)c1.__x << 8) | ((uint32_t)c2.__x << 16) |
+                            ((uint32_t)c3.__x << 24);
+    *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(cache) + e) = packed;
+    if (lane == 0) (kv ? p.v_scale : p.k_scale)[slot * p.Hkv + kvh] = scale;
   }
 }
+
+int ticket_words(int B, int N) {
+  return 2 * ((N + kBridgeCols - 1) / kBridgeCols) * ((B + kBridgeTokens - 1) / kBridgeTokens);
+}
+
+size_t align256_(size_t n) { return (n + 255) & ~size_t(255); }
 
 }  // namespace
 
 int bridge_splits(int d_model) { return d_model / kBridgeRows; }
 int bridge_row_multiple() { return kBridgeRows; }
 
-cudaError_t launch_bridge(const BridgeParams &p, cudaStream_t s) {
-  const dim3 g1(p.N / kBridgeCols, p.nsplit, 2 * ((p.B + kBridgeTokens - 1) / kBridgeTokens));
-  cudaError_t e = launch_ex(bridge_gemv_kernel, g1, dim3(kBridgeThreads), 0, s, 0, p);
-  if (e != cudaSuccess) return e;
-  return launch_ex(bridge_store_kernel, dim3(p.B, p.Hkv, 2), dim3(p.D), 0, s, 0, p);
+size_t bridge_workspace_bytes(int B, int d_model, int N) {
+  return align256_((size_t)ticket_words(B, N) * 4) + align256_((size_t)2 * bridge_splits(d_model) * B * N * 4);
+}
+
+cudaError_t launch_bridge(const BridgeParams &p0, void *workspace, cudaStream_t s) {
+  BridgeParams p = p0;
+  p.ntiles = (p.N + kBridgeCols - 1) / kBridgeCols;
+  p.ngroups = (p.B + kBridgeTokens - 1) / kBridgeTokens;
+  p.tickets = static_cast<int32_t *>(workspace);
+  p.partial = reinterpret_cast<float *>(static_cast<char *>(workspace) + align256_((size_t)ticket_words(p.B, p.N) * 4));
+  const dim3 grid(p.ntiles, p.nsplit, 2 * p.ngroups);
+  return launch_ex(bridge_kernel, grid, dim3(kBridgeThreads), 0, s, 0, p);
 }
 
 }  // namespace hs2

@@ -128,12 +128,16 @@ struct BridgeParams {
   int32_t B, d_model, Hkv, D, N;
   int32_t page_size, max_pages;
   int64_t t_cap, num_slots;
-  int32_t nsplit;                    // d_model / 256 row splits
+  int32_t nsplit;                    // row splits of d_model
+  int32_t ntiles, ngroups;           // column tiles, token groups (set by launch_bridge)
+  int32_t *tickets;                  // workspace [2][ntiles][ngroups], zero between calls
   float *partial;                    // workspace [2][nsplit][B][N]
 };
 int bridge_splits(int d_model);
 int bridge_row_multiple();
-cudaError_t launch_bridge(const BridgeParams &p, cudaStream_t s);
+size_t bridge_workspace_bytes(int B, int d_model, int N);
+// Splits `workspace` into tickets and partial sums and launches the append.
+cudaError_t launch_bridge(const BridgeParams &p, void *workspace, cudaStream_t s);
 
 // Sets the thread's hs2_last_error() text and returns `code`.
 int set_last_error(int code, const char *msg);

@@ -218,7 +218,8 @@ def kv_bridge_append(hidden, w_k, w_v, k, v, seq_lens, page_table=None, page_siz
                      workspace=None, stream=None):
     """KV Bridging append: writes the new token's K/V rows (hidden [B, d_model]
     bf16 times w_k / w_v [d_model, Hkv * d] bf16) at position seq_lens[b] - 1
-    of the caches k / v (and the E4M3 scales)."""
+    of the caches k / v (and the E4M3 scales).  A workspace passed in must
+    have been zero-filled once (see kv_bridge_workspace_bytes)."""
     assert hidden.dim() == 2 and hidden.is_contiguous() and w_k.is_contiguous() and w_v.is_contiguous()
     B, dm = hidden.shape
     if page_size is None:
@@ -229,7 +230,7 @@ def kv_bridge_append(hidden, w_k, w_v, k, v, seq_lens, page_table=None, page_siz
         n = kv_bridge_workspace_bytes(B, dm, k.shape[1], k.shape[2])
         if n == 0:
             raise HS2Error(ERR_INVALID_ARG, "invalid KV bridge shape")
-        workspace = torch.empty(n, dtype=torch.uint8, device=hidden.device)
+        workspace = torch.zeros(n, dtype=torch.uint8, device=hidden.device)
     kc, vc = cache_desc(k, k_scale, page_size), cache_desc(v, v_scale, page_size)
     _check(lib().hs2_kv_bridge_append(_ptr(hidden), B, dm, _ptr(w_k), _ptr(w_v), _ptr(seq_lens), _ptr(page_table),
                                       max_pages, ctypes.byref(kc), ctypes.byref(vc), _ptr(workspace),

@@ -154,5 +154,8 @@ def test_kv_bridge_rejects_bad_arguments(libhs2, kw, code):
 
 def test_kv_bridge_workspace_size_rule(libhs2):
     f = hs2.kv_bridge_workspace_bytes
-    assert f(4, 4096, 4, 128) == 2 * (4096 // 256) * 4 * 4 * 128 * 4
+    # 256 bytes of tickets (2 x 4 column tiles x 1 token group), then the
+    # partial sums [2][d_model / 128][batch][Hkv * d] fp32
+    assert f(4, 4096, 4, 128) == 256 + 2 * (4096 // 128) * 4 * 4 * 128 * 4
+    assert f(9, 128, 1, 64) == 256 + 2 * 1 * 9 * 64 * 4
     assert f(4, 4000, 4, 128) == 0 and f(0, 4096, 4, 128) == 0 and f(4, 4096, 4, 96) == 0

@@ -4,7 +4,7 @@ T_b - 1 of each sequence (bf16, fp32 or E4M3 with a per-row scale), and no
 other row of the cache changes.
 
 The kernel accumulates in fp32, the oracle in fp64.  Each kernel value is a
-chain of at most 32 + 8 + d_model / 256 fp32 additions (one warp's rows, the
+chain of at most 16 + 8 + d_model / 128 fp32 additions (one warp's rows, the
 warps, the splits), so it lies within (that depth + 2) * 2^-24 * sum_i
 |h_i w_i| of the exact dot product (the standard bound for recursive
 summation).  A stored code may differ from the oracle's only where the exact
@@ -50,6 +50,9 @@ CASES = {
     "e4m3_paged64": dict(dtype=torch.uint8, B=3, Hkv=4, d=128, dm=512, page=64),
     "e4m3_paged16": dict(dtype=torch.uint8, B=9, Hkv=4, d=128, dm=256, page=16),
     "f32_paged16_d64": dict(dtype=torch.float32, B=2, Hkv=1, d=64, dm=256, page=16),
+    # 3 heads of 64: the second 128-column tile is half empty; 11 sequences
+    # make two token groups; 3 row splits
+    "bf16_ragged_tile_b11": dict(dtype=torch.bfloat16, B=11, Hkv=3, d=64, dm=384, page=32),
 }
 
 
@@ -82,10 +85,16 @@ def test_kv_bridge_append_matches_oracle(oracle, name):
     dev = lambda t: None if t is None else t.cuda()
     k, v, ks, vs = dev(k0.clone()), dev(v0.clone()), dev(None if ks0 is None else ks0.clone()), \
         dev(None if vs0 is None else vs0.clone())
-    hs2.kv_bridge_append(h.cuda(), wk.cuda(), wv.cuda(), k, v, lens.cuda(), dev(pt), ps, ks, vs)
+    # two calls on one workspace: the first (another hidden state) checks that
+    # the call leaves its counters ready for the next; the second overwrites
+    # the same rows
+    ws = torch.zeros(hs2.kv_bridge_workspace_bytes(B, dm, Hkv, d), dtype=torch.uint8, device="cuda")
+    h_other = torch.randn(B, dm, generator=g).to(torch.bfloat16)
+    for hh in (h_other, h):
+        hs2.kv_bridge_append(hh.cuda(), wk.cuda(), wv.cuda(), k, v, lens.cuda(), dev(pt), ps, ks, vs, workspace=ws)
     torch.cuda.synchronize()
     ko, vo = oracle.kv_bridge(bf16_bits(h), bf16_bits(wk), bf16_bits(wv))
-    depth = 32 + 8 + dm // 256 + 2
+    depth = 16 + 8 + dm // 128 + 2
     habs = h.double().abs().numpy()
     eb = {"K": depth * U32 * habs @ wk.double().abs().numpy(), "V": depth * U32 * habs @ wv.double().abs().numpy()}
     k, v = k.cpu(), v.cpu()
