@@ -9,7 +9,11 @@ warps, the splits), so it lies within (that depth + 2) * 2^-24 * sum_i
 |h_i w_i| of the exact dot product (the standard bound for recursive
 summation).  A stored code may differ from the oracle's only where the exact
 value lies within that bound of the midpoint between the two codes, and at
-most 1% of the codes may differ at all."""
+most 1% of a case's codes may differ at all (one row of 64 can hold one such
+midpoint: a value 1.3e-8 from a bf16 midpoint, under a bound of 2e-5, has
+been seen to round the other way, as it may)."""
+import zlib
+
 import numpy as np
 import pytest
 import torch
@@ -36,12 +40,12 @@ def bf16_value(u):
 def check_rounded(got, ora_codes, exact, tol, decode, what):
     """got / ora_codes: stored codes; exact: the fp64 values they encode; tol:
     the kernel's error bound per value; decode: code -> value.  Codes differ
-    only next to a rounding midpoint."""
+    only next to a rounding midpoint.  Returns (differing, compared)."""
     bad = got != ora_codes
-    assert bad.mean() <= 0.01, f"{what}: {bad.sum()} of {bad.size} differ"
     for g, o, x, t in zip(got[bad], ora_codes[bad], exact[bad], tol[bad]):
         vg, vo = decode(g), decode(o)
         assert abs(x - (vg + vo) / 2) <= t, f"{what}: {x} stored as {vg}, oracle {vo}"
+    return int(bad.sum()), bad.size
 
 
 CASES = {
@@ -60,7 +64,7 @@ CASES = {
 def test_kv_bridge_append_matches_oracle(oracle, name):
     c = CASES[name]
     B, Hkv, d, dm, page = c["B"], c["Hkv"], c["d"], c["dm"], c["page"]
-    g = torch.Generator().manual_seed(hash(name) % 1000)
+    g = torch.Generator().manual_seed(zlib.crc32(name.encode()))  # stable across processes
     cap = 256
     lens = torch.randint(1, cap + 1, (B,), generator=g, dtype=torch.int32)
     lens[B // 2] = 0  # a sequence with no token: nothing is written
@@ -100,6 +104,7 @@ def test_kv_bridge_append_matches_oracle(oracle, name):
     k, v = k.cpu(), v.cpu()
     written = set()
     vals = e4m3_values(oracle)
+    differ = compared = 0
     for b in range(B):
         T = int(lens[b])
         if T < 1:
@@ -115,7 +120,8 @@ def test_kv_bridge_append_matches_oracle(oracle, name):
                 if c["dtype"] == torch.bfloat16:
                     got = bf16_bits(cache[slot, kvh])
                     ora = np.array([oracle.bf16_encode(e) for e in x], np.uint16)
-                    check_rounded(got, ora, x, tol, bf16_value, what)
+                    n, m = check_rounded(got, ora, x, tol, bf16_value, what)
+                    differ, compared = differ + n, compared + m
                 elif c["dtype"] == torch.float32:
                     err = np.abs(cache[slot, kvh].double().numpy() - x)
                     assert np.all(err <= tol), f"{what}: error {err.max()} above the bound"
@@ -131,7 +137,9 @@ def test_kv_bridge_append_matches_oracle(oracle, name):
                     y = x / s_o
                     ytol = tol / s_o + np.abs(y) * (s_tol / s_o + 2 * U32)
                     got = cache[slot, kvh].numpy()
-                    check_rounded(got, codes_o, y, ytol, lambda u: vals[int(u)], what)
+                    n, m = check_rounded(got, codes_o, y, ytol, lambda u: vals[int(u)], what)
+                    differ, compared = differ + n, compared + m
+    assert differ <= 0.01 * max(compared, 1), f"{name}: {differ} of {compared} codes differ"
     # every other row (and scale) is untouched
     for cache, orig in ((k, k0), (v, v0)):
         diff = (cache.view(torch.uint8) != orig.view(torch.uint8)).reshape(slots, Hkv, -1).any(-1)
