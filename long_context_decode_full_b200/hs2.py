@@ -98,6 +98,38 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _need(name, t, dtypes, dim=None, shape=None):
+    """The C ABI takes bare pointers: check what they cannot carry (element
+    type, rank, shape, contiguity, a CUDA device) before the call."""
+    if t is None:
+        return
+    dtypes = dtypes if isinstance(dtypes, tuple) else (dtypes,)
+    if t.dtype not in dtypes:
+        raise HS2Error(ERR_INVALID_ARG, f"{name}: dtype {t.dtype}, expected {' or '.join(map(str, dtypes))}")
+    if dim is not None and t.dim() != dim:
+        raise HS2Error(ERR_INVALID_ARG, f"{name}: {t.dim()} dimensions, expected {dim}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise HS2Error(ERR_INVALID_ARG, f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise HS2Error(ERR_INVALID_ARG, f"{name}: not contiguous")
+
+
+def _need_cuda(**tensors):
+    """Checked after every element type and shape, so a type error is
+    reported as such whatever the device."""
+    for name, t in tensors.items():
+        if t is not None and not t.is_cuda:
+            raise HS2Error(ERR_INVALID_ARG, f"{name}: not on a CUDA device")
+
+
+def _need_lens(seq_lens, page_table, B):
+    _need("seq_lens", seq_lens, torch.int32, shape=(B,))
+    if page_table is not None:
+        _need("page_table", page_table, torch.int32, dim=2)
+        if page_table.shape[0] != B:
+            raise HS2Error(ERR_INVALID_ARG, f"page_table: {page_table.shape[0]} rows for batch {B}")
+
+
 def _stream(stream) -> ctypes.c_void_p:
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
@@ -134,6 +166,9 @@ def full_attn_select(q, k, v, seq_lens, page_table=None, page_size=None, window=
     attention kernel and the selection kernels."""
     B, Hq, d = q.shape
     Hkv = k.shape[1]
+    _need_lens(seq_lens, page_table, B)
+    _need("idx_out", idx_out, torch.int32, shape=(B, Hkv, window + k_global))
+    _need_cuda(q=q, k=k, v=v, seq_lens=seq_lens, page_table=page_table, idx_out=idx_out)
     if page_size is None:
         assert page_table is None, "page_size is required with a page table"
         page_size = k.shape[0] // B
@@ -162,6 +197,9 @@ def full_attn_select_static(q, k, v, seq_lens, page_table=None, page_size=None, 
     overlap on the GPU race on that scratch."""
     B, Hq, d = q.shape
     Hkv = k.shape[1]
+    _need_lens(seq_lens, page_table, B)
+    _need("idx_out", idx_out, torch.int32, shape=(B, Hkv, window + k_global))
+    _need_cuda(q=q, k=k, v=v, seq_lens=seq_lens, page_table=page_table, idx_out=idx_out)
     if page_size is None:
         assert page_table is None, "page_size is required with a page table"
         page_size = k.shape[0] // B
@@ -180,6 +218,8 @@ def full_attn_select_static(q, k, v, seq_lens, page_table=None, page_size=None, 
 
 def sparse_attn(q_l, k, v, idx, k_scale=None, v_scale=None, page_size=1, out=None, stream=None):
     """Sparse-attention layer over the rows listed in ``idx`` (slots)."""
+    _need("idx", idx, torch.int32, dim=3)
+    _need_cuda(q=q_l, k=k, v=v, idx=idx)
     if out is None:
         out = torch.empty_like(q_l)
     kc, vc = cache_desc(k, k_scale, page_size), cache_desc(v, v_scale, page_size)
@@ -220,8 +260,18 @@ def kv_bridge_append(hidden, w_k, w_v, k, v, seq_lens, page_table=None, page_siz
     bf16 times w_k / w_v [d_model, Hkv * d] bf16) at position seq_lens[b] - 1
     of the caches k / v (and the E4M3 scales).  A workspace passed in must
     have been zero-filled once (see kv_bridge_workspace_bytes)."""
-    assert hidden.dim() == 2 and hidden.is_contiguous() and w_k.is_contiguous() and w_v.is_contiguous()
+    _need("hidden", hidden, torch.bfloat16, dim=2)
     B, dm = hidden.shape
+    if k.dim() != 3:
+        raise HS2Error(ERR_INVALID_ARG, "k: expected a [num_slots, Hkv, d] cache")
+    N = k.shape[1] * k.shape[2]
+    _need("w_k", w_k, torch.bfloat16, shape=(dm, N))
+    _need("w_v", w_v, torch.bfloat16, shape=(dm, N))
+    _need_lens(seq_lens, page_table, B)
+    _need("k_scale", k_scale, torch.float32, shape=k.shape[:2])
+    _need("v_scale", v_scale, torch.float32, shape=v.shape[:2])
+    _need_cuda(hidden=hidden, w_k=w_k, w_v=w_v, k=k, v=v, seq_lens=seq_lens, page_table=page_table,
+               k_scale=k_scale, v_scale=v_scale)
     if page_size is None:
         assert page_table is None, "page_size is required with a page table"
         page_size = k.shape[0] // B

@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from long_context_decode_full_b200 import hs2
 
@@ -159,3 +160,39 @@ def test_kv_bridge_workspace_size_rule(libhs2):
     assert f(4, 4096, 4, 128) == 256 + 2 * (4096 // 128) * 4 * 4 * 128 * 4
     assert f(9, 128, 1, 64) == 256 + 2 * 1 * 9 * 64 * 4
     assert f(4, 4000, 4, 128) == 0 and f(0, 4096, 4, 128) == 0 and f(4, 4096, 4, 96) == 0
+
+
+def _bridge_args(**over):
+    B, dm, Hkv, d, slots = 2, 256, 2, 128, 64
+    a = dict(hidden=torch.zeros(B, dm, dtype=torch.bfloat16), w_k=torch.zeros(dm, Hkv * d, dtype=torch.bfloat16),
+             w_v=torch.zeros(dm, Hkv * d, dtype=torch.bfloat16), k=torch.zeros(slots, Hkv, d, dtype=torch.bfloat16),
+             v=torch.zeros(slots, Hkv, d, dtype=torch.bfloat16), seq_lens=torch.ones(B, dtype=torch.int32),
+             page_table=torch.zeros(B, 2, dtype=torch.int32), page_size=16)
+    a.update(over)
+    return a
+
+
+@pytest.mark.parametrize("over,text", [
+    (dict(hidden=torch.zeros(2, 256)), "hidden: dtype"),
+    (dict(w_k=torch.zeros(256, 128, dtype=torch.bfloat16)), "w_k: shape"),
+    (dict(w_v=torch.zeros(256, 256, dtype=torch.float16)), "w_v: dtype"),
+    (dict(seq_lens=torch.ones(2, dtype=torch.int64)), "seq_lens: dtype"),
+    (dict(seq_lens=torch.ones(3, dtype=torch.int32)), "seq_lens: shape"),
+    (dict(page_table=torch.zeros(3, 2, dtype=torch.int32)), "page_table: 3 rows"),
+    (dict(k_scale=torch.zeros(64, 2, dtype=torch.float64)), "k_scale: dtype"),
+    (dict(), "not on a CUDA device"),
+])
+def test_binding_checks_what_pointers_cannot_carry(over, text):
+    """Element type, shape and device are checked in the binding, before the
+    C call (which only sees bare pointers)."""
+    with pytest.raises(hs2.HS2Error, match=text):
+        hs2.kv_bridge_append(**_bridge_args(**over))
+
+
+def test_binding_rejects_int64_lengths_and_lists():
+    q = torch.zeros(2, 16, 128, dtype=torch.bfloat16)
+    kv = torch.zeros(64, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(hs2.HS2Error, match="seq_lens: dtype"):
+        hs2.full_attn_select(q, kv, kv, torch.ones(2, dtype=torch.int64), torch.zeros(2, 2, dtype=torch.int32), 16)
+    with pytest.raises(hs2.HS2Error, match="idx: dtype"):
+        hs2.sparse_attn(q, kv, kv, torch.zeros(2, 2, 8, dtype=torch.int64), page_size=16)
