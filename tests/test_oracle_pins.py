@@ -414,3 +414,48 @@ def test_kv_bridge_closed_forms(oracle):
     k, v = oracle.kv_bridge(hb, wkb, wvb)
     np.testing.assert_allclose(k, h_exact @ wk_exact, rtol=0, atol=1e-12)
     np.testing.assert_allclose(v, h_exact @ wv_exact, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------- MQA (one KV head) -----
+
+def test_mqa_layer_matches_50_digit_brute_force(oracle):
+    """One KV head shared by 32 query heads: the group score sums all 32
+    heads' probabilities."""
+    spec = small_spec(num_kv_heads=1, group=32, seq_len=(9, 23))
+    w = synth.generate(spec, seed=13)
+    got = run_full(oracle, w)
+    ref = brute_full(w)
+    np.testing.assert_allclose(got["out"], ref["out"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got["lse"], ref["lse"], rtol=0, atol=1e-12)
+    for (b, kvh), sc in ref["score"].items():
+        T = int(w.seq_lens[b])
+        np.testing.assert_allclose(got["score"][b, kvh, :T], sc, rtol=1e-12, atol=0)
+        assert abs(sc.sum() - 32) < 1e-12
+
+
+def test_mqa_equals_gqa_over_copies_of_the_one_kv_head(oracle):
+    """MQA over 32 heads against GQA-8 over four identical copies of the KV
+    head: the same outputs; the MQA score is the sum of the four group
+    scores; the MQA selection is that sum's top-k (ties to the lower
+    position) plus the window."""
+    W, K = 5, 12
+    spec = small_spec(num_kv_heads=1, group=32, seq_len=(40, 90), window=W, k_global=K, page_size=8)
+    w = synth.generate(spec, seed=17)
+    mqa = run_full(oracle, w)
+    code = dtype_code(spec.kv_dtype)
+    k4 = np.repeat(synth.raw(w.k), 4, axis=1)
+    v4 = np.repeat(synth.raw(w.v), 4, axis=1)
+    gqa = oracle.full_attn_select(synth.raw(w.q_full), dtype_code(spec.q_dtype), k4, v4, code,
+                                  synth.raw(w.seq_lens), synth.raw(w.page_table), w.page_size, window=W, k_global=K)
+    np.testing.assert_allclose(mqa["out"], gqa["out"], rtol=0, atol=1e-14)
+    pt = w.page_table.numpy()
+    for b in range(spec.batch):
+        T = int(w.seq_lens[b])
+        summed = gqa["score"][b, :, :T].sum(axis=0)
+        np.testing.assert_allclose(mqa["score"][b, 0, :T], summed, rtol=1e-12, atol=0)
+        sc = mqa["score"][b, 0, :T - W]
+        order = np.lexsort((np.arange(T - W), -sc))
+        pos = sorted(order[:K].tolist() + list(range(T - W, T)))
+        slots = [int(pt[b, t // w.page_size]) * w.page_size + t % w.page_size for t in pos]
+        got = mqa["idx"][b, 0]
+        assert got[:len(slots)].tolist() == slots and np.all(got[len(slots):] == -1)
