@@ -54,6 +54,8 @@ def _load():
         lib.orc_e4m3_row.restype = None
         lib.orc_kv_bridge.argtypes = [P, I, I, P, P, I, P, P]
         lib.orc_kv_bridge.restype = I
+        lib.orc_select_blocks.argtypes = [P, I64, I, I, I, P, I, I, I, P]
+        lib.orc_select_blocks.restype = I
         _lib = lib
     return _lib
 
@@ -173,3 +175,46 @@ def kv_bridge(h, wk, wv):
     rc = _load().orc_kv_bridge(_ptr(h), B, dm, _ptr(wk), _ptr(wv), n, _ptr(k), _ptr(v))
     assert rc == 0
     return k, v
+
+
+def select_blocks(score, T, window, k_global, block):
+    """Block-level selection (first-generation HySparse) over one score row:
+    the taken positions, ascending (window included)."""
+    score = np.ascontiguousarray(np.asarray(score, np.float64)[:T])
+    idx = np.full(window + k_global, -1, np.int32)
+    n = _load().orc_select_blocks(_ptr(score), int(T), window, k_global, block, None, 1, max(int(T), 1), 0,
+                                  _ptr(idx))
+    if n < 0:
+        raise ValueError("block size must divide k_global")
+    return idx[:n].copy()
+
+
+def full_attn_select_blocks(q, q_dtype, k, v, kv_dtype, seq_lens, page_table=None, page_size=None,
+                            window=128, k_global=1024, block=64, k_scale=None, v_scale=None):
+    """The full layer with block-level instead of token-level selection: the
+    same attention output and group scores, and ``idx`` [B, Hkv, window +
+    k_global] slots of the taken blocks' positions plus the window."""
+    r = full_attn_select(q, q_dtype, k, v, kv_dtype, seq_lens, page_table, page_size, window, k_global,
+                         k_scale, v_scale)
+    seq_lens = _c(seq_lens, np.int32)
+    B, Hkv = r["idx"].shape[:2]
+    if page_table is not None:
+        page_table = _c(page_table, np.int32)
+        max_pages = page_table.shape[1]
+    else:
+        max_pages = 1
+        page_size = k.shape[0] // B if page_size is None else page_size
+    idx = np.full((B, Hkv, window + k_global), -1, np.int32)
+    n_sel = np.zeros((B, Hkv), np.int32)
+    for b in range(B):
+        T = int(seq_lens[b])
+        for h in range(Hkv):
+            row = np.ascontiguousarray(r["score"][b, h, :max(T, 1)])
+            out = idx[b, h]
+            n = _load().orc_select_blocks(_ptr(row), T, window, k_global, block, _ptr(page_table), max_pages,
+                                          page_size, b, out.ctypes.data_as(ctypes.c_void_p))
+            if n < 0:
+                raise ValueError("block size must divide k_global")
+            n_sel[b, h] = n
+    r["idx"], r["n_sel"] = idx, n_sel
+    return r

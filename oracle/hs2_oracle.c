@@ -17,6 +17,8 @@
  *     always taken, plus 1,024 global tokens chosen from outside that window;
  *   - the window and the global tokens are read from the same shared KV cache
  *     in one sparse-attention computation (no separate sliding-window branch);
+ *   - (paragraphs on first-generation HySparse) the block-level selection it
+ *     used, as a comparator at the same token budget (orc_select_blocks);
  *   - ("KV Bridging" paragraphs) each Cross-Decoder full-attention layer
  *     builds its KV cache from the matching Self-Decoder layer's input hidden
  *     state through its own K/V projections (orc_kv_bridge and the encoders
@@ -203,6 +205,58 @@ done:
   free(s);
   free(taken);
   free(cand);
+  return rc;
+}
+
+/*
+ * Block-level selection, the first-generation HySparse comparator (the
+ * announcement's paragraphs on HySparse v1: it selected whole blocks, so one
+ * important token brought in the block around it; HySparse2's token-level
+ * selection was compared with it at the same token budget).  Readings: the
+ * candidates [0, T-W) are cut into blocks [j*block, (j+1)*block), the last
+ * one cut short at T-W; a block's score is the sum of its positions' group
+ * scores; k_global / block blocks are taken by (block score descending, block
+ * index ascending), all of them when there are no more; the window
+ * [max(0,T-W), T) is always taken.  idx gets the slots of the taken positions
+ * in position order, -1 padded to window + k_global.  Returns the count, or
+ * -1 for a block size that does not divide k_global (or no memory).
+ */
+int orc_select_blocks(const double *score, int64_t T, int window, int k_global, int block,
+                      const int32_t *page_table, int max_pages, int page_size, int b, int32_t *idx) {
+  if (block < 1 || k_global % block != 0) return -1;
+  const int64_t n_cand = T > window ? T - window : 0;
+  const int64_t n_blocks = (n_cand + block - 1) / block, keep = k_global / block;
+  char *taken = calloc((size_t)(T > 0 ? T : 1), 1);
+  orc_cand *blk = NULL;
+  int rc = -1;
+  if (!taken) return -1;
+  for (int64_t t = n_cand; t < T; ++t) taken[t] = 1;
+  if (n_blocks <= keep) {
+    for (int64_t t = 0; t < n_cand; ++t) taken[t] = 1;
+  } else {
+    blk = malloc(sizeof(orc_cand) * (size_t)n_blocks);
+    if (!blk) goto done;
+    for (int64_t j = 0; j < n_blocks; ++j) {
+      const int64_t t1 = (j + 1) * block < n_cand ? (j + 1) * block : n_cand;
+      double sum = 0.0;
+      for (int64_t t = j * block; t < t1; ++t) sum += score[t];
+      blk[j].score = sum;
+      blk[j].t = j;
+    }
+    qsort(blk, (size_t)n_blocks, sizeof(orc_cand), cand_order);
+    for (int64_t i = 0; i < keep; ++i) {
+      const int64_t j = blk[i].t, t1 = (j + 1) * block < n_cand ? (j + 1) * block : n_cand;
+      for (int64_t t = j * block; t < t1; ++t) taken[t] = 1;
+    }
+  }
+  int n = 0;
+  for (int64_t t = 0; t < T; ++t)
+    if (taken[t]) idx[n++] = (int32_t)slot_of(page_table, max_pages, page_size, b, t);
+  for (int i = n; i < window + k_global; ++i) idx[i] = -1;
+  rc = n;
+done:
+  free(taken);
+  free(blk);
   return rc;
 }
 

@@ -459,3 +459,76 @@ def test_mqa_equals_gqa_over_copies_of_the_one_kv_head(oracle):
         slots = [int(pt[b, t // w.page_size]) * w.page_size + t % w.page_size for t in pos]
         got = mqa["idx"][b, 0]
         assert got[:len(slots)].tolist() == slots and np.all(got[len(slots):] == -1)
+
+
+# ------------------------------ block-level selection (HySparse v1) -----
+
+def _block_rank_reference(score, T, W, K, block):
+    """The definition, by counting: block j is taken when fewer than
+    K / block blocks beat it (a higher sum, or an equal sum and a lower
+    index).  Scores are dyadic here, so every sum is exact."""
+    n_cand = max(T - W, 0)
+    blocks = [list(range(j, min(j + block, n_cand))) for j in range(0, n_cand, block)]
+    sums = [sum(score[t] for t in blk) for blk in blocks]
+    keep = K // block
+    taken = set(range(n_cand, T))
+    for j, blk in enumerate(blocks):
+        beat = sum(1 for i in range(len(blocks)) if sums[i] > sums[j] or (sums[i] == sums[j] and i < j))
+        if beat < keep:
+            taken.update(blk)
+    return sorted(taken)
+
+
+@pytest.mark.parametrize("block", [1, 2, 3, 4, 6])
+def test_block_selection_matches_exhaustive_block_ranking(oracle, block):
+    g = np.random.default_rng(100 + block)
+    for _ in range(40):
+        T = int(g.integers(1, 120))
+        W = int(g.integers(0, 10))
+        K = block * int(g.integers(1, 6))
+        score = g.integers(0, 6, T) / 8.0  # dyadic: exact sums, frequent ties
+        got = oracle.select_blocks(score, T, W, K, block)
+        assert got.tolist() == _block_rank_reference(score, T, W, K, block), (T, W, K)
+
+
+def test_blocks_of_one_position_are_token_selection(oracle):
+    spec = small_spec(seq_len=(40, 90), window=5, k_global=12, page_size=8)
+    for seed, zero_q in ((3, False), (4, True)):
+        w = synth.generate(spec, seed=seed)
+        if zero_q:  # every score equal: the order is all ties
+            w.q_full = torch.zeros_like(w.q_full)
+        args = (synth.raw(w.q_full), dtype_code(spec.q_dtype), synth.raw(w.k), synth.raw(w.v),
+                dtype_code(spec.kv_dtype), synth.raw(w.seq_lens), synth.raw(w.page_table), w.page_size)
+        tok = oracle.full_attn_select(*args, window=5, k_global=12)
+        blk = oracle.full_attn_select_blocks(*args, window=5, k_global=12, block=1)
+        assert np.array_equal(tok["idx"], blk["idx"]) and np.array_equal(tok["n_sel"], blk["n_sel"])
+        assert np.array_equal(tok["out"], blk["out"])
+
+
+def test_one_needle_brings_its_whole_block(oracle):
+    T, W, K, block = 300, 20, 32, 16
+    score = np.full(T, 1e-4)
+    score[137] = 0.9  # block 8 = [128, 144)
+    score[30] = 0.05  # block 1 = [16, 32)
+    got = oracle.select_blocks(score, T, W, K, block)
+    assert got.tolist() == list(range(16, 32)) + list(range(128, 144)) + list(range(T - W, T))
+
+
+def test_ragged_last_block_and_short_contexts(oracle):
+    W, K, block = 4, 8, 4
+    # candidates [0, 10): blocks [0,4) [4,8) [8,10); the short last block wins
+    score = np.zeros(14)
+    score[8:10] = 1.0
+    score[0:4] = 0.25  # block sums: 1.0, 0, 2.0
+    got = oracle.select_blocks(score, 14, W, K, block)
+    assert got.tolist() == [0, 1, 2, 3, 8, 9, 10, 11, 12, 13]
+    # the short block stops at T - W: the window's scores are not part of it
+    # (block sums 1.0, 0.9, 0.5; running on into the window would make 1.1)
+    score = np.array([0.25] * 4 + [0.225] * 4 + [0.25] * 2 + [0.3] * 4)
+    assert oracle.select_blocks(score, 14, W, K, block).tolist() == list(range(8)) + [10, 11, 12, 13]
+    # no more candidate blocks than the budget: everything is taken
+    assert oracle.select_blocks(np.ones(11), 11, W, K, block).tolist() == list(range(11))
+    assert oracle.select_blocks(np.ones(3), 3, W, K, block).tolist() == [0, 1, 2]
+    assert oracle.select_blocks(np.ones(1), 0, W, K, block).tolist() == []
+    with pytest.raises(ValueError):
+        oracle.select_blocks(np.ones(20), 20, W, K, 3)
