@@ -204,7 +204,8 @@ FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged) {
   const int n = fp8 ? 4 : (D == 64 ? 2 : 3);
   if (const char *env = getenv("HS2_FULL_CFG")) {  // tuning override: "ncw,nstage[,nsl]"
     int a = 0, b = 0, c = 1;
-    if (sscanf(env, "%d,%d,%d", &a, &b, &c) >= 2 && tile_fits_pages(16 * a * c, page_size, paged))
+    if (sscanf(env, "%d,%d,%d", &a, &b, &c) >= 2 && a >= 1 && a <= 16 && b >= 1 && b <= 16 && (c == 1 || c == 2) &&
+        tile_fits_pages(16 * a * c, page_size, paged))
       return FullMmaConfig{a, b, c};
   }
   for (int i = 0; i < n; ++i)
