@@ -473,7 +473,9 @@ def run_gpu(args, rank, world, local):
         "clocks": clk,
         "device_status": status,
     }
-    if not args.no_bridge:
+    if not args.no_bridge and world == 1:
+        # a per-GPU figure; with one process there is no NCCL thread about
+        # while the graph is captured
         res["kv_bridge_append"] = time_kv_bridge(w, dev, stream, peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
