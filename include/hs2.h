@@ -114,6 +114,9 @@ size_t hs2_full_attn_select_workspace(int32_t batch, int32_t num_kv_heads, int32
  *              need no initialisation and are overwritten (except the sticky
  *              error flag).  One workspace must not serve two calls that
  *              run concurrently.
+ * Limits: W + K <= 4096 (else HS2_ERR_INVALID_ARG); batch <= 4096, a
+ * capacity t_cap <= 2^23 positions per sequence and
+ * B * ceil(t_cap / 16) * Hkv < 2^31 (else HS2_ERR_UNSUPPORTED).
  */
 int hs2_full_attn_select(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
                          const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
