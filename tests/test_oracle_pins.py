@@ -532,3 +532,21 @@ def test_ragged_last_block_and_short_contexts(oracle):
     assert oracle.select_blocks(np.ones(1), 0, W, K, block).tolist() == []
     with pytest.raises(ValueError):
         oracle.select_blocks(np.ones(20), 20, W, K, 3)
+
+
+@pytest.mark.parametrize("kv_dtype,page", [("bf16", 4), ("e4m3", 8), ("f32", None)])
+def test_rows_outside_the_sequences_are_never_read(oracle, kv_dtype, page):
+    """Every cache row no sequence position maps to is NaN (E4M3: the NaN
+    code): the full layer, the selection and a sparse layer over its list
+    are unchanged."""
+    spec = small_spec(kv_dtype=kv_dtype, q_dtype="f32" if kv_dtype == "f32" else "bf16", page_size=page,
+                      seq_len=(9, 30))
+    clean = synth.generate(spec, seed=23)
+    padded = synth.generate(spec, seed=23, pad_fill="nan")
+    assert np.isnan(dequant(padded, "k")).any()  # the fill is really there
+    a, b = run_full(oracle, clean), run_full(oracle, padded)
+    assert not np.isnan(b["out"]).any()
+    assert np.array_equal(a["out"], b["out"]) and np.array_equal(a["idx"], b["idx"])
+    sa = run_sparse(oracle, clean, clean.q_sparse[0], a["idx"])
+    sb = run_sparse(oracle, padded, padded.q_sparse[0], b["idx"])
+    assert np.array_equal(sa, sb)
