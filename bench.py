@@ -260,6 +260,15 @@ def cpu_baseline(w: synth.Workload, seconds: float = 10.0, max_units: int = 256)
 BRIDGE_D_MODEL = 4096  # the pages give no hidden size; a synthetic stand-in
 
 
+def bridge_bytes(batch, d_model, num_kv_heads, head_dim, elt, scales):
+    """Compulsory bytes of one KV Bridging append: both bf16 weight matrices
+    once, the bf16 hidden states, and the stored K and V rows (+ their fp32
+    scales for E4M3)."""
+    n = num_kv_heads * head_dim
+    return (2 * d_model * n * 2 + batch * d_model * 2 + 2 * batch * n * elt
+            + (2 * batch * num_kv_heads * 4 if scales else 0))
+
+
 def time_kv_bridge(w, dev, stream, peak, iters=20):
     """The decode-time KV Bridging append on the workload's batch and cache,
     L2 flushed before every launch so the weights come from HBM as they do
@@ -331,9 +340,8 @@ def time_kv_bridge(w, dev, stream, peak, iters=20):
         graph_us, us = None, isolated_us
         method = f"isolated launches (graph capture failed: {str(e).splitlines()[0][:120]})"
     torch.cuda.synchronize()
-    elt = w.k.element_size()
-    nbytes = (2 * BRIDGE_D_MODEL * N * 2 + s.batch * BRIDGE_D_MODEL * 2 + 2 * s.batch * N * elt
-              + (2 * s.batch * s.num_kv_heads * 4 if w.k_scale is not None else 0))
+    nbytes = bridge_bytes(s.batch, BRIDGE_D_MODEL, s.num_kv_heads, s.head_dim, w.k.element_size(),
+                          w.k_scale is not None)
     gbs = nbytes / (us * 1e-6) / 1e9
     return {"d_model": BRIDGE_D_MODEL, "us": us, "method": method, "graph_us": graph_us,
             "isolated_launch_us": isolated_us, "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
