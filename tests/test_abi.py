@@ -196,3 +196,33 @@ def test_binding_rejects_int64_lengths_and_lists():
         hs2.full_attn_select(q, kv, kv, torch.ones(2, dtype=torch.int64), torch.zeros(2, 2, dtype=torch.int32), 16)
     with pytest.raises(hs2.HS2Error, match="idx: dtype"):
         hs2.sparse_attn(q, kv, kv, torch.zeros(2, 2, 8, dtype=torch.int64), page_size=16)
+
+
+def test_header_is_plain_c_and_links(libhs2, tmp_path):
+    """include/hs2.h compiles as C99 and every entry point it declares links
+    against libhs2.so from a C program, which then makes the calls that need
+    no GPU (sizes, version, a rejected argument and its message)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    names = declared_functions()
+    src = tmp_path / "use_hs2.c"
+    src.write_text(
+        "#include <stdio.h>\n#include \"hs2.h\"\n"
+        "static void *const entry[] = {" + ", ".join(f"(void *){n}" for n in names) + "};\n"
+        "int main(void) {\n"
+        "  size_t ws = hs2_kv_bridge_workspace(4, 4096, 4, 128);\n"
+        "  int rc = hs2_copy_peak(NULL, NULL, 16, NULL);\n"
+        "  printf(\"%d %zu %d %d %s\\n\", hs2_version(), ws, rc, (int)(sizeof entry / sizeof entry[0]),\n"
+        "         hs2_last_error());\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "use_hs2"
+    libdir = os.path.dirname(hs2.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                    "-L", libdir, "-lhs2", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split(maxsplit=4)
+    assert int(out[0]) == hs2.version()
+    assert int(out[1]) == hs2.kv_bridge_workspace_bytes(4, 4096, 4, 128)
+    assert int(out[2]) == hs2.ERR_INVALID_ARG and int(out[3]) == len(names) and out[4].strip()
