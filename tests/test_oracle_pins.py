@@ -459,6 +459,11 @@ def test_mqa_equals_gqa_over_copies_of_the_one_kv_head(oracle):
         slots = [int(pt[b, t // w.page_size]) * w.page_size + t % w.page_size for t in pos]
         got = mqa["idx"][b, 0]
         assert got[:len(slots)].tolist() == slots and np.all(got[len(slots):] == -1)
+    # a sparse layer over the MQA list equals one over the same list given to each of the four copies
+    q_s = synth.raw(w.q_sparse[0])
+    s1 = oracle.sparse_attn(q_s, dtype_code(spec.q_dtype), synth.raw(w.k), synth.raw(w.v), code, mqa["idx"])
+    s4 = oracle.sparse_attn(q_s, dtype_code(spec.q_dtype), k4, v4, code, np.repeat(mqa["idx"], 4, axis=1))
+    np.testing.assert_allclose(s1, s4, rtol=0, atol=1e-14)
 
 
 # ------------------------------ block-level selection (HySparse v1) -----
