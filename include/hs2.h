@@ -93,6 +93,14 @@ size_t hs2_full_attn_select_workspace(int32_t batch, int32_t num_kv_heads, int32
 /*
  * Full-attention layer of a Hybrid Block, with token selection.
  *
+ * Passage: HySparse2 announcement for MiMo-V3, "KV Reuse" section -- the
+ * block's one full-attention layer attends over the whole shared KV cache and,
+ * while computing its own attention, picks the important positions from its
+ * attention scores (no separately trained selector); the next two paragraphs
+ * make the selection per token and fix the budget: the most recent 128 tokens
+ * always, plus 1,024 global tokens from outside that window.  (The same
+ * section is 02-03 of the Vietnamese translation of the announcement.)
+ *
  *   q          [B, Hq, d] device, the full layer's query of the new token.
  *   k_cache,
  *   v_cache    the shared cache (same dtype, heads, head_dim, page_size,
@@ -139,23 +147,26 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
  * The pages have no counterpart to this call; it exists for integration.
  *
  * Some callers only receive device pointers and a stream and are not allowed
- * to call cudaMalloc: a plugin inside a serving engine that has already
- * reserved nearly all HBM for its own KV-cache pool, or code whose launches
- * are later recorded into a CUDA graph, where allocating is not permitted.
- * They cannot provide the workspace hs2_full_attn_select() needs, so this
- * call uses a scratch array that the library itself owns: a fixed 32 MiB
- * device array that every GPU which loads the library keeps until the
+ * to call cudaMalloc: a plugin inside a serving engine that has reserved
+ * nearly all HBM for its own KV-cache pool up front, or an extension of a
+ * runtime that plans every buffer before execution and gives its kernels no
+ * scratch.  They cannot provide the workspace hs2_full_attn_select() needs,
+ * so this call uses a scratch array that the library itself owns: a fixed
+ * 32 MiB device array that every GPU which loads the library keeps until the
  * process exits.  The call allocates nothing.
  *
  *   Arguments and results are those of hs2_full_attn_select() without the
  *   workspace.  Shapes whose workspace (hs2_full_attn_select_workspace())
  *   exceeds 32 MiB are rejected with HS2_ERR_WORKSPACE and a message.
- *   The first call on each device looks up the array's device address on
- *   that device; make that first call before any stream capture begins.
+ *   The first call in each CUDA context (per device, for the runtime's primary
+ *   contexts) looks up the array's device address in that context; make that
+ *   first call before any stream capture begins.
  *   All calls share the one array and it keeps the last call's contents (the
  *   kernels clear what must start at zero themselves): calls that overlap on
  *   the GPU -- on different streams, or from different threads -- race and
  *   must be serialised by the caller.
+ *   Word 0 of the array is the sticky device-error flag of these calls; read
+ *   it with hs2_full_attn_select_static_status().
  */
 int hs2_full_attn_select_static(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
                                 const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
@@ -163,6 +174,21 @@ int hs2_full_attn_select_static(const hs2_heads *q, const hs2_cache *k_cache, co
                                 void *stream);
 
 /*
+ * Status of hs2_full_attn_select_static() calls in the current CUDA context
+ * (no counterpart in the pages): synchronises `stream`, then reads and clears
+ * the static scratch's sticky device-error flag.  HS2_OK, or HS2_ERR_TIMEOUT
+ * if a bounded device wait of an earlier static call expired (its out and
+ * idx_out are then incomplete).
+ */
+int hs2_full_attn_select_static_status(void *stream);
+
+/*
+ * Passage: HySparse2 announcement, "KV Reuse" section and the paragraph after
+ * the forced window -- every sparse layer of the block reuses the full
+ * layer's KV cache and its selection indices directly, and reads the window
+ * and the global tokens from that one cache in a single sparse-attention
+ * computation, with no sliding-window branch and no KV cache of its own.
+ *
  * Sparse-attention layer of a Hybrid Block: for each (b, query head h) the
  * softmax of q_l k^T / sqrt(d) over the rows idx[b, floor(h/G), :] (slots,
  * -1 entries skipped), times those V rows.  It reads the same shared cache as
@@ -245,6 +271,14 @@ int hs2_kv_bridge_append(const void *hidden, int32_t batch, int32_t d_model, con
  * Returns HS2_OK once launched (asynchronous on `stream`).
  */
 int hs2_selftest_bounded_wait(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The same self-test on the static scratch of hs2_full_attn_select_static()
+ * in the current CUDA context: afterwards hs2_full_attn_select_static_status()
+ * returns HS2_ERR_TIMEOUT once (and clears the flag).  Must not overlap a
+ * static call on the GPU.
+ */
+int hs2_selftest_bounded_wait_static(void *stream);
 
 const char *hs2_last_error(void);
 

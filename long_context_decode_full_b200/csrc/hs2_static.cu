@@ -4,15 +4,19 @@
 //
 // Who needs it: code that only receives device pointers and a stream and may
 // not call cudaMalloc -- for example a plugin inside a serving engine that
-// has already reserved almost all HBM for its own KV-cache pool and forbids
-// any further device allocation, or code whose calls are later recorded into
-// a CUDA graph, where allocating is not permitted.  Such callers cannot hand
-// hs2_full_attn_select() a workspace, so this entry point brings its own.
+// has reserved almost all HBM for its own KV-cache pool up front and forbids
+// any later device allocation, or an extension of a runtime that plans every
+// buffer before execution starts and hands its kernels no scratch.  Such
+// callers cannot give hs2_full_attn_select() a workspace, so this entry point
+// brings its own.
 //
 // The scratch is a file-scope __device__ array of kStaticScratchBytes (32 MiB);
-// every GPU that loads the library holds it until the process exits.  Its
-// device address is looked up once per device (cudaGetSymbolAddress, with
-// that device current) on the first call made on that device.
+// every GPU that loads the library holds it until the process exits.  In host
+// code the array's name is only a stand-in, so its device address is looked
+// up with cudaGetSymbolAddress once per CUDA context (with that context
+// current), on the first call made in that context, and cached.  Word 0 of
+// the array is the kernels' sticky error flag, which
+// hs2_full_attn_select_static_status() reads and clears.
 #include <stdio.h>
 
 #include <mutex>
@@ -25,9 +29,62 @@ namespace {
 constexpr size_t kStaticScratchBytes = size_t(32) << 20;
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-constexpr int kMaxDevices = 64;
-void *g_scratch_ptr[kMaxDevices] = {nullptr};
-std::mutex g_scratch_mu;
+// Device address of the array in each CUDA context seen so far.  A module is
+// loaded once per context, so the address is per context, not per device.
+constexpr int kMaxContexts = 64;
+struct CtxEntry {
+  void *ctx;
+  void *ptr;
+};
+CtxEntry g_entries[kMaxContexts];
+int g_num_entries = 0;
+std::mutex g_mu;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// The array's device address in the current context (looked up on first use).
+int scratch_address(void **out) {
+  CtxGetCurrentFn get = ctx_get_current();
+  if (!get) return hs2::set_last_error(HS2_ERR_CUDA, "cuCtxGetCurrent is not available from the driver");
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return hs2::set_last_error(HS2_ERR_CUDA, "cuCtxGetCurrent failed");
+  if (!ctx) {  // nothing bound yet: the symbol lookup binds the current device's primary context
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || get(&ctx) != CUDA_SUCCESS || !ctx)
+      return hs2::set_last_error(HS2_ERR_CUDA, "no usable current CUDA device");
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (int i = 0; i < g_num_entries; ++i)
+    if (g_entries[i].ctx == ctx) {
+      *out = g_entries[i].ptr;
+      return HS2_OK;
+    }
+  if (g_num_entries == kMaxContexts)
+    return hs2::set_last_error(HS2_ERR_CUDA, "more CUDA contexts than the static scratch keeps addresses for");
+  void *p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (e != cudaSuccess || !p) {
+    char msg[256];
+    snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+    return hs2::set_last_error(HS2_ERR_CUDA, msg);
+  }
+  g_entries[g_num_entries++] = CtxEntry{ctx, p};
+  *out = p;
+  return HS2_OK;
+}
 
 }  // namespace
 
@@ -49,24 +106,29 @@ extern "C" int hs2_full_attn_select_static(const hs2_heads *q, const hs2_cache *
       return hs2::set_last_error(HS2_ERR_WORKSPACE, msg);
     }
   }
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-    return hs2::set_last_error(HS2_ERR_CUDA, "no usable current CUDA device");
-  void *scratch;
-  {
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-      void *p = nullptr;
-      const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-      if (e != cudaSuccess || !p) {
-        char msg[256];
-        snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
-        return hs2::set_last_error(HS2_ERR_CUDA, msg);
-      }
-      g_scratch_ptr[dev] = p;
-    }
-    scratch = g_scratch_ptr[dev];
-  }
+  void *scratch = nullptr;
+  int rc = scratch_address(&scratch);
+  if (rc != HS2_OK) return rc;
   return hs2_full_attn_select(q, k_cache, v_cache, seq_lens, page_table, max_pages, window, k_global, out, idx_out,
                               scratch, kStaticScratchBytes, stream);
+}
+
+extern "C" int hs2_full_attn_select_static_status(void *stream) {
+  void *scratch = nullptr;
+  int rc = scratch_address(&scratch);
+  if (rc != HS2_OK) return rc;
+  return hs2_workspace_status(scratch, kStaticScratchBytes, stream);
+}
+
+extern "C" int hs2_selftest_bounded_wait_static(void *stream) {
+  void *scratch = nullptr;
+  int rc = scratch_address(&scratch);
+  if (rc != HS2_OK) return rc;
+  const cudaError_t e = hs2::launch_wait_selftest(static_cast<uint32_t *>(scratch), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    char msg[256];
+    snprintf(msg, sizeof msg, "self-test launch: %s", cudaGetErrorString(e));
+    return hs2::set_last_error(HS2_ERR_CUDA, msg);
+  }
+  return HS2_OK;
 }

@@ -42,7 +42,8 @@ class HS2Error(RuntimeError):
 
 _lib = None
 EXPORTS = ["hs2_full_attn_select_workspace", "hs2_full_attn_select", "hs2_full_attn_select_marked",
-           "hs2_full_attn_select_static", "hs2_sparse_attn",
+           "hs2_full_attn_select_static", "hs2_full_attn_select_static_status", "hs2_selftest_bounded_wait_static",
+           "hs2_sparse_attn",
            "hs2_workspace_status", "hs2_selftest_bounded_wait", "hs2_kv_bridge_workspace", "hs2_kv_bridge_append",
            "hs2_copy_peak", "hs2_last_error", "hs2_version"]
 
@@ -67,6 +68,10 @@ def lib():
                                                   ctypes.POINTER(Cache), P, P, I32, I32, I32,
                                                   ctypes.POINTER(Heads), P, P]
         L.hs2_full_attn_select_static.restype = ctypes.c_int
+        L.hs2_full_attn_select_static_status.argtypes = [P]
+        L.hs2_full_attn_select_static_status.restype = ctypes.c_int
+        L.hs2_selftest_bounded_wait_static.argtypes = [P]
+        L.hs2_selftest_bounded_wait_static.restype = ctypes.c_int
         L.hs2_sparse_attn.argtypes = [ctypes.POINTER(Heads), ctypes.POINTER(Cache), ctypes.POINTER(Cache), P, I32,
                                       ctypes.POINTER(Heads), P]
         L.hs2_sparse_attn.restype = ctypes.c_int
@@ -194,7 +199,8 @@ def full_attn_select_static(q, k, v, seq_lens, page_table=None, page_size=None, 
                             k_scale=None, v_scale=None, out=None, idx_out=None, stream=None):
     """full_attn_select() without a workspace: the library's own fixed 32 MiB
     device scratch is used (for callers that may not allocate).  Calls that
-    overlap on the GPU race on that scratch."""
+    overlap on the GPU race on that scratch; static_status() reports an
+    expired device wait of these calls."""
     B, Hq, d = q.shape
     Hkv = k.shape[1]
     _need_lens(seq_lens, page_table, B)
@@ -214,6 +220,12 @@ def full_attn_select_static(q, k, v, seq_lens, page_table=None, page_size=None, 
                                              _ptr(seq_lens), _ptr(page_table), max_pages, window, k_global,
                                              ctypes.byref(od), _ptr(idx_out), _stream(stream)))
     return out, idx_out
+
+
+def static_status(stream=None) -> int:
+    """Synchronises the stream, returns and clears the sticky device error flag
+    of full_attn_select_static() calls in the current CUDA context."""
+    return int(lib().hs2_full_attn_select_static_status(_stream(stream)))
 
 
 def sparse_attn(q_l, k, v, idx, k_scale=None, v_scale=None, page_size=1, out=None, stream=None):

@@ -1,10 +1,10 @@
 """hs2_full_attn_select_static: the full-attention + selection call for
-callers that may not allocate device memory (for instance a plugin inside a
+callers that may not allocate device memory -- for instance a plugin inside a
 serving engine that has reserved nearly all HBM for its own KV-cache pool, or
-code whose launches end up inside a CUDA graph, where allocating is not
-allowed).  It runs on the library's own fixed 32 MiB device scratch instead of
-a caller workspace.  This file runs last, so a failure here cannot hide the
-results of the other tests."""
+an extension of a runtime that plans every buffer before execution and gives
+its kernels no scratch.  It runs on the library's own fixed 32 MiB device
+scratch instead of a caller workspace.  This file runs last, so a failure here
+cannot hide the results of the other tests."""
 import ctypes
 
 import pytest
@@ -29,6 +29,10 @@ def _static_call(w, out, idx):
         s.k_global, ctypes.byref(od), ctypes.c_void_p(idx.data_ptr()), stream)
 
 
+def _status():
+    return hs2.lib().hs2_full_attn_select_static_status(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
 @pytest.mark.parametrize("kv_dtype", ["bf16", "e4m3"])
 def test_static_scratch_matches_workspace_call_twice_in_a_row(kv_dtype):
     spec = synth.WorkloadSpec("noalloc", batch=2, num_kv_heads=2, group=8, head_dim=128, seq_len=(2000, 6000),
@@ -40,10 +44,19 @@ def test_static_scratch_matches_workspace_call_twice_in_a_row(kv_dtype):
         out = torch.full_like(ref_out, float("nan"))
         idx = torch.full_like(ref_idx, -7)
         assert _static_call(w, out, idx) == hs2.OK, hs2.last_error()
-        torch.cuda.synchronize()
+        assert _status() == hs2.OK, hs2.last_error()  # synchronises; no device wait expired
         err = (out.float() - ref_out.float()).abs().max().item()
         assert err <= U.TOL[kv_dtype]
         assert torch.equal(idx, ref_idx)
+
+
+def test_static_status_reports_an_expired_wait_once():
+    assert _status() == hs2.OK
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert hs2.lib().hs2_selftest_bounded_wait_static(stream) == hs2.OK
+    assert _status() == hs2.ERR_TIMEOUT
+    assert "flag" in hs2.last_error()
+    assert _status() == hs2.OK  # read and cleared
 
 
 def test_static_scratch_rejects_shapes_beyond_its_size():
