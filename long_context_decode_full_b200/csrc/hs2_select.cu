@@ -37,6 +37,19 @@ namespace hs2 {
 namespace {
 
 constexpr double kLog2e = 1.4426950408889634074;
+constexpr double kLn2 = 0.69314718055994530942;
+
+// Far below the window, group probabilities can fall under fp32's normal
+// range (2^-126: logit margins above ~87 nats), where ex2 flushes them to 0.
+// When the k_global-th approximate score lies below 2^-96, the unit's scores
+// are recomputed with a common factor 2^E (a common factor keeps the order):
+// E is raised until the threshold bin sits near 2^-32, far from both ends of
+// fp32's range.  Scores far above it may overflow to +inf; they are certainly
+// selected and are counted as such.  E stops at 948, where a score still 0 in
+// fp32 is below 2^-1074 and so 0 in fp64 as well.
+constexpr int kTrustBin = 31 << 4;     // threshold bin of 2^-96 (biased exponent 31)
+constexpr int kTargetExponent = 95;    // biased exponent of 2^-32
+constexpr double kMaxShift = 948.0;
 
 constexpr int kMaxRecords = 1024;  // >= records per unit (4 * SMs / Hkv + 2)
 
@@ -220,6 +233,45 @@ __device__ __forceinline__ void load_logits(float (&raw)[kScoreLoads][G], const 
   }
 }
 
+// The unit's approximate scores and histogram again, each score scaled by
+// 2^E, until the threshold bin is at or above kTrustBin (whole block; runs
+// only when the first pass put the k-th score below 2^-96).  Rewrites the
+// scores sc[0, nC) and shifts the per-head LSE by E ln 2, so that the filter's
+// exact scores carry the same factor.  Returns the threshold bin.
+template <int G>
+__device__ int rescale_unit(const ScoreParams &p, int nC, const float *lg, float *sc, uint32_t *sh_hist,
+                            double *sh_lse, int bin, int *above, int *sh_warp, int *sh_res) {
+  const float a = (float)((double)p.c * kLog2e);
+  double E = 0.0;
+  for (int round = 0; round < 16 && bin < kTrustBin && E < kMaxShift; ++round) {
+    const int e_bin = bin >> 4;  // biased fp32 exponent of the threshold bin, 0 when it underflowed
+    E += e_bin > 0 ? (double)(kTargetExponent - e_bin) : 200.0;
+    if (E > kMaxShift) E = kMaxShift;
+    float bh[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) bh[h] = (float)(sh_lse[h] * kLog2e - E);
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh_hist[i] = 0u;
+    __syncthreads();
+    for (int t = threadIdx.x; t < nC; t += blockDim.x) {
+      float pr[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) pr[h] = ex2_approx(fmaf(__ldcg(lg + (size_t)t * G + h), a, -bh[h]));
+#pragma unroll
+      for (int w = 1; w < G; w <<= 1)
+#pragma unroll
+        for (int h = 0; h + w < G; h += 2 * w) pr[h] += pr[h + w];
+      const float sv = pr[0] >= 0.f ? pr[0] : 0.f;
+      sc[t] = sv;
+      atomicAdd(&sh_hist[__float_as_uint(sv) >> kHistShift], 1u);
+    }
+    __syncthreads();
+    bin = find_threshold_bin(sh_hist, kHistBins, p.k_global, above, sh_warp, sh_res);
+  }
+  if (threadIdx.x < G) sh_lse[threadIdx.x] -= E * kLn2;
+  __syncthreads();
+  return bin;
+}
+
 template <int G, int D>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams p) {
   __shared__ uint32_t sh_hist[kHistBins];
@@ -318,7 +370,8 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh_hist[i] = __ldcg(gh + i);
   __syncthreads();
   int above;
-  const int bin = find_threshold_bin(sh_hist, kHistBins, p.k_global, &above, sh_warp, sh_res);
+  int bin = find_threshold_bin(sh_hist, kHistBins, p.k_global, &above, sh_warp, sh_res);
+  if (bin < kTrustBin) bin = rescale_unit<G>(p, ui.nC, lg, sc, sh_hist, sh_lse, bin, &above, sh_warp, sh_res);
   if (threadIdx.x == 0) p.ws.thr[u] = make_int2(bin, above);
   if (threadIdx.x < G) p.ws.lse[u * 8 + threadIdx.x] = sh_lse[threadIdx.x];
 }
@@ -453,7 +506,7 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
   // the band keeps a 4e-4 margin on both sides.
   const int bin1 = p.ws.thr[u].x;
   const float lo = __uint_as_float((uint32_t)bin1 << kHistShift) * (1.f - kBandMargin);
-  const float hi = bin1 >= 0x7F7 ? INFINITY : __uint_as_float((uint32_t)(bin1 + 1) << kHistShift) * (1.f + kBandMargin);
+  const float hi = bin1 >= 0xFEF ? INFINITY : __uint_as_float((uint32_t)(bin1 + 1) << kHistShift) * (1.f + kBandMargin);
   double lse[8];
 #pragma unroll
   for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.lse[u * 8 + h] : 0.0;

@@ -163,3 +163,30 @@ def unit_oracle_sparse(oracle, w: synth.Workload, b: int, kvh: int, q, local_idx
     return oracle.sparse_attn(synth.raw(qq), DTYPE_CODE[s.q_dtype], synth.raw(k), synth.raw(v),
                               DTYPE_CODE[s.kv_dtype], np.asarray(local_idx, np.int32).reshape(1, 1, -1),
                               k_scale=synth.raw(ks), v_scale=synth.raw(vs))
+
+
+def check_idx_positions(gpos_row, opos_row, ora_score, T, window, k_global):
+    """check_idx_unit() on lists already mapped to logical positions: gpos_row
+    is the GPU's list (-1 padding, -2 for a slot outside the sequence),
+    opos_row the oracle's (-1 padded), ora_score its scores of [0, T).
+    Returns the number of positions that differ (all inside the near-tie band)."""
+    L = window + k_global
+    n = min(T, L)
+    g = np.asarray(gpos_row)
+    assert len(g) == L
+    assert np.all(g[n:] == -1), "padding must be -1"
+    gv = g[:n]
+    assert np.all(gv >= 0), "valid entries must be slots of the sequence"
+    assert np.all(np.diff(gv) > 0), "positions must be strictly ascending"
+    ov = np.asarray(opos_row)[:n]
+    win = set(range(max(0, T - window), T))
+    assert win <= set(gv.tolist()), "forced window missing"
+    diff = set(gv.tolist()) ^ set(ov.tolist())
+    if diff:
+        nC = max(0, T - window)
+        cand = np.sort(ora_score[:nC])[::-1]
+        sk = cand[k_global - 1]
+        bad = [t for t in diff if not (abs(ora_score[t] - sk) <= NEAR_TIE * sk)]
+        assert not bad, (f"{len(bad)} positions differ outside the near-tie band, e.g. {bad[:5]} "
+                         f"(scores {[ora_score[t] for t in bad[:5]]}, k-th {sk})")
+    return len(diff)

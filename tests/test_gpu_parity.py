@@ -242,3 +242,53 @@ def test_bounded_wait_expires_and_context_stays_usable(oracle, lib):
     out, idx = U.run_gpu(wd)
     torch.cuda.synchronize()
     U.check_full(wd, out, idx, ora)
+
+
+def planted_margins(kv_dtype, lo, hi, T=6000, seed=0):
+    """Keys along one axis so that every query head's logit is set exactly:
+    the window's keys are 0 (logit 0) and each selectable key sits lo..hi nats
+    (uniform) below it for head 0; head h has 1 + h/8 times that margin.
+    With margins beyond ~87 nats the group probabilities fall under fp32's
+    normal range, and the k-th score with them."""
+    sp = spec(batch=2, seq_len=T, kv_dtype=kv_dtype, sparse_layers=1, needles=0)
+    w = synth.generate(sp, seed=seed)
+    g = torch.Generator().manual_seed(seed)
+    c = 1.0 / np.sqrt(sp.head_dim)
+    w.q_full.zero_()
+    for h in range(sp.num_q_heads):
+        w.q_full[:, h, 0] = 8.0 + (h % sp.group)
+    rows = torch.zeros(w.num_slots, sp.num_kv_heads, sp.head_dim)
+    for b in range(sp.batch):
+        slots = synth.slots_of(w, b, torch.arange(T))
+        for kvh in range(sp.num_kv_heads):
+            margin = lo + (hi - lo) * torch.rand(T, generator=g)
+            x = margin / (8.0 * c)
+            x[T - sp.window:] = 0.0
+            rows[slots, kvh, 0] = x
+    if kv_dtype == "e4m3":
+        codes, scale = synth._quantize_e4m3(rows)
+        w.k.copy_(codes)
+        w.k_scale.copy_(scale)
+    else:
+        w.k.copy_(rows.to(w.k.dtype))
+    return w
+
+
+@pytest.mark.parametrize("kv_dtype,lo,hi", [
+    ("bf16", -200.0, -70.0),   # the k-th group probability underflows fp32 (the top ones do not)
+    ("bf16", -90.0, -60.0),    # it sits just above 2^-126, where single heads flush
+    ("bf16", -420.0, -260.0),  # two common factors are needed
+    ("e4m3", -200.0, -70.0),
+])
+def test_selection_below_fp32_range(oracle, lib, kv_dtype, lo, hi):
+    """Logit margins of 60-420 nats put the k-th score far below fp32's
+    normal range; the selection must still rank exactly like the fp64 oracle."""
+    w = planted_margins(kv_dtype, lo, hi, seed=int(-lo))
+    ora = U.run_oracle(oracle, w)
+    nC = int(w.seq_lens[0]) - w.spec.window
+    kth = np.sort(ora["score"][0, 0, :nC])[::-1][w.spec.k_global - 1]
+    assert kth < 2.0 ** -96, kth  # the case this test is about
+    wd = U.to_device(w)
+    out, idx = U.run_gpu(wd)
+    torch.cuda.synchronize()
+    U.check_full(wd, out, idx, ora)

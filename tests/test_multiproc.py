@@ -51,7 +51,7 @@ def test_max_over_ranks_two_gloo_ranks():
 def test_reference_arm_under_torchrun_prints_once():
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
            "--master-addr", "127.0.0.1", "--master-port", str(free_port()), os.path.join(ROOT, "bench.py"),
-           "--impl", "reference", "--gpus", "2", "--workload", "tiny_fp32_t2048", "--steps", "1", "--warmup", "0"]
+           "--impl", "reference", "--gpus", "2", "--workload", "tiny_fp32_t2048", "--steps", "3", "--warmup", "2"]
     r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
@@ -59,3 +59,5 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["config"]["workload"] == "tiny_fp32_t2048" and d["higher_is_better"] is True
+    assert (d["steps"], d["warmup"]) == (3, 2)  # the driver's --steps / --warmup, not clamped
+    assert abs(d["value"] * d["ms_per_step"] - 1000.0) < 1e-6 * 1000.0  # whole steps, measured
