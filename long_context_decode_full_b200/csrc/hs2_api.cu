@@ -6,6 +6,10 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <time.h>
+#include <unistd.h>
+
+#include <atomic>
 #include <mutex>
 
 #include "hs2.h"
@@ -80,7 +84,7 @@ int encode_cache_map(CUtensorMap *map, const hs2_cache *c, int box_rows) {
 
 // ---------------------------------------------------------------- workspace
 struct Layout {
-  size_t err, prefix, records, logits, scores, above, cand, subcnt, hist, thr, lse, total;
+  size_t err, prefix, records, logits, scores, above, cand, subcnt, hist, thr, lse, sel_lse, unit_ticket, total;
   int R, nsub;
 };
 
@@ -117,6 +121,10 @@ Layout layout(int B, int Hkv, int G, int D, int64_t t_cap_in) {
   o = align256(o + U * 8);
   L.lse = o;
   o = align256(o + U * 8 * sizeof(double));
+  L.sel_lse = o;
+  o = align256(o + U * 8 * sizeof(double));
+  L.unit_ticket = o;
+  o = align256(o + U * sizeof(unsigned long long));
   L.total = o;
   return L;
 }
@@ -137,10 +145,28 @@ FullWs bind(const Layout &L, void *ws, int B, int Hkv) {
   f.ticket = f.hist + U * kHistBins;
   f.thr = reinterpret_cast<int2 *>(w + L.thr);
   f.lse = reinterpret_cast<double *>(w + L.lse);
+  f.sel_lse = reinterpret_cast<double *>(w + L.sel_lse);
+  f.unit_ticket = reinterpret_cast<unsigned long long *>(w + L.unit_ticket);
   return f;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// A 40-bit id per call (never 0), stamped on the attention pass's unit
+// tickets; the process's first id is drawn from the clock and the pid so two
+// processes sharing a workspace are unlikely to meet the same id.
+unsigned long long next_call_id() {
+  static std::atomic<unsigned long long> ctr{[] {
+    struct timespec ts;
+    clock_gettime(CLOCK_REALTIME, &ts);
+    unsigned long long x = (unsigned long long)ts.tv_nsec * 0x9E3779B97F4A7C15ull ^ (unsigned long long)getpid() << 20;
+    return x ^ (x >> 29);
+  }()};
+  for (;;) {
+    const unsigned long long id = ++ctr & ((1ull << (64 - kTicketCountBits)) - 1ull);
+    if (id != 0) return id;
+  }
+}
 
 int group_ok(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
 
@@ -298,6 +324,7 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
   p.R = L.R;
   p.c = 1.0f / sqrtf((float)D);
   p.ws = bind(L, workspace, B, Hkv);
+  p.call_id = next_call_id();
   {  // the logits this call writes, bounded by the sequence capacity: small next to the 126 MB L2?
     const double logit_bytes = (double)B * Hkv * (double)t_cap * G * 4.0;
     p.kv_evict_first = logit_bytes <= 48.0 * (1 << 20) ? 1 : 0;
@@ -427,7 +454,7 @@ int hs2_workspace_status(void *workspace, size_t workspace_bytes, void *stream) 
   if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, 4, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "reading the workspace status");
-  if (flag) return fail(HS2_ERR_TIMEOUT, "device error flag 0x%x (1: consumer wait, 2: producer wait, 4: record)", flag);
+  if (flag) return fail(HS2_ERR_TIMEOUT, "device error flag 0x%x (1: consumer wait, 2: producer wait, 4: record, 8: unit ticket)", flag);
   return HS2_OK;
 }
 

@@ -28,6 +28,7 @@ struct FullParams {
   int32_t tile;              // positions per tile
   int32_t kv_evict_first;    // K/V loads marked evict-first in L2 (when the logits fit in L2 beside them)
   float c;                   // 1/sqrt(D)
+  unsigned long long call_id;  // stamped on the unit tickets (40 bits, never 0)
   FullWs ws;
 };
 
