@@ -6,10 +6,6 @@
 #include <stdlib.h>
 #include <string.h>
 
-#include <time.h>
-#include <unistd.h>
-
-#include <atomic>
 #include <mutex>
 
 #include "hs2.h"
@@ -84,7 +80,7 @@ int encode_cache_map(CUtensorMap *map, const hs2_cache *c, int box_rows) {
 
 // ---------------------------------------------------------------- workspace
 struct Layout {
-  size_t err, prefix, records, logits, scores, above, cand, subcnt, hist, thr, lse, sel_lse, unit_ticket, total;
+  size_t err, prefix, records, logits, scores, above, cand, subcnt, hist, thr, lse, total;
   int R, nsub;
 };
 
@@ -121,10 +117,6 @@ Layout layout(int B, int Hkv, int G, int D, int64_t t_cap_in) {
   o = align256(o + U * 8);
   L.lse = o;
   o = align256(o + U * 8 * sizeof(double));
-  L.sel_lse = o;
-  o = align256(o + U * 8 * sizeof(double));
-  L.unit_ticket = o;
-  o = align256(o + U * sizeof(unsigned long long));
   L.total = o;
   return L;
 }
@@ -145,28 +137,10 @@ FullWs bind(const Layout &L, void *ws, int B, int Hkv) {
   f.ticket = f.hist + U * kHistBins;
   f.thr = reinterpret_cast<int2 *>(w + L.thr);
   f.lse = reinterpret_cast<double *>(w + L.lse);
-  f.sel_lse = reinterpret_cast<double *>(w + L.sel_lse);
-  f.unit_ticket = reinterpret_cast<unsigned long long *>(w + L.unit_ticket);
   return f;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
-
-// A 40-bit id per call (never 0), stamped on the attention pass's unit
-// tickets; the process's first id is drawn from the clock and the pid so two
-// processes sharing a workspace are unlikely to meet the same id.
-unsigned long long next_call_id() {
-  static std::atomic<unsigned long long> ctr{[] {
-    struct timespec ts;
-    clock_gettime(CLOCK_REALTIME, &ts);
-    unsigned long long x = (unsigned long long)ts.tv_nsec * 0x9E3779B97F4A7C15ull ^ (unsigned long long)getpid() << 20;
-    return x ^ (x >> 29);
-  }()};
-  for (;;) {
-    const unsigned long long id = ++ctr & ((1ull << (64 - kTicketCountBits)) - 1ull);
-    if (id != 0) return id;
-  }
-}
 
 int group_ok(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
 
@@ -324,7 +298,6 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
   p.R = L.R;
   p.c = 1.0f / sqrtf((float)D);
   p.ws = bind(L, workspace, B, Hkv);
-  p.call_id = next_call_id();
   {  // the logits this call writes, bounded by the sequence capacity: small next to the 126 MB L2?
     const double logit_bytes = (double)B * Hkv * (double)t_cap * G * 4.0;
     p.kv_evict_first = logit_bytes <= 48.0 * (1 << 20) ? 1 : 0;
@@ -412,31 +385,50 @@ int hs2_sparse_attn(const hs2_heads *q_l, const hs2_cache *k_cache, const hs2_ca
   p.D = k_cache->head_dim;
   p.L = idx_stride;
   p.c = 1.0f / sqrtf((float)p.D);
-  // 8 warps per CTA take 16-row groups, each warp gathering up to `nbuf`
-  // groups at once: rows per CTA = 128 * nbuf, one cluster of S CTAs per
-  // (sequence, kv head).  nbuf starts at 2 and grows (up to what shared
-  // memory holds) while the units' CTAs would not fit in one wave of one CTA
-  // per SM or a cluster would exceed 16 CTAs; very long lists then take more
-  // rows per CTA than buffers, walked as a rolling pipeline.
+  // `warps` warps per CTA take groups of RG = 16 * nsl rows, each warp
+  // gathering up to `nbuf` groups at once: rows per CTA = warps * RG * nbuf,
+  // one cluster of S CTAs per (sequence, kv head).  nbuf starts at 2 and
+  // grows (up to what shared memory holds) while the units' CTAs would not
+  // fit in one wave of one CTA per SM or a cluster would exceed 16 CTAs; very
+  // long lists then take more rows per CTA than buffers, walked as a rolling
+  // pipeline.
   const int units = p.B * p.Hkv, sms = sm_count();
-  // a warp's gather buffers: 16 rows of K and V (+ scales); at most 192 KB per CTA
-  const int buf_bytes = 2 * 16 * p.D * (k_cache->dtype == HS2_E4M3 ? 1 : 2) + (k_cache->dtype == HS2_E4M3 ? 128 : 0);
-  int max_nbuf = (192 * 1024) / (8 * buf_bytes);
+  int warps = 4, nsl = 2, nbuf_env = 0, splits_env = 0;  // (8, 1) measured equal at 32K / 256K, 10% slower at 1M
+  if (const char *env = getenv("HS2_SPARSE_CFG")) {  // tuning override: "warps,nsl[,nbuf[,splits]]"
+    int a = 0, b2 = 0, c2 = 0, d2 = 0;
+    if (sscanf(env, "%d,%d,%d,%d", &a, &b2, &c2, &d2) >= 2 && (a == 4 || a == 8) && (b2 == 1 || b2 == 2)) {
+      warps = a;
+      nsl = b2;
+      nbuf_env = c2;
+      splits_env = d2 >= 1 && d2 <= 16 ? d2 : 0;
+    }
+  }
+  const int rg = 16 * nsl;
+  // a warp's gather buffer: RG rows of K and V (+ scales); at most 192 KB per CTA
+  const int buf_bytes = 2 * rg * p.D * (k_cache->dtype == HS2_E4M3 ? 1 : 2) + (k_cache->dtype == HS2_E4M3 ? 8 * rg : 0);
+  int max_nbuf = (192 * 1024) / (warps * buf_bytes);
   max_nbuf = max_nbuf < 1 ? 1 : (max_nbuf > 4 ? 4 : max_nbuf);
+  const int per_buf = warps * rg;  // rows per CTA per buffer round
   // two buffers per warp at least (one gather in flight while the other is
   // consumed), more while the CTAs would not fit in one wave
   int nbuf = max_nbuf < 2 ? max_nbuf : 2;
-  while (nbuf < max_nbuf && (units * ((idx_stride + 128 * nbuf - 1) / (128 * nbuf)) > sms ||
-                             (idx_stride + 128 * nbuf - 1) / (128 * nbuf) > 16))
+  while (nbuf < max_nbuf && (units * ((idx_stride + per_buf * nbuf - 1) / (per_buf * nbuf)) > sms ||
+                             (idx_stride + per_buf * nbuf - 1) / (per_buf * nbuf) > 16))
     ++nbuf;
-  if (const char *env = getenv("HS2_SPARSE_NBUF")) nbuf = atoi(env);  // tuning override
+  if (nbuf_env > 0) nbuf = nbuf_env;
   nbuf = nbuf < 1 ? 1 : (nbuf > max_nbuf ? max_nbuf : nbuf);
-  int rows = 128 * nbuf;
+  int rows = per_buf * nbuf;
   int S = (idx_stride + rows - 1) / rows;
   while (S > 16) {  // larger lists: more rows per CTA, never more than 16 per cluster
-    rows += 128;
+    rows += per_buf;
     S = (idx_stride + rows - 1) / rows;
   }
+  if (splits_env > 0) {
+    rows = ((idx_stride + splits_env - 1) / splits_env + per_buf - 1) / per_buf * per_buf;
+    S = (idx_stride + rows - 1) / rows;
+  }
+  p.warps = warps;
+  p.nsl = nsl;
   p.rows_per_cta = rows;
   p.splits = S;
   p.nbuf = nbuf;
@@ -454,7 +446,7 @@ int hs2_workspace_status(void *workspace, size_t workspace_bytes, void *stream) 
   if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, 4, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "reading the workspace status");
-  if (flag) return fail(HS2_ERR_TIMEOUT, "device error flag 0x%x (1: consumer wait, 2: producer wait, 4: record, 8: unit ticket)", flag);
+  if (flag) return fail(HS2_ERR_TIMEOUT, "device error flag 0x%x (1: consumer wait, 2: producer wait, 4: record)", flag);
   return HS2_OK;
 }
 
@@ -530,7 +522,7 @@ int hs2_selftest_bounded_wait(void *workspace, size_t workspace_bytes, void *str
 int hs2_copy_peak(void *dst, const void *src, size_t bytes, void *stream) {
   if (!dst || !src || (bytes & 15) || !aligned16(dst) || !aligned16(src))
     return fail(HS2_ERR_INVALID_ARG, "copy needs 16-byte aligned pointers and a multiple of 16 bytes");
-  cudaError_t e = launch_copy(dst, src, bytes, sm_count() * 4, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_copy(dst, src, bytes, sm_count() * 32, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "copy launch");
   return HS2_OK;
 }
@@ -557,18 +549,21 @@ cudaError_t launch_wait_selftest(uint32_t *err, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-__global__ void __launch_bounds__(512) copy_kernel(uint4 *__restrict__ dst, const uint4 *__restrict__ src, size_t n) {
+// Grid-strided 16-byte copy, four loads in flight per thread.  Measured on
+// B200 with 2 GiB: 32 CTAs of 256 threads per SM and plain loads/stores
+// reach ~6.3 TB/s (read + write); 4 CTAs per SM or streaming (.cs) hints
+// stay near 5.9 TB/s.
+__global__ void __launch_bounds__(256) copy_kernel(uint4 *__restrict__ dst, const uint4 *__restrict__ src, size_t n) {
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   for (; i + 3 * stride < n; i += 4 * stride) {
-    const uint4 a = __ldcs(src + i), b = __ldcs(src + i + stride), c = __ldcs(src + i + 2 * stride),
-                d = __ldcs(src + i + 3 * stride);
-    __stcs(dst + i, a);
-    __stcs(dst + i + stride, b);
-    __stcs(dst + i + 2 * stride, c);
-    __stcs(dst + i + 3 * stride, d);
+    const uint4 a = src[i], b = src[i + stride], c = src[i + 2 * stride], d = src[i + 3 * stride];
+    dst[i] = a;
+    dst[i + stride] = b;
+    dst[i + 2 * stride] = c;
+    dst[i + 3 * stride] = d;
   }
-  for (; i < n; i += stride) __stcs(dst + i, __ldcs(src + i));
+  for (; i < n; i += stride) dst[i] = src[i];
 }
 
 int set_last_error(int code, const char *msg) { return fail(code, "%s", msg); }
@@ -583,7 +578,7 @@ bool pdl_enabled() {
 
 cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int grid, cudaStream_t s) {
   if (bytes == 0) return cudaSuccess;
-  copy_kernel<<<grid, 512, 0, s>>>(static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), bytes / 16);
+  copy_kernel<<<grid, 256, 0, s>>>(static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), bytes / 16);
   return cudaGetLastError();
 }
 

@@ -30,7 +30,6 @@ constexpr int64_t kMaxContext = int64_t(1) << 23;  // positions per sequence
 constexpr uint32_t kErrFullWait = 1u;    // consumer timed out on a full barrier
 constexpr uint32_t kErrEmptyWait = 2u;   // producer timed out on an empty barrier
 constexpr uint32_t kErrRecord = 4u;      // record index outside its unit's slots
-constexpr uint32_t kErrTicket = 8u;      // a unit's tile count could not be updated
 
 // ---------------------------------------------------------------- workspace
 // Every array of the full-attention call lives in the caller's workspace.
@@ -46,37 +45,8 @@ struct FullWs {
   uint32_t *hist;        // [U, kHistBins], then ticket [U] and one spare word [U]
   uint32_t *ticket;      // [U]
   int2 *thr;             // [U] (threshold bin, count strictly above it)
-  double *lse;           // [U, 8] per-head log-sum-exp of the scaled logits (attention pass)
-  double *sel_lse;       // [U, 8] the same minus E ln 2, E the unit's score shift (selection)
-  unsigned long long *unit_ticket;  // [U] (call id << 24 | tiles done) of the attention pass
+  double *lse;           // [U, 8] per-head log-sum-exp of the scaled logits
 };
-
-// Tiles of unit u done so far in this call, counted by the CTAs that finish a
-// segment of it; the CTA whose count completes the unit's nb tiles gets true
-// and returns the word to zero.  Each word carries the call's id in its high
-// 40 bits, so a word left by another call (or never initialised) restarts the
-// count.  Lock-free: retries only when another CTA updated the word between
-// the load and the CAS, and gives up (false, error flag) after 1024 of them.
-constexpr int kTicketCountBits = 24;
-constexpr unsigned long long kTicketCountMask = (1ull << kTicketCountBits) - 1ull;
-__device__ __forceinline__ bool unit_ticket_completes(unsigned long long *word, unsigned long long call_id,
-                                                      int ntiles, int nb, uint32_t *err, uint32_t err_bit) {
-  unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(word);
-  for (int tries = 0; tries < 1024; ++tries) {
-    const unsigned long long want =
-        (cur >> kTicketCountBits) == call_id ? cur + (unsigned long long)ntiles
-                                             : (call_id << kTicketCountBits) | (unsigned long long)ntiles;
-    const unsigned long long prev = atomicCAS(word, cur, want);
-    if (prev == cur) {
-      if ((int)(want & kTicketCountMask) != nb) return false;
-      *reinterpret_cast<volatile unsigned long long *>(word) = 0ull;  // for the next call (and graph replays)
-      return true;
-    }
-    cur = prev;
-  }
-  atomicOr(err, err_bit);
-  return false;
-}
 
 // Balanced partition of the tile space over N persistent CTAs.  Tiles are
 // ordered by (sequence, kv head, tile); CTA c owns [c*total/N, (c+1)*total/N).

@@ -106,49 +106,6 @@ __device__ __forceinline__ int find_seq(const int32_t *prefix, int B, int Hkv, i
   return lo;
 }
 
-// Per-head log-sum-exp of unit u = (b, kvh) from its segment records, by one
-// warp of the CTA whose segment completed the unit.  Lane l folds the records
-// j = l / G, l / G + 32 / G, ... of head l % G into a running (max, sum) pair
-// (records of CTAs that own no tiles are skipped); the lanes of a head then
-// merge their pairs.  LSE_h = c M + log L with the sum L in fp64.
-__device__ void unit_lse_from_records(const FullParams &p, const int32_t *prefix, int b, int kvh) {
-  const int lane = threadIdx.x & 31;
-  const int G = p.G, h = lane % G;
-  const int nb = prefix[b + 1] - prefix[b];
-  const Partition part{(int64_t)p.Hkv * prefix[p.B], p.N};
-  const int64_t U = (int64_t)p.Hkv * prefix[b] + (int64_t)kvh * nb;
-  const int64_t c0 = part.cfirst(U);
-  const int nseg = (int)min((int64_t)p.R, part.cfirst(U + nb - 1) - c0 + 1);
-  const int64_t u = (int64_t)b * p.Hkv + kvh;
-  const int RS = G * (p.D + 2);
-  const float *rec0 = p.ws.records + (size_t)u * p.R * RS;
-  const double c = (double)p.c;
-  float M = -INFINITY;
-  double L = 0.0;
-#pragma unroll 4
-  for (int j = lane / G; j < nseg; j += 32 / G) {
-    if (!part.owns_tiles(c0 + j)) continue;
-    const float mj = __ldcg(rec0 + (size_t)j * RS + h);
-    const float lj = __ldcg(rec0 + (size_t)j * RS + G + h);
-    if (mj == -INFINITY) continue;
-    if (mj > M) {
-      L = L * exp(c * ((double)M - mj)) + (double)lj;  // (0 while M was -inf)
-      M = mj;
-    } else {
-      L += (double)lj * exp(c * ((double)mj - M));
-    }
-  }
-  for (int o = G; o < 32; o <<= 1) {  // lanes of the same head
-    const float Mo = __shfl_xor_sync(0xffffffffu, M, o);
-    const double Lo = __shfl_xor_sync(0xffffffffu, L, o);
-    const float Mn = fmaxf(M, Mo);
-    if (Mn != -INFINITY)
-      L = (M == -INFINITY ? 0.0 : L * exp(c * ((double)M - Mn))) + (Mo == -INFINITY ? 0.0 : Lo * exp(c * ((double)Mo - Mn)));
-    M = Mn;
-  }
-  if (lane < G) p.ws.lse[u * 8 + lane] = c * (double)M + log(L);
-}
-
 // producer warps: TMA (+ stage metadata), and for E4M3 the scale gathers
 template <bool FP8>
 constexpr int kProducerWarps = FP8 ? 2 : 1;
@@ -333,7 +290,6 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
   WarpAttn<D, FP8, NSL> st;
   st.reset();
   uint32_t cphase = 0;
-  int seg_tiles = 0;  // tiles of the current segment so far
   for (int it = 0;; ++it) {
     const int stage = it % NSTAGE;
     if (!mbar_wait(&full[stage], (it / NSTAGE) & 1)) {
@@ -348,7 +304,6 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
       st.load_q(reinterpret_cast<const __nv_bfloat16 *>(p.q) + ((int64_t)mt.b * p.Hkv * p.G + (int64_t)mt.kvh * p.G) * D,
                 p.G);
     }
-    ++seg_tiles;
     const int pos0 = mt.tile * C::TILE + C::RPW * warp;
     const int nvalid = max(0, min(C::RPW, mt.T - pos0));
     const uint32_t vmask = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
@@ -374,22 +329,10 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
         merge_warp_states<D>(scratch, C::WSTRIDE, NCW, p.G, p.c, p.ws.records + (size_t)mt.rec * p.G * (D + 2),
                              threadIdx.x, NCW * 32);
       fence_proxy_async_smem();  // before TMA refills the stage
-      __threadfence();           // the record reaches L2 before the unit's ticket counts it
       if (!consumer_sync(cbar, cphase)) {
         set_error(p.ws.err, kErrFullWait);
         break;
       }
-      if (warp == 0) {  // count the segment; the warp that completes the unit reduces its records
-        int done = 0;
-        if (lane == 0)
-          done = unit_ticket_completes(p.ws.unit_ticket + u, p.call_id, seg_tiles, prefix[mt.b + 1] - prefix[mt.b],
-                                       p.ws.err, kErrTicket);
-        if (__shfl_sync(0xffffffffu, done, 0)) {
-          __threadfence();
-          unit_lse_from_records(p, prefix, mt.b, mt.kvh);
-        }
-      }
-      seg_tiles = 0;
       st.reset();
     }
     __syncwarp();
@@ -423,7 +366,6 @@ __global__ void __launch_bounds__(32 * kF32Warps) full_attn_f32_kernel(const Ful
   const float *K = static_cast<const float *>(p.k), *V = static_cast<const float *>(p.v);
 
   float m[2], l[2], o[2][D / 32];
-  int seg_tiles = 0;
   int b = g0 < g1 ? find_seq(prefix, p.B, p.Hkv, g0) : 0;
   for (int64_t g = g0; g < g1; ++g) {
     while ((int64_t)p.Hkv * prefix[b + 1] <= g) ++b;
@@ -435,8 +377,6 @@ __global__ void __launch_bounds__(32 * kF32Warps) full_attn_f32_kernel(const Ful
     const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
     const bool first = i == 0 || g == g0, last = i == nb - 1 || g == g1 - 1;
     const int p0 = i * kF32Tile;
-    if (first) seg_tiles = 0;
-    ++seg_tiles;
     if (first) {
       const float *q = static_cast<const float *>(p.q) + ((int64_t)b * p.Hkv * p.G + (int64_t)kvh * p.G) * D;
       for (int e = threadIdx.x; e < p.G * D; e += nthr) Qs[e] = q[e];
@@ -509,16 +449,6 @@ __global__ void __launch_bounds__(32 * kF32Warps) full_attn_f32_kernel(const Ful
           rec[p.G + h] = l[hs];
         }
         for (int jj = 0; jj < D / 32; ++jj) rec[2 * p.G + h * D + lane + 32 * jj] = o[hs][jj];
-      }
-      __threadfence();  // the record reaches L2 before the unit's ticket counts it
-      __syncthreads();
-      if (warp == 0) {
-        int done = 0;
-        if (lane == 0) done = unit_ticket_completes(p.ws.unit_ticket + u, p.call_id, seg_tiles, nb, p.ws.err, kErrTicket);
-        if (__shfl_sync(0xffffffffu, done, 0)) {
-          __threadfence();
-          unit_lse_from_records(p, prefix, b, kvh);
-        }
       }
     }
   }

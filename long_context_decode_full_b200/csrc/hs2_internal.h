@@ -28,7 +28,6 @@ struct FullParams {
   int32_t tile;              // positions per tile
   int32_t kv_evict_first;    // K/V loads marked evict-first in L2 (when the logits fit in L2 beside them)
   float c;                   // 1/sqrt(D)
-  unsigned long long call_id;  // stamped on the unit tickets (40 bits, never 0)
   FullWs ws;
 };
 
@@ -61,7 +60,9 @@ struct SparseParams {
   int32_t L;                 // idx_stride
   int32_t rows_per_cta;      // multiple of 16
   int32_t splits;            // CTAs per unit (cluster size)
-  int32_t nbuf;              // 16-row gather buffers per warp (1..4)
+  int32_t nbuf;              // gather buffers (one group each) per warp (1..4)
+  int32_t warps;             // warps per CTA (4 or 8)
+  int32_t nsl;               // 16-row slices per group (1 or 2)
   float c;
 };
 

@@ -71,20 +71,11 @@ __device__ __forceinline__ void mark_records(UnitInfo &ui, uint8_t *sh_ok) {
   __syncthreads();
 }
 
-// T, the selectable count and whether the unit selects (no workspace reads).
-__device__ __forceinline__ UnitInfo unit_basic(const ScoreParams &p, int b) {
+__device__ __forceinline__ UnitInfo unit_info(const ScoreParams &p, int b, int kvh) {
   UnitInfo ui;
   ui.T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
   ui.nC = max(0, ui.T - p.window);
   ui.select = ui.nC > p.k_global && p.k_global > 0;
-  ui.nseg = 0;
-  ui.ok = nullptr;
-  return ui;
-}
-
-// The unit's place in the attention pass's partition: its record slots.
-__device__ __forceinline__ UnitInfo unit_info(const ScoreParams &p, int b, int kvh) {
-  UnitInfo ui = unit_basic(p, b);
   ui.nb = (ui.T + p.tile - 1) / p.tile;
   const int64_t total = (int64_t)p.Hkv * p.ws.prefix[p.B];
   ui.U = (int64_t)p.Hkv * p.ws.prefix[b] + (int64_t)kvh * ui.nb;
@@ -174,6 +165,45 @@ __device__ int find_threshold_bin(const uint32_t *hist, int nbins, int need, int
   return bin;
 }
 
+// Per-head LSE (fp64), max and normaliser of a unit from its segment
+// records, as a block-wide reduction: thread t folds the pairs (segment j,
+// head h) with h = t % G.
+template <int G, int D>
+__device__ void unit_lse(const float *rec0, const UnitInfo &ui, float c, double *sh_lse, float *sh_M, float *sh_L,
+                         double *sh_red) {
+  constexpr int RS = G * (D + 2);
+  const int nseg = ui.nseg;
+  const int tid = threadIdx.x, nt = blockDim.x, h = tid % G;
+  float m = -INFINITY;
+  for (int i = tid; i < nseg * G; i += nt)
+    if (ui.rec_ok(i / G)) m = fmaxf(m, rec0[(i / G) * RS + h]);
+  reinterpret_cast<float *>(sh_red)[tid] = m;
+  __syncthreads();
+  if (tid < G) {
+    float M = -INFINITY;
+    for (int t = tid; t < nt; t += G) M = fmaxf(M, reinterpret_cast<float *>(sh_red)[t]);
+    sh_M[tid] = M;
+  }
+  __syncthreads();
+  const float M = sh_M[h];
+  double L = 0.0;
+  for (int i = tid; i < nseg * G; i += nt) {
+    const int j = i / G;
+    if (!ui.rec_ok(j)) continue;
+    const float mj = rec0[j * RS + h];
+    if (mj != -INFINITY) L += (double)rec0[j * RS + G + h] * exp((double)c * ((double)mj - (double)M));
+  }
+  sh_red[tid] = L;
+  __syncthreads();
+  if (tid < G) {
+    double S = 0.0;
+    for (int t = tid; t < nt; t += G) S += sh_red[t];
+    sh_lse[tid] = (double)c * (double)sh_M[tid] + log(S);
+    sh_L[tid] = (float)S;
+  }
+  __syncthreads();
+}
+
 // ------------------------------------------------------------------ score
 // Loads the logits of positions tb + q * kScoreThreads (q < kScoreLoads) below t1.
 constexpr int kScoreLoads = 4;  // positions per thread in flight
@@ -245,7 +275,9 @@ __device__ int rescale_unit(const ScoreParams &p, int nC, const float *lg, float
 template <int G, int D>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams p) {
   __shared__ uint32_t sh_hist[kHistBins];
+  __shared__ double sh_red[kScoreThreads];
   __shared__ double sh_lse[G];
+  __shared__ float sh_M[G], sh_L[G];
   __shared__ int sh_warp[33], sh_res[2], sh_last;
   __shared__ uint8_t sh_ok[kMaxRecords];
   constexpr int RS = G * (D + 2);
@@ -253,45 +285,45 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   griddep_launch_dependents();
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const bool combine = chunk == (int)gridDim.x - 1;  // the unit's combine CTA
-  UnitInfo ui = combine ? unit_info(p, b, kvh) : unit_basic(p, b);
+  UnitInfo ui = unit_info(p, b, kvh);
   const int n_chunks = ui.select ? (ui.nC + p.score_chunk - 1) / p.score_chunk : 0;
   if (!combine && chunk >= n_chunks) return;
   const int64_t u = (int64_t)b * p.Hkv + kvh;
   const int t0 = chunk * p.score_chunk, t1 = min(ui.nC, t0 + p.score_chunk);
   const float *lg = p.ws.logits + (size_t)u * p.ustride * G;
-  // the per-head LSE comes from the attention pass (the CTA that completed the unit)
+  // the LSE first: its dependent record loads would otherwise queue behind
+  // every CTA's first batch of logits
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh_hist[i] = 0u;
+  mark_records(ui, sh_ok);
+  const float *rec0 = p.ws.records + (size_t)u * p.R * RS;
+  unit_lse<G, D>(rec0, ui, p.c, sh_lse, sh_M, sh_L, sh_red);
   float raw[kScoreLoads][G];
   if (!combine) load_logits<G>(raw, lg, t0 + threadIdx.x, t1);
-  if (threadIdx.x < G) sh_lse[threadIdx.x] = __ldcg(p.ws.lse + u * 8 + threadIdx.x);
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh_hist[i] = 0u;
-  if (combine) mark_records(ui, sh_ok);  // (a block barrier)
-  else __syncthreads();
 
-  if (combine) {  // out = sum_j o_j exp(c m_j - LSE)
-    const float *rec0 = p.ws.records + (size_t)u * p.R * RS;
+  if (combine) {  // out = sum_j o_j exp(c (m_j - M)) / L
     const int64_t ob = ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
     for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
       const int h = e / D;
-      const double lse = sh_lse[h];
+      const float M = sh_M[h];
       float acc = 0.f;
       int j = 0;
       for (; j + 4 <= ui.nseg; j += 4) {  // four records in flight
         float mv[4], ov[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          mv[q] = __ldcg(rec0 + (j + q) * RS + h);
-          ov[q] = __ldcg(rec0 + (j + q) * RS + 2 * G + e);
+          mv[q] = rec0[(j + q) * RS + h];
+          ov[q] = rec0[(j + q) * RS + 2 * G + e];
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          if (ui.rec_ok(j + q) && mv[q] != -INFINITY) acc += ov[q] * expf((float)((double)p.c * mv[q] - lse));
+          if (ui.rec_ok(j + q) && mv[q] != -INFINITY) acc += ov[q] * expf(p.c * (mv[q] - M));
       }
       for (; j < ui.nseg; ++j) {
         if (!ui.rec_ok(j)) continue;
-        const float mj = __ldcg(rec0 + j * RS + h);
-        if (mj != -INFINITY) acc += __ldcg(rec0 + j * RS + 2 * G + e) * expf((float)((double)p.c * mj - lse));
+        const float mj = rec0[j * RS + h];
+        if (mj != -INFINITY) acc += rec0[j * RS + 2 * G + e] * expf(p.c * (mj - M));
       }
-      const float val = ui.nseg > 0 && isfinite(lse) ? acc : 0.f;
+      const float val = ui.nseg > 0 && sh_L[h] > 0.f ? acc / sh_L[h] : 0.f;
       if (p.out_dtype == 0) static_cast<float *>(p.out)[ob + e] = val;
       else static_cast<__nv_bfloat16 *>(p.out)[ob + e] = __float2bfloat16_rn(val);
     }
@@ -341,7 +373,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   int bin = find_threshold_bin(sh_hist, kHistBins, p.k_global, &above, sh_warp, sh_res);
   if (bin < kTrustBin) bin = rescale_unit<G>(p, ui.nC, lg, sc, sh_hist, sh_lse, bin, &above, sh_warp, sh_res);
   if (threadIdx.x == 0) p.ws.thr[u] = make_int2(bin, above);
-  if (threadIdx.x < G) p.ws.sel_lse[u * 8 + threadIdx.x] = sh_lse[threadIdx.x];
+  if (threadIdx.x < G) p.ws.lse[u * 8 + threadIdx.x] = sh_lse[threadIdx.x];
 }
 
 // Exact group score of one position: p_h = 2^(raw_h * a - b_h) with
@@ -477,7 +509,7 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
   const float hi = bin1 >= 0xFEF ? INFINITY : __uint_as_float((uint32_t)(bin1 + 1) << kHistShift) * (1.f + kBandMargin);
   double lse[8];
 #pragma unroll
-  for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.sel_lse[u * 8 + h] : 0.0;
+  for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.lse[u * 8 + h] : 0.0;
 #pragma unroll
   for (int k = 0; k < kFilterSubsMax; ++k) {
     const int sub = sub0 + k * kWarps;

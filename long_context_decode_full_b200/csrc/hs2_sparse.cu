@@ -21,22 +21,23 @@ namespace hs2 {
 
 namespace {
 
-constexpr int kSparseWarps = 8;
-
-template <int D, bool FP8>
+// NW warps per CTA, each taking groups of RG = 16 NSL listed rows (NSL
+// 16-row slices per tensor-core step).
+template <int D, bool FP8, int NW, int NSL>
 struct SCfg {
+  static constexpr int RG = 16 * NSL;                               // rows per group
   static constexpr int ES = FP8 ? 1 : 2;
   static constexpr int ROWB = D * ES;
-  static constexpr int PANEL = 16 * 128;
-  static constexpr int KVB = 16 * ROWB;                             // 16 rows of K (or V)
-  static constexpr int BUF_BYTES = 2 * KVB + (FP8 ? 2 * 16 * 4 : 0);  // one 16-row group
+  static constexpr int PANEL = RG * 128;
+  static constexpr int KVB = RG * ROWB;                             // RG rows of K (or V)
+  static constexpr int BUF_BYTES = 2 * KVB + (FP8 ? 2 * RG * 4 : 0);  // one group
   static constexpr int WSTRIDE = 16 + 8 * D;                        // warp scratch floats
   // one CTA's partial record m[G], l[G], o[G][D], padded to whole float4s
   __host__ __device__ static int rec_floats(int G) { return (G * (D + 2) + 3) & ~3; }
-  __host__ __device__ static size_t staging(int nbuf) { return (size_t)kSparseWarps * nbuf * BUF_BYTES; }
+  __host__ __device__ static size_t staging(int nbuf) { return (size_t)NW * nbuf * BUF_BYTES; }
   // the warps' merge scratch reuses the staging buffers (idle by then) when
   // it fits, else gets a region of their own
-  __host__ __device__ static size_t scratch_bytes(int, int) { return (size_t)kSparseWarps * WSTRIDE * 4; }
+  __host__ __device__ static size_t scratch_bytes(int, int) { return (size_t)NW * WSTRIDE * 4; }
   __host__ __device__ static bool scratch_in_staging(int G, int S, int nbuf) {
     return scratch_bytes(G, S) <= staging(nbuf);
   }
@@ -58,9 +59,9 @@ __device__ __forceinline__ void cp_async_wait_n(int n) {  // n = groups allowed 
 // warps take 16-row groups round-robin.  Each warp issues the gathers of up
 // to `nbuf` groups at once, so their latencies overlap, and computes each
 // group on the tensor cores as it lands.
-template <int D, bool FP8>
-__global__ void __launch_bounds__(32 * kSparseWarps, 1) sparse_mma_kernel(const SparseParams p, int64_t num_slots) {
-  using C = SCfg<D, FP8>;
+template <int D, bool FP8, int NW, int NSL>
+__global__ void __launch_bounds__(32 * NW, 1) sparse_mma_kernel(const SparseParams p, int64_t num_slots) {
+  using C = SCfg<D, FP8, NW, NSL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -88,7 +89,7 @@ __global__ void __launch_bounds__(32 * kSparseWarps, 1) sparse_mma_kernel(const 
     const int sl = __ldg(p.idx + u * p.L + row_lo + r);
     slots[r] = (sl >= 0 && sl < num_slots) ? sl : -1;
   }
-  WarpAttn<D, FP8> st;
+  WarpAttn<D, FP8, NSL> st;
   st.reset();
   st.load_q(static_cast<const __nv_bfloat16 *>(p.q) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D, G);
   __syncthreads();
@@ -96,27 +97,27 @@ __global__ void __launch_bounds__(32 * kSparseWarps, 1) sparse_mma_kernel(const 
   constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
   const uint8_t *kg = static_cast<const uint8_t *>(p.k), *vg = static_cast<const uint8_t *>(p.v);
   uint8_t *wbase = smem + (size_t)warp * nbuf * C::BUF_BYTES;
-  // issue the loads of 16-row group `grp` into buffer `buf`; returns its row mask
+  // issue the loads of RG-row group `grp` into buffer `buf`; returns its row mask
   auto gather = [&](int grp, int buf) -> uint32_t {
     uint8_t *wb = wbase + buf * C::BUF_BYTES;
     const uint32_t kp = smem_u32(wb), vp = kp + C::KVB;
-    const int r = 16 * grp + (lane & 15);
+    const int r = C::RG * grp + (lane & (C::RG - 1));
     const int slot = r < nrows ? slots[r] : -1;
-    const uint32_t vm = __ballot_sync(0xffffffffu, slot >= 0) & 0xFFFFu;
+    const uint32_t vm = __ballot_sync(0xffffffffu, slot >= 0) & (C::RG == 32 ? 0xFFFFFFFFu : 0xFFFFu);
     if constexpr (FP8) {
       float *ks = reinterpret_cast<float *>(wb + 2 * C::KVB);
-      if (lane < 16) {
+      if (lane < C::RG) {
         if (slot >= 0) {
           cp_async_4(smem_u32(ks + lane), p.k_scale + (int64_t)slot * p.Hkv + kvh);
-          cp_async_4(smem_u32(ks + 16 + lane), p.v_scale + (int64_t)slot * p.Hkv + kvh);
+          cp_async_4(smem_u32(ks + C::RG + lane), p.v_scale + (int64_t)slot * p.Hkv + kvh);
         } else {
           ks[lane] = 0.f;
-          ks[16 + lane] = 0.f;
+          ks[C::RG + lane] = 0.f;
         }
       }
     }
 #pragma unroll 4
-    for (int e = lane; e < 16 * CPR; e += 32) {
+    for (int e = lane; e < C::RG * CPR; e += 32) {
       const int row = e / CPR, ch = e % CPR;
       const int sr = __shfl_sync(0xffffffffu, slot, row);
       const uint32_t off = (ch >> 3) * C::PANEL;
@@ -134,11 +135,11 @@ __global__ void __launch_bounds__(32 * kSparseWarps, 1) sparse_mma_kernel(const 
     return vm;
   };
 
-  const int ngroups = (nrows + 15) / 16;
-  const int mine = ngroups > warp ? (ngroups - warp + kSparseWarps - 1) / kSparseWarps : 0;  // groups of this warp
+  const int ngroups = (nrows + C::RG - 1) / C::RG;
+  const int mine = ngroups > warp ? (ngroups - warp + NW - 1) / NW : 0;  // groups of this warp
   uint32_t vm[4] = {0u, 0u, 0u, 0u};
   int issued = 0;
-  for (; issued < mine && issued < nbuf; ++issued) vm[issued & 3] = gather(warp + issued * kSparseWarps, issued % nbuf);
+  for (; issued < mine && issued < nbuf; ++issued) vm[issued & 3] = gather(warp + issued * NW, issued % nbuf);
   for (int k = 0; k < mine; ++k) {
     cp_async_wait_n(issued - k - 1);
     __syncwarp();
@@ -146,10 +147,10 @@ __global__ void __launch_bounds__(32 * kSparseWarps, 1) sparse_mma_kernel(const 
     const uint32_t kp = smem_u32(wb);
     const float *ks = reinterpret_cast<const float *>(wb + 2 * C::KVB);
     const uint32_t m = vm[k & 3];
-    if (m) st.step(kp, kp + C::KVB, C::PANEL, 0, m, p.c, nullptr, G, ks, ks + 16);
+    if (m) st.step(kp, kp + C::KVB, C::PANEL, 0, m, p.c, nullptr, G, ks, ks + C::RG);
     __syncwarp();  // the buffer is refilled by the next gather
     if (issued < mine) {
-      vm[issued & 3] = gather(warp + issued * kSparseWarps, issued % nbuf);
+      vm[issued & 3] = gather(warp + issued * NW, issued % nbuf);
       ++issued;
     }
   }
@@ -160,7 +161,7 @@ __global__ void __launch_bounds__(32 * kSparseWarps, 1) sparse_mma_kernel(const 
   float *scr = scratch + warp * C::WSTRIDE;
   st.store(scr, scr + 8, scr + 16);
   __syncthreads();
-  merge_warp_states<D>(scratch, C::WSTRIDE, kSparseWarps, G, p.c, partial, threadIdx.x, blockDim.x);
+  merge_warp_states<D>(scratch, C::WSTRIDE, NW, G, p.c, partial, threadIdx.x, blockDim.x);
   cluster.sync();  // every CTA's partial is complete
   // every CTA writes its share of the G x D outputs: the (m, l) pairs of all
   // partials (one per thread), the heads' weights, then its elements with the
@@ -250,18 +251,27 @@ __global__ void sparse_f32_kernel(const SparseParams p, int64_t num_slots) {
   for (int j = 0; j < D / 32; ++j) out[lane + 32 * j] = l > 0.f ? o[j] / l : 0.f;
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, int NW, int NSL>
 cudaError_t launch_mma_t(const SparseParams &p, int64_t num_slots, cudaStream_t s) {
-  using C = SCfg<D, FP8>;
+  using C = SCfg<D, FP8, NW, NSL>;
   const size_t smem = C::bytes(p.G, p.splits, p.rows_per_cta, p.nbuf);
-  auto kern = sparse_mma_kernel<D, FP8>;
+  auto kern = sparse_mma_kernel<D, FP8, NW, NSL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (p.splits > 8) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  return launch_ex(kern, dim3(p.splits, p.Hkv, p.B), dim3(32 * kSparseWarps), smem, s, p.splits, p, num_slots);
+  return launch_ex(kern, dim3(p.splits, p.Hkv, p.B), dim3(32 * NW), smem, s, p.splits, p, num_slots);
+}
+
+template <int D, bool FP8>
+cudaError_t launch_mma_shape(const SparseParams &p, int64_t num_slots, cudaStream_t s) {
+  if (p.warps == 8 && p.nsl == 1) return launch_mma_t<D, FP8, 8, 1>(p, num_slots, s);
+  if (p.warps == 4 && p.nsl == 2) return launch_mma_t<D, FP8, 4, 2>(p, num_slots, s);
+  if (p.warps == 8 && p.nsl == 2) return launch_mma_t<D, FP8, 8, 2>(p, num_slots, s);
+  if (p.warps == 4 && p.nsl == 1) return launch_mma_t<D, FP8, 4, 1>(p, num_slots, s);
+  return cudaErrorInvalidConfiguration;
 }
 
 }  // namespace
@@ -272,8 +282,9 @@ cudaError_t launch_sparse_impl(const SparseParams &p, int kv_dtype, int64_t num_
     if (p.D == 64) return launch_ex(sparse_f32_kernel<64>, dim3(p.Hkv, p.B), dim3(32 * p.G), smem, s, 0, p, num_slots);
     return launch_ex(sparse_f32_kernel<128>, dim3(p.Hkv, p.B), dim3(32 * p.G), smem, s, 0, p, num_slots);
   }
-  if (kv_dtype == 1) return p.D == 64 ? launch_mma_t<64, false>(p, num_slots, s) : launch_mma_t<128, false>(p, num_slots, s);
-  if (kv_dtype == 2 && p.D == 128) return launch_mma_t<128, true>(p, num_slots, s);
+  if (kv_dtype == 1)
+    return p.D == 64 ? launch_mma_shape<64, false>(p, num_slots, s) : launch_mma_shape<128, false>(p, num_slots, s);
+  if (kv_dtype == 2 && p.D == 128) return launch_mma_shape<128, true>(p, num_slots, s);
   return cudaErrorInvalidValue;
 }
 
