@@ -116,7 +116,7 @@ Layout layout(int B, int Hkv, int G, int D, int64_t t_cap_in) {
   L.thr = o;
   o = align256(o + U * 8);
   L.lse = o;
-  o = align256(o + U * 8 * sizeof(double));
+  o = align256(o + U * kMaxGroup * sizeof(double));
   L.total = o;
   return L;
 }
@@ -142,7 +142,7 @@ FullWs bind(const Layout &L, void *ws, int B, int Hkv) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-int group_ok(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
+int group_ok(int G) { return G == 1 || G == 2 || G == 4 || G == 8 || G == 16 || G == 32; }
 
 // Checks a q/out descriptor against the cache; `what` names it in errors.
 int check_heads(const hs2_heads *h, const hs2_cache *k, const char *what) {
@@ -155,7 +155,9 @@ int check_heads(const hs2_heads *h, const hs2_cache *k, const char *what) {
     return fail(HS2_ERR_INVALID_ARG, "%s num_heads %d is not a multiple of num_kv_heads %d", what, h->num_heads,
                 k->num_kv_heads);
   if (!group_ok(h->num_heads / k->num_kv_heads))
-    return fail(HS2_ERR_UNSUPPORTED, "GQA group %d not built (1, 2, 4 or 8)", h->num_heads / k->num_kv_heads);
+    return fail(HS2_ERR_UNSUPPORTED, "GQA group %d not built (1, 2, 4, 8, 16 or 32)", h->num_heads / k->num_kv_heads);
+  if (k->dtype == HS2_F32 && h->num_heads / k->num_kv_heads > 8)
+    return fail(HS2_ERR_UNSUPPORTED, "fp32 caches take GQA groups of at most 8 heads");
   const int want = k->dtype == HS2_F32 ? HS2_F32 : HS2_BF16;
   if (h->dtype != want)
     return fail(HS2_ERR_UNSUPPORTED, "%s dtype %d with cache dtype %d (need %s)", what, h->dtype, k->dtype,
@@ -196,20 +198,26 @@ bool tile_fits_pages(int tile, int page_size, bool paged) {
   return tile % page_size == 0 && tile / page_size <= 8;
 }
 
-FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged) {
+// The consumer warps split into (G + 7) / 8 head groups, so their count must
+// divide by it.
+FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged, int G) {
+  const int nhg = (G + 7) / 8;
   static const FullMmaConfig bf16_128[] = {{4, 3, 2}, {8, 3, 1}, {4, 6, 1}};
+  // groups above 8 heads give every warp several 8-head steps per tile: more
+  // consumer warps (measured at 256K, G = 32: 154 us against 179 us)
+  static const FullMmaConfig bf16_128_wide[] = {{8, 3, 1}, {4, 3, 2}, {4, 6, 1}};
   static const FullMmaConfig bf16_64[] = {{8, 6, 1}, {4, 6, 1}};
   static const FullMmaConfig e4m3[] = {{8, 3, 2}, {12, 4, 1}, {8, 6, 1}, {4, 8, 1}};
-  const FullMmaConfig *list = fp8 ? e4m3 : (D == 64 ? bf16_64 : bf16_128);
+  const FullMmaConfig *list = fp8 ? e4m3 : (D == 64 ? bf16_64 : (nhg > 1 ? bf16_128_wide : bf16_128));
   const int n = fp8 ? 4 : (D == 64 ? 2 : 3);
   if (const char *env = getenv("HS2_FULL_CFG")) {  // tuning override: "ncw,nstage[,nsl]"
     int a = 0, b = 0, c = 1;
     if (sscanf(env, "%d,%d,%d", &a, &b, &c) >= 2 && a >= 1 && a <= 16 && b >= 1 && b <= 16 && (c == 1 || c == 2) &&
-        tile_fits_pages(16 * a * c, page_size, paged))
+        a % nhg == 0 && tile_fits_pages(16 * a * c, page_size, paged))
       return FullMmaConfig{a, b, c};
   }
   for (int i = 0; i < n; ++i)
-    if (tile_fits_pages(16 * list[i].ncw * list[i].nsl, page_size, paged)) return list[i];
+    if (list[i].ncw % nhg == 0 && tile_fits_pages(16 * list[i].ncw * list[i].nsl, page_size, paged)) return list[i];
   return list[n - 1];
 }
 
@@ -311,7 +319,7 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
     if (e != cudaSuccess) return cuda_fail(e, "full-attention (fp32) launch");
   } else {
     const bool fp8 = k_cache->dtype == HS2_E4M3;
-    const FullMmaConfig cfg = pick_full_config(D, fp8, ps, paged);
+    const FullMmaConfig cfg = pick_full_config(D, fp8, ps, paged, G);
     p.tile = 16 * cfg.ncw * cfg.nsl;
     p.N = sms;
     const int box_rows = paged ? (ps < p.tile ? ps : p.tile) : p.tile;
@@ -355,6 +363,7 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
     sp.filter_subs = positions / 4096.0 > 5.0 * sms ? 2 : 1;  // 8 warps x 512 positions per sub-range
   }
   sp.c = p.c;
+  sp.ncomb = (G * D + 255) / 256;
   sp.ws = p.ws;
   e = launch_select(sp, s);
   if (e != cudaSuccess) return cuda_fail(e, "selection launch");
@@ -392,7 +401,7 @@ int hs2_sparse_attn(const hs2_heads *q_l, const hs2_cache *k_cache, const hs2_ca
   // fit in one wave of one CTA per SM or a cluster would exceed 16 CTAs; very
   // long lists then take more rows per CTA than buffers, walked as a rolling
   // pipeline.
-  const int units = p.B * p.Hkv, sms = sm_count();
+  const int units = p.B * p.Hkv * ((p.G + 7) / 8), sms = sm_count();  // clusters: one per 8 query heads
   int warps = 4, nsl = 2, nbuf_env = 0, splits_env = 0;  // (8, 1) measured equal at 32K / 256K, 10% slower at 1M
   if (const char *env = getenv("HS2_SPARSE_CFG")) {  // tuning override: "warps,nsl[,nbuf[,splits]]"
     int a = 0, b2 = 0, c2 = 0, d2 = 0;

@@ -25,6 +25,7 @@ constexpr int kSubRange = 512;           // positions per filter-warp list
 constexpr float kBandMargin = 4e-4f;     // relative margin of the selection guard band
 constexpr int kMaxSelect = 4096;         // window + k_global upper bound
 constexpr int64_t kMaxContext = int64_t(1) << 23;  // positions per sequence
+constexpr int kMaxGroup = 32;            // query heads per KV head (MQA: all of them)
 
 // Error bits of the sticky workspace flag.
 constexpr uint32_t kErrFullWait = 1u;    // consumer timed out on a full barrier
@@ -45,7 +46,7 @@ struct FullWs {
   uint32_t *hist;        // [U, kHistBins], then ticket [U] and one spare word [U]
   uint32_t *ticket;      // [U]
   int2 *thr;             // [U] (threshold bin, count strictly above it)
-  double *lse;           // [U, 8] per-head log-sum-exp of the scaled logits
+  double *lse;           // [U, kMaxGroup] per-head log-sum-exp of the scaled logits
 };
 
 // Balanced partition of the tile space over N persistent CTAs.  Tiles are

@@ -287,6 +287,13 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
   }
 
   // -------------------------------------------------------------- consumers
+  // Heads come in groups of 8 (one MMA N-tile).  With G > 8 (MQA-style
+  // groups) warp w serves head group hg = w % NHG and, of each tile, the row
+  // blocks j = w / NHG + k * (NCW / NHG), k < NHG: every head group sees every
+  // row of the tile from the same shared-memory stage.
+  const int NHG = (p.G + 7) >> 3, WPG = NCW / NHG;
+  const int hg = warp % NHG, wig = warp / NHG;
+  const int Gl = min(8, p.G - 8 * hg);  // heads of this warp's group
   WarpAttn<D, FP8, NSL> st;
   st.reset();
   uint32_t cphase = 0;
@@ -301,17 +308,21 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
     const int64_t u = (int64_t)mt.b * p.Hkv + mt.kvh;
     if (mt.flags & kFirst) {
       st.reset();
-      st.load_q(reinterpret_cast<const __nv_bfloat16 *>(p.q) + ((int64_t)mt.b * p.Hkv * p.G + (int64_t)mt.kvh * p.G) * D,
-                p.G);
+      st.load_q(reinterpret_cast<const __nv_bfloat16 *>(p.q) +
+                    ((int64_t)mt.b * p.Hkv * p.G + (int64_t)mt.kvh * p.G + 8 * hg) * D,
+                Gl);
     }
-    const int pos0 = mt.tile * C::TILE + C::RPW * warp;
-    const int nvalid = max(0, min(C::RPW, mt.T - pos0));
-    const uint32_t vmask = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
     const uint32_t kp = sbase + stage * C::STAGE;
-    const float *ks = reinterpret_cast<const float *>(smem + (size_t)stage * C::STAGE + 2 * C::KVB) + C::RPW * warp;
-    if (nvalid > 0)
-      st.step(kp, kp + C::KVB, C::PANEL, C::RPW * warp, vmask, p.c, p.ws.logits + (u * p.ustride + pos0) * p.G, p.G,
-              ks, ks + C::TILE);
+    for (int k = 0; k < NHG; ++k) {
+      const int j = wig + k * WPG;  // row block of the tile
+      const int pos0 = mt.tile * C::TILE + C::RPW * j;
+      const int nvalid = max(0, min(C::RPW, mt.T - pos0));
+      const uint32_t vmask = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
+      const float *ks = reinterpret_cast<const float *>(smem + (size_t)stage * C::STAGE + 2 * C::KVB) + C::RPW * j;
+      if (nvalid > 0)
+        st.step(kp, kp + C::KVB, C::PANEL, C::RPW * j, vmask, p.c,
+                p.ws.logits + (u * p.ustride + pos0) * p.G + 8 * hg, Gl, ks, ks + C::TILE, p.G);
+    }
     if (mt.flags & kLast) {
       // segment end: merge the warps' states inside this stage, then release it
       if (!consumer_sync(cbar, cphase)) {  // every warp is done reading the tile
@@ -326,8 +337,9 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
         break;
       }
       if (mt.rec >= 0)
-        merge_warp_states<D>(scratch, C::WSTRIDE, NCW, p.G, p.c, p.ws.records + (size_t)mt.rec * p.G * (D + 2),
-                             threadIdx.x, NCW * 32);
+        for (int g8 = 0; g8 < NHG; ++g8)  // the warps of head group g8 are g8, g8 + NHG, ...
+          merge_warp_states<D>(scratch + g8 * C::WSTRIDE, NHG * C::WSTRIDE, WPG, min(8, p.G - 8 * g8), p.c,
+                               p.ws.records + (size_t)mt.rec * p.G * (D + 2), threadIdx.x, NCW * 32, 8 * g8, p.G);
       fence_proxy_async_smem();  // before TMA refills the stage
       if (!consumer_sync(cbar, cphase)) {
         set_error(p.ws.err, kErrFullWait);

@@ -46,6 +46,7 @@ struct ScoreParams {
   int32_t nsub;              // 512-position lists per unit: ceil(t_cap / 512)
   int32_t score_chunk;       // positions per score CTA (a power of two, 2048 .. 65536)
   int32_t filter_subs;       // 512-position sub-ranges per filter warp (1 or 2)
+  int32_t ncomb;             // combine CTAs per unit (256 output elements each)
   float c;
   FullWs ws;
 };

@@ -7,7 +7,7 @@
 // group of the softmax probability p_{h,t} = exp(c * s_{h,t} - LSE_h).
 //
 // Three kernels on the CUDA cores:
-//   score  -- grid (chunk, kv head, sequence) + one combine CTA per unit; a
+//   score  -- grid (chunk, kv head, sequence) + combine CTAs per unit; a
 //             chunk (2048..65536 positions) is sized per call so the grid is
 //             one wave.  Score CTAs rebuild each head's LSE from the segment
 //             records (a parallel fp64 reduction), then turn the raw logits of
@@ -15,7 +15,7 @@
 //             per head, relative error below 1e-5) and a 4096-bin histogram of
 //             their top bits (16 bins per octave); the last chunk to finish
 //             (atomic ticket, no waiting) finds the bin b holding the
-//             k_global-th largest approximate score.  The combine CTA merges
+//             k_global-th largest approximate score.  The combine CTAs merge
 //             the records into the attention output.
 //   filter -- each warp owns one or two 512-position sub-ranges and writes,
 //             in position order, the positions whose approximate score is
@@ -52,6 +52,9 @@ constexpr int kTargetExponent = 95;    // biased exponent of 2^-32
 constexpr double kMaxShift = 948.0;
 
 constexpr int kMaxRecords = 1024;  // >= records per unit (4 * SMs / Hkv + 2)
+constexpr int kCombineElems = 256;  // output elements per combine CTA (one per thread)
+// e0 is a multiple of 256, so a combine CTA covers 256 / D whole heads (at most 4 with D = 64)
+static_assert(kMaxRecords * (kCombineElems / 64) <= kHistBins, "combine weights fit in the histogram");
 
 struct UnitInfo {
   int T, nC, nb;
@@ -205,10 +208,14 @@ __device__ void unit_lse(const float *rec0, const UnitInfo &ui, float c, double 
 }
 
 // ------------------------------------------------------------------ score
-// Loads the logits of positions tb + q * kScoreThreads (q < kScoreLoads) below t1.
-constexpr int kScoreLoads = 4;  // positions per thread in flight
+// Positions per thread in flight: 32 logits per thread in every case.
 template <int G>
-__device__ __forceinline__ void load_logits(float (&raw)[kScoreLoads][G], const float *lg, int tb, int t1) {
+constexpr int score_loads() { return G >= 32 ? 1 : (G >= 16 ? 2 : 4); }
+
+// Loads the logits of positions tb + q * kScoreThreads (q < score_loads) below t1.
+template <int G>
+__device__ __forceinline__ void load_logits(float (&raw)[score_loads<G>()][G], const float *lg, int tb, int t1) {
+  constexpr int kScoreLoads = score_loads<G>();
 #pragma unroll
   for (int q = 0; q < kScoreLoads; ++q) {
     const int t = tb + q * kScoreThreads;
@@ -284,7 +291,10 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   griddep_wait();
   griddep_launch_dependents();
   const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const bool combine = chunk == (int)gridDim.x - 1;  // the unit's combine CTA
+  // the last p.ncomb x-indices are the unit's combine CTAs, kCombineElems
+  // output elements each
+  const int comb = chunk - ((int)gridDim.x - p.ncomb);
+  const bool combine = comb >= 0;
   UnitInfo ui = unit_info(p, b, kvh);
   const int n_chunks = ui.select ? (ui.nC + p.score_chunk - 1) / p.score_chunk : 0;
   if (!combine && chunk >= n_chunks) return;
@@ -297,35 +307,32 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   mark_records(ui, sh_ok);
   const float *rec0 = p.ws.records + (size_t)u * p.R * RS;
   unit_lse<G, D>(rec0, ui, p.c, sh_lse, sh_M, sh_L, sh_red);
+  constexpr int kScoreLoads = score_loads<G>();
   float raw[kScoreLoads][G];
   if (!combine) load_logits<G>(raw, lg, t0 + threadIdx.x, t1);
 
-  if (combine) {  // out = sum_j o_j exp(c (m_j - M)) / L
+  if (combine) {  // out = sum_j o_j exp(c (m_j - M)) / L over elements [e0, e1)
+    const int e0 = comb * kCombineElems, e1 = min(G * D, e0 + kCombineElems);
+    const int h0 = e0 / D, nh = e1 > e0 ? (e1 - 1) / D - h0 + 1 : 0;
+    // the weights exp(c (m_j - M_h)) / L_h of this CTA's heads, once per (record, head)
+    float *wts = reinterpret_cast<float *>(sh_hist);  // [nseg][nh] (nseg * nh <= kHistBins)
+    for (int i = threadIdx.x; i < ui.nseg * nh; i += blockDim.x) {
+      const int j = i / nh, h = h0 + i % nh;
+      const float mj = ui.rec_ok(j) ? rec0[j * RS + h] : -INFINITY;
+      wts[i] = mj != -INFINITY && sh_L[h] > 0.f ? expf(p.c * (mj - sh_M[h])) / sh_L[h] : 0.f;
+    }
+    __syncthreads();
     const int64_t ob = ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
-    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-      const int h = e / D;
-      const float M = sh_M[h];
+    for (int e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
+      const int hi = e / D - h0;
       float acc = 0.f;
-      int j = 0;
-      for (; j + 4 <= ui.nseg; j += 4) {  // four records in flight
-        float mv[4], ov[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          mv[q] = rec0[(j + q) * RS + h];
-          ov[q] = rec0[(j + q) * RS + 2 * G + e];
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (ui.rec_ok(j + q) && mv[q] != -INFINITY) acc += ov[q] * expf(p.c * (mv[q] - M));
+#pragma unroll 8
+      for (int j = 0; j < ui.nseg; ++j) {
+        const float w = wts[j * nh + hi];
+        if (w != 0.f) acc += rec0[j * RS + 2 * G + e] * w;
       }
-      for (; j < ui.nseg; ++j) {
-        if (!ui.rec_ok(j)) continue;
-        const float mj = rec0[j * RS + h];
-        if (mj != -INFINITY) acc += rec0[j * RS + 2 * G + e] * expf(p.c * (mj - M));
-      }
-      const float val = ui.nseg > 0 && sh_L[h] > 0.f ? acc / sh_L[h] : 0.f;
-      if (p.out_dtype == 0) static_cast<float *>(p.out)[ob + e] = val;
-      else static_cast<__nv_bfloat16 *>(p.out)[ob + e] = __float2bfloat16_rn(val);
+      if (p.out_dtype == 0) static_cast<float *>(p.out)[ob + e] = acc;
+      else static_cast<__nv_bfloat16 *>(p.out)[ob + e] = __float2bfloat16_rn(acc);
     }
     return;
   }
@@ -373,7 +380,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   int bin = find_threshold_bin(sh_hist, kHistBins, p.k_global, &above, sh_warp, sh_res);
   if (bin < kTrustBin) bin = rescale_unit<G>(p, ui.nC, lg, sc, sh_hist, sh_lse, bin, &above, sh_warp, sh_res);
   if (threadIdx.x == 0) p.ws.thr[u] = make_int2(bin, above);
-  if (threadIdx.x < G) p.ws.lse[u * 8 + threadIdx.x] = sh_lse[threadIdx.x];
+  if (threadIdx.x < G) p.ws.lse[u * kMaxGroup + threadIdx.x] = sh_lse[threadIdx.x];
 }
 
 // Exact group score of one position: p_h = 2^(raw_h * a - b_h) with
@@ -383,28 +390,33 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
 __device__ __forceinline__ float exact_score(const float *raw, int G, float c, const double *lse) {
   const double ad = (double)c * kLog2e;
   const float a_hi = (float)ad, a_lo = (float)(ad - (double)a_hi);
-  float pr[8];
+  float total = 0.f;
+  for (int h0 = 0; h0 < G; h0 += 8) {  // groups of 8 heads, each summed pairwise
+    float pr[8];
 #pragma unroll
-  for (int h = 0; h < 8; ++h) {
-    pr[h] = 0.f;
-    if (h >= G) continue;
-    const double bd = lse[h] * kLog2e;
-    const float b_hi = (float)bd, b_lo = (float)(bd - (double)b_hi);
-    const float x = __ldcg(raw + h);
-    const float ph = __fmul_rn(x, a_hi);
-    const float pl = fmaf(x, a_lo, fmaf(x, a_hi, -ph));  // x*a = ph + pl
-    const float sh = __fsub_rn(ph, b_hi);                // two-sum: sh + se = ph - b_hi exactly
-    const float z = __fsub_rn(sh, ph);
-    const float se = __fadd_rn(__fsub_rn(ph, __fsub_rn(sh, z)), __fsub_rn(-b_hi, z));
-    const float yl = (se + pl) - b_lo;
-    const float e = ex2_approx(sh);
-    pr[h] = fmaf(e, yl * 0.69314718055994531f, e);  // 2^(sh + yl) = 2^sh (1 + yl ln 2)
+    for (int i = 0; i < 8; ++i) {
+      const int h = h0 + i;
+      pr[i] = 0.f;
+      if (h >= G) continue;
+      const double bd = lse[h] * kLog2e;
+      const float b_hi = (float)bd, b_lo = (float)(bd - (double)b_hi);
+      const float x = __ldcg(raw + h);
+      const float ph = __fmul_rn(x, a_hi);
+      const float pl = fmaf(x, a_lo, fmaf(x, a_hi, -ph));  // x*a = ph + pl
+      const float sh = __fsub_rn(ph, b_hi);                // two-sum: sh + se = ph - b_hi exactly
+      const float z = __fsub_rn(sh, ph);
+      const float se = __fadd_rn(__fsub_rn(ph, __fsub_rn(sh, z)), __fsub_rn(-b_hi, z));
+      const float yl = (se + pl) - b_lo;
+      const float e = ex2_approx(sh);
+      pr[i] = fmaf(e, yl * 0.69314718055994531f, e);  // 2^(sh + yl) = 2^sh (1 + yl ln 2)
+    }
+#pragma unroll
+    for (int w = 1; w < 8; w <<= 1)
+#pragma unroll
+      for (int i = 0; i + w < 8; i += 2 * w) pr[i] += pr[i + w];
+    total += pr[0];
   }
-#pragma unroll
-  for (int w = 1; w < 8; w <<= 1)
-#pragma unroll
-    for (int h = 0; h + w < 8; h += 2 * w) pr[h] += pr[h + w];
-  return pr[0] >= 0.f ? pr[0] : 0.f;  // NaN (bad inputs) ranks lowest
+  return total >= 0.f ? total : 0.f;  // NaN (bad inputs) ranks lowest
 }
 
 // ------------------------------------------------------------------ filter
@@ -507,9 +519,9 @@ __global__ void __launch_bounds__(kScoreThreads) filter_kernel(const ScoreParams
   const int bin1 = p.ws.thr[u].x;
   const float lo = __uint_as_float((uint32_t)bin1 << kHistShift) * (1.f - kBandMargin);
   const float hi = bin1 >= 0xFEF ? INFINITY : __uint_as_float((uint32_t)(bin1 + 1) << kHistShift) * (1.f + kBandMargin);
-  double lse[8];
-#pragma unroll
-  for (int h = 0; h < 8; ++h) lse[h] = h < p.G ? p.ws.lse[u * 8 + h] : 0.0;
+  __shared__ double lse[kMaxGroup];
+  if (threadIdx.x < p.G) lse[threadIdx.x] = p.ws.lse[u * kMaxGroup + threadIdx.x];
+  __syncthreads();
 #pragma unroll
   for (int k = 0; k < kFilterSubsMax; ++k) {
     const int sub = sub0 + k * kWarps;
@@ -794,12 +806,14 @@ size_t final_smem_bytes(int nsub) { return (size_t)(2 * (nsub + 1) + 5 * kMaxSel
 cudaError_t launch_select(const ScoreParams &p, cudaStream_t s) {
   const int chunks = (int)((p.t_cap + p.score_chunk - 1) / p.score_chunk);
   cudaError_t e;
-  const dim3 sgrid(chunks + 1, p.Hkv, p.B);  // + the combine CTA of each unit
+  const dim3 sgrid(chunks + p.ncomb, p.Hkv, p.B);  // + the combine CTAs of each unit
   switch (p.G) {
     case 1: e = launch_score_g<1>(p, sgrid, s); break;
     case 2: e = launch_score_g<2>(p, sgrid, s); break;
     case 4: e = launch_score_g<4>(p, sgrid, s); break;
     case 8: e = launch_score_g<8>(p, sgrid, s); break;
+    case 16: e = launch_score_g<16>(p, sgrid, s); break;
+    case 32: e = launch_score_g<32>(p, sgrid, s); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;

@@ -41,7 +41,7 @@ struct SCfg {
   __host__ __device__ static bool scratch_in_staging(int G, int S, int nbuf) {
     return scratch_bytes(G, S) <= staging(nbuf);
   }
-  static size_t bytes(int G, int S, int rows, int nbuf) {
+  static size_t bytes(int G, int S, int rows, int nbuf) {  // G: heads of one cluster (<= 8)
     return 128 + staging(nbuf) + (scratch_in_staging(G, S, nbuf) ? 0 : scratch_bytes(G, S)) +
            (size_t)rec_floats(G) * 4 + (size_t)(3 * S + 1) * 8 * 4 + (size_t)rows * 4;
   }
@@ -67,9 +67,10 @@ __global__ void __launch_bounds__(32 * NW, 1) sparse_mma_kernel(const SparsePara
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   cg::cluster_group cluster = cg::this_cluster();
   const int S = (int)cluster.num_blocks();
-  const int RSP = C::rec_floats(p.G);
+  const int Gc = p.G < 8 ? p.G : 8;  // heads of one cluster (the shared-memory layout)
+  const int RSP = C::rec_floats(Gc);
   const int nbuf = p.nbuf;
-  const bool in_staging = C::scratch_in_staging(p.G, S, nbuf);
+  const bool in_staging = C::scratch_in_staging(Gc, S, nbuf);
   uint8_t *after = smem + C::staging(nbuf) + (in_staging ? 0 : C::scratch_bytes(p.G, S));
   float *scratch = reinterpret_cast<float *>(in_staging ? smem : smem + C::staging(nbuf));
   float *partial = reinterpret_cast<float *>(after);             // m[G], l[G], o[G][D] of this CTA
@@ -78,8 +79,13 @@ __global__ void __launch_bounds__(32 * NW, 1) sparse_mma_kernel(const SparsePara
   float *ms_ = inv_l + 8, *ls_ = ms_ + S * 8;                    // (m, l) of (CTA, head)
   int *slots = reinterpret_cast<int *>(ls_ + S * 8);             // this CTA's index entries
   const int rank = (int)cluster.block_rank();
-  const int kvh = blockIdx.y, b = blockIdx.z, G = p.G;
+  // blockIdx.y = (kv head, group of 8 query heads): groups above 8 heads
+  // (MQA-style) take one cluster per 8 heads, each gathering the rows itself
+  const int nhg = (p.G + 7) >> 3;
+  const int kvh = blockIdx.y / nhg, hg = blockIdx.y % nhg, b = blockIdx.z;
+  const int G = min(8, p.G - 8 * hg);  // heads of this cluster
   const int64_t u = (int64_t)b * p.Hkv + kvh;
+  const int64_t head0 = (int64_t)b * p.Hkv * p.G + (int64_t)kvh * p.G + 8 * hg;  // first query head
   const int row_lo = rank * p.rows_per_cta, nrows = max(0, min(p.L, row_lo + p.rows_per_cta) - row_lo);
   griddep_wait();  // the index list and the query come from earlier kernels
   griddep_launch_dependents();
@@ -91,7 +97,7 @@ __global__ void __launch_bounds__(32 * NW, 1) sparse_mma_kernel(const SparsePara
   }
   WarpAttn<D, FP8, NSL> st;
   st.reset();
-  st.load_q(static_cast<const __nv_bfloat16 *>(p.q) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D, G);
+  st.load_q(static_cast<const __nv_bfloat16 *>(p.q) + head0 * D, G);
   __syncthreads();
 
   constexpr int CPR = C::ROWB / 16;  // 16-byte chunks per row
@@ -189,7 +195,7 @@ __global__ void __launch_bounds__(32 * NW, 1) sparse_mma_kernel(const SparsePara
   __syncthreads();
   {
     const int per = (G * D + S - 1) / S, e0 = rank * per, e1 = min(G * D, e0 + per);
-    const int64_t ob = ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
+    const int64_t ob = head0 * D;
     for (int e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
       const int h = e / D;
       float acc = 0.f;
@@ -254,7 +260,7 @@ __global__ void sparse_f32_kernel(const SparseParams p, int64_t num_slots) {
 template <int D, bool FP8, int NW, int NSL>
 cudaError_t launch_mma_t(const SparseParams &p, int64_t num_slots, cudaStream_t s) {
   using C = SCfg<D, FP8, NW, NSL>;
-  const size_t smem = C::bytes(p.G, p.splits, p.rows_per_cta, p.nbuf);
+  const size_t smem = C::bytes(p.G < 8 ? p.G : 8, p.splits, p.rows_per_cta, p.nbuf);
   auto kern = sparse_mma_kernel<D, FP8, NW, NSL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -262,7 +268,7 @@ cudaError_t launch_mma_t(const SparseParams &p, int64_t num_slots, cudaStream_t 
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  return launch_ex(kern, dim3(p.splits, p.Hkv, p.B), dim3(32 * NW), smem, s, p.splits, p, num_slots);
+  return launch_ex(kern, dim3(p.splits, p.Hkv * ((p.G + 7) / 8), p.B), dim3(32 * NW), smem, s, p.splits, p, num_slots);
 }
 
 template <int D, bool FP8>

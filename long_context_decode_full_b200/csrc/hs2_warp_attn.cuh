@@ -96,10 +96,13 @@ struct WarpAttn {
   // tile; pstride: bytes between panels; row0: first row of the first slice
   // inside the panel (slice sl starts at row0 + 16 sl); vmask: bit r set when
   // row row0 + r holds a real position; c: 1/sqrt(D) in the logit domain.
-  // logit_dst (or nullptr): raw logits [16 NSL][G] of these rows.  ks / vs
-  // (E4M3): the rows' K / V scales in shared memory.
+  // logit_dst (or nullptr): raw logits of these rows for the G heads of this
+  // warp, row r at logit_dst + r * ldl.  ks / vs (E4M3): the rows' K / V
+  // scales in shared memory.
   __device__ __forceinline__ void step(uint32_t kp, uint32_t vp, uint32_t pstride, int row0, uint32_t vmask,
-                                       float c, float *logit_dst, int G, const float *ks, const float *vs) {
+                                       float c, float *logit_dst, int G, const float *ks, const float *vs,
+                                       int ldl = -1) {
+    if (ldl < 0) ldl = G;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     // two accumulator chains per slice (even / odd k-steps) halve the
     // dependent-MMA latency; their fp32 sum is the logit
@@ -174,7 +177,7 @@ struct WarpAttn {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           if (!ok[sl][j]) continue;
-          float *dst = logit_dst + (16 * sl + 8 * j + g) * G + 2 * t;
+          float *dst = logit_dst + (16 * sl + 8 * j + g) * ldl + 2 * t;
           if ((G & 1) == 0) st_global_hint(dst, x[sl][j][0], x[sl][j][1], keep);
           else {
             st_global_hint(dst, x[sl][j][0], keep);
@@ -347,11 +350,13 @@ struct WarpAttn {
 };
 
 // Merges NW warp states in shared scratch (stride `wstride` floats per warp:
-// m[8], l[8], o[8][D]) into one record m[G], l[G], o[G][D] at `rec` (global or
-// shared).  Threads tid .. nthreads cooperate.
+// m[8], l[8], o[8][D]) of G <= 8 heads into heads hoff .. hoff + G - 1 of a
+// record of Gtot heads, m[Gtot], l[Gtot], o[Gtot][D], at `rec` (global or
+// shared; Gtot = G, hoff = 0 by default).  Threads tid .. nthreads cooperate.
 template <int D>
 __device__ __forceinline__ void merge_warp_states(const float *scr, int wstride, int NW, int G, float c,
-                                                  float *rec, int tid, int nthreads) {
+                                                  float *rec, int tid, int nthreads, int hoff = 0, int Gtot = -1) {
+  if (Gtot < 0) Gtot = G;
   for (int h = tid; h < G; h += nthreads) {
     float M = -INFINITY;
     for (int w = 0; w < NW; ++w) M = fmaxf(M, scr[w * wstride + h]);
@@ -360,9 +365,10 @@ __device__ __forceinline__ void merge_warp_states(const float *scr, int wstride,
       const float mw = scr[w * wstride + h];
       if (mw != -INFINITY) L += expf(c * (mw - M)) * scr[w * wstride + 8 + h];
     }
-    rec[h] = M;
-    rec[G + h] = L;
+    rec[hoff + h] = M;
+    rec[Gtot + hoff + h] = L;
   }
+  rec += 2 * Gtot + hoff * D;  // o of head hoff
   // thread -> (dim, first head); each head's warp weights computed once per thread
   const int dim = tid % D, h0 = tid / D, hstep = nthreads / D;
   if (hstep == 0) {  // fewer threads than head dims
@@ -375,7 +381,7 @@ __device__ __forceinline__ void merge_warp_states(const float *scr, int wstride,
         const float mw = scr[w * wstride + h];
         if (mw != -INFINITY) acc += expf(c * (mw - M)) * scr[w * wstride + 16 + e];
       }
-      rec[2 * G + e] = acc;
+      rec[e] = acc;
     }
     return;
   }
@@ -388,7 +394,7 @@ __device__ __forceinline__ void merge_warp_states(const float *scr, int wstride,
       const float mw = scr[w * wstride + h];
       if (mw != -INFINITY) acc += expf(c * (mw - M)) * scr[w * wstride + 16 + h * D + dim];
     }
-    rec[2 * G + h * D + dim] = acc;
+    rec[h * D + dim] = acc;
   }
 }
 

@@ -65,6 +65,10 @@ WORKLOADS = {
         WorkloadSpec("ctx256k_b4_bf16_paged", 4, 4, 8, 128, 262144, "bf16", "bf16", 64, 3,
                      needles=256, needle_bursts=8),
         WorkloadSpec("ctx1m_b1_fp8_paged", 1, 4, 8, 128, 1048576, "e4m3", "bf16", 64, 3, needles=1024),
+        # the compact MQA configuration: one KV head shared by all 32 query heads
+        WorkloadSpec("mqa_ctx256k_b4_bf16_paged", 4, 1, 32, 128, 262144, "bf16", "bf16", 64, 3,
+                     needles=256, needle_bursts=8),
+        WorkloadSpec("mqa_ctx1m_b1_fp8_paged", 1, 1, 32, 128, 1048576, "e4m3", "bf16", 64, 3, needles=1024),
     ]
 }
 

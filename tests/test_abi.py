@@ -61,7 +61,10 @@ def sparse(q=None, k=None, v=None, idx=FAKE, stride=1152, out=None):
     (dict(k=cache(dim=96), v=cache(dim=96)), hs2.ERR_UNSUPPORTED),
     (dict(k=cache(heads=4)), hs2.ERR_INVALID_ARG),
     (dict(q=heads(h=6), out=heads(h=6)), hs2.ERR_UNSUPPORTED),
-    (dict(q=heads(h=64), out=heads(h=64)), hs2.ERR_UNSUPPORTED),
+    (dict(q=heads(h=128), out=heads(h=128)), hs2.ERR_UNSUPPORTED),  # G = 64
+    (dict(q=heads(h=24), out=heads(h=24)), hs2.ERR_UNSUPPORTED),    # G = 12
+    (dict(k=cache(dtype=0, dim=64), v=cache(dtype=0, dim=64), q=heads(dtype=0, h=32, dim=64),
+          out=heads(dtype=0, h=32, dim=64)), hs2.ERR_UNSUPPORTED),  # fp32 cache, G = 16
     (dict(q=heads(dtype=0), out=heads(dtype=0)), hs2.ERR_UNSUPPORTED),
     (dict(out=heads(b=3)), hs2.ERR_INVALID_ARG),
     (dict(seq=0), hs2.ERR_INVALID_ARG),

@@ -1,4 +1,4 @@
-"""Parity at the full sizes of the five decode workloads, in the launch
+"""Parity at the full sizes of the seven decode workloads (five GQA-8, two MQA), in the launch
 configuration the benchmark times.  Every (sequence, KV head) unit of every
 workload is recomputed by the oracle (one unit per task, in a pool of spawned
 CPU processes) and compared element by element: the full layer's output, the
@@ -22,7 +22,7 @@ import oracle_pool
 pytestmark = pytest.mark.gpu
 
 WORKLOADS = ["tiny_fp32_t2048", "decode_b8_32k_bf16", "paged_b64_8k_128k_bf16", "ctx256k_b4_bf16_paged",
-             "ctx1m_b1_fp8_paged"]
+             "ctx1m_b1_fp8_paged", "mqa_ctx256k_b4_bf16_paged", "mqa_ctx1m_b1_fp8_paged"]
 
 
 @pytest.fixture(scope="module")

@@ -37,6 +37,10 @@ CASES = {
     "e4m3_paged32_nanpad": spec(kv_dtype="e4m3", page_size=32, batch=2, seq_len=(1200, 2600)),
     "e4m3_paged16": spec(kv_dtype="e4m3", page_size=16, batch=2, seq_len=(1100, 2700)),
     "e4m3_contiguous_g4": spec(kv_dtype="e4m3", page_size=None, group=4, num_kv_heads=3, batch=2),
+    "bf16_g16": spec(group=16, num_kv_heads=2, batch=2),
+    "bf16_mqa_g32": spec(group=32, num_kv_heads=1, batch=3),
+    "bf16_mqa_g32_d64_contiguous": spec(group=32, num_kv_heads=1, batch=2, head_dim=64, page_size=None),
+    "e4m3_mqa_g32": spec(kv_dtype="e4m3", group=32, num_kv_heads=1, batch=2, seq_len=(1500, 4000)),
     "f32_tiny": synth.WORKLOADS["tiny_fp32_t2048"],
     "f32_paged_ragged": spec(kv_dtype="f32", q_dtype="f32", head_dim=64, group=4, page_size=16,
                              seq_len=(1200, 2500)),
