@@ -78,7 +78,7 @@ typedef struct {
   void *data;          /* device; 16-byte aligned */
   int32_t dtype;       /* HS2_F32 (with an HS2_F32 cache) or HS2_BF16 */
   int32_t batch;
-  int32_t num_heads;   /* num_kv_heads * G, G in {1, 2, 4, 8} */
+  int32_t num_heads;   /* num_kv_heads * G, G in {1, 2, 4, 8, 16, 32} (above 8: bf16 / E4M3 caches) */
   int32_t head_dim;
 } hs2_heads;
 
@@ -141,6 +141,29 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
                                 const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
                                 int32_t window, int32_t k_global, hs2_heads *out, int32_t *idx_out,
                                 void *workspace, size_t workspace_bytes, void *stream, void *mark_event);
+
+/*
+ * The full-attention layer with BLOCK-level instead of token-level selection:
+ * the first-generation HySparse selection, kept as a comparator (HySparse2
+ * announcement, the paragraphs contrasting token-level with HySparse's
+ * block-level selection: v1 chose whole blocks, so an important token brought
+ * the block around it; the two were compared at the same token budget).
+ * Readings: the selectable positions [0, T_b - W) are cut into blocks of
+ * `block` positions, the last one cut short at T_b - W; a block's score is
+ * the sum of its positions' group scores (as for hs2_full_attn_select());
+ * k_global / block blocks are taken by (block score desc, block index asc),
+ * all of them when there are no more; the window is always taken.
+ *
+ *   Arguments as hs2_full_attn_select(), plus block >= 1 dividing k_global
+ *   (else HS2_ERR_INVALID_ARG).  out is the same attention output; idx_out
+ *   holds the slots of the taken positions in ascending position order (the
+ *   taken blocks' positions, then the window), the rest -1.  The workspace is
+ *   that of hs2_full_attn_select() (same size function).
+ */
+int hs2_full_attn_select_blocks(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                                const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
+                                int32_t window, int32_t k_global, int32_t block, hs2_heads *out, int32_t *idx_out,
+                                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * hs2_full_attn_select() for callers that cannot allocate device memory.

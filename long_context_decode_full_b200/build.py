@@ -21,8 +21,9 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
                 "-I", os.path.join(ROOT, "include"), "-I", CSRC]
-SOURCES = ["hs2_api.cu", "hs2_full_attn.cu", "hs2_select.cu", "hs2_sparse.cu", "hs2_static.cu", "hs2_bridge.cu"]
-HEADERS = ["hs2_common.cuh", "hs2_internal.h", "hs2_warp_attn.cuh"]
+SOURCES = ["hs2_api.cu", "hs2_full_attn.cu", "hs2_select.cu", "hs2_blocks.cu", "hs2_sparse.cu", "hs2_static.cu",
+           "hs2_bridge.cu"]
+HEADERS = ["hs2_common.cuh", "hs2_internal.h", "hs2_warp_attn.cuh", "hs2_select_common.cuh"]
 
 
 def _stale(target: str, deps) -> bool:

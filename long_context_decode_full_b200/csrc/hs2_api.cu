@@ -221,6 +221,11 @@ FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged, int G
   return list[n - 1];
 }
 
+int full_attn_select_impl(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                          const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages, int32_t window,
+                          int32_t k_global, int32_t block, hs2_heads *out, int32_t *idx_out, void *workspace,
+                          size_t workspace_bytes, void *stream, void *mark_event);
+
 }  // namespace
 
 extern "C" {
@@ -249,6 +254,30 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
                                 const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
                                 int32_t window, int32_t k_global, hs2_heads *out, int32_t *idx_out,
                                 void *workspace, size_t workspace_bytes, void *stream, void *mark_event) {
+  return full_attn_select_impl(q, k_cache, v_cache, seq_lens, page_table, max_pages, window, k_global, 0, out,
+                               idx_out, workspace, workspace_bytes, stream, mark_event);
+}
+
+int hs2_full_attn_select_blocks(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                                const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
+                                int32_t window, int32_t k_global, int32_t block, hs2_heads *out, int32_t *idx_out,
+                                void *workspace, size_t workspace_bytes, void *stream) {
+  if (block < 1 || k_global < 0 || k_global % block != 0)
+    return fail(HS2_ERR_INVALID_ARG, "block %d must be >= 1 and divide k_global %d", block, k_global);
+  return full_attn_select_impl(q, k_cache, v_cache, seq_lens, page_table, max_pages, window, k_global, block, out,
+                               idx_out, workspace, workspace_bytes, stream, nullptr);
+}
+
+}  // extern "C"
+
+namespace {
+
+// The full layer, then token-level selection (block = 0) or block-level
+// selection with blocks of `block` positions.
+int full_attn_select_impl(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                          const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages, int32_t window,
+                          int32_t k_global, int32_t block, hs2_heads *out, int32_t *idx_out, void *workspace,
+                          size_t workspace_bytes, void *stream, void *mark_event) {
   int rc;
   if ((rc = check_caches(k_cache, v_cache))) return rc;
   if ((rc = check_heads(q, k_cache, "q"))) return rc;
@@ -365,10 +394,14 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
   sp.c = p.c;
   sp.ncomb = (G * D + 255) / 256;
   sp.ws = p.ws;
-  e = launch_select(sp, s);
+  e = block > 0 ? launch_block_select(sp, block, s) : launch_select(sp, s);
   if (e != cudaSuccess) return cuda_fail(e, "selection launch");
   return HS2_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 int hs2_sparse_attn(const hs2_heads *q_l, const hs2_cache *k_cache, const hs2_cache *v_cache, const int32_t *idx,
                     int32_t idx_stride, hs2_heads *out, void *stream) {

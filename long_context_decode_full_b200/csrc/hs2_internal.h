@@ -112,6 +112,8 @@ int full_f32_tile();
 int full_f32_ctas_per_sm();
 
 cudaError_t launch_select(const ScoreParams &p, cudaStream_t s);
+// Block-level selection (first-generation comparator) in place of launch_select.
+cudaError_t launch_block_select(const ScoreParams &p, int block, cudaStream_t s);
 
 cudaError_t launch_sparse_impl(const SparseParams &p, int kv_dtype, int64_t num_slots, cudaStream_t s);
 

@@ -42,6 +42,7 @@ class HS2Error(RuntimeError):
 
 _lib = None
 EXPORTS = ["hs2_full_attn_select_workspace", "hs2_full_attn_select", "hs2_full_attn_select_marked",
+           "hs2_full_attn_select_blocks",
            "hs2_full_attn_select_static", "hs2_full_attn_select_static_status", "hs2_selftest_bounded_wait_static",
            "hs2_sparse_attn",
            "hs2_workspace_status", "hs2_selftest_bounded_wait", "hs2_kv_bridge_workspace", "hs2_kv_bridge_append",
@@ -64,6 +65,9 @@ def lib():
         L.hs2_full_attn_select.restype = ctypes.c_int
         L.hs2_full_attn_select_marked.argtypes = L.hs2_full_attn_select.argtypes + [P]
         L.hs2_full_attn_select_marked.restype = ctypes.c_int
+        L.hs2_full_attn_select_blocks.argtypes = [ctypes.POINTER(Heads), ctypes.POINTER(Cache), ctypes.POINTER(Cache),
+                                                  P, P, I32, I32, I32, I32, ctypes.POINTER(Heads), P, P, SZ, P]
+        L.hs2_full_attn_select_blocks.restype = ctypes.c_int
         L.hs2_full_attn_select_static.argtypes = [ctypes.POINTER(Heads), ctypes.POINTER(Cache),
                                                   ctypes.POINTER(Cache), P, P, I32, I32, I32,
                                                   ctypes.POINTER(Heads), P, P]
@@ -192,6 +196,36 @@ def full_attn_select(q, k, v, seq_lens, page_table=None, page_size=None, window=
                                              _ptr(seq_lens), _ptr(page_table), max_pages, window, k_global,
                                              ctypes.byref(od), _ptr(idx_out), _ptr(workspace), workspace.numel(),
                                              _stream(stream), ev))
+    return out, idx_out
+
+
+def full_attn_select_blocks(q, k, v, seq_lens, page_table=None, page_size=None, window=128, k_global=1024,
+                            block=16, k_scale=None, v_scale=None, out=None, idx_out=None, workspace=None,
+                            stream=None):
+    """Full-attention layer + BLOCK-level selection (the first-generation
+    comparator): the same attention output, and idx [B, Hkv, window + k_global]
+    with the slots of the k_global / block best blocks' positions and the
+    window, ascending, -1 padded."""
+    B, Hq, d = q.shape
+    Hkv = k.shape[1]
+    _need_lens(seq_lens, page_table, B)
+    _need("idx_out", idx_out, torch.int32, shape=(B, Hkv, window + k_global))
+    _need_cuda(q=q, k=k, v=v, seq_lens=seq_lens, page_table=page_table, idx_out=idx_out)
+    if page_size is None:
+        assert page_table is None, "page_size is required with a page table"
+        page_size = k.shape[0] // B
+    max_pages = 1 if page_table is None else page_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if idx_out is None:
+        idx_out = torch.empty(B, Hkv, window + k_global, dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, Hkv, Hq // Hkv, d, page_size * max_pages, q.device)
+    kc, vc = cache_desc(k, k_scale, page_size), cache_desc(v, v_scale, page_size)
+    qd, od = heads_desc(q), heads_desc(out)
+    _check(lib().hs2_full_attn_select_blocks(ctypes.byref(qd), ctypes.byref(kc), ctypes.byref(vc), _ptr(seq_lens),
+                                             _ptr(page_table), max_pages, window, k_global, block, ctypes.byref(od),
+                                             _ptr(idx_out), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out, idx_out
 
 

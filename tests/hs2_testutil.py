@@ -190,3 +190,36 @@ def check_idx_positions(gpos_row, opos_row, ora_score, T, window, k_global):
         assert not bad, (f"{len(bad)} positions differ outside the near-tie band, e.g. {bad[:5]} "
                          f"(scores {[ora_score[t] for t in bad[:5]]}, k-th {sk})")
     return len(diff)
+
+
+def check_block_positions(gpos_row, opos_row, ora_score, T, window, k_global, block):
+    """Block-level index lists as positions: the GPU's (gpos_row, -1 padded)
+    against the oracle's (opos_row).  Both must hold the window and whole
+    blocks in ascending order; a block may differ only when its oracle block
+    sum lies within 1e-6 relative of the oracle's (k_global / block)-th block
+    sum.  Returns the number of blocks that differ."""
+    L = window + k_global
+    g = np.asarray(gpos_row)
+    assert len(g) == L
+    gv = g[g >= 0]
+    assert np.all(g[len(gv):] == -1), "padding must be -1 and last"
+    assert np.all(np.diff(gv) > 0), "positions must be strictly ascending"
+    nC = max(0, T - window)
+    win = set(range(nC, T))
+    assert win <= set(gv.tolist()), "forced window missing"
+    ov = np.asarray(opos_row)
+    ov = ov[ov >= 0]
+    gblk = {int(t) // block for t in gv if t < nC}
+    oblk = {int(t) // block for t in ov if t < nC}
+    for j in gblk:  # whole blocks only
+        lo, hi = j * block, min((j + 1) * block, nC)
+        assert set(range(lo, hi)) <= set(gv.tolist()), f"block {j} taken in part"
+    diff = gblk ^ oblk
+    if diff:
+        nblk = (nC + block - 1) // block
+        sums = np.array([ora_score[j * block:min((j + 1) * block, nC)].sum() for j in range(nblk)])
+        keep = k_global // block
+        sk = np.sort(sums)[::-1][keep - 1]
+        bad = [j for j in diff if not (abs(sums[j] - sk) <= NEAR_TIE * sk)]
+        assert not bad, f"{len(bad)} blocks differ outside the near-tie band, e.g. {bad[:5]} (k-th sum {sk})"
+    return len(diff)

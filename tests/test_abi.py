@@ -229,3 +229,14 @@ def test_header_is_plain_c_and_links(libhs2, tmp_path):
     assert int(out[0]) == hs2.version()
     assert int(out[1]) == hs2.kv_bridge_workspace_bytes(4, 4096, 4, 128)
     assert int(out[2]) == hs2.ERR_INVALID_ARG and int(out[3]) == len(names) and out[4].strip()
+
+
+def test_block_selection_rejects_a_block_that_does_not_divide_the_budget(libhs2):
+    q, k, v, out = heads(), cache(), cache(), heads()
+    call = lambda K, blk: hs2.lib().hs2_full_attn_select_blocks(
+        ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), FAKE, FAKE, 64, 128, K, blk, ctypes.byref(out), FAKE,
+        FAKE * 16, 1 << 40, None)
+    assert call(1024, 3) == hs2.ERR_INVALID_ARG
+    assert call(1024, 0) == hs2.ERR_INVALID_ARG
+    assert call(1024, -4) == hs2.ERR_INVALID_ARG
+    assert "divide" in hs2.last_error()

@@ -25,6 +25,15 @@ WORKLOADS = ["tiny_fp32_t2048", "decode_b8_32k_bf16", "paged_b64_8k_128k_bf16", 
              "ctx1m_b1_fp8_paged", "mqa_ctx256k_b4_bf16_paged", "mqa_ctx1m_b1_fp8_paged"]
 
 
+# workloads whose every unit is also checked with block-level selection (block size)
+BLOCK_WORKLOADS = {"decode_b8_32k_bf16": 16, "ctx256k_b4_bf16_paged": 16, "ctx1m_b1_fp8_paged": 64}
+
+
+@pytest.fixture(scope="module")
+def oracle_mod(oracle):
+    return oracle
+
+
 @pytest.fixture(scope="module")
 def pool(oracle):
     # spawned workers (no fork of a process that holds a CUDA context)
@@ -82,7 +91,7 @@ def check_unit(w, res, gpos_row, outs):
 
 
 @pytest.mark.parametrize("name", WORKLOADS)
-def test_full_size_workload_every_unit(pool, name):
+def test_full_size_workload_every_unit(pool, oracle_mod, name):
     ex, nworkers = pool
     spec = synth.WORKLOADS[name]
     w = synth.generate(spec, seed=0, device="cuda")
@@ -95,7 +104,7 @@ def test_full_size_workload_every_unit(pool, name):
         assert torch.isfinite(o.float()).all()
     gpos = gpu_positions(w, idx)
     units = [(b, h) for b in range(spec.batch) for h in range(spec.num_kv_heads)]
-    pending, done, worst, ndiff = set(), 0, 0.0, 0
+    pending, done, worst, ndiff, scores = set(), 0, 0.0, 0, {}
     it = iter(units)
     while True:
         while len(pending) < 2 * nworkers:
@@ -112,9 +121,27 @@ def test_full_size_workload_every_unit(pool, name):
             res = f.result()
             b, h = res["key"]
             err, nd = check_unit(w, res, gpos[b, h], outs)
+            if name in BLOCK_WORKLOADS:
+                scores[(b, h)] = res["score"]
             worst = max(worst, err)
             ndiff += nd
             done += 1
     assert done == len(units)
     print(f"{name}: {done} units, worst full-layer max-abs {worst:.2e}, "
           f"positions differing inside the near-tie band {ndiff}")
+    if name in BLOCK_WORKLOADS:  # block-level selection on the same inputs, every unit
+        block = BLOCK_WORKLOADS[name]
+        _, bidx = hs2.full_attn_select_blocks(w.q_full, w.k, w.v, w.seq_lens, w.page_table, w.page_size,
+                                              spec.window, spec.k_global, block, w.k_scale, w.v_scale,
+                                              workspace=ws)
+        torch.cuda.synchronize()
+        assert hs2.workspace_status(ws) == 0
+        bpos = gpu_positions(w, bidx)
+        nb = 0
+        for (b, h), score in scores.items():
+            T = int(w.seq_lens[b])
+            ora = oracle_mod.select_blocks(score, T, spec.window, spec.k_global, block)
+            opos = np.full(spec.window + spec.k_global, -1)
+            opos[:len(ora)] = ora
+            nb += U.check_block_positions(bpos[b, h], opos, score, T, spec.window, spec.k_global, block)
+        print(f"{name}: block-level selection (block {block}), blocks differing inside the near-tie band {nb}")

@@ -296,3 +296,58 @@ def test_selection_below_fp32_range(oracle, lib, kv_dtype, lo, hi):
     out, idx = U.run_gpu(wd)
     torch.cuda.synchronize()
     U.check_full(wd, out, idx, ora)
+
+
+BLOCK_CASES = {
+    "bf16_paged64_b16": (spec(), 16, 128, 1024),
+    "bf16_contiguous_b1": (spec(page_size=None, batch=2), 1, 128, 1024),
+    "e4m3_paged32_b8": (spec(kv_dtype="e4m3", page_size=32, batch=2, seq_len=(1500, 4000)), 8, 128, 1024),
+    "f32_tiny_b64": (synth.WORKLOADS["tiny_fp32_t2048"], 64, 128, 1024),
+    "mqa_g32_b32": (spec(group=32, num_kv_heads=1, batch=2), 32, 128, 1024),
+    "short_contexts_b16": (spec(seq_len=(1, 1400), batch=4), 16, 128, 1024),
+    "one_block_of_k": (spec(batch=2), 1024, 128, 1024),
+    "odd_budget_b5": (spec(batch=2, seq_len=(900, 2500)), 5, 64, 300),
+    "no_global_budget": (spec(batch=2), 4, 128, 0),
+}
+
+
+@pytest.mark.parametrize("name", list(BLOCK_CASES))
+def test_block_selection_matches_oracle(oracle, lib, name):
+    """Block-level selection (the first-generation comparator) against the
+    oracle's block ranking of its own group scores, every unit."""
+    sp, block, W, K = BLOCK_CASES[name]
+    w = synth.generate(sp, seed=zlib.crc32(name.encode()) % 1000)
+    s = w.spec
+    code = U.DTYPE_CODE
+    ora = oracle.full_attn_select_blocks(synth.raw(w.q_full), code[s.q_dtype], synth.raw(w.k), synth.raw(w.v),
+                                         code[s.kv_dtype], synth.raw(w.seq_lens), synth.raw(w.page_table),
+                                         w.page_size, window=W, k_global=K, block=block,
+                                         k_scale=synth.raw(w.k_scale), v_scale=synth.raw(w.v_scale))
+    wd = U.to_device(w)
+    out, idx = lib.full_attn_select_blocks(wd.q_full, wd.k, wd.v, wd.seq_lens, wd.page_table, wd.page_size, W, K,
+                                           block, wd.k_scale, wd.v_scale, workspace=U.garbage_workspace(wd))
+    torch.cuda.synchronize()
+    U.check_out(out, ora["out"], s.kv_dtype)
+    gi = idx.cpu().numpy()
+    for b in range(s.batch):
+        T = int(w.seq_lens[b])
+        s2p = U.slot_to_pos(w, b)
+        for h in range(s.num_kv_heads):
+            gpos = np.array([s2p[int(x)] if x >= 0 else -1 for x in gi[b, h]])
+            opos = np.array([s2p[int(x)] if x >= 0 else -1 for x in ora["idx"][b, h]])
+            U.check_block_positions(gpos, opos, ora["score"][b, h], T, W, K, block)
+
+
+def test_block_selection_with_zero_query_takes_the_lowest_blocks(oracle, lib):
+    """q = 0: every position scores alike, every full block ties, so the
+    lowest k_global / block blocks are taken (bit-exact)."""
+    sp = spec(seq_len=3000, batch=2)
+    w = synth.generate(sp, seed=8)
+    w.q_full.zero_()
+    ora = oracle.full_attn_select_blocks(synth.raw(w.q_full), 1, synth.raw(w.k), synth.raw(w.v), 1,
+                                         synth.raw(w.seq_lens), synth.raw(w.page_table), w.page_size,
+                                         window=128, k_global=1024, block=16)
+    wd = U.to_device(w)
+    _, idx = lib.full_attn_select_blocks(wd.q_full, wd.k, wd.v, wd.seq_lens, wd.page_table, wd.page_size, 128,
+                                         1024, 16)
+    assert np.array_equal(idx.cpu().numpy(), ora["idx"])
