@@ -38,9 +38,9 @@ namespace hs2 {
 namespace {
 
 // ------------------------------------------------------------------ score
-// Positions per thread in flight: 32 logits per thread in every case.
+// Positions per thread and batch (two batches in flight): 16 logits per batch.
 template <int G>
-constexpr int score_loads() { return G >= 32 ? 1 : (G >= 16 ? 2 : 4); }
+constexpr int score_loads() { return G >= 16 ? 1 : 16 / G; }
 
 // Loads the logits of positions tb + q * kScoreThreads (q < score_loads) below t1.
 template <int G>
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
   const float *rec0 = p.ws.records + (size_t)u * p.R * RS;
   unit_lse<G, D>(rec0, ui, p.c, sh_lse, sh_M, sh_L, sh_red);
   constexpr int kScoreLoads = score_loads<G>();
-  float raw[kScoreLoads][G];
+  float raw[kScoreLoads][G], raw2[kScoreLoads][G];
   if (!combine) load_logits<G>(raw, lg, t0 + threadIdx.x, t1);
 
   if (combine) {
@@ -155,15 +155,14 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
 #pragma unroll
   for (int h = 0; h < G; ++h) bh[h] = (float)(sh_lse[h] * kLog2e);
   constexpr int kStep = kScoreLoads * kScoreThreads;
-  for (int tb = t0 + threadIdx.x; tb < t1; tb += kStep) {
-    if (tb > t0 + (int)threadIdx.x) load_logits<G>(raw, lg, tb, t1);  // (the first batch is loaded)
+  auto score_batch = [&](const float (&r)[kScoreLoads][G], int tb) {
 #pragma unroll
     for (int q = 0; q < kScoreLoads; ++q) {
       const int t = tb + q * kScoreThreads;
       if (t >= t1) break;
       float pr[G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) pr[h] = ex2_approx(fmaf(raw[q][h], a, -bh[h]));
+      for (int h = 0; h < G; ++h) pr[h] = ex2_approx(fmaf(r[q][h], a, -bh[h]));
 #pragma unroll
       for (int w = 1; w < G; w <<= 1)  // pairwise sum of the group's probabilities
 #pragma unroll
@@ -172,6 +171,14 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams 
       sc[t] = s;
       atomicAdd(&sh_hist[__float_as_uint(s) >> kHistShift], 1u);
     }
+  };
+  // two batches in flight: the next one loads while the current one is scored
+  // (the first batch was loaded before the LSE)
+  for (int tb = t0 + threadIdx.x; tb < t1; tb += 2 * kStep) {
+    load_logits<G>(raw2, lg, tb + kStep, t1);
+    score_batch(raw, tb);
+    load_logits<G>(raw, lg, tb + 2 * kStep, t1);
+    score_batch(raw2, tb + kStep);
   }
   __syncthreads();
   uint32_t *gh = p.ws.hist + (size_t)u * kHistBins;
