@@ -389,6 +389,39 @@ def time_kv_bridge(w, dev, stream, peak, iters=20):
                     "(E4M3: per-(token, kv head) scale); bytes = both weight matrices + hidden + stored rows"}
 
 
+# ------------------------------------------------------------------ block-level selection
+def time_block_selection(w, ws, out, idx, stream, block=16, iters=50):
+    """The full layer with the first-generation block-level selection in
+    place of the token-level one (the comparator), on the same inputs: mean
+    time of `iters` back-to-back calls, and of the same number of token-level
+    calls for reference (both CUDA events around the whole run)."""
+    from long_context_decode_full_b200 import hs2
+
+    s = w.spec
+    if s.k_global % block:
+        return None
+
+    def run(fn):
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(iters):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+
+    blk = run(lambda: hs2.full_attn_select_blocks(w.q_full, w.k, w.v, w.seq_lens, w.page_table, w.page_size,
+                                                  s.window, s.k_global, block, w.k_scale, w.v_scale, out=out,
+                                                  idx_out=idx, workspace=ws))
+    tok = run(lambda: hs2.full_attn_select(w.q_full, w.k, w.v, w.seq_lens, w.page_table, w.page_size, s.window,
+                                           s.k_global, w.k_scale, w.v_scale, out=out, idx_out=idx, workspace=ws))
+    return {"block": block, "full_layer_ms_block_selection": blk, "full_layer_ms_token_selection": tok,
+            "calls": iters, "what": "full layer (attention + selection) per call, back to back, CUDA events"}
+
+
 # ------------------------------------------------------------------ GPU arm
 def run_gpu(args, rank, world, local):
     from long_context_decode_full_b200 import hs2
@@ -537,6 +570,8 @@ def run_gpu(args, rank, world, local):
         "clocks": clk,
         "device_status": status,
     }
+    if world == 1 and not args.no_block_timing:
+        res["block_selection"] = time_block_selection(w, ws, outs[0], idx, stream)
     if not args.no_bridge and world == 1:
         # a per-GPU figure; with one process there is no NCCL thread about
         # while the graph is captured
@@ -592,6 +627,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time for the CPU baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-copy-peak", action="store_true", help="skip the same-run copy-bandwidth measurement")
+    ap.add_argument("--no-block-timing", action="store_true", help="skip the block-level selection timing")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's context (profiling runs)")
     ap.add_argument("--kv-heads", type=int, default=0, help="override the workload's KV heads (experiments)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (experiments)")

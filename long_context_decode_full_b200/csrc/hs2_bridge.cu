@@ -16,8 +16,10 @@
 //   - the 8 warps' partial sums meet in shared memory and the CTA's tile of
 //     partial sums goes to the workspace;
 //   - the last CTA of each (K or V, column tile, token group) to finish -- a
-//     ticket counter in the workspace -- adds the splits' tiles in split order
-//     (so the result does not depend on which CTA came last), stores the rows
+//     ticket counter in the workspace -- adds the splits' tiles: 8 / (tokens)
+//     warps per token, each a fixed share of the splits in split order, then
+//     the shares in warp order (so the result does not depend on which CTA
+//     came last), stores the rows
 //     (E4M3: one warp per token holds a whole head of 128 columns, so the
 //     row max is a warp reduction) and resets its ticket to zero.
 #include "hs2.h"
@@ -102,27 +104,42 @@ __global__ void __launch_bounds__(kBridgeThreads) bridge_kernel(const BridgePara
   for (int w8 = 0; w8 < kBridgeWarps; ++w8) s = add4(s, *reinterpret_cast<const float4 *>(&sh_red[w8][tok][4 * lane]));
   if (tok < nb && active)
     __stcg(reinterpret_cast<float4 *>(p.partial + (((int64_t)kv * p.nsplit + split) * p.B + b0 + tok) * p.N + col), s);
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
+    // one gpu-scope fence after the barrier orders every thread's partial
+    // store (fences are cumulative) before the ticket
+    __threadfence();
     int *ticket = p.tickets + ((int64_t)kv * p.ntiles + tile) * p.ngroups + grp;
     const int last = atomicAdd(ticket, 1) == p.nsplit - 1;
     if (last) *ticket = 0;  // every split has counted: ready for the next call
     sh_last = last;
   }
   __syncthreads();
-  if (!sh_last || tok >= nb) return;
+  if (!sh_last) return;
   __threadfence();
 
-  // last CTA: the splits in order, then the store (warp-uniform from here on)
+  // last CTA: the splits of token t are read by the warps t * wpt .. (t + 1)
+  // * wpt - 1 at once, each a fixed share of the splits in split order (one
+  // round of loads), and the shares are then added in warp order: the result
+  // does not depend on timing
+  const int wpt = kBridgeWarps / nb;  // warps per token
+  {
+    const int t = warp / wpt, k = warp % wpt;
+    float4 x4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t < nb && active) {
+      const int s0 = k * p.nsplit / wpt, s1 = (k + 1) * p.nsplit / wpt;
+      const float *src = p.partial + ((int64_t)kv * p.nsplit * p.B + b0 + t) * p.N + col;
+      const int64_t step = (int64_t)p.B * p.N;
+#pragma unroll 16
+      for (int sp = s0; sp < s1; ++sp) x4 = add4(x4, __ldcg(reinterpret_cast<const float4 *>(src + sp * step)));
+    }
+    *reinterpret_cast<float4 *>(&sh_red[warp][0][4 * lane]) = x4;
+  }
+  __syncthreads();
+  if (tok >= nb) return;
   const int b = b0 + tok;
   float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (active) {
-    const float *src = p.partial + ((int64_t)kv * p.nsplit * p.B + b) * p.N + col;
-    const int64_t step = (int64_t)p.B * p.N;
-#pragma unroll 8
-    for (int sp = 0; sp < p.nsplit; ++sp) x = add4(x, __ldcg(reinterpret_cast<const float4 *>(src + sp * step)));
-  }
+  for (int k = 0; k < wpt; ++k) x = add4(x, *reinterpret_cast<const float4 *>(&sh_red[tok * wpt + k][0][4 * lane]));
   const int T = clamp_len(__ldg(p.seq_lens + b), (int)p.t_cap);
   if (T < 1) return;  // no token to append
   const int64_t pos = T - 1;
