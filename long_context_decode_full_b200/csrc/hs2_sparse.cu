@@ -207,54 +207,92 @@ __global__ void __launch_bounds__(32 * NW, 1) sparse_mma_kernel(const SparsePara
 }
 
 // ------------------------------------------------------------ fp32 caches
+// One CTA of 4 warps per (sequence, kv head): the listed rows are gathered 64
+// at a time into shared memory (coalesced row loads), then warp w serves the
+// heads w and w + 4 of the group with an online softmax on the CUDA cores
+// (FFMA keeps fp32 logits exact to fp32 rounding).
+constexpr int kSpF32Tile = 64;
+constexpr int kSpF32Warps = 4;
+
 template <int D>
-__global__ void sparse_f32_kernel(const SparseParams p, int64_t num_slots) {
-  extern __shared__ float qs[];  // [G][D]
+__global__ void __launch_bounds__(32 * kSpF32Warps) sparse_f32_kernel(const SparseParams p, int64_t num_slots) {
+  extern __shared__ float fsm[];
+  float *Ks = fsm;                          // [64][D + 1]
+  float *Vs = Ks + kSpF32Tile * (D + 1);    // [64][D + 1]
+  float *Qs = Vs + kSpF32Tile * (D + 1);    // [G <= 8][D]
+  int *slots = reinterpret_cast<int *>(Qs + 8 * D);  // [64]
   const int kvh = blockIdx.x, b = blockIdx.y, G = p.G;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nthr = blockDim.x;
   griddep_wait();
   griddep_launch_dependents();
   const float *q = static_cast<const float *>(p.q) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
-  for (int e = threadIdx.x; e < G * D; e += blockDim.x) qs[e] = q[e];
-  __syncthreads();
-  const int h = warp;
-  if (h >= G) return;
+  for (int e = threadIdx.x; e < G * D; e += nthr) Qs[e] = q[e];
   const float *K = static_cast<const float *>(p.k), *V = static_cast<const float *>(p.v);
   const int32_t *idx = p.idx + ((int64_t)b * p.Hkv + kvh) * p.L;
-  float m = -INFINITY, l = 0.f, o[D / 32];
+  float m[2], l[2], o[2][D / 32];
 #pragma unroll
-  for (int j = 0; j < D / 32; ++j) o[j] = 0.f;
-  for (int base = 0; base < p.L; base += 32) {
-    int slot = base + lane < p.L ? __ldg(idx + base + lane) : -1;
-    if (slot >= num_slots) slot = -1;
-    float s = -INFINITY;
-    if (slot >= 0) {
-      const float *kr = K + ((int64_t)slot * p.Hkv + kvh) * D;
-      float acc = 0.f;
-      for (int e = 0; e < D; ++e) acc = fmaf(qs[h * D + e], kr[e], acc);
-      s = acc;
-    }
-    const float mx = warp_max(s);
-    if (mx == -INFINITY) continue;
-    const float m_new = fmaxf(m, mx);
-    const float alpha = expf(p.c * (m - m_new));
-    const float pr = slot >= 0 ? expf(p.c * (s - m_new)) : 0.f;
-    l = l * alpha + warp_sum(pr);
-    m = m_new;
+  for (int hs = 0; hs < 2; ++hs) {
+    m[hs] = -INFINITY;
+    l[hs] = 0.f;
 #pragma unroll
-    for (int j = 0; j < D / 32; ++j) {
-      float acc = o[j] * alpha;
-      for (int r = 0; r < 32; ++r) {
-        const int sr = __shfl_sync(0xffffffffu, slot, r);
-        const float pp = __shfl_sync(0xffffffffu, pr, r);
-        if (sr >= 0) acc = fmaf(pp, V[((int64_t)sr * p.Hkv + kvh) * D + lane + 32 * j], acc);
-      }
-      o[j] = acc;
-    }
+    for (int j = 0; j < D / 32; ++j) o[hs][j] = 0.f;
   }
-  float *out = static_cast<float *>(p.out) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G + h) * D;
+  for (int base = 0; base < p.L; base += kSpF32Tile) {
+    for (int r = threadIdx.x; r < kSpF32Tile; r += nthr) {
+      const int sl = base + r < p.L ? __ldg(idx + base + r) : -1;
+      slots[r] = (sl >= 0 && sl < num_slots) ? sl : -1;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kSpF32Tile * D; e += nthr) {
+      const int rr = e / D, col = e % D;
+      const int sl = slots[rr];
+      Ks[rr * (D + 1) + col] = sl >= 0 ? K[((int64_t)sl * p.Hkv + kvh) * D + col] : 0.f;
+      Vs[rr * (D + 1) + col] = sl >= 0 ? V[((int64_t)sl * p.Hkv + kvh) * D + col] : 0.f;
+    }
+    __syncthreads();
 #pragma unroll
-  for (int j = 0; j < D / 32; ++j) out[lane + 32 * j] = l > 0.f ? o[j] / l : 0.f;
+    for (int hs = 0; hs < 2; ++hs) {
+      const int h = warp + kSpF32Warps * hs;
+      if (h >= G) break;
+      float s[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int rr = lane + 32 * j;
+        float acc = 0.f;
+#pragma unroll 4
+        for (int e = 0; e < D; ++e) acc = fmaf(Qs[h * D + e], Ks[rr * (D + 1) + e], acc);
+        s[j] = slots[rr] >= 0 ? acc : -INFINITY;
+      }
+      const float mx = warp_max(fmaxf(s[0], s[1]));
+      if (mx == -INFINITY) continue;  // no listed row in this tile
+      const float m_new = fmaxf(m[hs], mx);
+      const float alpha = expf(p.c * (m[hs] - m_new));
+      float pr[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) pr[j] = s[j] == -INFINITY ? 0.f : expf(p.c * (s[j] - m_new));
+      l[hs] = l[hs] * alpha + warp_sum(pr[0] + pr[1]);
+      m[hs] = m_new;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        float acc = o[hs][j] * alpha;
+#pragma unroll 4
+        for (int rr = 0; rr < kSpF32Tile; ++rr) {
+          const float pp = __shfl_sync(0xffffffffu, pr[rr >> 5], rr & 31);
+          acc = fmaf(pp, Vs[rr * (D + 1) + lane + 32 * j], acc);
+        }
+        o[hs][j] = acc;
+      }
+    }
+    __syncthreads();  // the tile is consumed before the next gather
+  }
+#pragma unroll
+  for (int hs = 0; hs < 2; ++hs) {
+    const int h = warp + kSpF32Warps * hs;
+    if (h >= G) break;
+    float *out = static_cast<float *>(p.out) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G + h) * D;
+#pragma unroll
+    for (int j = 0; j < D / 32; ++j) out[lane + 32 * j] = l[hs] > 0.f ? o[hs][j] / l[hs] : 0.f;
+  }
 }
 
 template <int D, bool FP8, int NW, int NSL>
@@ -284,9 +322,16 @@ cudaError_t launch_mma_shape(const SparseParams &p, int64_t num_slots, cudaStrea
 
 cudaError_t launch_sparse_impl(const SparseParams &p, int kv_dtype, int64_t num_slots, cudaStream_t s) {
   if (kv_dtype == 0) {
-    const size_t smem = (size_t)p.G * p.D * 4;
-    if (p.D == 64) return launch_ex(sparse_f32_kernel<64>, dim3(p.Hkv, p.B), dim3(32 * p.G), smem, s, 0, p, num_slots);
-    return launch_ex(sparse_f32_kernel<128>, dim3(p.Hkv, p.B), dim3(32 * p.G), smem, s, 0, p, num_slots);
+    const size_t smem = (size_t)(2 * kSpF32Tile * (p.D + 1) + 8 * p.D) * 4 + kSpF32Tile * 4;
+    cudaError_t e;
+    if (p.D == 64) {
+      e = cudaFuncSetAttribute(sparse_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      return launch_ex(sparse_f32_kernel<64>, dim3(p.Hkv, p.B), dim3(32 * kSpF32Warps), smem, s, 0, p, num_slots);
+    }
+    e = cudaFuncSetAttribute(sparse_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_ex(sparse_f32_kernel<128>, dim3(p.Hkv, p.B), dim3(32 * kSpF32Warps), smem, s, 0, p, num_slots);
   }
   if (kv_dtype == 1)
     return p.D == 64 ? launch_mma_shape<64, false>(p, num_slots, s) : launch_mma_shape<128, false>(p, num_slots, s);
