@@ -198,26 +198,43 @@ bool tile_fits_pages(int tile, int page_size, bool paged) {
   return tile % page_size == 0 && tile / page_size <= 8;
 }
 
-// The consumer warps split into (G + 7) / 8 head groups, so their count must
-// divide by it.
+// A warp serves 8 nt query heads, so with more heads per group than that the
+// consumer warps split into ceil(G / (8 nt)) head groups and their count must
+// divide by it.  Groups of 16 and more heads take nt = 2 where a configuration
+// is built for it (each shared-memory fragment then feeds two MMAs).
 FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged, int G) {
-  const int nhg = (G + 7) / 8;
-  static const FullMmaConfig bf16_128[] = {{4, 3, 2}, {8, 3, 1}, {4, 6, 1}};
-  // groups above 8 heads give every warp several 8-head steps per tile: more
-  // consumer warps (measured at 256K, G = 32: 154 us against 179 us)
-  static const FullMmaConfig bf16_128_wide[] = {{8, 3, 1}, {4, 3, 2}, {4, 6, 1}};
-  static const FullMmaConfig bf16_64[] = {{8, 6, 1}, {4, 6, 1}};
-  static const FullMmaConfig e4m3[] = {{8, 3, 2}, {12, 4, 1}, {8, 6, 1}, {4, 8, 1}};
-  const FullMmaConfig *list = fp8 ? e4m3 : (D == 64 ? bf16_64 : (nhg > 1 ? bf16_128_wide : bf16_128));
-  const int n = fp8 ? 4 : (D == 64 ? 2 : 3);
-  if (const char *env = getenv("HS2_FULL_CFG")) {  // tuning override: "ncw,nstage[,nsl]"
-    int a = 0, b = 0, c = 1;
-    if (sscanf(env, "%d,%d,%d", &a, &b, &c) >= 2 && a >= 1 && a <= 16 && b >= 1 && b <= 16 && (c == 1 || c == 2) &&
-        a % nhg == 0 && tile_fits_pages(16 * a * c, page_size, paged))
-      return FullMmaConfig{a, b, c};
+  static const FullMmaConfig bf16_128[] = {{4, 3, 2, 1}, {8, 3, 1, 1}, {4, 6, 1, 1}};
+  static const FullMmaConfig bf16_64[] = {{8, 6, 1, 1}, {4, 6, 1, 1}};
+  static const FullMmaConfig e4m3[] = {{8, 3, 2, 1}, {12, 4, 1, 1}, {8, 6, 1, 1}, {4, 8, 1, 1}};
+  // 16 heads per warp: one consumer warp per SM sub-partition with all 255
+  // registers measured fastest (MQA at 256K bf16: 136 us against 144 us with
+  // 8 warps x 1 slice and 154 us with 8-head warps; at 1M E4M3: 151 us
+  // against 160 us with 8-head warps; 8-warp E4M3 variants spilled, 179 us)
+  static const FullMmaConfig bf16_128_wide[] = {{4, 3, 2, 2}, {8, 3, 1, 2}};
+  static const FullMmaConfig bf16_64_wide[] = {{8, 6, 1, 2}};
+  static const FullMmaConfig e4m3_wide[] = {{4, 6, 2, 2}};
+  auto heads_split = [&](const FullMmaConfig &c) { return c.ncw % ((G + 8 * c.nt - 1) / (8 * c.nt)) == 0; };
+  auto fits = [&](const FullMmaConfig &c) {
+    return heads_split(c) && tile_fits_pages(16 * c.ncw * c.nsl, page_size, paged);
+  };
+  if (const char *env = getenv("HS2_FULL_CFG")) {  // tuning override: "ncw,nstage[,nsl[,nt]]"
+    int a = 0, b = 0, c = 1, d = 1;
+    if (sscanf(env, "%d,%d,%d,%d", &a, &b, &c, &d) >= 2 && a >= 1 && a <= 16 && b >= 1 && b <= 16 &&
+        (c == 1 || c == 2) && (d == 1 || (d == 2 && G >= 16))) {
+      const FullMmaConfig e{a, b, c, d};
+      if (fits(e)) return e;
+    }
   }
+  if (G >= 16) {
+    const FullMmaConfig *wide = fp8 ? e4m3_wide : (D == 64 ? bf16_64_wide : bf16_128_wide);
+    const int nw = fp8 ? 1 : (D == 64 ? 1 : 2);
+    for (int i = 0; i < nw; ++i)
+      if (fits(wide[i])) return wide[i];
+  }
+  const FullMmaConfig *list = fp8 ? e4m3 : (D == 64 ? bf16_64 : bf16_128);
+  const int n = fp8 ? 4 : (D == 64 ? 2 : 3);
   for (int i = 0; i < n; ++i)
-    if (list[i].ncw % nhg == 0 && tile_fits_pages(16 * list[i].ncw * list[i].nsl, page_size, paged)) return list[i];
+    if (fits(list[i])) return list[i];
   return list[n - 1];
 }
 
@@ -357,8 +374,8 @@ int full_attn_select_impl(const hs2_heads *q, const hs2_cache *k_cache, const hs
     if ((rc = encode_cache_map(&tmv, v_cache, box_rows))) return rc;
     e = launch_full_mma(p, tmk, tmv, fp8, cfg, p.N, s);
     if (e == cudaErrorInvalidConfiguration)
-      return fail(HS2_ERR_UNSUPPORTED, "no full-attention kernel built for ncw=%d nstage=%d nsl=%d", cfg.ncw, cfg.nstage,
-                  cfg.nsl);
+      return fail(HS2_ERR_UNSUPPORTED, "no full-attention kernel built for ncw=%d nstage=%d nsl=%d nt=%d", cfg.ncw,
+                  cfg.nstage, cfg.nsl, cfg.nt);
     if (e != cudaSuccess) return cuda_fail(e, "full-attention launch");
   }
   if (mark_event) {

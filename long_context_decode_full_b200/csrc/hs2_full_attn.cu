@@ -29,7 +29,7 @@ struct StageMeta {
 };
 constexpr int kFirst = 1, kLast = 2, kDone = 4;
 
-template <int D, bool FP8, int NCW, int NSTAGE, int NSL>
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT>
 struct Cfg {
   static constexpr int RPW = 16 * NSL;  // rows per consumer warp
   static constexpr int TILE = RPW * NCW;
@@ -41,13 +41,16 @@ struct Cfg {
   static constexpr int SCB = FP8 ? 2 * TILE * 4 : 0;                // K and V scales of a tile
   static constexpr int STAGE = (2 * KVB + SCB + 1023) / 1024 * 1024;  // K, V, scales; 1 KB aligned for TMA
   static constexpr int WSTRIDE = 16 + 8 * D;
+  // NT = 2: one saved warp state per sender of the first merge round
+  static constexpr int SLOT = WarpAttn<D, FP8, NSL, NT>::kSaveBytes / 4;
   static constexpr size_t OFF_BAR = (size_t)NSTAGE * STAGE;
   static constexpr size_t OFF_META = OFF_BAR + (2 * NSTAGE + 1) * 8;
   static constexpr size_t OFF_PREFIX = OFF_META + NSTAGE * sizeof(StageMeta);
   static size_t bytes(int B) { return OFF_PREFIX + (size_t)(B + 1) * 4 + 1024; }
   static_assert(ROWB % 128 == 0, "rows are whole 128-byte panels");
   // the warps merge a segment's states inside the stage they last read
-  static_assert((size_t)NCW * WSTRIDE * 4 <= (size_t)STAGE, "merge scratch must fit in one stage");
+  static_assert(NT == 2 || (size_t)NCW * WSTRIDE * 4 <= (size_t)STAGE, "merge scratch must fit in one stage");
+  static_assert(NT == 1 || (size_t)(NCW / 2) * SLOT * 4 <= (size_t)STAGE, "merge scratch must fit in one stage");
 };
 
 __device__ __forceinline__ int64_t slot_of(const int32_t *pt, int max_pages, int ps, int b, int64_t pos) {
@@ -110,11 +113,11 @@ __device__ __forceinline__ int find_seq(const int32_t *prefix, int B, int Hkv, i
 template <bool FP8>
 constexpr int kProducerWarps = FP8 ? 2 : 1;
 
-template <int D, bool FP8, int NCW, int NSTAGE, int NSL>
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT>
 __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
     full_attn_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                          const FullParams p) {
-  using C = Cfg<D, FP8, NCW, NSTAGE, NSL>;
+  using C = Cfg<D, FP8, NCW, NSTAGE, NSL, NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -287,14 +290,15 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
   }
 
   // -------------------------------------------------------------- consumers
-  // Heads come in groups of 8 (one MMA N-tile).  With G > 8 (MQA-style
-  // groups) warp w serves head group hg = w % NHG and, of each tile, the row
-  // blocks j = w / NHG + k * (NCW / NHG), k < NHG: every head group sees every
-  // row of the tile from the same shared-memory stage.
-  const int NHG = (p.G + 7) >> 3, WPG = NCW / NHG;
+  // A warp serves HPW = 8 NT heads (NT MMA N-tiles).  With more heads than
+  // that (MQA-style groups) warp w serves head group hg = w % NHG and, of
+  // each tile, the row blocks j = w / NHG + k * (NCW / NHG), k < NHG: every
+  // head group sees every row of the tile from the same shared-memory stage.
+  constexpr int HPW = 8 * NT;
+  const int NHG = (p.G + HPW - 1) / HPW, WPG = NCW / NHG;
   const int hg = warp % NHG, wig = warp / NHG;
-  const int Gl = min(8, p.G - 8 * hg);  // heads of this warp's group
-  WarpAttn<D, FP8, NSL> st;
+  const int Gl = min(HPW, p.G - HPW * hg);  // heads of this warp's group
+  WarpAttn<D, FP8, NSL, NT> st;
   st.reset();
   uint32_t cphase = 0;
   for (int it = 0;; ++it) {
@@ -309,7 +313,7 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
     if (mt.flags & kFirst) {
       st.reset();
       st.load_q(reinterpret_cast<const __nv_bfloat16 *>(p.q) +
-                    ((int64_t)mt.b * p.Hkv * p.G + (int64_t)mt.kvh * p.G + 8 * hg) * D,
+                    ((int64_t)mt.b * p.Hkv * p.G + (int64_t)mt.kvh * p.G + HPW * hg) * D,
                 Gl);
     }
     const uint32_t kp = sbase + stage * C::STAGE;
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
       const float *ks = reinterpret_cast<const float *>(smem + (size_t)stage * C::STAGE + 2 * C::KVB) + C::RPW * j;
       if (nvalid > 0)
         st.step(kp, kp + C::KVB, C::PANEL, C::RPW * j, vmask, p.c,
-                p.ws.logits + (u * p.ustride + pos0) * p.G + 8 * hg, Gl, ks, ks + C::TILE, p.G);
+                p.ws.logits + (u * p.ustride + pos0) * p.G + HPW * hg, Gl, ks, ks + C::TILE, p.G);
     }
     if (mt.flags & kLast) {
       // segment end: merge the warps' states inside this stage, then release it
@@ -330,16 +334,38 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
         break;
       }
       float *scratch = reinterpret_cast<float *>(smem + (size_t)stage * C::STAGE);
-      float *scr = scratch + warp * C::WSTRIDE;
-      st.store(scr, scr + 8, scr + 16);
-      if (!consumer_sync(cbar, cphase)) {
-        set_error(p.ws.err, kErrFullWait);
-        break;
+      float *rec = p.ws.records + (size_t)(mt.rec >= 0 ? mt.rec : 0) * p.G * (D + 2);
+      if constexpr (NT == 1) {
+        float *scr = scratch + warp * C::WSTRIDE;
+        st.store(scr, scr + 8, scr + 16);
+        if (!consumer_sync(cbar, cphase)) {
+          set_error(p.ws.err, kErrFullWait);
+          break;
+        }
+        if (mt.rec >= 0)
+          for (int g8 = 0; g8 < NHG; ++g8)  // the warps of head group g8 are g8, g8 + NHG, ...
+            merge_warp_states<D>(scratch + g8 * C::WSTRIDE, NHG * C::WSTRIDE, WPG, min(8, p.G - 8 * g8), p.c, rec,
+                                 threadIdx.x, NCW * 32, 8 * g8, p.G);
+      } else {
+        // a tree over the WPG warps of each head group, in registers: in the
+        // round of span s, warp wig = 2 s k + s hands its state to 2 s k
+        // through slot (hg, k) of the stage; warp wig = 0 writes the record
+        st.finish();
+        bool sync_ok = true;
+        for (int span = 1; span < WPG && sync_ok; span *= 2) {
+          const int r = wig % (2 * span);
+          float *slot = scratch + (size_t)(hg + NHG * (wig / (2 * span))) * C::SLOT;
+          if (r == span) st.save(slot);
+          sync_ok = consumer_sync(cbar, cphase);
+          if (sync_ok && r == 0 && wig + span < WPG) st.absorb(slot, p.c);
+          sync_ok = sync_ok && consumer_sync(cbar, cphase);  // the slots are read before the next round
+        }
+        if (!sync_ok) {
+          set_error(p.ws.err, kErrFullWait);
+          break;
+        }
+        if (wig == 0 && mt.rec >= 0) st.write_record(rec, Gl, HPW * hg, p.G);
       }
-      if (mt.rec >= 0)
-        for (int g8 = 0; g8 < NHG; ++g8)  // the warps of head group g8 are g8, g8 + NHG, ...
-          merge_warp_states<D>(scratch + g8 * C::WSTRIDE, NHG * C::WSTRIDE, WPG, min(8, p.G - 8 * g8), p.c,
-                               p.ws.records + (size_t)mt.rec * p.G * (D + 2), threadIdx.x, NCW * 32, 8 * g8, p.G);
       fence_proxy_async_smem();  // before TMA refills the stage
       if (!consumer_sync(cbar, cphase)) {
         set_error(p.ws.err, kErrFullWait);
@@ -466,12 +492,12 @@ __global__ void __launch_bounds__(32 * kF32Warps) full_attn_f32_kernel(const Ful
   }
 }
 
-template <int D, bool FP8, int NCW, int NSTAGE, int NSL>
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT>
 cudaError_t launch_mma_t(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, int grid,
                          cudaStream_t s) {
-  using C = Cfg<D, FP8, NCW, NSTAGE, NSL>;
+  using C = Cfg<D, FP8, NCW, NSTAGE, NSL, NT>;
   const size_t smem = C::bytes(p.B);
-  auto kern = full_attn_mma_kernel<D, FP8, NCW, NSTAGE, NSL>;
+  auto kern = full_attn_mma_kernel<D, FP8, NCW, NSTAGE, NSL, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_ex(kern, dim3(grid), dim3(32 * (NCW + kProducerWarps<FP8>)), smem, s, 0, tmk, tmv, p);
@@ -481,21 +507,26 @@ cudaError_t launch_mma_t(const FullParams &p, const CUtensorMap &tmk, const CUte
 
 cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, bool fp8,
                             const FullMmaConfig &cfg, int grid, cudaStream_t s) {
-#define HS2_FULL_CASE(D_, F_, W_, S_, L_)                                               \
-  if (p.D == D_ && fp8 == F_ && cfg.ncw == W_ && cfg.nstage == S_ && cfg.nsl == L_)     \
-    return launch_mma_t<D_, F_, W_, S_, L_>(p, tmk, tmv, grid, s);
-  HS2_FULL_CASE(128, false, 8, 3, 1)
-  HS2_FULL_CASE(128, false, 4, 6, 1)
-  HS2_FULL_CASE(128, false, 4, 3, 2)
-  HS2_FULL_CASE(64, false, 8, 6, 1)
-  HS2_FULL_CASE(64, false, 4, 6, 1)
-  HS2_FULL_CASE(128, true, 8, 3, 2)
-  HS2_FULL_CASE(128, true, 6, 4, 2)
-  HS2_FULL_CASE(128, true, 4, 6, 2)
-  HS2_FULL_CASE(128, true, 16, 3, 1)
-  HS2_FULL_CASE(128, true, 12, 4, 1)
-  HS2_FULL_CASE(128, true, 8, 6, 1)
-  HS2_FULL_CASE(128, true, 4, 8, 1)
+#define HS2_FULL_CASE(D_, F_, W_, S_, L_, N_)                                                        \
+  if (p.D == D_ && fp8 == F_ && cfg.ncw == W_ && cfg.nstage == S_ && cfg.nsl == L_ && cfg.nt == N_) \
+    return launch_mma_t<D_, F_, W_, S_, L_, N_>(p, tmk, tmv, grid, s);
+  HS2_FULL_CASE(128, false, 8, 3, 1, 1)
+  HS2_FULL_CASE(128, false, 4, 6, 1, 1)
+  HS2_FULL_CASE(128, false, 4, 3, 2, 1)
+  HS2_FULL_CASE(64, false, 8, 6, 1, 1)
+  HS2_FULL_CASE(64, false, 4, 6, 1, 1)
+  HS2_FULL_CASE(128, true, 8, 3, 2, 1)
+  HS2_FULL_CASE(128, true, 6, 4, 2, 1)
+  HS2_FULL_CASE(128, true, 4, 6, 2, 1)
+  HS2_FULL_CASE(128, true, 16, 3, 1, 1)
+  HS2_FULL_CASE(128, true, 12, 4, 1, 1)
+  HS2_FULL_CASE(128, true, 8, 6, 1, 1)
+  HS2_FULL_CASE(128, true, 4, 8, 1, 1)
+  // 16 heads per warp (groups of 16 and 32 query heads)
+  HS2_FULL_CASE(128, false, 8, 3, 1, 2)
+  HS2_FULL_CASE(128, false, 4, 3, 2, 2)
+  HS2_FULL_CASE(64, false, 8, 6, 1, 2)
+  HS2_FULL_CASE(128, true, 4, 6, 2, 2)
 #undef HS2_FULL_CASE
   return cudaErrorInvalidConfiguration;
 }

@@ -72,6 +72,7 @@ struct FullMmaConfig {
   int ncw;     // consumer warps
   int nstage;  // pipeline stages
   int nsl;     // 16-row slices per warp and tile (tile = 16 * ncw * nsl positions)
+  int nt;      // 8-head MMA N-tiles per warp (1, or 2 for groups of 16 and more heads)
 };
 
 // Launch with programmatic stream serialization (unless HS2_PDL=0) and an

@@ -27,67 +27,78 @@ namespace hs2 {
 
 // NSL: 16-row slices per step.  Two slices give the warp two independent
 // instruction streams (MMA chains, conversions, exponentials) to interleave.
-template <int D, bool FP8, int NSL = 1>
+// NT: 8-head N-tiles per step.  With two (16 heads per warp, MQA-style
+// groups), every K and V fragment read from shared memory (and, for E4M3,
+// widened) feeds two MMAs instead of being read again by another warp.
+template <int D, bool FP8, int NSL = 1, int NT = 1>
 struct WarpAttn {
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(NSL == 1 || NSL == 2, "slices per step");
+  static_assert(NT == 1 || NT == 2, "8-head N-tiles per step");
   static_assert(!FP8 || D == 128, "E4M3 path is built for head_dim 128");
   static constexpr int KS = D / 16;  // k-steps of Q K^T and m-tiles of V^T P^T
 
-  uint32_t qa[KS][2];  // B-fragments of Q^T (head g; zero for heads >= G)
-  float qscale[2];     // E4M3: 2^-e undoing the prescale of heads 2t, 2t+1
-  float m[2];          // running max of raw logits of heads 2t, 2t+1 (uniform over g)
-  float l[2];          // this lane's share of sum exp(c (s - m)) for heads 2t, 2t+1
-  float sig;           // E4M3: running max of the V scale (warp uniform)
-  float inv_sig;       // E4M3: 1 / sig (0 while sig is 0)
-  float o[KS][4];      // O^T accumulator: dims x heads (2t, 2t+1)
+  uint32_t qa[NT][KS][2];  // B-fragments of Q^T (N-tile n: head 8n + g; zero for heads >= G)
+  float qscale[NT][2];     // E4M3: 2^-e undoing the prescale of heads 8n + 2t, 8n + 2t + 1
+  float m[NT][2];          // running max of raw logits of heads 8n + 2t, 8n + 2t + 1 (uniform over g)
+  float l[NT][2];          // this lane's share of sum exp(c (s - m)) for those heads
+  float sig;               // E4M3: running max of the V scale (warp uniform)
+  float inv_sig;           // E4M3: 1 / sig (0 while sig is 0)
+  float o[NT][KS][4];      // O^T accumulators: dims x heads (8n + 2t, 8n + 2t + 1)
 
   __device__ __forceinline__ void reset() {
-    m[0] = m[1] = -INFINITY;
-    l[0] = l[1] = 0.f;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      m[n][0] = m[n][1] = -INFINITY;
+      l[n][0] = l[n][1] = 0.f;
+#pragma unroll
+      for (int i = 0; i < KS; ++i) o[n][i][0] = o[n][i][1] = o[n][i][2] = o[n][i][3] = 0.f;
+    }
     sig = 0.f;
     inv_sig = 0.f;
-#pragma unroll
-    for (int i = 0; i < KS; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   }
 
-  // Query of the group (G consecutive heads, bf16 [G][D]) into B-fragments.
+  // Query of the warp's heads (G <= 8 NT consecutive heads, bf16 [G][D]) into B-fragments.
   __device__ __forceinline__ void load_q(const __nv_bfloat16 *q, int G) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const uint32_t *q32 = reinterpret_cast<const uint32_t *>(q);
-    if constexpr (!FP8) {
 #pragma unroll
-      for (int kk = 0; kk < KS; ++kk) {
-        qa[kk][0] = g < G ? __ldg(q32 + ((g * D + 16 * kk + 2 * t) >> 1)) : 0u;
-        qa[kk][1] = g < G ? __ldg(q32 + ((g * D + 16 * kk + 8 + 2 * t) >> 1)) : 0u;
-      }
-      qscale[0] = qscale[1] = 1.f;
-    } else {
-      // k-step kk of lane t covers dims 32t + 4kk + {0,1} (MMA k = 2t, 2t+1)
-      // and 32t + 4kk + {2,3} (MMA k = 2t+8, 2t+9).
-      float v[KS][4];
-      float amax = 0.f;
+    for (int n = 0; n < NT; ++n) {
+      const int hh = 8 * n + g;  // this lane's head of N-tile n
+      if constexpr (!FP8) {
 #pragma unroll
-      for (int kk = 0; kk < KS; ++kk) {
-        uint2 w = g < G ? __ldg(reinterpret_cast<const uint2 *>(q + g * D + 32 * t + 4 * kk)) : make_uint2(0, 0);
-        v[kk][0] = __uint_as_float(w.x << 16);
-        v[kk][1] = __uint_as_float(w.x & 0xFFFF0000u);
-        v[kk][2] = __uint_as_float(w.y << 16);
-        v[kk][3] = __uint_as_float(w.y & 0xFFFF0000u);
+        for (int kk = 0; kk < KS; ++kk) {
+          qa[n][kk][0] = hh < G ? __ldg(q32 + ((hh * D + 16 * kk + 2 * t) >> 1)) : 0u;
+          qa[n][kk][1] = hh < G ? __ldg(q32 + ((hh * D + 16 * kk + 8 + 2 * t) >> 1)) : 0u;
+        }
+        qscale[n][0] = qscale[n][1] = 1.f;
+      } else {
+        // k-step kk of lane t covers dims 32t + 4kk + {0,1} (MMA k = 2t, 2t+1)
+        // and 32t + 4kk + {2,3} (MMA k = 2t+8, 2t+9).
+        float v[KS][4];
+        float amax = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(v[kk][e]));
-      }
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      const int e = amax > 0.f ? 14 - ilogbf(amax) : 0;
-      const float up = ldexpf(1.f, e);
-      // the logits of this lane belong to heads 2t, 2t+1 (lanes 8t, 8t + 4 hold their exponents)
-      qscale[0] = ldexpf(1.f, -__shfl_sync(0xffffffffu, e, 8 * t));
-      qscale[1] = ldexpf(1.f, -__shfl_sync(0xffffffffu, e, 8 * t + 4));
+        for (int kk = 0; kk < KS; ++kk) {
+          uint2 w = hh < G ? __ldg(reinterpret_cast<const uint2 *>(q + hh * D + 32 * t + 4 * kk)) : make_uint2(0, 0);
+          v[kk][0] = __uint_as_float(w.x << 16);
+          v[kk][1] = __uint_as_float(w.x & 0xFFFF0000u);
+          v[kk][2] = __uint_as_float(w.y << 16);
+          v[kk][3] = __uint_as_float(w.y & 0xFFFF0000u);
 #pragma unroll
-      for (int kk = 0; kk < KS; ++kk) {
-        qa[kk][0] = pack_f16(v[kk][0] * up, v[kk][1] * up);
-        qa[kk][1] = pack_f16(v[kk][2] * up, v[kk][3] * up);
+          for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(v[kk][e]));
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const int e = amax > 0.f ? 14 - ilogbf(amax) : 0;
+        const float up = ldexpf(1.f, e);
+        // the logits of this lane belong to heads 8n + 2t, 8n + 2t + 1 (lanes 8t, 8t + 4 hold their exponents)
+        qscale[n][0] = ldexpf(1.f, -__shfl_sync(0xffffffffu, e, 8 * t));
+        qscale[n][1] = ldexpf(1.f, -__shfl_sync(0xffffffffu, e, 8 * t + 4));
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+          qa[n][kk][0] = pack_f16(v[kk][0] * up, v[kk][1] * up);
+          qa[n][kk][1] = pack_f16(v[kk][2] * up, v[kk][3] * up);
+        }
       }
     }
   }
@@ -104,13 +115,15 @@ struct WarpAttn {
                                        int ldl = -1) {
     if (ldl < 0) ldl = G;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    // two accumulator chains per slice (even / odd k-steps) halve the
-    // dependent-MMA latency; their fp32 sum is the logit
-    float s[NSL][4], s2[NSL][4];
+    // two accumulator chains per slice and N-tile (even / odd k-steps) halve
+    // the dependent-MMA latency; their fp32 sum is the logit
+    float s[NSL][NT][4], s2[NSL][NT][4];
 #pragma unroll
     for (int sl = 0; sl < NSL; ++sl)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s[sl][e] = s2[sl][e] = 0.f;
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[sl][n][e] = s2[sl][n][e] = 0.f;
 
     // ---- S^T = K Q^T
     if constexpr (!FP8) {
@@ -123,8 +136,11 @@ struct WarpAttn {
         for (int sl = 0; sl < NSL; ++sl) {
           uint32_t r[4];
           ldsm_x4(r, swz(kp + (cb >> 7) * pstride, row + 16 * sl, (cb & 127) >> 4));
-          if (kk & 1) mma_bf16(s2[sl], r[0], r[1], r[2], r[3], qa[kk][0], qa[kk][1]);
-          else mma_bf16(s[sl], r[0], r[1], r[2], r[3], qa[kk][0], qa[kk][1]);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            if (kk & 1) mma_bf16(s2[sl][n], r[0], r[1], r[2], r[3], qa[n][kk][0], qa[n][kk][1]);
+            else mma_bf16(s[sl][n], r[0], r[1], r[2], r[3], qa[n][kk][0], qa[n][kk][1]);
+          }
         }
       }
     } else {
@@ -144,14 +160,17 @@ struct WarpAttn {
           uint32_t lo0, hi0, lo1, hi1;
           e4m3x4_to_f16x2x2(w[sl][0][kk], lo0, hi0);
           e4m3x4_to_f16x2x2(w[sl][1][kk], lo1, hi1);
-          if (kk & 1) mma_f16(s2[sl], lo0, lo1, hi0, hi1, qa[kk][0], qa[kk][1]);
-          else mma_f16(s[sl], lo0, lo1, hi0, hi1, qa[kk][0], qa[kk][1]);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            if (kk & 1) mma_f16(s2[sl][n], lo0, lo1, hi0, hi1, qa[n][kk][0], qa[n][kk][1]);
+            else mma_f16(s[sl][n], lo0, lo1, hi0, hi1, qa[n][kk][0], qa[n][kk][1]);
+          }
         }
       }
     }
 
-    // ---- logits, online softmax: x[sl][j][h] = row 16 sl + g + 8j, head 2t + h
-    float x[NSL][2][2];
+    // ---- logits, online softmax: x[sl][n][j][h] = row 16 sl + g + 8j, head 8n + 2t + h
+    float x[NSL][NT][2][2];
     bool ok[NSL][2];
     float sv[NSL][2];
 #pragma unroll
@@ -159,31 +178,41 @@ struct WarpAttn {
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int r = 16 * sl + 8 * j + g;
-        x[sl][j][0] = s[sl][2 * j] + s2[sl][2 * j];
-        x[sl][j][1] = s[sl][2 * j + 1] + s2[sl][2 * j + 1];
         ok[sl][j] = ((vmask >> r) & 1u) != 0u;
         sv[sl][j] = 0.f;
+        float kj = 1.f;
         if constexpr (FP8) {
-          const float kj = ok[sl][j] ? ks[r] : 0.f;
-          x[sl][j][0] *= kj * qscale[0];
-          x[sl][j][1] *= kj * qscale[1];
+          kj = ok[sl][j] ? ks[r] : 0.f;
           sv[sl][j] = ok[sl][j] ? vs[r] : 0.f;
         }
-      }
-    if (logit_dst != nullptr && 2 * t < G) {
-      const uint64_t keep = l2_policy_evict_last();  // read back by the score pass
 #pragma unroll
-      for (int sl = 0; sl < NSL; ++sl)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          if (!ok[sl][j]) continue;
-          float *dst = logit_dst + (16 * sl + 8 * j + g) * ldl + 2 * t;
-          if ((G & 1) == 0) st_global_hint(dst, x[sl][j][0], x[sl][j][1], keep);
-          else {
-            st_global_hint(dst, x[sl][j][0], keep);
-            if (2 * t + 1 < G) st_global_hint(dst + 1, x[sl][j][1], keep);
+        for (int n = 0; n < NT; ++n) {
+          x[sl][n][j][0] = s[sl][n][2 * j] + s2[sl][n][2 * j];
+          x[sl][n][j][1] = s[sl][n][2 * j + 1] + s2[sl][n][2 * j + 1];
+          if constexpr (FP8) {
+            x[sl][n][j][0] *= kj * qscale[n][0];
+            x[sl][n][j][1] *= kj * qscale[n][1];
           }
         }
+      }
+    if (logit_dst != nullptr) {
+      const uint64_t keep = l2_policy_evict_last();  // read back by the score pass
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        if (8 * n + 2 * t >= G) continue;
+#pragma unroll
+        for (int sl = 0; sl < NSL; ++sl)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (!ok[sl][j]) continue;
+            float *dst = logit_dst + (16 * sl + 8 * j + g) * ldl + 8 * n + 2 * t;
+            if ((G & 1) == 0) st_global_hint(dst, x[sl][n][j][0], x[sl][n][j][1], keep);
+            else {
+              st_global_hint(dst, x[sl][n][j][0], keep);
+              if (8 * n + 2 * t + 1 < G) st_global_hint(dst + 1, x[sl][n][j][1], keep);
+            }
+          }
+      }
     }
     // Lazy rescaling: the reference m only moves when a logit would lift
     // exp(c (x - m)) above 2^8 (and sig when a V scale exceeds it); p <= 2^8
@@ -191,17 +220,27 @@ struct WarpAttn {
     // result equals an eager online softmax.  The common case costs one vote.
     const float cl = c * 1.44269504088896341f;  // exp(c x) = 2^(x cl)
     const float thr = 8.f / cl;
-    float mloc[2] = {-INFINITY, -INFINITY}, sloc = 0.f;
+    float mloc[NT][2], sloc = 0.f;
+    bool grow = false;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      mloc[n][0] = mloc[n][1] = -INFINITY;
+#pragma unroll
+      for (int sl = 0; sl < NSL; ++sl)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) mloc[n][h] = fmaxf(mloc[n][h], ok[sl][j] ? x[sl][n][j][h] : -INFINITY);
+      grow = grow || mloc[n][0] > m[n][0] + thr || mloc[n][1] > m[n][1] + thr;
+    }
 #pragma unroll
     for (int sl = 0; sl < NSL; ++sl)
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      for (int j = 0; j < 2; ++j) sloc = fmaxf(sloc, sv[sl][j]);
+    grow = grow || (FP8 && sloc > sig);
+    float alpha[NT][2];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) mloc[h] = fmaxf(mloc[h], ok[sl][j] ? x[sl][j][h] : -INFINITY);
-        sloc = fmaxf(sloc, sv[sl][j]);
-      }
-    const bool grow = mloc[0] > m[0] + thr || mloc[1] > m[1] + thr || (FP8 && sloc > sig);
-    float alpha[2] = {1.f, 1.f};
+    for (int n = 0; n < NT; ++n) alpha[n][0] = alpha[n][1] = 1.f;
     if (__any_sync(0xffffffffu, grow)) {
       float beta = 1.f;
       if constexpr (FP8) {
@@ -215,49 +254,62 @@ struct WarpAttn {
           sig = sig_new;
         }
       }
-      float f[2];
+      float f[NT][2];
+      bool any_f = false;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {  // max over the rows: lanes of equal t
-        float mx = fmaxf(mloc[h], __shfl_xor_sync(0xffffffffu, mloc[h], 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float m_new = fmaxf(m[h], mx);
-        if (m_new != m[h]) alpha[h] = ex2_approx((m[h] - m_new) * cl);  // 0 when m was -inf
-        m[h] = m_new;
-        f[h] = alpha[h] * beta;
-      }
-      // rescale the O^T columns of heads 2t, 2t+1
-      if (__any_sync(0xffffffffu, f[0] != 1.f || f[1] != 1.f)) {
+      for (int n = 0; n < NT; ++n)
 #pragma unroll
-        for (int i = 0; i < KS; ++i) {
-          o[i][0] *= f[0];
-          o[i][1] *= f[1];
-          o[i][2] *= f[0];
-          o[i][3] *= f[1];
+        for (int h = 0; h < 2; ++h) {  // max over the rows: lanes of equal t
+          float mx = fmaxf(mloc[n][h], __shfl_xor_sync(0xffffffffu, mloc[n][h], 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float m_new = fmaxf(m[n][h], mx);
+          if (m_new != m[n][h]) alpha[n][h] = ex2_approx((m[n][h] - m_new) * cl);  // 0 when m was -inf
+          m[n][h] = m_new;
+          f[n][h] = alpha[n][h] * beta;
+          any_f = any_f || f[n][h] != 1.f;
         }
+      // rescale the O^T columns of heads 8n + 2t, 8n + 2t + 1
+      if (__any_sync(0xffffffffu, any_f)) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int i = 0; i < KS; ++i) {
+            o[n][i][0] *= f[n][0];
+            o[n][i][1] *= f[n][1];
+            o[n][i][2] *= f[n][0];
+            o[n][i][3] *= f[n][1];
+          }
       }
     }
-    uint32_t pb[NSL][2];  // P^T fragments: the transposed 8x8 halves (rows 0-7, 8-15 x heads)
-    float lsum[2] = {0.f, 0.f};
+    uint32_t pb[NSL][NT][2];  // P^T fragments: the transposed 8x8 halves (rows 0-7, 8-15 x heads)
+    float lsum[NT][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) lsum[n][0] = lsum[n][1] = 0.f;
 #pragma unroll
     for (int sl = 0; sl < NSL; ++sl)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        float p[2];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // the difference first: dominant terms exact
-          p[h] = ok[sl][j] ? ex2_approx((x[sl][j][h] - m[h]) * cl) : 0.f;
-          lsum[h] += p[h];
-        }
-        if constexpr (FP8) {
-          const float w8 = sv[sl][j] * inv_sig;
-          pb[sl][j] = movmatrix_t(pack_f16(p[0] * w8, p[1] * w8));
-        } else {
-          pb[sl][j] = movmatrix_t(pack_bf16(p[0], p[1]));
+        for (int n = 0; n < NT; ++n) {
+          float pr[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {  // the difference first: dominant terms exact
+            pr[h] = ok[sl][j] ? ex2_approx((x[sl][n][j][h] - m[n][h]) * cl) : 0.f;
+            lsum[n][h] += pr[h];
+          }
+          if constexpr (FP8) {
+            const float w8 = sv[sl][j] * inv_sig;
+            pb[sl][n][j] = movmatrix_t(pack_f16(pr[0] * w8, pr[1] * w8));
+          } else {
+            pb[sl][n][j] = movmatrix_t(pack_bf16(pr[0], pr[1]));
+          }
         }
       }
 #pragma unroll
-    for (int h = 0; h < 2; ++h) l[h] = l[h] * alpha[h] + lsum[h];
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) l[n][h] = l[n][h] * alpha[n][h] + lsum[n][h];
 
     // ---- O^T += V^T P^T (A rows 2t, 2t+1, 8+2t, 9+2t of each slice)
     const bool full = vmask == (NSL == 2 ? 0xFFFFFFFFu : 0xFFFFu);
@@ -283,7 +335,8 @@ struct WarpAttn {
             a[2] &= m23[sl];
             a[3] &= m23[sl];
           }
-          mma_bf16(o[mt], a[0], a[1], a[2], a[3], pb[sl][0], pb[sl][1]);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) mma_bf16(o[n][mt], a[0], a[1], a[2], a[3], pb[sl][n][0], pb[sl][n][1]);
         }
       }
     } else {
@@ -315,37 +368,154 @@ struct WarpAttn {
           uint32_t a0, a1, a2, a3;
           e4m3x4_to_f16x2x2(x01, a0, a1);
           e4m3x4_to_f16x2x2(x23, a2, a3);
-          mma_f16(o[mt], a0, a1, a2, a3, pb[sl][0], pb[sl][1]);
+#pragma unroll
+          for (int n = 0; n < NT; ++n) mma_f16(o[n][mt], a0, a1, a2, a3, pb[sl][n][0], pb[sl][n][1]);
         }
       }
     }
   }
 
-  // Writes this warp's state to shared scratch: m[8], l[8], o[8][D] (true
-  // scale, not yet normalised).  Heads >= G are written too and ignored.
+  // Writes this warp's state to shared scratch: m[8 NT], l[8 NT], o[8 NT][D]
+  // (true scale, not yet normalised) at sm, sl, so.  Heads >= G are written
+  // too and ignored.
   __device__ __forceinline__ void store(float *sm, float *sl, float *so) const {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {  // sum over the rows: lanes of equal t
-      float lt = l[h];
-      lt += __shfl_xor_sync(0xffffffffu, lt, 4);
-      lt += __shfl_xor_sync(0xffffffffu, lt, 8);
-      lt += __shfl_xor_sync(0xffffffffu, lt, 16);
-      if (g == 0) {
-        sm[2 * t + h] = m[h];
-        sl[2 * t + h] = lt;
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // sum over the rows: lanes of equal t
+        float lt = l[n][h];
+        lt += __shfl_xor_sync(0xffffffffu, lt, 4);
+        lt += __shfl_xor_sync(0xffffffffu, lt, 8);
+        lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+        if (g == 0) {
+          sm[8 * n + 2 * t + h] = m[n][h];
+          sl[8 * n + 2 * t + h] = lt;
+        }
       }
-    }
     const float os = FP8 ? sig : 1.f;
 #pragma unroll
-    for (int mt = 0; mt < KS; ++mt) {
-      const int d0 = FP8 ? 16 * g + 2 * mt : 16 * mt + g;
-      const int d1 = FP8 ? d0 + 1 : d0 + 8;
-      so[(2 * t) * D + d0] = o[mt][0] * os;
-      so[(2 * t + 1) * D + d0] = o[mt][1] * os;
-      so[(2 * t) * D + d1] = o[mt][2] * os;
-      so[(2 * t + 1) * D + d1] = o[mt][3] * os;
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        const int d0 = FP8 ? 16 * g + 2 * mt : 16 * mt + g;
+        const int d1 = FP8 ? d0 + 1 : d0 + 8;
+        float *on = so + 8 * n * D;
+        on[(2 * t) * D + d0] = o[n][mt][0] * os;
+        on[(2 * t + 1) * D + d0] = o[n][mt][1] * os;
+        on[(2 * t) * D + d1] = o[n][mt][2] * os;
+        on[(2 * t + 1) * D + d1] = o[n][mt][3] * os;
+      }
+  }
+
+  // ---- Merging the states of warps that served the same heads, in registers
+  // (a tree over shared memory, one partner at a time).  The saved state is
+  // o lane-major (element i of lane L at dst[32 i + L]) followed by (m, l) of
+  // the 8 NT heads, which are uniform over g after finish().
+  static constexpr int kSaveFloats = NT * 4 * KS + NT * 16 / 32 + 1;  // per lane, rounded up
+  static constexpr int kSaveBytes = (NT * 4 * KS * 32 + NT * 16) * 4;
+
+  // Sums l over the rows (lanes of equal t), so every lane holds its heads'
+  // whole-warp normaliser, and brings o to its true scale (E4M3: sig = 1
+  // afterwards).  Call once before save / absorb / write_record.
+  __device__ __forceinline__ void finish() {
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float lt = l[n][h];
+        lt += __shfl_xor_sync(0xffffffffu, lt, 4);
+        lt += __shfl_xor_sync(0xffffffffu, lt, 8);
+        lt += __shfl_xor_sync(0xffffffffu, lt, 16);
+        l[n][h] = lt;
+      }
+    if constexpr (FP8) {
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < KS; ++i)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[n][i][e] *= sig;
+      sig = 1.f;
+      inv_sig = 1.f;
     }
+  }
+
+  __device__ __forceinline__ void save(float *dst) const {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    float *ml = dst + NT * 4 * KS * 32;  // m then l of head 8n + 2t + h at [16 n + 4 h + t], [.. + 8]
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      if (g == 0)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          ml[16 * n + 4 * h + t] = m[n][h];
+          ml[16 * n + 8 + 4 * h + t] = l[n][h];
+        }
+#pragma unroll
+      for (int k = 0; k < KS; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[32 * (4 * (KS * n + k) + e) + lane] = o[n][k][e];
+    }
+  }
+
+  // Folds a partner's saved state (same heads, same lane layout) into this one.
+  __device__ __forceinline__ void absorb(const float *src, float c) {
+    const int lane = threadIdx.x & 31, t = lane & 3;
+    const float cl = c * 1.44269504088896341f;
+    const float *ml = src + NT * 4 * KS * 32;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      float fa[2], fb[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float mb = ml[16 * n + 4 * h + t];
+        const float lb = ml[16 * n + 8 + 4 * h + t];
+        const float M = fmaxf(m[n][h], mb);
+        fa[h] = m[n][h] == -INFINITY ? 0.f : ex2_approx((m[n][h] - M) * cl);
+        fb[h] = mb == -INFINITY ? 0.f : ex2_approx((mb - M) * cl);
+        l[n][h] = l[n][h] * fa[h] + lb * fb[h];
+        m[n][h] = M;
+      }
+#pragma unroll
+      for (int k = 0; k < KS; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          o[n][k][e] = o[n][k][e] * fa[e & 1] + src[32 * (4 * (KS * n + k) + e) + lane] * fb[e & 1];
+    }
+  }
+
+  // Writes the (finished) state of heads [0, G) into a record of Gtot heads
+  // m[Gtot], l[Gtot], o[Gtot][D] at rec (global), as heads hoff + h.
+  __device__ __forceinline__ void write_record(float *rec, int G, int hoff, int Gtot) const {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int hh = 8 * n + 2 * t + h;
+        if (g == 0 && hh < G) {
+          rec[hoff + hh] = m[n][h];
+          rec[Gtot + hoff + hh] = l[n][h];
+        }
+      }
+    float *ro = rec + 2 * Gtot + hoff * D;
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        const int d0 = FP8 ? 16 * g + 2 * mt : 16 * mt + g;
+        const int d1 = FP8 ? d0 + 1 : d0 + 8;
+        const int h0 = 8 * n + 2 * t;
+        if (h0 < G) {
+          ro[h0 * D + d0] = o[n][mt][0];
+          ro[h0 * D + d1] = o[n][mt][2];
+        }
+        if (h0 + 1 < G) {
+          ro[(h0 + 1) * D + d0] = o[n][mt][1];
+          ro[(h0 + 1) * D + d1] = o[n][mt][3];
+        }
+      }
   }
 };
 

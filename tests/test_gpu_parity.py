@@ -232,6 +232,46 @@ def test_every_attention_config(oracle, lib, monkeypatch, kv_dtype, cfg):
     U.check_full(wd, out, idx, ora)
 
 
+# configurations for groups of 16 and more heads (ncw, nstage, nsl, nt): nt = 2
+# gives each warp 16 heads; the nt = 1 entries are the 8-head fallbacks
+WIDE_CONFIGS = {
+    "bf16": ["4,3,2,2", "8,3,1,2", "8,3,1,1", "4,3,2,1"],
+    "e4m3": ["4,6,2,2", "8,3,2,1"],
+}
+WIDE_SHAPES = {  # (spec fields, sequence lengths)
+    "mqa_g32": (dict(group=32, num_kv_heads=1, batch=3), [90, 4100, 1300]),
+    "g16": (dict(group=16, num_kv_heads=2, batch=2), [2500, 700]),
+}
+
+
+@pytest.mark.parametrize("shape", list(WIDE_SHAPES))
+@pytest.mark.parametrize("kv_dtype,cfg", [(d, c) for d, cs in WIDE_CONFIGS.items() for c in cs])
+def test_every_wide_attention_config(oracle, lib, monkeypatch, kv_dtype, cfg, shape):
+    """Every configuration built for groups above 8 heads, on short and
+    ragged sequences (warps whose row blocks lie past the end merge empty
+    states)."""
+    fields, lens = WIDE_SHAPES[shape]
+    sp = spec(kv_dtype=kv_dtype, sparse_layers=1, seq_len=max(lens), **fields)
+    w = synth.generate(sp, seed=11, seq_lens=lens)
+    ora = U.run_oracle(oracle, w)
+    wd = U.to_device(w)
+    monkeypatch.setenv("HS2_FULL_CFG", cfg)
+    out, idx = U.run_gpu(wd)
+    torch.cuda.synchronize()
+    U.check_full(wd, out, idx, ora)
+
+
+def test_wide_d64_config(oracle, lib, monkeypatch):
+    sp = spec(group=32, num_kv_heads=1, batch=2, head_dim=64, page_size=None, sparse_layers=1, seq_len=3000)
+    w = synth.generate(sp, seed=12, seq_lens=[3000, 333])
+    ora = U.run_oracle(oracle, w)
+    wd = U.to_device(w)
+    monkeypatch.setenv("HS2_FULL_CFG", "8,6,1,2")
+    out, idx = U.run_gpu(wd)
+    torch.cuda.synchronize()
+    U.check_full(wd, out, idx, ora)
+
+
 def test_bounded_wait_expires_and_context_stays_usable(oracle, lib):
     """A device wait that nothing completes gives up, flags the workspace,
     and the next status read reports it once; the context keeps working."""
