@@ -445,9 +445,10 @@ def run_gpu(args, rank, world, local):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(KB)]
 
     def step(e=None):
+        # the marked breakdown steps run the separate kernels (their boundary carries the event)
         hs2.full_attn_select(w.q_full, w.k, w.v, w.seq_lens, w.page_table, w.page_size, s.window, s.k_global,
                              w.k_scale, w.v_scale, out=outs[0], idx_out=idx, workspace=ws,
-                             mark_event=None if e is None else e[1])
+                             mark_event=None if e is None else e[1], fused=args.fused and e is None)
         if e is not None:
             e[2].record(stream)
         for l in range(s.sparse_layers):
@@ -507,7 +508,7 @@ def run_gpu(args, rank, world, local):
             a.copy_(b, non_blocking=True)
         lens_dev.copy_(lens_host, non_blocking=True)
         hs2.full_attn_select(q_dev[0], w.k, w.v, lens_dev, w.page_table, w.page_size, s.window, s.k_global,
-                             w.k_scale, w.v_scale, out=outs[0], idx_out=idx, workspace=ws)
+                             w.k_scale, w.v_scale, out=outs[0], idx_out=idx, workspace=ws, fused=args.fused)
         for l in range(s.sparse_layers):
             hs2.sparse_attn(q_dev[1 + l], w.k, w.v, idx, w.k_scale, w.v_scale, w.page_size, out=outs[1 + l])
         for a, b in zip(outs_host, outs):
@@ -546,7 +547,7 @@ def run_gpu(args, rank, world, local):
         "vs_baseline": None,
         "dtype": {"bf16": "bf16", "e4m3": "e4m3", "f32": "f32"}[s.kv_dtype],
         "data": "synthetic",
-        "config": workload_config(w, world),
+        "config": dict(workload_config(w, world), full_layer_call="fused" if args.fused else "separate kernels"),
         "roofline": {"bound": "hbm", "kernel": "full_attn_mma_kernel", "achieved": attn_gbs, "peak": peak,
                      "unit": "GB/s", "frac": attn_gbs / peak, "traffic": traffic,
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
@@ -566,7 +567,7 @@ def run_gpu(args, rank, world, local):
                 "d2h_bytes_per_step": d2h, "steps": K2,
                 "what": "queries copied in from pinned host memory, outputs and index list copied out and synced, "
                         "every step; the KV cache stays resident"},
-        "gpu_launches": K * (4 + s.sparse_layers),
+        "gpu_launches": K * ((3 if args.fused else 4) + s.sparse_layers),
         "clocks": clk,
         "device_status": status,
     }
@@ -605,7 +606,7 @@ def run_reference(args, rank, world, local):
     return {"metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": workload_config(w, world),
+            "config": dict(workload_config(w, world), full_layer_call="fused" if args.fused else "separate kernels"),
             "cpu_baseline": {"value": v, "unit": "steps/s", "cores": threads, "kind": "oracle", "cpu": host_cpu(),
                              "sample": f"whole steps: all {len(units)} (sequence, kv head) units of the workload, "
                                        f"each through the full layer, the selection and {spec.sparse_layers} sparse "
@@ -628,6 +629,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-copy-peak", action="store_true", help="skip the same-run copy-bandwidth measurement")
     ap.add_argument("--no-block-timing", action="store_true", help="skip the block-level selection timing")
+    ap.add_argument("--fused", action="store_true",
+                    help="time the fused full-layer call (attention + score pass in one persistent kernel)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's context (profiling runs)")
     ap.add_argument("--kv-heads", type=int, default=0, help="override the workload's KV heads (experiments)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (experiments)")

@@ -143,6 +143,28 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
                                 void *workspace, size_t workspace_bytes, void *stream, void *mark_event);
 
 /*
+ * hs2_full_attn_select() as one fused persistent pass: the attention kernel's
+ * CTAs, after their last tile, wait at a grid barrier and run the selection's
+ * score pass over the positions they attended (logits still in L2), so the
+ * full layer selects as it finishes its own computation (HySparse2
+ * announcement, "KV Reuse" section: the full layer's attention scores pick
+ * the positions the sparse layers read).  Same arguments and results as
+ * hs2_full_attn_select(); two more kernels (filter, final) follow on `stream`.
+ *   The kernel is launched cooperatively (every CTA resident at once; no
+ *   programmatic overlap with the previous kernel); the call first clears
+ *   the barrier's counter with cudaMemsetAsync.  The barrier wait is bounded
+ *   (about 2 s): on expiry the sticky flag reports HS2_ERR_TIMEOUT through
+ *   hs2_workspace_status() and the selection of that call is not valid.
+ *   Tensor-core caches (bf16, E4M3) in the default configuration of their
+ *   shape only; fp32 caches run the unfused call.  HS2_ERR_UNSUPPORTED for
+ *   shapes with no fused kernel built.
+ */
+int hs2_full_attn_select_fused(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                               const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
+                               int32_t window, int32_t k_global, hs2_heads *out, int32_t *idx_out,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * The full-attention layer with BLOCK-level instead of token-level selection:
  * the first-generation HySparse selection, kept as a comparator (HySparse2
  * announcement, the paragraphs contrasting token-level with HySparse's

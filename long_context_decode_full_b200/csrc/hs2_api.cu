@@ -241,7 +241,7 @@ FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged, int G
 int full_attn_select_impl(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
                           const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages, int32_t window,
                           int32_t k_global, int32_t block, hs2_heads *out, int32_t *idx_out, void *workspace,
-                          size_t workspace_bytes, void *stream, void *mark_event);
+                          size_t workspace_bytes, void *stream, void *mark_event, bool fused = false);
 
 }  // namespace
 
@@ -275,6 +275,14 @@ int hs2_full_attn_select_marked(const hs2_heads *q, const hs2_cache *k_cache, co
                                idx_out, workspace, workspace_bytes, stream, mark_event);
 }
 
+int hs2_full_attn_select_fused(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
+                               const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
+                               int32_t window, int32_t k_global, hs2_heads *out, int32_t *idx_out, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+  return full_attn_select_impl(q, k_cache, v_cache, seq_lens, page_table, max_pages, window, k_global, 0, out,
+                               idx_out, workspace, workspace_bytes, stream, nullptr, true);
+}
+
 int hs2_full_attn_select_blocks(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
                                 const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages,
                                 int32_t window, int32_t k_global, int32_t block, hs2_heads *out, int32_t *idx_out,
@@ -294,7 +302,7 @@ namespace {
 int full_attn_select_impl(const hs2_heads *q, const hs2_cache *k_cache, const hs2_cache *v_cache,
                           const int32_t *seq_lens, const int32_t *page_table, int32_t max_pages, int32_t window,
                           int32_t k_global, int32_t block, hs2_heads *out, int32_t *idx_out, void *workspace,
-                          size_t workspace_bytes, void *stream, void *mark_event) {
+                          size_t workspace_bytes, void *stream, void *mark_event, bool fused) {
   int rc;
   if ((rc = check_caches(k_cache, v_cache))) return rc;
   if ((rc = check_heads(q, k_cache, "q"))) return rc;
@@ -358,29 +366,15 @@ int full_attn_select_impl(const hs2_heads *q, const hs2_cache *k_cache, const hs
   }
   const int sms = sm_count();
   cudaError_t e;
+  const bool fp8 = k_cache->dtype == HS2_E4M3;
+  FullMmaConfig cfg{};
   if (!mma) {
     p.tile = full_f32_tile();
     p.N = sms * full_f32_ctas_per_sm();
-    e = launch_full_f32(p, p.N, s);
-    if (e != cudaSuccess) return cuda_fail(e, "full-attention (fp32) launch");
   } else {
-    const bool fp8 = k_cache->dtype == HS2_E4M3;
-    const FullMmaConfig cfg = pick_full_config(D, fp8, ps, paged, G);
+    cfg = pick_full_config(D, fp8, ps, paged, G);
     p.tile = 16 * cfg.ncw * cfg.nsl;
     p.N = sms;
-    const int box_rows = paged ? (ps < p.tile ? ps : p.tile) : p.tile;
-    CUtensorMap tmk, tmv;
-    if ((rc = encode_cache_map(&tmk, k_cache, box_rows))) return rc;
-    if ((rc = encode_cache_map(&tmv, v_cache, box_rows))) return rc;
-    e = launch_full_mma(p, tmk, tmv, fp8, cfg, p.N, s);
-    if (e == cudaErrorInvalidConfiguration)
-      return fail(HS2_ERR_UNSUPPORTED, "no full-attention kernel built for ncw=%d nstage=%d nsl=%d nt=%d", cfg.ncw,
-                  cfg.nstage, cfg.nsl, cfg.nt);
-    if (e != cudaSuccess) return cuda_fail(e, "full-attention launch");
-  }
-  if (mark_event) {
-    e = cudaEventRecord(static_cast<cudaEvent_t>(mark_event), s);
-    if (e != cudaSuccess) return cuda_fail(e, "recording the mark event");
   }
   ScoreParams sp{};
   sp.seq_lens = seq_lens;
@@ -411,7 +405,36 @@ int full_attn_select_impl(const hs2_heads *q, const hs2_cache *k_cache, const hs
   sp.c = p.c;
   sp.ncomb = (G * D + 255) / 256;
   sp.ws = p.ws;
-  e = block > 0 ? launch_block_select(sp, block, s) : launch_select(sp, s);
+  // the fused call: token-level selection on the tensor-core path only
+  const bool fuse = fused && mma && block == 0;
+  if (fuse && (G >= 16) != (cfg.nt == 2))
+    return fail(HS2_ERR_UNSUPPORTED, "fused call: no kernel for %d heads per group with %d-head warps", G, 8 * cfg.nt);
+  if (!mma) {
+    e = launch_full_f32(p, p.N, s);
+    if (e != cudaSuccess) return cuda_fail(e, "full-attention (fp32) launch");
+  } else {
+    const int box_rows = paged ? (ps < p.tile ? ps : p.tile) : p.tile;
+    CUtensorMap tmk, tmv;
+    if ((rc = encode_cache_map(&tmk, k_cache, box_rows))) return rc;
+    if ((rc = encode_cache_map(&tmv, v_cache, box_rows))) return rc;
+    if (fuse) {
+      // the grid barrier's arrival counter (word 16 of the flag block) starts at zero
+      e = cudaMemsetAsync(p.ws.err + 16, 0, sizeof(uint32_t), s);
+      if (e != cudaSuccess) return cuda_fail(e, "clearing the grid-barrier counter");
+      e = launch_full_fused(p, sp, tmk, tmv, fp8, cfg, p.N, s);
+    } else {
+      e = launch_full_mma(p, tmk, tmv, fp8, cfg, p.N, s);
+    }
+    if (e == cudaErrorInvalidConfiguration)
+      return fail(HS2_ERR_UNSUPPORTED, "no %sfull-attention kernel built for ncw=%d nstage=%d nsl=%d nt=%d",
+                  fuse ? "fused " : "", cfg.ncw, cfg.nstage, cfg.nsl, cfg.nt);
+    if (e != cudaSuccess) return cuda_fail(e, fuse ? "fused full-attention launch" : "full-attention launch");
+  }
+  if (mark_event) {
+    e = cudaEventRecord(static_cast<cudaEvent_t>(mark_event), s);
+    if (e != cudaSuccess) return cuda_fail(e, "recording the mark event");
+  }
+  e = block > 0 ? launch_block_select(sp, block, s) : (fuse ? launch_select_after_score(sp, s) : launch_select(sp, s));
   if (e != cudaSuccess) return cuda_fail(e, "selection launch");
   return HS2_OK;
 }
@@ -505,7 +528,9 @@ int hs2_workspace_status(void *workspace, size_t workspace_bytes, void *stream) 
   if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, 4, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "reading the workspace status");
-  if (flag) return fail(HS2_ERR_TIMEOUT, "device error flag 0x%x (1: consumer wait, 2: producer wait, 4: record)", flag);
+  if (flag)
+    return fail(HS2_ERR_TIMEOUT, "device error flag 0x%x (1: consumer wait, 2: producer wait, 4: record, 8: grid barrier)",
+                flag);
   return HS2_OK;
 }
 

@@ -136,6 +136,14 @@ __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
+// Untiled bulk copy of `bytes` (a multiple of 16) from global memory into
+// this CTA's shared memory, both addresses 16-byte aligned, completing on
+// `bar` (no multicast).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
 // L2 eviction policies.  The logits are read back by the score pass right
 // after the attention kernel (evict last), so most of them are still in L2
 // then.  Marking the K/V stream (read once) evict-first helps only when the

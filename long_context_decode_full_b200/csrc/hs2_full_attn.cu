@@ -16,6 +16,7 @@
 //
 // The fp32 cache variant runs the same partition on the CUDA cores (FFMA), so
 // fp32 logits keep full fp32 accuracy.
+#include "hs2_fused_tail.cuh"
 #include "hs2_internal.h"
 #include "hs2_warp_attn.cuh"
 
@@ -113,10 +114,11 @@ __device__ __forceinline__ int find_seq(const int32_t *prefix, int B, int Hkv, i
 template <bool FP8>
 constexpr int kProducerWarps = FP8 ? 2 : 1;
 
-template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT>
-__global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
-    full_attn_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                         const FullParams p) {
+// The attention pass of one CTA; with FUSED the CTA then runs the score pass
+// of the selection (hs2_fused_tail.cuh) over the tiles it attended.
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT, bool FUSED>
+__device__ __forceinline__ void full_attn_body(const CUtensorMap &tmk, const CUtensorMap &tmv, const FullParams &p,
+                                               const ScoreParams *sp) {
   using C = Cfg<D, FP8, NCW, NSTAGE, NSL, NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -155,10 +157,14 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
     for (int i = threadIdx.x; i <= p.B; i += blockDim.x) p.ws.prefix[i] = prefix[i];
 
   const int64_t total = (int64_t)p.Hkv * prefix[p.B];
-  if (total == 0) return;
+  if (total == 0) {  // every sequence is empty (the same for all CTAs: no barrier)
+    if constexpr (FUSED) fused_zero_empty(*sp);
+    return;
+  }
   const Partition part{total, p.N};
   const int64_t g0 = part.start(blockIdx.x), g1 = part.start(blockIdx.x + 1);
 
+  [&]() {  // producers and consumers; both return here when their work is done
   if (producer) {
     // ------------------------------------------------------------ producers
     // Boxes of RB rows (one page, or the whole tile when pages are larger).
@@ -376,6 +382,34 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[stage]);
   }
+  }();
+
+  if constexpr (FUSED) {
+    // every segment record and logit of the call is written once all CTAs
+    // pass the barrier; the K/V stages are idle from here on
+    TailSmem *ts = reinterpret_cast<TailSmem *>(smem);
+    if (!grid_barrier(p.ws.err + 16, p.ws.err + 32, gridDim.x, &ts->ok_flag)) {
+      if (threadIdx.x == 0) set_error(p.ws.err, kErrGridWait);
+      return;
+    }
+    fused_tail_dispatch<D, NT>(*sp, g0, g1, ts, (size_t)C::STAGE * NSTAGE);
+  }
+}
+
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT>
+__global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
+    full_attn_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                         const FullParams p) {
+  full_attn_body<D, FP8, NCW, NSTAGE, NSL, NT, false>(tmk, tmv, p, nullptr);
+}
+
+// The fused call: attention, a grid barrier, then the score pass.  Launched
+// cooperatively (every CTA resident at once).
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT>
+__global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
+    full_attn_fused_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                           const FullParams p, const ScoreParams sp) {
+  full_attn_body<D, FP8, NCW, NSTAGE, NSL, NT, true>(tmk, tmv, p, &sp);
 }
 
 // ------------------------------------------------------------ fp32 caches
@@ -503,6 +537,18 @@ cudaError_t launch_mma_t(const FullParams &p, const CUtensorMap &tmk, const CUte
   return launch_ex(kern, dim3(grid), dim3(32 * (NCW + kProducerWarps<FP8>)), smem, s, 0, tmk, tmv, p);
 }
 
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT>
+cudaError_t launch_fused_t(const FullParams &p, const ScoreParams &sp, const CUtensorMap &tmk,
+                           const CUtensorMap &tmv, int grid, cudaStream_t s) {
+  using C = Cfg<D, FP8, NCW, NSTAGE, NSL, NT>;
+  static_assert(kTailBufOffset + 4 * kTailChunk <= (size_t)C::STAGE * NSTAGE, "score-pass arrays fit in the stages");
+  const size_t smem = C::bytes(p.B);
+  auto kern = full_attn_fused_kernel<D, FP8, NCW, NSTAGE, NSL, NT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_coop(kern, dim3(grid), dim3(32 * (NCW + kProducerWarps<FP8>)), smem, s, tmk, tmv, p, sp);
+}
+
 }  // namespace
 
 cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, bool fp8,
@@ -528,6 +574,21 @@ cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const C
   HS2_FULL_CASE(64, false, 8, 6, 1, 2)
   HS2_FULL_CASE(128, true, 4, 6, 2, 2)
 #undef HS2_FULL_CASE
+  return cudaErrorInvalidConfiguration;
+}
+
+cudaError_t launch_full_fused(const FullParams &p, const ScoreParams &sp, const CUtensorMap &tmk,
+                              const CUtensorMap &tmv, bool fp8, const FullMmaConfig &cfg, int grid, cudaStream_t s) {
+#define HS2_FUSED_CASE(D_, F_, W_, S_, L_, N_)                                                       \
+  if (p.D == D_ && fp8 == F_ && cfg.ncw == W_ && cfg.nstage == S_ && cfg.nsl == L_ && cfg.nt == N_) \
+    return launch_fused_t<D_, F_, W_, S_, L_, N_>(p, sp, tmk, tmv, grid, s);
+  // the default configuration of each case
+  HS2_FUSED_CASE(128, false, 4, 3, 2, 1)
+  HS2_FUSED_CASE(64, false, 8, 6, 1, 1)
+  HS2_FUSED_CASE(128, true, 8, 3, 2, 1)
+  HS2_FUSED_CASE(128, false, 4, 3, 2, 2)
+  HS2_FUSED_CASE(128, true, 4, 6, 2, 2)
+#undef HS2_FUSED_CASE
   return cudaErrorInvalidConfiguration;
 }
 

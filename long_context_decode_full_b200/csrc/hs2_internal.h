@@ -105,14 +105,45 @@ cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// Cooperative launch (every CTA resident at once), with programmatic stream
+// serialization as well where the runtime accepts the pair (else without it).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_coop(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess && cfg.numAttrs == 2) {
+    (void)cudaGetLastError();  // the refused pair is not the caller's error
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, args...);
+  }
+  return e;
+}
+
 // ---- launchers (return cudaError_t of the launch) -------------------------
 cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, bool fp8,
                             const FullMmaConfig &cfg, int grid, cudaStream_t s);
+// Attention and the selection's score pass in one cooperative persistent
+// launch (cudaErrorInvalidConfiguration when no fused kernel is built for cfg).
+cudaError_t launch_full_fused(const FullParams &p, const ScoreParams &sp, const CUtensorMap &tmk,
+                              const CUtensorMap &tmv, bool fp8, const FullMmaConfig &cfg, int grid, cudaStream_t s);
 cudaError_t launch_full_f32(const FullParams &p, int grid, cudaStream_t s);
 int full_f32_tile();
 int full_f32_ctas_per_sm();
 
 cudaError_t launch_select(const ScoreParams &p, cudaStream_t s);
+// The filter and final kernels alone (after the fused call's score pass).
+cudaError_t launch_select_after_score(const ScoreParams &p, cudaStream_t s);
 // Block-level selection (first-generation comparator) in place of launch_select.
 cudaError_t launch_block_select(const ScoreParams &p, int block, cudaStream_t s);
 

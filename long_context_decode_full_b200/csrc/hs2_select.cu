@@ -70,45 +70,6 @@ __device__ __forceinline__ void load_logits(float (&raw)[score_loads<G>()][G], c
   }
 }
 
-// The unit's approximate scores and histogram again, each score scaled by
-// 2^E, until the threshold bin is at or above kTrustBin (whole block; runs
-// only when the first pass put the k-th score below 2^-96).  Rewrites the
-// scores sc[0, nC) and shifts the per-head LSE by E ln 2, so that the filter's
-// exact scores carry the same factor.  Returns the threshold bin.
-template <int G>
-__device__ int rescale_unit(const ScoreParams &p, int nC, const float *lg, float *sc, uint32_t *sh_hist,
-                            double *sh_lse, int bin, int *above, int *sh_warp, int *sh_res) {
-  const float a = (float)((double)p.c * kLog2e);
-  double E = 0.0;
-  for (int round = 0; round < 16 && bin < kTrustBin && E < kMaxShift; ++round) {
-    const int e_bin = bin >> 4;  // biased fp32 exponent of the threshold bin, 0 when it underflowed
-    E += e_bin > 0 ? (double)(kTargetExponent - e_bin) : 200.0;
-    if (E > kMaxShift) E = kMaxShift;
-    float bh[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) bh[h] = (float)(sh_lse[h] * kLog2e - E);
-    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) sh_hist[i] = 0u;
-    __syncthreads();
-    for (int t = threadIdx.x; t < nC; t += blockDim.x) {
-      float pr[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) pr[h] = ex2_approx(fmaf(__ldcg(lg + (size_t)t * G + h), a, -bh[h]));
-#pragma unroll
-      for (int w = 1; w < G; w <<= 1)
-#pragma unroll
-        for (int h = 0; h + w < G; h += 2 * w) pr[h] += pr[h + w];
-      const float sv = pr[0] >= 0.f ? pr[0] : 0.f;
-      sc[t] = sv;
-      atomicAdd(&sh_hist[__float_as_uint(sv) >> kHistShift], 1u);
-    }
-    __syncthreads();
-    bin = find_threshold_bin(sh_hist, kHistBins, p.k_global, above, sh_warp, sh_res);
-  }
-  if (threadIdx.x < G) sh_lse[threadIdx.x] -= E * kLn2;
-  __syncthreads();
-  return bin;
-}
-
 template <int G, int D>
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(const ScoreParams p) {
   __shared__ uint32_t sh_hist[kHistBins];
@@ -597,9 +558,13 @@ cudaError_t launch_select(const ScoreParams &p, cudaStream_t s) {
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
+  return launch_select_after_score(p, s);
+}
+
+cudaError_t launch_select_after_score(const ScoreParams &p, cudaStream_t s) {
   const int fchunk = kSubRange * (kScoreThreads / 32) * p.filter_subs;
   const int fchunks = (int)((p.t_cap + fchunk - 1) / fchunk);
-  e = launch_ex(filter_kernel, dim3(fchunks, p.Hkv, p.B), dim3(kScoreThreads), 0, s, 0, p);
+  cudaError_t e = launch_ex(filter_kernel, dim3(fchunks, p.Hkv, p.B), dim3(kScoreThreads), 0, s, 0, p);
   if (e != cudaSuccess) return e;
   const size_t smem = final_smem_bytes(p.nsub);
   e = cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -42,7 +42,7 @@ class HS2Error(RuntimeError):
 
 _lib = None
 EXPORTS = ["hs2_full_attn_select_workspace", "hs2_full_attn_select", "hs2_full_attn_select_marked",
-           "hs2_full_attn_select_blocks",
+           "hs2_full_attn_select_blocks", "hs2_full_attn_select_fused",
            "hs2_full_attn_select_static", "hs2_full_attn_select_static_status", "hs2_selftest_bounded_wait_static",
            "hs2_sparse_attn",
            "hs2_workspace_status", "hs2_selftest_bounded_wait", "hs2_kv_bridge_workspace", "hs2_kv_bridge_append",
@@ -65,6 +65,8 @@ def lib():
         L.hs2_full_attn_select.restype = ctypes.c_int
         L.hs2_full_attn_select_marked.argtypes = L.hs2_full_attn_select.argtypes + [P]
         L.hs2_full_attn_select_marked.restype = ctypes.c_int
+        L.hs2_full_attn_select_fused.argtypes = L.hs2_full_attn_select.argtypes
+        L.hs2_full_attn_select_fused.restype = ctypes.c_int
         L.hs2_full_attn_select_blocks.argtypes = [ctypes.POINTER(Heads), ctypes.POINTER(Cache), ctypes.POINTER(Cache),
                                                   P, P, I32, I32, I32, I32, ctypes.POINTER(Heads), P, P, SZ, P]
         L.hs2_full_attn_select_blocks.restype = ctypes.c_int
@@ -168,11 +170,13 @@ def alloc_workspace(batch, num_kv_heads, group, head_dim, t_cap, device="cuda") 
 
 def full_attn_select(q, k, v, seq_lens, page_table=None, page_size=None, window=128, k_global=1024,
                      k_scale=None, v_scale=None, out=None, idx_out=None, workspace=None, stream=None,
-                     mark_event=None):
+                     mark_event=None, fused=False):
     """Full-attention layer + token selection.  Returns (out, idx) where idx
     holds selected slots [B, Hkv, window + k_global], ascending, -1 padded.
     ``mark_event`` (a recorded-once torch.cuda.Event) is recorded between the
-    attention kernel and the selection kernels."""
+    attention kernel and the selection kernels.  ``fused`` runs the attention
+    and the selection's score pass in one cooperative persistent kernel
+    (hs2_full_attn_select_fused; no mark event)."""
     B, Hq, d = q.shape
     Hkv = k.shape[1]
     _need_lens(seq_lens, page_table, B)
@@ -191,6 +195,13 @@ def full_attn_select(q, k, v, seq_lens, page_table=None, page_size=None, window=
         workspace = alloc_workspace(B, Hkv, Hq // Hkv, d, t_cap, q.device)
     kc, vc = cache_desc(k, k_scale, page_size), cache_desc(v, v_scale, page_size)
     qd, od = heads_desc(q), heads_desc(out)
+    if fused:
+        assert mark_event is None, "the fused call records no mark event"
+        _check(lib().hs2_full_attn_select_fused(ctypes.byref(qd), ctypes.byref(kc), ctypes.byref(vc),
+                                                _ptr(seq_lens), _ptr(page_table), max_pages, window, k_global,
+                                                ctypes.byref(od), _ptr(idx_out), _ptr(workspace), workspace.numel(),
+                                                _stream(stream)))
+        return out, idx_out
     ev = None if mark_event is None else ctypes.c_void_p(mark_event.cuda_event)
     _check(lib().hs2_full_attn_select_marked(ctypes.byref(qd), ctypes.byref(kc), ctypes.byref(vc),
                                              _ptr(seq_lens), _ptr(page_table), max_pages, window, k_global,
@@ -277,13 +288,14 @@ def sparse_attn(q_l, k, v, idx, k_scale=None, v_scale=None, page_size=1, out=Non
 
 def hybrid_block_step(q_full, q_sparse: Sequence[torch.Tensor], k, v, seq_lens, page_table=None, page_size=None,
                       window=128, k_global=1024, k_scale=None, v_scale=None, outs=None, idx_out=None,
-                      workspace=None, stream=None):
+                      workspace=None, stream=None, fused=False):
     """One decode step of a Hybrid Block: the full layer (attention + token
     selection) then every sparse layer with its own query, all reusing the
-    same cache and the same index list.  Returns (outs, idx)."""
+    same cache and the same index list.  Returns (outs, idx).  ``fused``
+    selects the fused full-layer call (see full_attn_select)."""
     outs = outs if outs is not None else [None] * (1 + len(q_sparse))
     o0, idx = full_attn_select(q_full, k, v, seq_lens, page_table, page_size, window, k_global, k_scale, v_scale,
-                               outs[0], idx_out, workspace, stream)
+                               outs[0], idx_out, workspace, stream, fused=fused)
     ps = page_size if page_size is not None else k.shape[0] // q_full.shape[0]
     res = [o0]
     for i, q in enumerate(q_sparse):

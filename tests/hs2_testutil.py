@@ -37,14 +37,14 @@ def garbage_workspace(w: synth.Workload, seed=0):
     return ws
 
 
-def run_gpu(w: synth.Workload, q=None, window=None, k_global=None, workspace=None):
+def run_gpu(w: synth.Workload, q=None, window=None, k_global=None, workspace=None, fused=False):
     from long_context_decode_full_b200 import hs2
     s = w.spec
     if workspace is None:
         workspace = garbage_workspace(w)
     return hs2.full_attn_select(w.q_full if q is None else q, w.k, w.v, w.seq_lens, w.page_table, w.page_size,
                                 s.window if window is None else window, s.k_global if k_global is None else k_global,
-                                w.k_scale, w.v_scale, workspace=workspace)
+                                w.k_scale, w.v_scale, workspace=workspace, fused=fused)
 
 
 def run_gpu_sparse(w: synth.Workload, q, idx):

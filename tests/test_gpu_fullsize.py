@@ -145,3 +145,21 @@ def test_full_size_workload_every_unit(pool, oracle_mod, name):
             opos[:len(ora)] = ora
             nb += U.check_block_positions(bpos[b, h], opos, score, T, spec.window, spec.k_global, block)
         print(f"{name}: block-level selection (block {block}), blocks differing inside the near-tie band {nb}")
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_full_size_fused_call_equals_separate_kernels(name):
+    """The fused full-layer call gives the separate kernels' output and index
+    list bit for bit at full size (those are compared with the oracle on
+    every unit above)."""
+    spec = synth.WORKLOADS[name]
+    w = synth.generate(spec, seed=0, device="cuda")
+    ws = U.garbage_workspace(w)
+    args = (w.q_full, w.k, w.v, w.seq_lens, w.page_table, w.page_size, spec.window, spec.k_global, w.k_scale,
+            w.v_scale)
+    o_sep, i_sep = hs2.full_attn_select(*args, workspace=ws)
+    o_fus, i_fus = hs2.full_attn_select(*args, workspace=ws, fused=True)
+    torch.cuda.synchronize()
+    assert hs2.workspace_status(ws) == 0
+    assert torch.equal(i_fus, i_sep)
+    assert torch.equal(o_fus, o_sep)
