@@ -318,6 +318,18 @@ int hs2_kv_bridge_append(const void *hidden, int32_t batch, int32_t d_model, con
 int hs2_selftest_bounded_wait(void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Self-test of the fused call's grid barrier (no counterpart in the pages):
+ * two CTAs meet at a barrier sized for three, both give up after about 10 ms
+ * of clock cycles and set the workspace's sticky flag (bit 8), so a
+ * following hs2_workspace_status() returns HS2_ERR_TIMEOUT (and clears it);
+ * the context stays usable and the next fused call on the workspace clears
+ * the barrier's counter.  No fault, trap or hang is involved.
+ *   workspace  device, >= 256 bytes, 256-byte aligned (its flag block is used).
+ * Returns HS2_OK once launched (asynchronous on `stream`).
+ */
+int hs2_selftest_grid_barrier(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * The same self-test on the static scratch of hs2_full_attn_select_static()
  * in the current CUDA context: afterwards hs2_full_attn_select_static_status()
  * returns HS2_ERR_TIMEOUT once (and clears the flag).  Must not overlap a

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "hs2.h"
+#include "hs2_fused_tail.cuh"
 #include "hs2_internal.h"
 
 using namespace hs2;
@@ -603,6 +604,14 @@ int hs2_selftest_bounded_wait(void *workspace, size_t workspace_bytes, void *str
   return HS2_OK;
 }
 
+int hs2_selftest_grid_barrier(void *workspace, size_t workspace_bytes, void *stream) {
+  if (!workspace || workspace_bytes < 256) return fail(HS2_ERR_WORKSPACE, "workspace is NULL or too small");
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return fail(HS2_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  cudaError_t e = launch_grid_barrier_selftest(static_cast<uint32_t *>(workspace), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return HS2_OK;
+}
+
 int hs2_copy_peak(void *dst, const void *src, size_t bytes, void *stream) {
   if (!dst || !src || (bytes & 15) || !aligned16(dst) || !aligned16(src))
     return fail(HS2_ERR_INVALID_ARG, "copy needs 16-byte aligned pointers and a multiple of 16 bytes");
@@ -630,6 +639,22 @@ __global__ void wait_selftest_kernel(uint32_t *err) {
 
 cudaError_t launch_wait_selftest(uint32_t *err, cudaStream_t s) {
   wait_selftest_kernel<<<1, 32, 0, s>>>(err);
+  return cudaGetLastError();
+}
+
+// Two CTAs meet at the fused call's grid barrier sized for three: neither is
+// the last arrival, so both give up (after ~10 ms) and set the sticky flag's
+// grid-barrier bit, then return.
+__global__ void grid_barrier_selftest_kernel(uint32_t *err) {
+  __shared__ int flag;
+  if (!grid_barrier(err + 16, err + 32, gridDim.x + 1, &flag, 20000000LL) && threadIdx.x == 0)
+    set_error(err, kErrGridWait);
+}
+
+cudaError_t launch_grid_barrier_selftest(uint32_t *err, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(err + 16, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return e;
+  grid_barrier_selftest_kernel<<<2, 32, 0, s>>>(err);
   return cudaGetLastError();
 }
 

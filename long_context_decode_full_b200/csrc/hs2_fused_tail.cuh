@@ -56,8 +56,9 @@ struct TailStream {
 
 // Grid-wide barrier over `nblocks` co-resident CTAs.  `count` is zero between
 // calls (the last arriver returns it to zero before it releases the others by
-// bumping `gen`); the wait gives up after kSpinLimitCycles.  Whole block.
-__device__ bool grid_barrier(uint32_t *count, uint32_t *gen, uint32_t nblocks, int *flag) {
+// bumping `gen`); the wait gives up after `limit` clock cycles.  Whole block.
+__device__ bool grid_barrier(uint32_t *count, uint32_t *gen, uint32_t nblocks, int *flag,
+                             long long limit = kSpinLimitCycles) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();  // this CTA's records, logits and counters before its arrival
@@ -70,7 +71,7 @@ __device__ bool grid_barrier(uint32_t *count, uint32_t *gen, uint32_t nblocks, i
     } else {
       const long long t0 = clock64();
       while (*reinterpret_cast<volatile uint32_t *>(gen) == g0) {
-        if (clock64() - t0 > kSpinLimitCycles) {
+        if (clock64() - t0 > limit) {
           ok = false;
           break;
         }

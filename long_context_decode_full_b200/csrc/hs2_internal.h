@@ -152,6 +152,7 @@ cudaError_t launch_sparse_impl(const SparseParams &p, int kv_dtype, int64_t num_
 cudaError_t launch_copy(void *dst, const void *src, size_t bytes, int grid, cudaStream_t s);
 
 cudaError_t launch_wait_selftest(uint32_t *err, cudaStream_t s);
+cudaError_t launch_grid_barrier_selftest(uint32_t *err, cudaStream_t s);
 
 // KV Bridging append of one decode step.
 struct BridgeParams {

@@ -45,7 +45,8 @@ EXPORTS = ["hs2_full_attn_select_workspace", "hs2_full_attn_select", "hs2_full_a
            "hs2_full_attn_select_blocks", "hs2_full_attn_select_fused",
            "hs2_full_attn_select_static", "hs2_full_attn_select_static_status", "hs2_selftest_bounded_wait_static",
            "hs2_sparse_attn",
-           "hs2_workspace_status", "hs2_selftest_bounded_wait", "hs2_kv_bridge_workspace", "hs2_kv_bridge_append",
+           "hs2_workspace_status", "hs2_selftest_bounded_wait", "hs2_selftest_grid_barrier",
+           "hs2_kv_bridge_workspace", "hs2_kv_bridge_append",
            "hs2_copy_peak", "hs2_last_error", "hs2_version"]
 
 
@@ -90,6 +91,8 @@ def lib():
         L.hs2_kv_bridge_append.restype = ctypes.c_int
         L.hs2_selftest_bounded_wait.argtypes = [P, SZ, P]
         L.hs2_selftest_bounded_wait.restype = ctypes.c_int
+        L.hs2_selftest_grid_barrier.argtypes = [P, SZ, P]
+        L.hs2_selftest_grid_barrier.restype = ctypes.c_int
         L.hs2_copy_peak.argtypes = [P, P, SZ, P]
         L.hs2_copy_peak.restype = ctypes.c_int
         L.hs2_last_error.argtypes = []
@@ -348,6 +351,12 @@ def kv_bridge_append(hidden, w_k, w_v, k, v, seq_lens, page_table=None, page_siz
 def selftest_bounded_wait(workspace: torch.Tensor, stream=None):
     """Makes one bounded device wait expire on purpose (it sets the sticky flag)."""
     _check(lib().hs2_selftest_bounded_wait(_ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def selftest_grid_barrier(workspace: torch.Tensor, stream=None):
+    """Makes the fused call's grid barrier expire on purpose (two CTAs wait for
+    a third that never comes; it sets the sticky flag)."""
+    _check(lib().hs2_selftest_grid_barrier(_ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def copy_peak(dst: torch.Tensor, src: torch.Tensor, stream=None):

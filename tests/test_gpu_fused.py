@@ -95,3 +95,20 @@ def test_fused_fp32_cache_runs_separate_kernels(oracle, lib):
     out, idx = U.run_gpu(wd, fused=True)
     torch.cuda.synchronize()
     U.check_full(wd, out, idx, ora)
+
+
+def test_grid_barrier_expires_and_next_fused_call_works(lib):
+    """A grid barrier that cannot complete gives up, the status reports it
+    once, and the next fused call on the same workspace (which clears the
+    barrier's counter) still gives the separate kernels' results."""
+    w = U.to_device(synth.generate(spec(batch=2, seq_len=(2000, 3000)), seed=10))
+    ws = U.garbage_workspace(w)
+    ref_out, ref_idx = U.run_gpu(w, workspace=ws)
+    hs2.selftest_grid_barrier(ws)
+    assert hs2.workspace_status(ws) == hs2.ERR_TIMEOUT
+    assert hs2.workspace_status(ws) == 0
+    out, idx = U.run_gpu(w, workspace=ws, fused=True)
+    torch.cuda.synchronize()
+    assert hs2.workspace_status(ws) == 0
+    assert torch.equal(idx, ref_idx)
+    assert torch.equal(out, ref_out)
