@@ -23,7 +23,8 @@ FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt
                 "-I", os.path.join(ROOT, "include"), "-I", CSRC]
 SOURCES = ["hs2_api.cu", "hs2_full_attn.cu", "hs2_select.cu", "hs2_blocks.cu", "hs2_sparse.cu", "hs2_static.cu",
            "hs2_bridge.cu"]
-HEADERS = ["hs2_common.cuh", "hs2_internal.h", "hs2_warp_attn.cuh", "hs2_select_common.cuh", "hs2_fused_tail.cuh"]
+HEADERS = ["hs2_common.cuh", "hs2_internal.h", "hs2_warp_attn.cuh", "hs2_select_common.cuh", "hs2_fused_tail.cuh",
+           "hs2_tc.cuh"]
 
 
 def _stale(target: str, deps) -> bool:

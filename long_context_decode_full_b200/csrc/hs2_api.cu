@@ -203,26 +203,35 @@ bool tile_fits_pages(int tile, int page_size, bool paged) {
 // consumer warps split into ceil(G / (8 nt)) head groups and their count must
 // divide by it.  Groups of 16 and more heads take nt = 2 where a configuration
 // is built for it (each shared-memory fragment then feeds two MMAs).
-FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged, int G) {
-  static const FullMmaConfig bf16_128[] = {{4, 3, 2, 1}, {8, 3, 1, 1}, {4, 6, 1, 1}};
-  static const FullMmaConfig bf16_64[] = {{8, 6, 1, 1}, {4, 6, 1, 1}};
-  static const FullMmaConfig e4m3[] = {{8, 3, 2, 1}, {12, 4, 1, 1}, {8, 6, 1, 1}, {4, 8, 1, 1}};
+FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged, int G, int batch) {
+  static const FullMmaConfig bf16_128[] = {{4, 3, 2, 1, 0}, {8, 3, 1, 1, 0}, {4, 6, 1, 1, 0}};
+  static const FullMmaConfig bf16_64[] = {{8, 6, 1, 1, 0}, {4, 6, 1, 1, 0}};
+  static const FullMmaConfig e4m3[] = {{8, 3, 2, 1, 0}, {12, 4, 1, 1, 0}, {8, 6, 1, 1, 0}, {4, 8, 1, 1, 0}};
   // 16 heads per warp: one consumer warp per SM sub-partition with all 255
   // registers measured fastest (MQA at 256K bf16: 136 us against 144 us with
   // 8 warps x 1 slice and 154 us with 8-head warps; at 1M E4M3: 151 us
   // against 160 us with 8-head warps; 8-warp E4M3 variants spilled, 179 us)
-  static const FullMmaConfig bf16_128_wide[] = {{4, 3, 2, 2}, {8, 3, 1, 2}};
-  static const FullMmaConfig bf16_64_wide[] = {{8, 6, 1, 2}};
-  static const FullMmaConfig e4m3_wide[] = {{4, 6, 2, 2}};
+  static const FullMmaConfig bf16_128_wide[] = {{4, 3, 2, 2, 0}, {8, 3, 1, 2, 0}};
+  static const FullMmaConfig bf16_64_wide[] = {{8, 6, 1, 2, 0}};
+  static const FullMmaConfig e4m3_wide[] = {{4, 6, 2, 2, 0}};
+  // Groups of 16 or 32 heads over a bf16 cache with d 128 can run both
+  // products on tcgen05 (accumulators in tensor memory; "4,3,2,2,1" below).
+  // Measured at MQA 256K: attention 133 us against 134 us for the 16-head
+  // mma.sync warps (the logit write-back, not the tensor math, bounds it),
+  // and the step 3% slower (at 223 KB of shared memory no score CTA fits
+  // beside the attention CTA at the kernel boundary), so it is opt-in.
+  const bool tc_ok = !fp8 && D == 128 && (G == 16 || G == 32) && full_tc_smem_bytes(batch) <= 232448 &&
+                     tile_fits_pages(128, page_size, paged);
   auto heads_split = [&](const FullMmaConfig &c) { return c.ncw % ((G + 8 * c.nt - 1) / (8 * c.nt)) == 0; };
   auto fits = [&](const FullMmaConfig &c) {
     return heads_split(c) && tile_fits_pages(16 * c.ncw * c.nsl, page_size, paged);
   };
-  if (const char *env = getenv("HS2_FULL_CFG")) {  // tuning override: "ncw,nstage[,nsl[,nt]]"
-    int a = 0, b = 0, c = 1, d = 1;
-    if (sscanf(env, "%d,%d,%d,%d", &a, &b, &c, &d) >= 2 && a >= 1 && a <= 16 && b >= 1 && b <= 16 &&
-        (c == 1 || c == 2) && (d == 1 || (d == 2 && G >= 16))) {
-      const FullMmaConfig e{a, b, c, d};
+  if (const char *env = getenv("HS2_FULL_CFG")) {  // tuning override: "ncw,nstage[,nsl[,nt[,tc]]]"
+    int a = 0, b = 0, c = 1, d = 1, t = 0;
+    if (sscanf(env, "%d,%d,%d,%d,%d", &a, &b, &c, &d, &t) >= 2 && a >= 1 && a <= 16 && b >= 1 && b <= 16 &&
+        (c == 1 || c == 2) && (d == 1 || (d == 2 && G >= 16)) &&
+        (t == 0 || (t == 1 && tc_ok && a == 4 && b == 3 && c == 2 && d == 2))) {
+      const FullMmaConfig e{a, b, c, d, t};
       if (fits(e)) return e;
     }
   }
@@ -373,7 +382,7 @@ int full_attn_select_impl(const hs2_heads *q, const hs2_cache *k_cache, const hs
     p.tile = full_f32_tile();
     p.N = sms * full_f32_ctas_per_sm();
   } else {
-    cfg = pick_full_config(D, fp8, ps, paged, G);
+    cfg = pick_full_config(D, fp8, ps, paged, G, B);
     p.tile = 16 * cfg.ncw * cfg.nsl;
     p.N = sms;
   }
@@ -427,8 +436,8 @@ int full_attn_select_impl(const hs2_heads *q, const hs2_cache *k_cache, const hs
       e = launch_full_mma(p, tmk, tmv, fp8, cfg, p.N, s);
     }
     if (e == cudaErrorInvalidConfiguration)
-      return fail(HS2_ERR_UNSUPPORTED, "no %sfull-attention kernel built for ncw=%d nstage=%d nsl=%d nt=%d",
-                  fuse ? "fused " : "", cfg.ncw, cfg.nstage, cfg.nsl, cfg.nt);
+      return fail(HS2_ERR_UNSUPPORTED, "no %sfull-attention kernel built for ncw=%d nstage=%d nsl=%d nt=%d tc=%d",
+                  fuse ? "fused " : "", cfg.ncw, cfg.nstage, cfg.nsl, cfg.nt, cfg.tc);
     if (e != cudaSuccess) return cuda_fail(e, fuse ? "fused full-attention launch" : "full-attention launch");
   }
   if (mark_event) {

@@ -18,6 +18,7 @@
 // fp32 logits keep full fp32 accuracy.
 #include "hs2_fused_tail.cuh"
 #include "hs2_internal.h"
+#include "hs2_tc.cuh"
 #include "hs2_warp_attn.cuh"
 
 namespace hs2 {
@@ -30,7 +31,23 @@ struct StageMeta {
 };
 constexpr int kFirst = 1, kLast = 2, kDone = 4;
 
-template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT>
+// Shared-memory region of the tcgen05 path (after the stage metadata): the
+// query as the Q K^T product's B operand (heads x d, 128-byte swizzle), two
+// P^T buffers (rows x heads, core matrices of 8 rows x 8 heads), a reduction
+// scratch, its mbarriers and the tensor-memory base address.
+struct TcShared {
+  static constexpr int kQ = 0, kP = 8192, kPBuf = 8192, kRed = kP + 2 * kPBuf, kBar = kRed + 4 * 32 * 4;
+  static constexpr int kBytes = kBar + 8 * 8 + 16;
+  uint8_t *base;
+  __device__ uint64_t *s_full() const { return reinterpret_cast<uint64_t *>(base + kBar); }      // [2]
+  __device__ uint64_t *p_full() const { return reinterpret_cast<uint64_t *>(base + kBar) + 2; }  // [2]
+  __device__ uint64_t *o_done() const { return reinterpret_cast<uint64_t *>(base + kBar) + 4; }  // [2]
+  __device__ uint64_t *o_free() const { return reinterpret_cast<uint64_t *>(base + kBar) + 6; }
+  __device__ uint32_t *tmem() const { return reinterpret_cast<uint32_t *>(base + kBar + 64); }
+  __device__ float *red() const { return reinterpret_cast<float *>(base + kRed); }  // [4 warps][32 heads]
+};
+
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT, bool TC = false>
 struct Cfg {
   static constexpr int RPW = 16 * NSL;  // rows per consumer warp
   static constexpr int TILE = RPW * NCW;
@@ -46,7 +63,8 @@ struct Cfg {
   static constexpr int SLOT = WarpAttn<D, FP8, NSL, NT>::kSaveBytes / 4;
   static constexpr size_t OFF_BAR = (size_t)NSTAGE * STAGE;
   static constexpr size_t OFF_META = OFF_BAR + (2 * NSTAGE + 1) * 8;
-  static constexpr size_t OFF_PREFIX = OFF_META + NSTAGE * sizeof(StageMeta);
+  static constexpr size_t OFF_TC = (OFF_META + NSTAGE * sizeof(StageMeta) + 1023) / 1024 * 1024;
+  static constexpr size_t OFF_PREFIX = TC ? OFF_TC + TcShared::kBytes : OFF_META + NSTAGE * sizeof(StageMeta);
   static size_t bytes(int B) { return OFF_PREFIX + (size_t)(B + 1) * 4 + 1024; }
   static_assert(ROWB % 128 == 0, "rows are whole 128-byte panels");
   // the warps merge a segment's states inside the stage they last read
@@ -114,12 +132,268 @@ __device__ __forceinline__ int find_seq(const int32_t *prefix, int B, int Hkv, i
 template <bool FP8>
 constexpr int kProducerWarps = FP8 ? 2 : 1;
 
+
+// ------------------------------------------------------------ tcgen05 path
+// Groups of 16 or 32 query heads over a bf16 cache with d 128 (MQA-style):
+// the group is a real M x N tile, so both products of a 128-row tile run on
+// tcgen05 with the accumulators in tensor memory.  One warp issues the MMAs
+// (one elected lane): S^T = K Q^T (M = 128 rows, N = G heads, K = d; A the
+// K tile as TMA left it, K-major with the 128-byte swizzle; B the query in
+// shared memory, same layout) into one of two S^T buffers, then
+// O^T += V^T P^T (M = d, N = G, K = 128 rows; A the V tile read MN-major,
+// B the P^T buffer the softmax warps wrote) into O^T.  Four softmax warps
+// own one tensor-memory lane (one row of S^T, one dim of O^T) per thread:
+// they load the row's G logits, store them for the score pass, keep the
+// online softmax (lazy rescaling as in the warp path, decided for the whole
+// CTA by a barrier reduction), write p as bf16, and at a segment end read
+// O^T and reduce l into the record.  Each loop runs the CTA's tile count, so
+// the warps stay in step even when a bounded wait gives up.
+constexpr uint32_t kTmemCols = 128;  // S^T buffers at columns 0 and 32, O^T at 64
+constexpr int kTcThreads = 128;      // softmax threads (= tensor-memory lanes = tile rows)
+
+__device__ __forceinline__ bool bar_any(bool x) {  // OR over the 128 softmax threads (named barrier 1)
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+      "barrier.cta.red.or.pred p, 1, 128, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)x)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void bar_softmax() { asm volatile("barrier.cta.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ void st_global_v4_hint(float *addr, float a, float b, float c, float d, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d), "l"(pol)
+               : "memory");
+}
+
+template <int NSTAGE>
+__device__ void tc_mma_loop(const FullParams &p, uint8_t *smem, uint64_t *full, uint64_t *empty,
+                            const StageMeta *meta, const TcShared &ts, int64_t ntiles) {
+  using C = Cfg<128, false, 4, NSTAGE, 2, 2, true>;
+  const int lane = threadIdx.x & 31, G = p.G;
+  const uint32_t tmem = *ts.tmem();
+  const uint32_t qs = smem_u32(ts.base + TcShared::kQ);
+  const uint32_t id_qk = tc::idesc(128, G, 1, 0, 0), id_pv = tc::idesc(128, G, 1, 1, 1);
+  bool ok = true;
+  int segs = 0;             // segments begun
+  bool pv_first = false;    // the tile whose PV is next starts a segment
+  int pv_stage = 0;
+  for (int64_t it = 0; it <= ntiles; ++it) {
+    int stage = 0;
+    bool first = false;
+    if (it < ntiles) {
+      stage = (int)(it % NSTAGE);
+      ok = ok && mbar_wait(&full[stage], (uint32_t)(it / NSTAGE) & 1u);
+      const StageMeta mt = meta[stage];
+      first = (mt.flags & kFirst) != 0;
+      if (first) {
+        // the last Q K^T with the previous query is done before it is replaced
+        if (it > 0) ok = ok && mbar_wait(&ts.s_full()[(it - 1) & 1], (uint32_t)((it - 1) >> 1) & 1u);
+        if (lane < G) {  // lane h: query head h, 16 chunks of 16 B into its swizzled row
+          const uint4 *q = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p.q) +
+                                                           ((int64_t)mt.b * p.Hkv * G + (int64_t)mt.kvh * G + lane) * 128);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const uint4 v = __ldg(q + c);
+            const int panel = c >> 3, cc = c & 7;
+            *reinterpret_cast<uint4 *>(ts.base + TcShared::kQ + panel * G * 128 + lane * 128 + ((cc ^ (lane & 7)) << 4)) = v;
+          }
+        }
+        tc::fence_async_smem();
+        __syncwarp();
+      }
+      tc::fence_after();
+      if (lane == 0) {  // S^T = K Q^T into buffer it & 1
+        const uint32_t kb = smem_u32(smem) + (uint32_t)stage * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (uint32_t)(kk & 3) * 32;
+          const uint64_t a = tc::sdesc(kb + (uint32_t)(kk >> 2) * C::PANEL + off, 16, 1024, 2);
+          const uint64_t b = tc::sdesc(qs + (uint32_t)(kk >> 2) * (uint32_t)(G * 128) + off, 16, 1024, 2);
+          tc::mma_f16(tmem + 32u * (uint32_t)(it & 1), a, b, id_qk, kk > 0);
+        }
+        tc::commit(&ts.s_full()[it & 1]);
+      }
+      __syncwarp();
+    }
+    if (it >= 1) {  // O^T += V^T P^T of the previous tile
+      const int64_t j = it - 1;
+      ok = ok && mbar_wait(&ts.p_full()[j & 1], (uint32_t)(j >> 1) & 1u);
+      if (pv_first && segs > 1)  // the previous segment's O^T has been read
+        ok = ok && mbar_wait(ts.o_free(), (uint32_t)(segs - 2) & 1u);
+      tc::fence_after();
+      if (lane == 0) {
+        const uint32_t vb = smem_u32(smem) + (uint32_t)pv_stage * C::STAGE + C::KVB;
+        const uint32_t pb = smem_u32(ts.base + TcShared::kP) + (uint32_t)(j & 1) * TcShared::kPBuf;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t a = tc::sdesc(vb + (uint32_t)k * 2048, C::PANEL, 1024, 2);  // V^T: MN-major, swizzled
+          const uint64_t b = tc::sdesc(pb + (uint32_t)k * 256, 128, 2048, 0);       // P^T: MN-major, core matrices
+          tc::mma_f16(tmem + 64u, a, b, id_pv, !(pv_first && k == 0));
+        }
+        tc::commit(&empty[pv_stage]);        // the K/V stage can be refilled
+        tc::commit(&ts.o_done()[j & 1]);
+      }
+      __syncwarp();
+    }
+    if (it < ntiles) {
+      pv_first = first;
+      pv_stage = stage;
+      if (first) ++segs;
+    }
+  }
+  // the last commit covers every MMA this warp issued: they are done before
+  // the tensor memory is freed (bounded, also after an earlier expiry)
+  if (ntiles > 0) mbar_wait(&ts.o_done()[(ntiles - 1) & 1], (uint32_t)((ntiles - 1) >> 1) & 1u, 40000000LL);
+  if (!ok && lane == 0) set_error(p.ws.err, kErrFullWait);
+}
+
+template <int NSTAGE>
+__device__ void tc_softmax_loop(const FullParams &p, uint8_t *smem, uint64_t *full, const StageMeta *meta,
+                                const TcShared &ts, int64_t ntiles) {
+  using C = Cfg<128, false, 4, NSTAGE, 2, 2, true>;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, G = p.G;
+  const uint32_t tmem = *ts.tmem();
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;  // warp w reads lanes 32 w .. 32 w + 31
+  const float cl = p.c * 1.44269504088896341f;            // exp(c x) = 2^(x cl)
+  const float thr = 8.f / cl;                              // p stays <= 2^8
+  float m[32], l[32];
+  bool ok = true;
+  float *red = ts.red();
+  for (int64_t it = 0; it < ntiles; ++it) {
+    const int stage = (int)(it % NSTAGE);
+    ok = ok && mbar_wait(&full[stage], (uint32_t)(it / NSTAGE) & 1u);
+    const StageMeta mt = meta[stage];
+    const bool first = (mt.flags & kFirst) != 0, last = (mt.flags & kLast) != 0;
+    if (first) {
+#pragma unroll
+      for (int h = 0; h < 32; ++h) {
+        m[h] = -INFINITY;
+        l[h] = 0.f;
+      }
+    }
+    const int pos = mt.tile * C::TILE + tid;
+    const bool valid = pos < mt.T;
+    ok = ok && mbar_wait(&ts.s_full()[it & 1], (uint32_t)(it >> 1) & 1u);
+    tc::fence_after();
+    float x[32];
+    tc::ld32(tmem + lane_base + 32u * (uint32_t)(it & 1), x);
+    const int64_t u = (int64_t)mt.b * p.Hkv + mt.kvh;
+    if (valid) {  // raw logits for the score pass (evict-last in L2)
+      float *dst = p.ws.logits + (u * p.ustride + pos) * G;
+      const uint64_t keep = l2_policy_evict_last();
+#pragma unroll
+      for (int h4 = 0; h4 < 8; ++h4)
+        if (4 * h4 < G) st_global_v4_hint(dst + 4 * h4, x[4 * h4], x[4 * h4 + 1], x[4 * h4 + 2], x[4 * h4 + 3], keep);
+    }
+    bool grow = false;
+#pragma unroll
+    for (int h = 0; h < 32; ++h) grow = grow || (h < G && valid && x[h] > m[h] + thr);
+    if (bar_any(grow)) {
+      // the new per-head maxima over the tile's rows, for the whole CTA
+#pragma unroll
+      for (int h = 0; h < 32; ++h) {
+        if (h >= G) break;
+        const float v = warp_max(valid ? x[h] : -INFINITY);
+        if (lane == 0) red[warp * 32 + h] = v;
+      }
+      bar_softmax();
+      float alpha[32];
+#pragma unroll
+      for (int h = 0; h < 32; ++h) {
+        alpha[h] = 1.f;
+        if (h >= G) continue;
+        const float mx = fmaxf(fmaxf(red[h], red[32 + h]), fmaxf(red[64 + h], red[96 + h]));
+        const float m_new = fmaxf(m[h], mx);
+        if (m_new != m[h]) alpha[h] = m[h] == -INFINITY ? 0.f : ex2_approx((m[h] - m_new) * cl);
+        m[h] = m_new;
+        l[h] *= alpha[h];
+      }
+      bar_softmax();  // red is read before it is written again
+      if (!first) {   // O^T holds this segment's earlier tiles: rescale its columns
+        ok = ok && mbar_wait(&ts.o_done()[(it - 1) & 1], (uint32_t)((it - 1) >> 1) & 1u);
+        tc::fence_after();
+        float o[32];
+        tc::ld32(tmem + lane_base + 64u, o);
+#pragma unroll
+        for (int h = 0; h < 32; ++h) o[h] *= alpha[h];
+        tc::st32(tmem + lane_base + 64u, o);
+      }
+    }
+    // p = 2^((x - m) cl) as bf16 pairs; l sums the unrounded values
+    uint32_t pk[16];
+#pragma unroll
+    for (int h2 = 0; h2 < 16; ++h2) {
+      float p0 = 0.f, p1 = 0.f;
+      if (valid && 2 * h2 < G) {
+        p0 = ex2_approx((x[2 * h2] - m[2 * h2]) * cl);
+        p1 = ex2_approx((x[2 * h2 + 1] - m[2 * h2 + 1]) * cl);
+        l[2 * h2] += p0;
+        l[2 * h2 + 1] += p1;
+      }
+      pk[h2] = pack_bf16(p0, p1);
+    }
+    if (it >= 2)  // the P^T buffer's previous tile has been multiplied
+      ok = ok && mbar_wait(&ts.o_done()[it & 1], (uint32_t)((it - 2) >> 1) & 1u);
+    uint8_t *pbuf = ts.base + TcShared::kP + (size_t)(it & 1) * TcShared::kPBuf;
+#pragma unroll
+    for (int n8 = 0; n8 < 4; ++n8)
+      if (8 * n8 < G)
+        *reinterpret_cast<uint4 *>(pbuf + n8 * 2048 + tid * 16) =
+            make_uint4(pk[4 * n8], pk[4 * n8 + 1], pk[4 * n8 + 2], pk[4 * n8 + 3]);
+    if (!valid) {  // rows past the end may hold anything (NaN included): zero the V row
+      uint8_t *vrow = smem + (size_t)stage * C::STAGE + C::KVB + tid * 128;
+#pragma unroll
+      for (int pn = 0; pn < 2; ++pn)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(vrow + pn * C::PANEL + c * 16) = make_uint4(0, 0, 0, 0);
+    }
+    tc::fence_async_smem();
+    tc::fence_before();
+    mbar_arrive(&ts.p_full()[it & 1]);
+    if (last) {  // segment end: the record from O^T, m and the rows' l
+      ok = ok && mbar_wait(&ts.o_done()[it & 1], (uint32_t)(it >> 1) & 1u);
+      tc::fence_after();
+      float o[32];
+      tc::ld32(tmem + lane_base + 64u, o);
+#pragma unroll
+      for (int h = 0; h < 32; ++h) {
+        if (h >= G) break;
+        const float v = warp_sum(l[h]);
+        if (lane == 0) red[warp * 32 + h] = v;
+      }
+      bar_softmax();
+      if (mt.rec >= 0) {
+        float *rec = p.ws.records + (size_t)mt.rec * G * 130;
+#pragma unroll
+        for (int h = 0; h < 32; ++h)
+          if (h < G) rec[2 * G + h * 128 + tid] = o[h];
+        if (tid < G) {
+          float mh = -INFINITY;
+#pragma unroll
+          for (int h = 0; h < 32; ++h)
+            if (h == tid) mh = m[h];
+          rec[tid] = mh;
+          rec[G + tid] = (red[tid] + red[32 + tid]) + (red[64 + tid] + red[96 + tid]);
+        }
+      }
+      tc::fence_before();
+      bar_softmax();  // red and O^T are read
+      mbar_arrive(ts.o_free());
+    }
+  }
+  if (!ok) set_error(p.ws.err, kErrFullWait);
+}
+
 // The attention pass of one CTA; with FUSED the CTA then runs the score pass
 // of the selection (hs2_fused_tail.cuh) over the tiles it attended.
-template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT, bool FUSED>
+template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT, bool FUSED, bool TC = false>
 __device__ __forceinline__ void full_attn_body(const CUtensorMap &tmk, const CUtensorMap &tmv, const FullParams &p,
                                                const ScoreParams *sp) {
-  using C = Cfg<D, FP8, NCW, NSTAGE, NSL, NT>;
+  using C = Cfg<D, FP8, NCW, NSTAGE, NSL, NT, TC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -130,15 +404,26 @@ __device__ __forceinline__ void full_attn_body(const CUtensorMap &tmk, const CUt
   int32_t *prefix = reinterpret_cast<int32_t *>(smem + C::OFF_PREFIX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool producer = warp >= NCW;
-  const bool tma_role = warp == NCW;  // the other producer warp (E4M3) gathers scales
+  constexpr int kMmaWarps = TC ? 1 : 0;  // the tcgen05 path's MMA-issuing warp follows the consumers
+  const bool producer = warp >= NCW + kMmaWarps;
+  const bool tma_role = warp == NCW + kMmaWarps;  // the other producer warp (E4M3) gathers scales
+  const bool mma_role = TC && warp == NCW;
+  const TcShared ts{smem + C::OFF_TC};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&full[s], FP8 ? 33u : 1u);
-      mbar_init(&empty[s], (uint32_t)NCW);
+      mbar_init(&empty[s], TC ? 1u : (uint32_t)NCW);  // tcgen05: one commit releases a stage
     }
     mbar_init(cbar, (uint32_t)NCW);
+    if constexpr (TC) {
+      for (int k = 0; k < 2; ++k) {
+        mbar_init(&ts.s_full()[k], 1u);
+        mbar_init(&ts.p_full()[k], (uint32_t)kTcThreads);
+        mbar_init(&ts.o_done()[k], 1u);
+      }
+      mbar_init(ts.o_free(), (uint32_t)kTcThreads);
+    }
     fence_mbar_init();
   }
   if (tma_role && lane == 0) {
@@ -149,7 +434,7 @@ __device__ __forceinline__ void full_attn_body(const CUtensorMap &tmk, const CUt
   griddep_launch_dependents();  // the score kernel may be scheduled as SMs free up
   if (tma_role) {
     compute_prefix(p, prefix, C::TILE);
-  } else if (!producer) {
+  } else if (warp < NCW) {
     zero_counters(p, threadIdx.x, NCW * 32);
   }
   __syncthreads();
@@ -163,6 +448,15 @@ __device__ __forceinline__ void full_attn_body(const CUtensorMap &tmk, const CUt
   }
   const Partition part{total, p.N};
   const int64_t g0 = part.start(blockIdx.x), g1 = part.start(blockIdx.x + 1);
+  if constexpr (TC) {  // tensor memory for the S^T buffers and O^T
+    if (mma_role) {
+      tc::tmem_alloc(ts.tmem(), kTmemCols);
+      tc::tmem_relinquish();
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+  }
 
   [&]() {  // producers and consumers; both return here when their work is done
   if (producer) {
@@ -295,6 +589,12 @@ __device__ __forceinline__ void full_attn_body(const CUtensorMap &tmk, const CUt
     return;
   }
 
+  if constexpr (TC) {
+    if (mma_role) tc_mma_loop<NSTAGE>(p, smem, full, empty, meta, ts, g1 - g0);
+    else tc_softmax_loop<NSTAGE>(p, smem, full, meta, ts, g1 - g0);
+    return;
+  }
+
   // -------------------------------------------------------------- consumers
   // A warp serves HPW = 8 NT heads (NT MMA N-tiles).  With more heads than
   // that (MQA-style groups) warp w serves head group hg = w % NHG and, of
@@ -384,6 +684,12 @@ __device__ __forceinline__ void full_attn_body(const CUtensorMap &tmk, const CUt
   }
   }();
 
+  if constexpr (TC) {  // every tcgen05 operation has completed: free the tensor memory
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    if (mma_role) tc::tmem_dealloc(*ts.tmem(), kTmemCols);
+  }
   if constexpr (FUSED) {
     // every segment record and logit of the call is written once all CTAs
     // pass the barrier; the K/V stages are idle from here on
@@ -401,6 +707,22 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
     full_attn_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                          const FullParams p) {
   full_attn_body<D, FP8, NCW, NSTAGE, NSL, NT, false>(tmk, tmv, p, nullptr);
+}
+
+// Groups of 16 or 32 heads, bf16, d 128: the tcgen05 consumers (4 softmax
+// warps, 1 MMA warp) and the TMA producer.
+template <int NSTAGE>
+__global__ void __launch_bounds__(32 * (4 + 1 + 1), 1)
+    full_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                        const FullParams p) {
+  full_attn_body<128, false, 4, NSTAGE, 2, 2, false, true>(tmk, tmv, p, nullptr);
+}
+
+template <int NSTAGE>
+__global__ void __launch_bounds__(32 * (4 + 1 + 1), 1)
+    full_attn_fused_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                              const FullParams p, const ScoreParams sp) {
+  full_attn_body<128, false, 4, NSTAGE, 2, 2, true, true>(tmk, tmv, p, &sp);
 }
 
 // The fused call: attention, a grid barrier, then the score pass.  Launched
@@ -537,6 +859,17 @@ cudaError_t launch_mma_t(const FullParams &p, const CUtensorMap &tmk, const CUte
   return launch_ex(kern, dim3(grid), dim3(32 * (NCW + kProducerWarps<FP8>)), smem, s, 0, tmk, tmv, p);
 }
 
+template <int NSTAGE>
+cudaError_t launch_tc_t(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, int grid,
+                        cudaStream_t s) {
+  using C = Cfg<128, false, 4, NSTAGE, 2, 2, true>;
+  const size_t smem = C::bytes(p.B);
+  auto kern = full_attn_tc_kernel<NSTAGE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_ex(kern, dim3(grid), dim3(32 * (4 + 1 + 1)), smem, s, 0, tmk, tmv, p);
+}
+
 template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT>
 cudaError_t launch_fused_t(const FullParams &p, const ScoreParams &sp, const CUtensorMap &tmk,
                            const CUtensorMap &tmv, int grid, cudaStream_t s) {
@@ -551,8 +884,16 @@ cudaError_t launch_fused_t(const FullParams &p, const ScoreParams &sp, const CUt
 
 }  // namespace
 
+size_t full_tc_smem_bytes(int B) { return Cfg<128, false, 4, 3, 2, 2, true>::bytes(B); }
+
 cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, bool fp8,
                             const FullMmaConfig &cfg, int grid, cudaStream_t s) {
+  if (cfg.tc) {
+    if (!(p.D == 128 && !fp8 && cfg.ncw == 4 && cfg.nsl == 2 && (p.G == 16 || p.G == 32)))
+      return cudaErrorInvalidConfiguration;
+    if (cfg.nstage == 3) return launch_tc_t<3>(p, tmk, tmv, grid, s);  // (2 stages: 181 us against 133 at MQA 256K)
+    return cudaErrorInvalidConfiguration;
+  }
 #define HS2_FULL_CASE(D_, F_, W_, S_, L_, N_)                                                        \
   if (p.D == D_ && fp8 == F_ && cfg.ncw == W_ && cfg.nstage == S_ && cfg.nsl == L_ && cfg.nt == N_) \
     return launch_mma_t<D_, F_, W_, S_, L_, N_>(p, tmk, tmv, grid, s);
@@ -579,6 +920,17 @@ cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const C
 
 cudaError_t launch_full_fused(const FullParams &p, const ScoreParams &sp, const CUtensorMap &tmk,
                               const CUtensorMap &tmv, bool fp8, const FullMmaConfig &cfg, int grid, cudaStream_t s) {
+  if (cfg.tc) {
+    if (!(p.D == 128 && !fp8 && cfg.ncw == 4 && cfg.nstage == 3 && cfg.nsl == 2 && (p.G == 16 || p.G == 32)))
+      return cudaErrorInvalidConfiguration;
+    using C = Cfg<128, false, 4, 3, 2, 2, true>;
+    static_assert(kTailBufOffset + 4 * kTailChunk <= (size_t)C::STAGE * 3, "score-pass arrays fit in the stages");
+    const size_t smem = C::bytes(p.B);
+    auto kern = full_attn_fused_tc_kernel<3>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_coop(kern, dim3(grid), dim3(32 * (4 + 1 + 1)), smem, s, tmk, tmv, p, sp);
+  }
 #define HS2_FUSED_CASE(D_, F_, W_, S_, L_, N_)                                                       \
   if (p.D == D_ && fp8 == F_ && cfg.ncw == W_ && cfg.nstage == S_ && cfg.nsl == L_ && cfg.nt == N_) \
     return launch_fused_t<D_, F_, W_, S_, L_, N_>(p, sp, tmk, tmv, grid, s);

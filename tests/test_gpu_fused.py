@@ -112,3 +112,17 @@ def test_grid_barrier_expires_and_next_fused_call_works(lib):
     assert hs2.workspace_status(ws) == 0
     assert torch.equal(idx, ref_idx)
     assert torch.equal(out, ref_out)
+
+
+def test_fused_call_with_tcgen05_attention(oracle, lib, monkeypatch):
+    """The tcgen05 attention configuration (groups of 32 heads, bf16) through
+    the fused call equals its separate kernels and the oracle."""
+    monkeypatch.setenv("HS2_FULL_CFG", "4,3,2,2,1")
+    sp = spec(group=32, num_kv_heads=1, batch=3)
+    w = synth.generate(sp, seed=6, seq_lens=[4100, 90, 2600])
+    ora = U.run_oracle(oracle, w)
+    wd = U.to_device(w)
+    out_u, idx_u, out_f, idx_f = _both(wd)
+    assert torch.equal(idx_f, idx_u)
+    assert torch.equal(out_f, out_u)
+    U.check_full(wd, out_f, idx_f, ora)

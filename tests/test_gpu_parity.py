@@ -232,10 +232,10 @@ def test_every_attention_config(oracle, lib, monkeypatch, kv_dtype, cfg):
     U.check_full(wd, out, idx, ora)
 
 
-# configurations for groups of 16 and more heads (ncw, nstage, nsl, nt): nt = 2
+# configurations for groups of 16 and more heads (ncw, nstage, nsl, nt[, tc]): nt = 2
 # gives each warp 16 heads; the nt = 1 entries are the 8-head fallbacks
 WIDE_CONFIGS = {
-    "bf16": ["4,3,2,2", "8,3,1,2", "8,3,1,1", "4,3,2,1"],
+    "bf16": ["4,3,2,2,1", "4,3,2,2", "8,3,1,2", "8,3,1,1", "4,3,2,1"],
     "e4m3": ["4,6,2,2", "8,3,2,1"],
 }
 WIDE_SHAPES = {  # (spec fields, sequence lengths)
