@@ -220,7 +220,7 @@ FullMmaConfig pick_full_config(int D, bool fp8, int page_size, bool paged, int G
   // mma.sync warps (the logit write-back, not the tensor math, bounds it),
   // and the step 3% slower (at 223 KB of shared memory no score CTA fits
   // beside the attention CTA at the kernel boundary), so it is opt-in.
-  const bool tc_ok = !fp8 && D == 128 && (G == 16 || G == 32) && full_tc_smem_bytes(batch) <= 232448 &&
+  const bool tc_ok = D == 128 && (G == 16 || G == 32) && full_tc_smem_bytes(batch, fp8) <= 232448 &&
                      tile_fits_pages(128, page_size, paged);
   auto heads_split = [&](const FullMmaConfig &c) { return c.ncw % ((G + 8 * c.nt - 1) / (8 * c.nt)) == 0; };
   auto fits = [&](const FullMmaConfig &c) {

@@ -33,18 +33,27 @@ constexpr int kFirst = 1, kLast = 2, kDone = 4;
 
 // Shared-memory region of the tcgen05 path (after the stage metadata): the
 // query as the Q K^T product's B operand (heads x d, 128-byte swizzle), two
-// P^T buffers (rows x heads, core matrices of 8 rows x 8 heads), a reduction
-// scratch, its mbarriers and the tensor-memory base address.
+// P^T buffers (rows x heads, core matrices of 8 rows x 8 heads), reduction
+// scratch, the query's per-head scales (E4M3), the mbarriers and the
+// tensor-memory base address; for E4M3 caches then the f16 copies of the
+// K tile (two buffers) and of the V tile, in the bf16 tile's layout.
+template <bool FP8>
 struct TcShared {
-  static constexpr int kQ = 0, kP = 8192, kPBuf = 8192, kRed = kP + 2 * kPBuf, kBar = kRed + 4 * 32 * 4;
-  static constexpr int kBytes = kBar + 8 * 8 + 16;
+  static constexpr int kQ = 0, kP = 8192, kPBuf = 8192, kRed = kP + 2 * kPBuf, kSig = kRed + 4 * 32 * 4;
+  static constexpr int kQs = kSig + 16, kBar = kQs + 32 * 4, kEnd = kBar + 12 * 8;
+  static constexpr int kK16 = (kEnd + 1023) / 1024 * 1024, kV16 = kK16 + 2 * 32768;
+  static constexpr int kBytes = FP8 ? kV16 + 32768 : kEnd;
   uint8_t *base;
   __device__ uint64_t *s_full() const { return reinterpret_cast<uint64_t *>(base + kBar); }      // [2]
   __device__ uint64_t *p_full() const { return reinterpret_cast<uint64_t *>(base + kBar) + 2; }  // [2]
   __device__ uint64_t *o_done() const { return reinterpret_cast<uint64_t *>(base + kBar) + 4; }  // [2]
   __device__ uint64_t *o_free() const { return reinterpret_cast<uint64_t *>(base + kBar) + 6; }
-  __device__ uint32_t *tmem() const { return reinterpret_cast<uint32_t *>(base + kBar + 64); }
+  __device__ uint64_t *k_full() const { return reinterpret_cast<uint64_t *>(base + kBar) + 7; }  // [2] (E4M3)
+  __device__ uint64_t *q_ready() const { return reinterpret_cast<uint64_t *>(base + kBar) + 9; }  // (E4M3)
+  __device__ uint32_t *tmem() const { return reinterpret_cast<uint32_t *>(base + kBar + 80); }
   __device__ float *red() const { return reinterpret_cast<float *>(base + kRed); }  // [4 warps][32 heads]
+  __device__ float *sig_red() const { return reinterpret_cast<float *>(base + kSig); }  // [4 warps]
+  __device__ float *qscale() const { return reinterpret_cast<float *>(base + kQs); }   // [32 heads]
 };
 
 template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT, bool TC = false>
@@ -64,7 +73,7 @@ struct Cfg {
   static constexpr size_t OFF_BAR = (size_t)NSTAGE * STAGE;
   static constexpr size_t OFF_META = OFF_BAR + (2 * NSTAGE + 1) * 8;
   static constexpr size_t OFF_TC = (OFF_META + NSTAGE * sizeof(StageMeta) + 1023) / 1024 * 1024;
-  static constexpr size_t OFF_PREFIX = TC ? OFF_TC + TcShared::kBytes : OFF_META + NSTAGE * sizeof(StageMeta);
+  static constexpr size_t OFF_PREFIX = TC ? OFF_TC + TcShared<FP8>::kBytes : OFF_META + NSTAGE * sizeof(StageMeta);
   static size_t bytes(int B) { return OFF_PREFIX + (size_t)(B + 1) * 4 + 1024; }
   static_assert(ROWB % 128 == 0, "rows are whole 128-byte panels");
   // the warps merge a segment's states inside the stage they last read
@@ -169,14 +178,35 @@ __device__ __forceinline__ void st_global_v4_hint(float *addr, float a, float b,
                : "memory");
 }
 
-template <int NSTAGE>
+// E4M3 tile rows into the f16 tile layout (two 128-byte-swizzled panels of
+// 64 dims): thread r widens row r of the 128-row code tile at `codes`
+// (one 128-byte swizzled row per position) into `dst`.  Exact.
+__device__ __forceinline__ void tc_widen_row(const uint8_t *codes, uint8_t *dst, int r) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {  // codes 16 c .. 16 c + 15
+    const uint4 w = *reinterpret_cast<const uint4 *>(codes + r * 128 + ((c ^ (r & 7)) << 4));
+    uint32_t f[8];
+    e4m3x4_to_f16x2x2(w.x, f[0], f[1]);
+    e4m3x4_to_f16x2x2(w.y, f[2], f[3]);
+    e4m3x4_to_f16x2x2(w.z, f[4], f[5]);
+    e4m3x4_to_f16x2x2(w.w, f[6], f[7]);
+    uint8_t *panel = dst + (c >> 2) * 16384 + r * 128;
+    const int c0 = 2 * (c & 3);
+    *reinterpret_cast<uint4 *>(panel + ((c0 ^ (r & 7)) << 4)) = make_uint4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<uint4 *>(panel + (((c0 + 1) ^ (r & 7)) << 4)) = make_uint4(f[4], f[5], f[6], f[7]);
+  }
+}
+
+template <int NSTAGE, bool FP8>
 __device__ void tc_mma_loop(const FullParams &p, uint8_t *smem, uint64_t *full, uint64_t *empty,
-                            const StageMeta *meta, const TcShared &ts, int64_t ntiles) {
-  using C = Cfg<128, false, 4, NSTAGE, 2, 2, true>;
+                            const StageMeta *meta, const TcShared<FP8> &ts, int64_t ntiles) {
+  using C = Cfg<128, FP8, 4, NSTAGE, 2, 2, true>;
+  using TS = TcShared<FP8>;
   const int lane = threadIdx.x & 31, G = p.G;
   const uint32_t tmem = *ts.tmem();
-  const uint32_t qs = smem_u32(ts.base + TcShared::kQ);
-  const uint32_t id_qk = tc::idesc(128, G, 1, 0, 0), id_pv = tc::idesc(128, G, 1, 1, 1);
+  const uint32_t qs = smem_u32(ts.base + TS::kQ);
+  const uint32_t fmt = FP8 ? 0u : 1u;  // f16 (widened codes, prescaled query) or bf16
+  const uint32_t id_qk = tc::idesc(128, G, fmt, 0, 0), id_pv = tc::idesc(128, G, fmt, 1, 1);
   bool ok = true;
   int segs = 0;             // segments begun
   bool pv_first = false;    // the tile whose PV is next starts a segment
@@ -195,23 +225,51 @@ __device__ void tc_mma_loop(const FullParams &p, uint8_t *smem, uint64_t *full, 
         if (lane < G) {  // lane h: query head h, 16 chunks of 16 B into its swizzled row
           const uint4 *q = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p.q) +
                                                            ((int64_t)mt.b * p.Hkv * G + (int64_t)mt.kvh * G + lane) * 128);
+          uint4 v[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) v[c] = __ldg(q + c);
+          if constexpr (FP8) {
+            // f16 with a power-of-two prescale (exact for bf16 values), undone on the logit
+            float amax = 0.f;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[e] << 16)), fabsf(__uint_as_float(w[e] & 0xFFFF0000u))));
+            }
+            const int ex = amax > 0.f ? 14 - ilogbf(amax) : 0;
+            const float up = ldexpf(1.f, ex);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                w[e] = pack_f16(__uint_as_float(w[e] << 16) * up, __uint_as_float(w[e] & 0xFFFF0000u) * up);
+              v[c] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            ts.qscale()[lane] = ldexpf(1.f, -ex);
+          }
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const uint4 v = __ldg(q + c);
             const int panel = c >> 3, cc = c & 7;
-            *reinterpret_cast<uint4 *>(ts.base + TcShared::kQ + panel * G * 128 + lane * 128 + ((cc ^ (lane & 7)) << 4)) = v;
+            *reinterpret_cast<uint4 *>(ts.base + TS::kQ + panel * G * 128 + lane * 128 + ((cc ^ (lane & 7)) << 4)) = v[c];
           }
         }
         tc::fence_async_smem();
         __syncwarp();
+        if (FP8 && lane == 0) mbar_arrive(ts.q_ready());  // the query's scales, for the softmax warps
       }
+      if constexpr (FP8)  // the widened K tile
+        ok = ok && mbar_wait(&ts.k_full()[it & 1], (uint32_t)(it >> 1) & 1u);
       tc::fence_after();
       if (lane == 0) {  // S^T = K Q^T into buffer it & 1
-        const uint32_t kb = smem_u32(smem) + (uint32_t)stage * C::STAGE;
+        const uint32_t kb = FP8 ? smem_u32(ts.base + TS::kK16) + (uint32_t)(it & 1) * 32768u
+                                : smem_u32(smem) + (uint32_t)stage * C::STAGE;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (uint32_t)(kk & 3) * 32;
-          const uint64_t a = tc::sdesc(kb + (uint32_t)(kk >> 2) * C::PANEL + off, 16, 1024, 2);
+          const uint64_t a = tc::sdesc(kb + (uint32_t)(kk >> 2) * 16384u + off, 16, 1024, 2);
           const uint64_t b = tc::sdesc(qs + (uint32_t)(kk >> 2) * (uint32_t)(G * 128) + off, 16, 1024, 2);
           tc::mma_f16(tmem + 32u * (uint32_t)(it & 1), a, b, id_qk, kk > 0);
         }
@@ -226,15 +284,15 @@ __device__ void tc_mma_loop(const FullParams &p, uint8_t *smem, uint64_t *full, 
         ok = ok && mbar_wait(ts.o_free(), (uint32_t)(segs - 2) & 1u);
       tc::fence_after();
       if (lane == 0) {
-        const uint32_t vb = smem_u32(smem) + (uint32_t)pv_stage * C::STAGE + C::KVB;
-        const uint32_t pb = smem_u32(ts.base + TcShared::kP) + (uint32_t)(j & 1) * TcShared::kPBuf;
+        const uint32_t vb = FP8 ? smem_u32(ts.base + TS::kV16) : smem_u32(smem) + (uint32_t)pv_stage * C::STAGE + C::KVB;
+        const uint32_t pb = smem_u32(ts.base + TS::kP) + (uint32_t)(j & 1) * TS::kPBuf;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint64_t a = tc::sdesc(vb + (uint32_t)k * 2048, C::PANEL, 1024, 2);  // V^T: MN-major, swizzled
-          const uint64_t b = tc::sdesc(pb + (uint32_t)k * 256, 128, 2048, 0);       // P^T: MN-major, core matrices
+          const uint64_t a = tc::sdesc(vb + (uint32_t)k * 2048, 16384, 1024, 2);  // V^T: MN-major, swizzled
+          const uint64_t b = tc::sdesc(pb + (uint32_t)k * 256, 128, 2048, 0);    // P^T: MN-major, core matrices
           tc::mma_f16(tmem + 64u, a, b, id_pv, !(pv_first && k == 0));
         }
-        tc::commit(&empty[pv_stage]);        // the K/V stage can be refilled
+        if constexpr (!FP8) tc::commit(&empty[pv_stage]);  // the K/V stage can be refilled
         tc::commit(&ts.o_done()[j & 1]);
       }
       __syncwarp();
@@ -251,18 +309,31 @@ __device__ void tc_mma_loop(const FullParams &p, uint8_t *smem, uint64_t *full, 
   if (!ok && lane == 0) set_error(p.ws.err, kErrFullWait);
 }
 
-template <int NSTAGE>
-__device__ void tc_softmax_loop(const FullParams &p, uint8_t *smem, uint64_t *full, const StageMeta *meta,
-                                const TcShared &ts, int64_t ntiles) {
-  using C = Cfg<128, false, 4, NSTAGE, 2, 2, true>;
+template <int NSTAGE, bool FP8>
+__device__ void tc_softmax_loop(const FullParams &p, uint8_t *smem, uint64_t *full, uint64_t *empty,
+                                const StageMeta *meta, const TcShared<FP8> &ts, int64_t ntiles) {
+  using C = Cfg<128, FP8, 4, NSTAGE, 2, 2, true>;
+  using TS = TcShared<FP8>;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, G = p.G;
   const uint32_t tmem = *ts.tmem();
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;  // warp w reads lanes 32 w .. 32 w + 31
   const float cl = p.c * 1.44269504088896341f;            // exp(c x) = 2^(x cl)
   const float thr = 8.f / cl;                              // p stays <= 2^8
-  float m[32], l[32];
+  float m[32], l[32], qsc[32];
+  float sig = 0.f, inv_sig = 0.f;                          // E4M3: running max of the V scale
   bool ok = true;
+  int segs = 0;
   float *red = ts.red();
+#pragma unroll
+  for (int h = 0; h < 32; ++h) qsc[h] = 1.f;
+  if constexpr (FP8) {  // the first tile's K codes, widened
+    if (ntiles > 0) {
+      ok = ok && mbar_wait(&full[0], 0u);
+      tc_widen_row(smem, ts.base + TS::kK16, tid);
+      tc::fence_async_smem();
+      mbar_arrive(&ts.k_full()[0]);
+    }
+  }
   for (int64_t it = 0; it < ntiles; ++it) {
     const int stage = (int)(it % NSTAGE);
     ok = ok && mbar_wait(&full[stage], (uint32_t)(it / NSTAGE) & 1u);
@@ -274,13 +345,40 @@ __device__ void tc_softmax_loop(const FullParams &p, uint8_t *smem, uint64_t *fu
         m[h] = -INFINITY;
         l[h] = 0.f;
       }
+      sig = 0.f;
+      inv_sig = 0.f;
+      if constexpr (FP8) {  // the query's per-head scales
+        ok = ok && mbar_wait(ts.q_ready(), (uint32_t)segs & 1u);
+#pragma unroll
+        for (int h = 0; h < 32; ++h) qsc[h] = h < G ? ts.qscale()[h] : 1.f;
+      }
+      ++segs;
+    }
+    if constexpr (FP8) {  // the next tile's K codes, widened, while this tile's S^T is computed
+      if (it + 1 < ntiles) {
+        const int st1 = (int)((it + 1) % NSTAGE);
+        ok = ok && mbar_wait(&full[st1], (uint32_t)((it + 1) / NSTAGE) & 1u);
+        tc_widen_row(smem + (size_t)st1 * C::STAGE, ts.base + TS::kK16 + (size_t)((it + 1) & 1) * 32768, tid);
+        tc::fence_async_smem();
+        mbar_arrive(&ts.k_full()[(it + 1) & 1]);
+      }
     }
     const int pos = mt.tile * C::TILE + tid;
     const bool valid = pos < mt.T;
+    float kr = 1.f, vr = 0.f;  // E4M3: this row's K and V scales
+    if constexpr (FP8) {
+      const float *sc = reinterpret_cast<const float *>(smem + (size_t)stage * C::STAGE + 2 * C::KVB);
+      kr = valid ? sc[tid] : 0.f;
+      vr = valid ? sc[C::TILE + tid] : 0.f;
+    }
     ok = ok && mbar_wait(&ts.s_full()[it & 1], (uint32_t)(it >> 1) & 1u);
     tc::fence_after();
     float x[32];
     tc::ld32(tmem + lane_base + 32u * (uint32_t)(it & 1), x);
+    if constexpr (FP8) {
+#pragma unroll
+      for (int h = 0; h < 32; ++h) x[h] *= kr * qsc[h];
+    }
     const int64_t u = (int64_t)mt.b * p.Hkv + mt.kvh;
     if (valid) {  // raw logits for the score pass (evict-last in L2)
       float *dst = p.ws.logits + (u * p.ustride + pos) * G;
@@ -289,28 +387,44 @@ __device__ void tc_softmax_loop(const FullParams &p, uint8_t *smem, uint64_t *fu
       for (int h4 = 0; h4 < 8; ++h4)
         if (4 * h4 < G) st_global_v4_hint(dst + 4 * h4, x[4 * h4], x[4 * h4 + 1], x[4 * h4 + 2], x[4 * h4 + 3], keep);
     }
-    bool grow = false;
+    bool grow = FP8 && vr > sig;
 #pragma unroll
     for (int h = 0; h < 32; ++h) grow = grow || (h < G && valid && x[h] > m[h] + thr);
     if (bar_any(grow)) {
-      // the new per-head maxima over the tile's rows, for the whole CTA
+      // the new per-head maxima (and E4M3: the V scales' maximum) over the tile, for the whole CTA
 #pragma unroll
       for (int h = 0; h < 32; ++h) {
         if (h >= G) break;
         const float v = warp_max(valid ? x[h] : -INFINITY);
         if (lane == 0) red[warp * 32 + h] = v;
       }
+      if constexpr (FP8) {
+        const float v = warp_max(vr);
+        if (lane == 0) ts.sig_red()[warp] = v;
+      }
       bar_softmax();
-      float alpha[32];
+      float beta = 1.f;
+      if constexpr (FP8) {
+        const float smax = fmaxf(fmaxf(ts.sig_red()[0], ts.sig_red()[1]), fmaxf(ts.sig_red()[2], ts.sig_red()[3]));
+        if (smax > sig) {
+          const float inv_new = __frcp_rn(smax);
+          beta = sig * inv_new;
+          sig = smax;
+          inv_sig = inv_new;
+        }
+      }
+      float f[32];
 #pragma unroll
       for (int h = 0; h < 32; ++h) {
-        alpha[h] = 1.f;
-        if (h >= G) continue;
-        const float mx = fmaxf(fmaxf(red[h], red[32 + h]), fmaxf(red[64 + h], red[96 + h]));
-        const float m_new = fmaxf(m[h], mx);
-        if (m_new != m[h]) alpha[h] = m[h] == -INFINITY ? 0.f : ex2_approx((m[h] - m_new) * cl);
-        m[h] = m_new;
-        l[h] *= alpha[h];
+        float alpha = 1.f;
+        if (h < G) {
+          const float mx = fmaxf(fmaxf(red[h], red[32 + h]), fmaxf(red[64 + h], red[96 + h]));
+          const float m_new = fmaxf(m[h], mx);
+          if (m_new != m[h]) alpha = m[h] == -INFINITY ? 0.f : ex2_approx((m[h] - m_new) * cl);
+          m[h] = m_new;
+          l[h] *= alpha;
+        }
+        f[h] = alpha * beta;
       }
       bar_softmax();  // red is read before it is written again
       if (!first) {   // O^T holds this segment's earlier tiles: rescale its columns
@@ -319,11 +433,13 @@ __device__ void tc_softmax_loop(const FullParams &p, uint8_t *smem, uint64_t *fu
         float o[32];
         tc::ld32(tmem + lane_base + 64u, o);
 #pragma unroll
-        for (int h = 0; h < 32; ++h) o[h] *= alpha[h];
+        for (int h = 0; h < 32; ++h) o[h] *= f[h];
         tc::st32(tmem + lane_base + 64u, o);
       }
     }
-    // p = 2^((x - m) cl) as bf16 pairs; l sums the unrounded values
+    // p = 2^((x - m) cl); l sums it; the P^T operand carries p (bf16), or
+    // p times the row's V scale over sig (f16, E4M3)
+    const float w8 = FP8 ? vr * inv_sig : 1.f;
     uint32_t pk[16];
 #pragma unroll
     for (int h2 = 0; h2 < 16; ++h2) {
@@ -334,25 +450,40 @@ __device__ void tc_softmax_loop(const FullParams &p, uint8_t *smem, uint64_t *fu
         l[2 * h2] += p0;
         l[2 * h2 + 1] += p1;
       }
-      pk[h2] = pack_bf16(p0, p1);
+      pk[h2] = FP8 ? pack_f16(p0 * w8, p1 * w8) : pack_bf16(p0, p1);
     }
-    if (it >= 2)  // the P^T buffer's previous tile has been multiplied
-      ok = ok && mbar_wait(&ts.o_done()[it & 1], (uint32_t)((it - 2) >> 1) & 1u);
-    uint8_t *pbuf = ts.base + TcShared::kP + (size_t)(it & 1) * TcShared::kPBuf;
+    if (FP8 ? it >= 1 : it >= 2)  // E4M3: the V copy and P^T buffers' previous tile has been multiplied
+      ok = ok && mbar_wait(&ts.o_done()[FP8 ? (it - 1) & 1 : it & 1],
+                           (uint32_t)((FP8 ? it - 1 : it - 2) >> 1) & 1u);
+    if constexpr (FP8) {  // this tile's V codes, widened (zeros past the end), then the stage is free
+      uint8_t *v16 = ts.base + TS::kV16;
+      if (valid) {
+        tc_widen_row(smem + (size_t)stage * C::STAGE + C::KVB, v16, tid);
+      } else {
+#pragma unroll
+        for (int pn = 0; pn < 2; ++pn)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(v16 + pn * 16384 + tid * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    uint8_t *pbuf = ts.base + TS::kP + (size_t)(it & 1) * TS::kPBuf;
 #pragma unroll
     for (int n8 = 0; n8 < 4; ++n8)
       if (8 * n8 < G)
         *reinterpret_cast<uint4 *>(pbuf + n8 * 2048 + tid * 16) =
             make_uint4(pk[4 * n8], pk[4 * n8 + 1], pk[4 * n8 + 2], pk[4 * n8 + 3]);
-    if (!valid) {  // rows past the end may hold anything (NaN included): zero the V row
-      uint8_t *vrow = smem + (size_t)stage * C::STAGE + C::KVB + tid * 128;
+    if constexpr (!FP8) {
+      if (!valid) {  // rows past the end may hold anything (NaN included): zero the V row
+        uint8_t *vrow = smem + (size_t)stage * C::STAGE + C::KVB + tid * 128;
 #pragma unroll
-      for (int pn = 0; pn < 2; ++pn)
+        for (int pn = 0; pn < 2; ++pn)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(vrow + pn * C::PANEL + c * 16) = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(vrow + pn * C::PANEL + c * 16) = make_uint4(0, 0, 0, 0);
+      }
     }
     tc::fence_async_smem();
     tc::fence_before();
+    if constexpr (FP8) mbar_arrive(&empty[stage]);  // codes and scales of this tile are consumed
     mbar_arrive(&ts.p_full()[it & 1]);
     if (last) {  // segment end: the record from O^T, m and the rows' l
       ok = ok && mbar_wait(&ts.o_done()[it & 1], (uint32_t)(it >> 1) & 1u);
@@ -368,9 +499,10 @@ __device__ void tc_softmax_loop(const FullParams &p, uint8_t *smem, uint64_t *fu
       bar_softmax();
       if (mt.rec >= 0) {
         float *rec = p.ws.records + (size_t)mt.rec * G * 130;
+        const float os = FP8 ? sig : 1.f;
 #pragma unroll
         for (int h = 0; h < 32; ++h)
-          if (h < G) rec[2 * G + h * 128 + tid] = o[h];
+          if (h < G) rec[2 * G + h * 128 + tid] = o[h] * os;
         if (tid < G) {
           float mh = -INFINITY;
 #pragma unroll
@@ -408,12 +540,13 @@ __device__ __forceinline__ void full_attn_body(const CUtensorMap &tmk, const CUt
   const bool producer = warp >= NCW + kMmaWarps;
   const bool tma_role = warp == NCW + kMmaWarps;  // the other producer warp (E4M3) gathers scales
   const bool mma_role = TC && warp == NCW;
-  const TcShared ts{smem + C::OFF_TC};
+  const TcShared<FP8> ts{smem + C::OFF_TC};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&full[s], FP8 ? 33u : 1u);
-      mbar_init(&empty[s], TC ? 1u : (uint32_t)NCW);  // tcgen05: one commit releases a stage
+      // tcgen05: one commit releases a stage (E4M3: the softmax threads, once its codes are widened)
+      mbar_init(&empty[s], TC ? (FP8 ? (uint32_t)kTcThreads : 1u) : (uint32_t)NCW);
     }
     mbar_init(cbar, (uint32_t)NCW);
     if constexpr (TC) {
@@ -423,6 +556,8 @@ __device__ __forceinline__ void full_attn_body(const CUtensorMap &tmk, const CUt
         mbar_init(&ts.o_done()[k], 1u);
       }
       mbar_init(ts.o_free(), (uint32_t)kTcThreads);
+      for (int k = 0; k < 2; ++k) mbar_init(&ts.k_full()[k], (uint32_t)kTcThreads);
+      mbar_init(ts.q_ready(), 1u);
     }
     fence_mbar_init();
   }
@@ -590,8 +725,8 @@ __device__ __forceinline__ void full_attn_body(const CUtensorMap &tmk, const CUt
   }
 
   if constexpr (TC) {
-    if (mma_role) tc_mma_loop<NSTAGE>(p, smem, full, empty, meta, ts, g1 - g0);
-    else tc_softmax_loop<NSTAGE>(p, smem, full, meta, ts, g1 - g0);
+    if (mma_role) tc_mma_loop<NSTAGE, FP8>(p, smem, full, empty, meta, ts, g1 - g0);
+    else tc_softmax_loop<NSTAGE, FP8>(p, smem, full, empty, meta, ts, g1 - g0);
     return;
   }
 
@@ -709,13 +844,13 @@ __global__ void __launch_bounds__(32 * (NCW + kProducerWarps<FP8>), 1)
   full_attn_body<D, FP8, NCW, NSTAGE, NSL, NT, false>(tmk, tmv, p, nullptr);
 }
 
-// Groups of 16 or 32 heads, bf16, d 128: the tcgen05 consumers (4 softmax
-// warps, 1 MMA warp) and the TMA producer.
-template <int NSTAGE>
-__global__ void __launch_bounds__(32 * (4 + 1 + 1), 1)
+// Groups of 16 or 32 heads, d 128: the tcgen05 consumers (4 softmax warps,
+// 1 MMA warp) and the producers (TMA; E4M3: and the scale gathers).
+template <int NSTAGE, bool FP8>
+__global__ void __launch_bounds__(32 * (4 + 1 + kProducerWarps<FP8>), 1)
     full_attn_tc_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                         const FullParams p) {
-  full_attn_body<128, false, 4, NSTAGE, 2, 2, false, true>(tmk, tmv, p, nullptr);
+  full_attn_body<128, FP8, 4, NSTAGE, 2, 2, false, true>(tmk, tmv, p, nullptr);
 }
 
 template <int NSTAGE>
@@ -859,15 +994,15 @@ cudaError_t launch_mma_t(const FullParams &p, const CUtensorMap &tmk, const CUte
   return launch_ex(kern, dim3(grid), dim3(32 * (NCW + kProducerWarps<FP8>)), smem, s, 0, tmk, tmv, p);
 }
 
-template <int NSTAGE>
+template <int NSTAGE, bool FP8>
 cudaError_t launch_tc_t(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, int grid,
                         cudaStream_t s) {
-  using C = Cfg<128, false, 4, NSTAGE, 2, 2, true>;
+  using C = Cfg<128, FP8, 4, NSTAGE, 2, 2, true>;
   const size_t smem = C::bytes(p.B);
-  auto kern = full_attn_tc_kernel<NSTAGE>;
+  auto kern = full_attn_tc_kernel<NSTAGE, FP8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_ex(kern, dim3(grid), dim3(32 * (4 + 1 + 1)), smem, s, 0, tmk, tmv, p);
+  return launch_ex(kern, dim3(grid), dim3(32 * (4 + 1 + kProducerWarps<FP8>)), smem, s, 0, tmk, tmv, p);
 }
 
 template <int D, bool FP8, int NCW, int NSTAGE, int NSL, int NT>
@@ -884,15 +1019,16 @@ cudaError_t launch_fused_t(const FullParams &p, const ScoreParams &sp, const CUt
 
 }  // namespace
 
-size_t full_tc_smem_bytes(int B) { return Cfg<128, false, 4, 3, 2, 2, true>::bytes(B); }
+size_t full_tc_smem_bytes(int B, bool fp8) {
+  return fp8 ? Cfg<128, true, 4, 3, 2, 2, true>::bytes(B) : Cfg<128, false, 4, 3, 2, 2, true>::bytes(B);
+}
 
 cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const CUtensorMap &tmv, bool fp8,
                             const FullMmaConfig &cfg, int grid, cudaStream_t s) {
-  if (cfg.tc) {
-    if (!(p.D == 128 && !fp8 && cfg.ncw == 4 && cfg.nsl == 2 && (p.G == 16 || p.G == 32)))
+  if (cfg.tc) {  // 3 stages (bf16 with 2: 181 us against 133 at MQA 256K)
+    if (!(p.D == 128 && cfg.ncw == 4 && cfg.nstage == 3 && cfg.nsl == 2 && (p.G == 16 || p.G == 32)))
       return cudaErrorInvalidConfiguration;
-    if (cfg.nstage == 3) return launch_tc_t<3>(p, tmk, tmv, grid, s);  // (2 stages: 181 us against 133 at MQA 256K)
-    return cudaErrorInvalidConfiguration;
+    return fp8 ? launch_tc_t<3, true>(p, tmk, tmv, grid, s) : launch_tc_t<3, false>(p, tmk, tmv, grid, s);
   }
 #define HS2_FULL_CASE(D_, F_, W_, S_, L_, N_)                                                        \
   if (p.D == D_ && fp8 == F_ && cfg.ncw == W_ && cfg.nstage == S_ && cfg.nsl == L_ && cfg.nt == N_) \
@@ -920,7 +1056,7 @@ cudaError_t launch_full_mma(const FullParams &p, const CUtensorMap &tmk, const C
 
 cudaError_t launch_full_fused(const FullParams &p, const ScoreParams &sp, const CUtensorMap &tmk,
                               const CUtensorMap &tmv, bool fp8, const FullMmaConfig &cfg, int grid, cudaStream_t s) {
-  if (cfg.tc) {
+  if (cfg.tc) {  // (bf16 only)
     if (!(p.D == 128 && !fp8 && cfg.ncw == 4 && cfg.nstage == 3 && cfg.nsl == 2 && (p.G == 16 || p.G == 32)))
       return cudaErrorInvalidConfiguration;
     using C = Cfg<128, false, 4, 3, 2, 2, true>;

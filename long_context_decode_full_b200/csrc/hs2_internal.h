@@ -73,10 +73,10 @@ struct FullMmaConfig {
   int nstage;  // pipeline stages
   int nsl;     // 16-row slices per warp and tile (tile = 16 * ncw * nsl positions)
   int nt;      // 8-head MMA N-tiles per warp (1, or 2 for groups of 16 and more heads)
-  int tc;      // 1: tcgen05 consumers (groups of 16 or 32 heads, bf16, d 128; ncw 4, nstage 3, nsl 2, nt 2)
+  int tc;      // 1: tcgen05 consumers (groups of 16 or 32 heads, d 128; ncw 4, nstage 3, nsl 2, nt 2)
 };
 // Shared memory of the tcgen05 attention kernel for a batch of B sequences.
-size_t full_tc_smem_bytes(int B);
+size_t full_tc_smem_bytes(int B, bool fp8);
 
 // Launch with programmatic stream serialization (unless HS2_PDL=0) and an
 // optional 1-D cluster.

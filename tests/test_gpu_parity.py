@@ -236,7 +236,7 @@ def test_every_attention_config(oracle, lib, monkeypatch, kv_dtype, cfg):
 # gives each warp 16 heads; the nt = 1 entries are the 8-head fallbacks
 WIDE_CONFIGS = {
     "bf16": ["4,3,2,2,1", "4,3,2,2", "8,3,1,2", "8,3,1,1", "4,3,2,1"],
-    "e4m3": ["4,6,2,2", "8,3,2,1"],
+    "e4m3": ["4,3,2,2,1", "4,6,2,2", "8,3,2,1"],
 }
 WIDE_SHAPES = {  # (spec fields, sequence lengths)
     "mqa_g32": (dict(group=32, num_kv_heads=1, batch=3), [90, 4100, 1300]),
