@@ -492,28 +492,41 @@ def run_gpu(args, rank, world, local):
     sel_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(KB))
     marked_ms = statistics.mean(ev[i][0].elapsed_time(ev[i + 1][0]) for i in range(KB - 1))
 
-    # e2e: queries in from pinned host memory, outputs + index list back, every step
-    q_host = [w.q_full.cpu().pin_memory()] + [w.q_sparse[l].cpu().pin_memory() for l in range(s.sparse_layers)]
-    lens_host = w.seq_lens.cpu().pin_memory()
-    outs_host = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
-    idx_host = torch.empty_like(idx, device="cpu").pin_memory()
-    q_dev = [torch.empty_like(x, device=dev) for x in q_host]
-    lens_dev = torch.empty_like(lens_host, device=dev)
-    h2d = sum(x.numel() * x.element_size() for x in q_host) + lens_host.numel() * 4
-    d2h = sum(x.numel() * x.element_size() for x in outs_host) + idx_host.numel() * 4
+    # e2e: queries in from pinned host memory, outputs + index list back, every step.
+    # The step's inputs travel in one pinned buffer and its results in one device
+    # buffer (one copy each way); the kernels read and write views of them.
+    def packed(tensors, device):
+        offs, n = [], 0
+        for t in tensors:
+            offs.append(n)
+            n += (t.numel() * t.element_size() + 255) // 256 * 256
+        buf = torch.empty(n, dtype=torch.uint8, device=device)
+        views = [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape) for o, t in zip(offs, tensors)]
+        return buf, views
+
+    ins = [w.q_full] + [w.q_sparse[l] for l in range(s.sparse_layers)] + [w.seq_lens]
+    in_dev, in_views = packed(ins, dev)
+    in_host = torch.empty_like(in_dev, device="cpu").pin_memory()
+    off = 0
+    for t in ins:  # the inputs laid out in the pinned buffer as in the device one
+        nb = t.numel() * t.element_size()
+        in_host[off:off + nb].view(t.dtype).view(t.shape).copy_(t.cpu())
+        off += (nb + 255) // 256 * 256
+    q_dev, lens_dev = in_views[:-1], in_views[-1]
+    out_dev, out_views = packed(outs + [idx], dev)
+    outs_e2e, idx_e2e = out_views[:-1], out_views[-1]
+    out_host = torch.empty_like(out_dev, device="cpu").pin_memory()
+    h2d = in_host.numel()
+    d2h = out_host.numel()
     K2 = max(3, min(K, args.e2e_steps))
 
     def e2e_step():
-        for a, b in zip(q_dev, q_host):
-            a.copy_(b, non_blocking=True)
-        lens_dev.copy_(lens_host, non_blocking=True)
+        in_dev.copy_(in_host, non_blocking=True)
         hs2.full_attn_select(q_dev[0], w.k, w.v, lens_dev, w.page_table, w.page_size, s.window, s.k_global,
-                             w.k_scale, w.v_scale, out=outs[0], idx_out=idx, workspace=ws, fused=args.fused)
+                             w.k_scale, w.v_scale, out=outs_e2e[0], idx_out=idx_e2e, workspace=ws, fused=args.fused)
         for l in range(s.sparse_layers):
-            hs2.sparse_attn(q_dev[1 + l], w.k, w.v, idx, w.k_scale, w.v_scale, w.page_size, out=outs[1 + l])
-        for a, b in zip(outs_host, outs):
-            a.copy_(b, non_blocking=True)
-        idx_host.copy_(idx, non_blocking=True)
+            hs2.sparse_attn(q_dev[1 + l], w.k, w.v, idx_e2e, w.k_scale, w.v_scale, w.page_size, out=outs_e2e[1 + l])
+        out_host.copy_(out_dev, non_blocking=True)
         torch.cuda.current_stream().synchronize()
 
     for _ in range(3):
@@ -565,7 +578,8 @@ def run_gpu(args, rank, world, local):
         "nominal_hbm_gbs": NOMINAL_HBM_GBS,
         "e2e": {"value": world * 1000.0 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K2,
-                "what": "queries copied in from pinned host memory, outputs and index list copied out and synced, "
+                "what": "queries and lengths copied in from one pinned host buffer, outputs and index list copied "
+                        "out as one buffer and synced, "
                         "every step; the KV cache stays resident"},
         "gpu_launches": K * ((3 if args.fused else 4) + s.sparse_layers),
         "clocks": clk,
