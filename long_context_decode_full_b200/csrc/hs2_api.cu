@@ -686,6 +686,33 @@ __global__ void __launch_bounds__(256) copy_kernel(uint4 *__restrict__ dst, cons
 
 int set_last_error(int code, const char *msg) { return fail(code, "%s", msg); }
 
+namespace {
+struct SmemAttr {
+  const void *kern;
+  int dev, bytes;
+};
+std::mutex g_attr_mu;
+SmemAttr g_attr[512];
+int g_nattr = 0;
+}  // namespace
+
+cudaError_t set_smem_once(const void *kern, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  for (int i = 0; i < g_nattr; ++i) {
+    if (g_attr[i].kern != kern || g_attr[i].dev != dev) continue;
+    if (g_attr[i].bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) g_attr[i].bytes = bytes;
+    return e;
+  }
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && g_nattr < 512) g_attr[g_nattr++] = SmemAttr{kern, dev, bytes};
+  return e;
+}
+
 bool pdl_enabled() {
   static const bool on = [] {
     const char *env = getenv("HS2_PDL");

@@ -989,7 +989,7 @@ cudaError_t launch_mma_t(const FullParams &p, const CUtensorMap &tmk, const CUte
   using C = Cfg<D, FP8, NCW, NSTAGE, NSL, NT>;
   const size_t smem = C::bytes(p.B);
   auto kern = full_attn_mma_kernel<D, FP8, NCW, NSTAGE, NSL, NT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   return launch_ex(kern, dim3(grid), dim3(32 * (NCW + kProducerWarps<FP8>)), smem, s, 0, tmk, tmv, p);
 }
@@ -1000,7 +1000,7 @@ cudaError_t launch_tc_t(const FullParams &p, const CUtensorMap &tmk, const CUten
   using C = Cfg<128, FP8, 4, NSTAGE, 2, 2, true>;
   const size_t smem = C::bytes(p.B);
   auto kern = full_attn_tc_kernel<NSTAGE, FP8>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   return launch_ex(kern, dim3(grid), dim3(32 * (4 + 1 + kProducerWarps<FP8>)), smem, s, 0, tmk, tmv, p);
 }
@@ -1012,7 +1012,7 @@ cudaError_t launch_fused_t(const FullParams &p, const ScoreParams &sp, const CUt
   static_assert(kTailBufOffset + 4 * kTailChunk <= (size_t)C::STAGE * NSTAGE, "score-pass arrays fit in the stages");
   const size_t smem = C::bytes(p.B);
   auto kern = full_attn_fused_kernel<D, FP8, NCW, NSTAGE, NSL, NT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   return launch_coop(kern, dim3(grid), dim3(32 * (NCW + kProducerWarps<FP8>)), smem, s, tmk, tmv, p, sp);
 }
@@ -1063,7 +1063,7 @@ cudaError_t launch_full_fused(const FullParams &p, const ScoreParams &sp, const 
     static_assert(kTailBufOffset + 4 * kTailChunk <= (size_t)C::STAGE * 3, "score-pass arrays fit in the stages");
     const size_t smem = C::bytes(p.B);
     auto kern = full_attn_fused_tc_kernel<3>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), (int)smem);
     if (e != cudaSuccess) return e;
     return launch_coop(kern, dim3(grid), dim3(32 * (4 + 1 + 1)), smem, s, tmk, tmv, p, sp);
   }
@@ -1087,11 +1087,11 @@ cudaError_t launch_full_f32(const FullParams &p, int grid, cudaStream_t s) {
   const size_t smem = (size_t)(2 * kF32Tile * (p.D + 1) + 8 * p.D) * 4 + (size_t)(p.B + 1) * 4;
   cudaError_t e;
   if (p.D == 64) {
-    e = cudaFuncSetAttribute(full_attn_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = set_smem_once(reinterpret_cast<const void *>(full_attn_f32_kernel<64>), (int)smem);
     if (e != cudaSuccess) return e;
     return launch_ex(full_attn_f32_kernel<64>, dim3(grid), dim3(32 * kF32Warps), smem, s, 0, p);
   } else if (p.D == 128) {
-    e = cudaFuncSetAttribute(full_attn_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = set_smem_once(reinterpret_cast<const void *>(full_attn_f32_kernel<128>), (int)smem);
     if (e != cudaSuccess) return e;
     return launch_ex(full_attn_f32_kernel<128>, dim3(grid), dim3(32 * kF32Warps), smem, s, 0, p);
   }

@@ -78,6 +78,11 @@ struct FullMmaConfig {
 // Shared memory of the tcgen05 attention kernel for a batch of B sequences.
 size_t full_tc_smem_bytes(int B, bool fp8);
 
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel and
+// device (again only to raise it): the attribute call costs host time on
+// every launch otherwise.
+cudaError_t set_smem_once(const void *kern, int bytes);
+
 // Launch with programmatic stream serialization (unless HS2_PDL=0) and an
 // optional 1-D cluster.
 bool pdl_enabled();

@@ -567,7 +567,7 @@ cudaError_t launch_select_after_score(const ScoreParams &p, cudaStream_t s) {
   cudaError_t e = launch_ex(filter_kernel, dim3(fchunks, p.Hkv, p.B), dim3(kScoreThreads), 0, s, 0, p);
   if (e != cudaSuccess) return e;
   const size_t smem = final_smem_bytes(p.nsub);
-  e = cudaFuncSetAttribute(final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = set_smem_once(reinterpret_cast<const void *>(final_kernel), (int)smem);
   if (e != cudaSuccess) return e;
   return launch_ex(final_kernel, dim3(p.Hkv, p.B), dim3(kFinalThreads), smem, s, 0, p);
 }

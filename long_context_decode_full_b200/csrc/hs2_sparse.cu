@@ -300,7 +300,7 @@ cudaError_t launch_mma_t(const SparseParams &p, int64_t num_slots, cudaStream_t 
   using C = SCfg<D, FP8, NW, NSL>;
   const size_t smem = C::bytes(p.G < 8 ? p.G : 8, p.splits, p.rows_per_cta, p.nbuf);
   auto kern = sparse_mma_kernel<D, FP8, NW, NSL>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   if (p.splits > 8) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -325,11 +325,11 @@ cudaError_t launch_sparse_impl(const SparseParams &p, int kv_dtype, int64_t num_
     const size_t smem = (size_t)(2 * kSpF32Tile * (p.D + 1) + 8 * p.D) * 4 + kSpF32Tile * 4;
     cudaError_t e;
     if (p.D == 64) {
-      e = cudaFuncSetAttribute(sparse_f32_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      e = set_smem_once(reinterpret_cast<const void *>(sparse_f32_kernel<64>), (int)smem);
       if (e != cudaSuccess) return e;
       return launch_ex(sparse_f32_kernel<64>, dim3(p.Hkv, p.B), dim3(32 * kSpF32Warps), smem, s, 0, p, num_slots);
     }
-    e = cudaFuncSetAttribute(sparse_f32_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = set_smem_once(reinterpret_cast<const void *>(sparse_f32_kernel<128>), (int)smem);
     if (e != cudaSuccess) return e;
     return launch_ex(sparse_f32_kernel<128>, dim3(p.Hkv, p.B), dim3(32 * kSpF32Warps), smem, s, 0, p, num_slots);
   }
