@@ -79,6 +79,46 @@ int encode_cache_map(CUtensorMap *map, const hs2_cache *c, int box_rows) {
   return HS2_OK;
 }
 
+// The tensor map of a cache depends only on its pointer, shape, element type
+// and box: the last few are kept, so a decode loop encodes them once.
+struct MapKey {
+  const void *data;
+  int dtype, heads, dim, box, dev;
+  int64_t slots;
+  bool operator==(const MapKey &o) const {
+    return data == o.data && dtype == o.dtype && heads == o.heads && dim == o.dim && box == o.box && dev == o.dev &&
+           slots == o.slots;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  bool used;
+};
+std::mutex g_map_mu;
+MapEntry g_maps[16];
+int g_map_next = 0;
+
+int cache_map(CUtensorMap *map, const hs2_cache *c, int box_rows) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  const MapKey key{c->data, (int)c->dtype, c->num_kv_heads, c->head_dim, box_rows, dev, c->num_slots};
+  {
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    for (const MapEntry &e : g_maps)
+      if (e.used && e.key == key) {
+        *map = e.map;
+        return HS2_OK;
+      }
+  }
+  const int rc = encode_cache_map(map, c, box_rows);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  g_maps[g_map_next] = MapEntry{key, *map, true};
+  g_map_next = (g_map_next + 1) % 16;
+  return HS2_OK;
+}
+
 // ---------------------------------------------------------------- workspace
 struct Layout {
   size_t err, prefix, records, logits, scores, above, cand, subcnt, hist, thr, lse, total;
@@ -425,8 +465,8 @@ int full_attn_select_impl(const hs2_heads *q, const hs2_cache *k_cache, const hs
   } else {
     const int box_rows = paged ? (ps < p.tile ? ps : p.tile) : p.tile;
     CUtensorMap tmk, tmv;
-    if ((rc = encode_cache_map(&tmk, k_cache, box_rows))) return rc;
-    if ((rc = encode_cache_map(&tmv, v_cache, box_rows))) return rc;
+    if ((rc = cache_map(&tmk, k_cache, box_rows))) return rc;
+    if ((rc = cache_map(&tmv, v_cache, box_rows))) return rc;
     if (fuse) {
       // the grid barrier's arrival counter (word 16 of the flag block) starts at zero
       e = cudaMemsetAsync(p.ws.err + 16, 0, sizeof(uint32_t), s);
