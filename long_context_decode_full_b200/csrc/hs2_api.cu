@@ -570,6 +570,15 @@ int hs2_sparse_attn(const hs2_heads *q_l, const hs2_cache *k_cache, const hs2_ca
   p.rows_per_cta = rows;
   p.splits = S;
   p.nbuf = nbuf;
+  if (k_cache->dtype == HS2_F32) {
+    // fp32 caches: a cluster of up to 16 CTAs per (sequence, kv head), each
+    // taking a share of the list's 64-row tiles, as long as the clusters fit
+    // one CTA per SM
+    const int ntiles = (idx_stride + 63) / 64, per_unit = sms / (p.B * p.Hkv);
+    int s32 = per_unit < 1 ? 1 : (per_unit > 16 ? 16 : per_unit);
+    if (s32 > ntiles) s32 = ntiles < 1 ? 1 : ntiles;
+    p.splits = s32;
+  }
   cudaError_t e = launch_sparse_impl(p, k_cache->dtype, k_cache->num_slots, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "sparse-attention launch");
   return HS2_OK;

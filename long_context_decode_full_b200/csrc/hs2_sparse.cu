@@ -207,12 +207,21 @@ __global__ void __launch_bounds__(32 * NW, 1) sparse_mma_kernel(const SparsePara
 }
 
 // ------------------------------------------------------------ fp32 caches
-// One CTA of 4 warps per (sequence, kv head): the listed rows are gathered 64
-// at a time into shared memory (coalesced row loads), then warp w serves the
-// heads w and w + 4 of the group with an online softmax on the CUDA cores
-// (FFMA keeps fp32 logits exact to fp32 rounding).
+// A cluster of S CTAs (4 warps each) per (sequence, kv head): CTA r takes the
+// 64-row tiles [r * ntiles / S, (r + 1) * ntiles / S) of the index list.  A
+// tile's listed rows are gathered into shared memory (coalesced row loads),
+// then warp w serves the heads w and w + 4 of the group with an online softmax
+// on the CUDA cores (FFMA keeps fp32 logits exact to fp32 rounding).  The CTAs'
+// (m, l, o) meet through distributed shared memory: each CTA writes 1/S of the
+// group's G x D outputs.
 constexpr int kSpF32Tile = 64;
 constexpr int kSpF32Warps = 4;
+constexpr int kSpF32MaxSplits = 16;
+
+template <int D>
+constexpr int sp_f32_floats() {  // shared floats before the tile's slot list
+  return 2 * kSpF32Tile * (D + 1) + 8 * D + (16 + 8 * D) + 8 * kSpF32MaxSplits + 8;
+}
 
 template <int D>
 __global__ void __launch_bounds__(32 * kSpF32Warps) sparse_f32_kernel(const SparseParams p, int64_t num_slots) {
@@ -220,8 +229,13 @@ __global__ void __launch_bounds__(32 * kSpF32Warps) sparse_f32_kernel(const Spar
   float *Ks = fsm;                          // [64][D + 1]
   float *Vs = Ks + kSpF32Tile * (D + 1);    // [64][D + 1]
   float *Qs = Vs + kSpF32Tile * (D + 1);    // [G <= 8][D]
-  int *slots = reinterpret_cast<int *>(Qs + 8 * D);  // [64]
-  const int kvh = blockIdx.x, b = blockIdx.y, G = p.G;
+  float *part = Qs + 8 * D;                 // this CTA's m[8], l[8], o[8][D]
+  float *wts = part + 16 + 8 * D;           // [rank][8] weights of the partials
+  float *inv_l = wts + 8 * kSpF32MaxSplits; // [8]
+  int *slots = reinterpret_cast<int *>(inv_l + 8);  // [64]
+  cg::cluster_group cluster = cg::this_cluster();
+  const int S = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
+  const int kvh = blockIdx.y, b = blockIdx.z, G = p.G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nthr = blockDim.x;
   griddep_wait();
   griddep_launch_dependents();
@@ -237,7 +251,10 @@ __global__ void __launch_bounds__(32 * kSpF32Warps) sparse_f32_kernel(const Spar
 #pragma unroll
     for (int j = 0; j < D / 32; ++j) o[hs][j] = 0.f;
   }
-  for (int base = 0; base < p.L; base += kSpF32Tile) {
+  const int ntiles = (p.L + kSpF32Tile - 1) / kSpF32Tile;
+  const int tile0 = rank * ntiles / S, tile1 = (rank + 1) * ntiles / S;
+  for (int tile = tile0; tile < tile1; ++tile) {
+    const int base = tile * kSpF32Tile;
     for (int r = threadIdx.x; r < kSpF32Tile; r += nthr) {
       const int sl = base + r < p.L ? __ldg(idx + base + r) : -1;
       slots[r] = (sl >= 0 && sl < num_slots) ? sl : -1;
@@ -285,14 +302,59 @@ __global__ void __launch_bounds__(32 * kSpF32Warps) sparse_f32_kernel(const Spar
     }
     __syncthreads();  // the tile is consumed before the next gather
   }
+  // this CTA's partial state (m = -inf, l = 0 where it saw no listed row)
 #pragma unroll
   for (int hs = 0; hs < 2; ++hs) {
     const int h = warp + kSpF32Warps * hs;
     if (h >= G) break;
-    float *out = static_cast<float *>(p.out) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G + h) * D;
+    if (lane == 0) {
+      part[h] = m[hs];
+      part[8 + h] = l[hs];
+    }
 #pragma unroll
-    for (int j = 0; j < D / 32; ++j) out[lane + 32 * j] = l[hs] > 0.f ? o[hs][j] / l[hs] : 0.f;
+    for (int j = 0; j < D / 32; ++j) part[16 + h * D + lane + 32 * j] = o[hs][j];
   }
+  cluster.sync();  // every CTA's partial is complete
+  if (threadIdx.x < G) {  // the partials' weights per head: exp(c (m_r - M)), and 1 / sum_r w_r l_r
+    const int h = threadIdx.x;
+    float M = -INFINITY;
+    for (int r = 0; r < S; ++r) M = fmaxf(M, cluster.map_shared_rank(part, r)[h]);
+    float L = 0.f;
+    for (int r = 0; r < S; ++r) {
+      const float *pr = cluster.map_shared_rank(part, r);
+      const float w = pr[h] == -INFINITY ? 0.f : expf(p.c * (pr[h] - M));
+      wts[r * 8 + h] = w;
+      L += w * pr[8 + h];
+    }
+    inv_l[h] = L > 0.f ? 1.f / L : 0.f;
+  }
+  __syncthreads();
+  {  // this CTA's share of the outputs, the partials added in rank order
+    const int per = (G * D + S - 1) / S, e0 = rank * per, e1 = min(G * D, e0 + per);
+    float *out = static_cast<float *>(p.out) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
+    for (int e = e0 + threadIdx.x; e < e1; e += nthr) {
+      const int h = e / D;
+      float acc = 0.f;
+      for (int r = 0; r < S; ++r) acc += wts[r * 8 + h] * cluster.map_shared_rank(part, r)[16 + e];
+      out[e] = acc * inv_l[h];
+    }
+  }
+  cluster.sync();  // keep every CTA's shared memory alive until all have read it
+}
+
+template <int D>
+cudaError_t launch_f32_t(const SparseParams &p, int64_t num_slots, cudaStream_t s) {
+  const size_t smem = (size_t)sp_f32_floats<D>() * 4 + kSpF32Tile * 4;
+  auto kern = sparse_f32_kernel<D>;
+  cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), (int)smem);
+  if (e != cudaSuccess) return e;
+  static bool wide_ok = false;  // clusters above 8 CTAs need the non-portable size allowed (once)
+  if (p.splits > 8 && !wide_ok) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    wide_ok = true;
+  }
+  return launch_ex(kern, dim3(p.splits, p.Hkv, p.B), dim3(32 * kSpF32Warps), smem, s, p.splits, p, num_slots);
 }
 
 template <int D, bool FP8, int NW, int NSL>
@@ -321,17 +383,9 @@ cudaError_t launch_mma_shape(const SparseParams &p, int64_t num_slots, cudaStrea
 }  // namespace
 
 cudaError_t launch_sparse_impl(const SparseParams &p, int kv_dtype, int64_t num_slots, cudaStream_t s) {
-  if (kv_dtype == 0) {
-    const size_t smem = (size_t)(2 * kSpF32Tile * (p.D + 1) + 8 * p.D) * 4 + kSpF32Tile * 4;
-    cudaError_t e;
-    if (p.D == 64) {
-      e = set_smem_once(reinterpret_cast<const void *>(sparse_f32_kernel<64>), (int)smem);
-      if (e != cudaSuccess) return e;
-      return launch_ex(sparse_f32_kernel<64>, dim3(p.Hkv, p.B), dim3(32 * kSpF32Warps), smem, s, 0, p, num_slots);
-    }
-    e = set_smem_once(reinterpret_cast<const void *>(sparse_f32_kernel<128>), (int)smem);
-    if (e != cudaSuccess) return e;
-    return launch_ex(sparse_f32_kernel<128>, dim3(p.Hkv, p.B), dim3(32 * kSpF32Warps), smem, s, 0, p, num_slots);
+  if (kv_dtype == 0) {  // p.splits CTAs per (sequence, kv head), 1 .. 16
+    if (p.splits < 1 || p.splits > kSpF32MaxSplits) return cudaErrorInvalidValue;
+    return p.D == 64 ? launch_f32_t<64>(p, num_slots, s) : launch_f32_t<128>(p, num_slots, s);
   }
   if (kv_dtype == 1)
     return p.D == 64 ? launch_mma_shape<64, false>(p, num_slots, s) : launch_mma_shape<128, false>(p, num_slots, s);
