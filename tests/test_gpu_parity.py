@@ -44,6 +44,11 @@ CASES = {
     "f32_tiny": synth.WORKLOADS["tiny_fp32_t2048"],
     "f32_paged_ragged": spec(kv_dtype="f32", q_dtype="f32", head_dim=64, group=4, page_size=16,
                              seq_len=(1200, 2500)),
+    # fp32 sparse layers run as clusters of min(16, SMs / units, tiles) CTAs:
+    # d 128 with two heads per warp (16 CTAs of 75 KB), and 20 units (7 CTAs each)
+    "f32_d128_g8": spec(kv_dtype="f32", q_dtype="f32", batch=2, seq_len=(1300, 3000)),
+    "f32_g2_b10_contiguous": spec(kv_dtype="f32", q_dtype="f32", head_dim=64, group=2, batch=10, page_size=None,
+                                  seq_len=(100, 2000)),
     "short_window_only": spec(seq_len=(1, 127), batch=4),
     "exactly_window_plus_k": spec(batch=2, seq_len=1152),
     "one_more_than_fits": spec(batch=2, seq_len=1153),
