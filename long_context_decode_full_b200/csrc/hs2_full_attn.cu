@@ -879,7 +879,8 @@ __global__ void __launch_bounds__(32 * kF32Warps) full_attn_f32_kernel(const Ful
   float *Ks = fsm;                        // [64][D+1]
   float *Vs = Ks + kF32Tile * (D + 1);    // [64][D+1]
   float *Qs = Vs + kF32Tile * (D + 1);    // [8][D]
-  int32_t *prefix = reinterpret_cast<int32_t *>(Qs + 8 * D);
+  int64_t *slots = reinterpret_cast<int64_t *>(Qs + 8 * D);  // the tile's cache slots (-1: none)
+  int32_t *prefix = reinterpret_cast<int32_t *>(slots + kF32Tile);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nthr = blockDim.x;
   griddep_wait();
   griddep_launch_dependents();
@@ -908,7 +909,7 @@ __global__ void __launch_bounds__(32 * kF32Warps) full_attn_f32_kernel(const Ful
     const int p0 = i * kF32Tile;
     if (first) {
       const float *q = static_cast<const float *>(p.q) + ((int64_t)b * p.Hkv * p.G + (int64_t)kvh * p.G) * D;
-      for (int e = threadIdx.x; e < p.G * D; e += nthr) Qs[e] = q[e];
+      for (int e = threadIdx.x; e < p.G * D; e += nthr) cp_async_4(smem_u32(Qs + e), q + e);
 #pragma unroll
       for (int hs = 0; hs < 2; ++hs) {
         m[hs] = -INFINITY;
@@ -916,17 +917,29 @@ __global__ void __launch_bounds__(32 * kF32Warps) full_attn_f32_kernel(const Ful
         for (int j = 0; j < D / 32; ++j) o[hs][j] = 0.f;
       }
     }
-    for (int e = threadIdx.x; e < kF32Tile * D; e += nthr) {
-      const int rr = e / D, col = e % D, pos = p0 + rr;
-      float kv = 0.f, vv = 0.f;
+    // the tile's slots once, then every element of its K and V rows in flight
+    // at once (4-byte cp.async into the padded rows)
+    for (int rr = threadIdx.x; rr < kF32Tile; rr += nthr) {
+      const int pos = p0 + rr;
       const int64_t slot = pos < T ? slot_of(p.page_table, p.max_pages, p.page_size, b, pos) : -1;
-      if (slot >= 0 && slot < p.num_slots) {
-        kv = K[(slot * p.Hkv + kvh) * D + col];
-        vv = V[(slot * p.Hkv + kvh) * D + col];
-      }
-      Ks[rr * (D + 1) + col] = kv;
-      Vs[rr * (D + 1) + col] = vv;
+      slots[rr] = slot >= 0 && slot < p.num_slots ? slot : -1;
     }
+    __syncthreads();
+#pragma unroll 8
+    for (int e = threadIdx.x; e < kF32Tile * D; e += 32 * kF32Warps) {
+      const int rr = e / D, col = e % D;
+      const int64_t slot = slots[rr];
+      float *kd = Ks + rr * (D + 1) + col, *vd = Vs + rr * (D + 1) + col;
+      if (slot >= 0) {
+        cp_async_4(smem_u32(kd), K + (slot * p.Hkv + kvh) * D + col);
+        cp_async_4(smem_u32(vd), V + (slot * p.Hkv + kvh) * D + col);
+      } else {
+        *kd = 0.f;
+        *vd = 0.f;
+      }
+    }
+    cp_async_commit();
+    cp_async_wait_all();
     __syncthreads();
 #pragma unroll
     for (int hs = 0; hs < 2; ++hs) {
@@ -1084,7 +1097,7 @@ int full_f32_tile() { return kF32Tile; }
 int full_f32_ctas_per_sm() { return 2; }
 
 cudaError_t launch_full_f32(const FullParams &p, int grid, cudaStream_t s) {
-  const size_t smem = (size_t)(2 * kF32Tile * (p.D + 1) + 8 * p.D) * 4 + (size_t)(p.B + 1) * 4;
+  const size_t smem = (size_t)(2 * kF32Tile * (p.D + 1) + 8 * p.D) * 4 + kF32Tile * 8 + (size_t)(p.B + 1) * 4;
   cudaError_t e;
   if (p.D == 64) {
     e = set_smem_once(reinterpret_cast<const void *>(full_attn_f32_kernel<64>), (int)smem);

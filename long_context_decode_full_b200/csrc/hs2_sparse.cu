@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(32 * kSpF32Warps) sparse_f32_kernel(const Spar
   griddep_wait();
   griddep_launch_dependents();
   const float *q = static_cast<const float *>(p.q) + ((int64_t)b * p.Hkv * G + (int64_t)kvh * G) * D;
-  for (int e = threadIdx.x; e < G * D; e += nthr) Qs[e] = q[e];
+  for (int e = threadIdx.x; e < G * D; e += nthr) cp_async_4(smem_u32(Qs + e), q + e);  // waited on with the first tile
   const float *K = static_cast<const float *>(p.k), *V = static_cast<const float *>(p.v);
   const int32_t *idx = p.idx + ((int64_t)b * p.Hkv + kvh) * p.L;
   float m[2], l[2], o[2][D / 32];
@@ -260,12 +260,23 @@ __global__ void __launch_bounds__(32 * kSpF32Warps) sparse_f32_kernel(const Spar
       slots[r] = (sl >= 0 && sl < num_slots) ? sl : -1;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < kSpF32Tile * D; e += nthr) {
+    // every element of the tile's K and V rows in flight at once (4-byte
+    // cp.async into the padded rows)
+#pragma unroll 8
+    for (int e = threadIdx.x; e < kSpF32Tile * D; e += 32 * kSpF32Warps) {
       const int rr = e / D, col = e % D;
       const int sl = slots[rr];
-      Ks[rr * (D + 1) + col] = sl >= 0 ? K[((int64_t)sl * p.Hkv + kvh) * D + col] : 0.f;
-      Vs[rr * (D + 1) + col] = sl >= 0 ? V[((int64_t)sl * p.Hkv + kvh) * D + col] : 0.f;
+      float *kd = Ks + rr * (D + 1) + col, *vd = Vs + rr * (D + 1) + col;
+      if (sl >= 0) {
+        cp_async_4(smem_u32(kd), K + ((int64_t)sl * p.Hkv + kvh) * D + col);
+        cp_async_4(smem_u32(vd), V + ((int64_t)sl * p.Hkv + kvh) * D + col);
+      } else {
+        *kd = 0.f;
+        *vd = 0.f;
+      }
     }
+    cp_async_commit();
+    cp_async_wait_all();
     __syncthreads();
 #pragma unroll
     for (int hs = 0; hs < 2; ++hs) {
@@ -302,6 +313,7 @@ __global__ void __launch_bounds__(32 * kSpF32Warps) sparse_f32_kernel(const Spar
     }
     __syncthreads();  // the tile is consumed before the next gather
   }
+  cp_async_wait_all();  // (the query's copies, should this CTA have had no tile)
   // this CTA's partial state (m = -inf, l = 0 where it saw no listed row)
 #pragma unroll
   for (int hs = 0; hs < 2; ++hs) {
