@@ -147,6 +147,29 @@ def test_window_and_budget_variants(oracle, lib):
         U.check_full(wd, out, idx, ora, window=W, k_global=K)
 
 
+@pytest.mark.parametrize("kv_dtype", ["f32", "bf16", "e4m3"])
+def test_sparse_ragged_lists(oracle, lib, kv_dtype):
+    """Sparse layers over index lists of 12, 364 and 1,100 rows (W + K for
+    three budgets): shorter than one 64-row tile, and ragged last tiles, with
+    the oracle's list as input.  The fp32 clusters' merge is repeatable bit
+    for bit."""
+    kw = dict(kv_dtype=kv_dtype, q_dtype="f32" if kv_dtype == "f32" else "bf16", batch=3, seq_len=(700, 2600))
+    if kv_dtype == "f32":
+        kw.update(head_dim=64, group=4)
+    w = synth.generate(spec(**kw), seed=31)
+    wd = U.to_device(w)
+    for W, K in [(5, 7), (64, 300), (100, 1000)]:
+        ora = U.run_oracle(oracle, w, window=W, k_global=K)
+        ora_idx = torch.from_numpy(ora["idx"]).cuda()
+        assert ora_idx.shape[-1] == W + K
+        g = U.run_gpu_sparse(wd, wd.q_sparse[0], ora_idx)
+        g2 = U.run_gpu_sparse(wd, wd.q_sparse[0], ora_idx)
+        torch.cuda.synchronize()
+        ref = U.run_oracle_sparse(oracle, w, w.q_sparse[0], ora["idx"])
+        U.check_out(g, ref, kv_dtype, f"sparse layer, list of {W + K}")
+        assert torch.equal(g, g2)
+
+
 def test_repeatable_bitwise(lib):
     sp = spec(kv_dtype="bf16")
     w = U.to_device(synth.generate(sp, seed=4))
