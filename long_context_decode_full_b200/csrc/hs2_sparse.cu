@@ -10,6 +10,8 @@
 // attention step for the G query heads of the group, the CTA merges its
 // warps, and the CTAs merge through distributed shared memory, each writing
 // its share of the output elements.  No workspace, no atomics, one launch.
+// fp32 caches take the same cluster shape on the CUDA cores (FFMA): 64-row
+// tiles gathered with 4-byte cp.async, one warp per query head.
 #include <cooperative_groups.h>
 
 #include "hs2_internal.h"
