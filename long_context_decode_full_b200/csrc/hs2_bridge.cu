@@ -48,9 +48,13 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
   return __bfloat1622float2(v);  // .x is the lower address
 }
 
+// TOK token slots per CTA (1, 2, 4 or 8: the batch rounded up to a power of
+// two, 8 above 4), so a small batch does not pay for 8 tokens' FMAs.
+template <int TOK>
 __global__ void __launch_bounds__(kBridgeThreads) bridge_kernel(const BridgeParams p) {
-  __shared__ float sh_h[kBridgeTokens][kBridgeRows];                                 // the tokens' hidden slice
-  __shared__ __align__(16) float sh_red[kBridgeWarps][kBridgeTokens][kBridgeCols];   // per-warp partial sums
+  static_assert(TOK >= 1 && TOK <= kBridgeTokens, "token slots");
+  __shared__ float sh_h[TOK][kBridgeRows];                                 // the tokens' hidden slice
+  __shared__ __align__(16) float sh_red[kBridgeWarps][TOK][kBridgeCols];   // per-warp partial sums
   __shared__ int sh_last;
   griddep_wait();
   griddep_launch_dependents();
@@ -70,21 +74,21 @@ __global__ void __launch_bounds__(kBridgeThreads) bridge_kernel(const BridgePara
     const int r = r0 + warp + j * kBridgeWarps;
     wr[j] = active ? __ldg(reinterpret_cast<const uint2 *>(w + (int64_t)r * p.N + col)) : make_uint2(0u, 0u);
   }
-  for (int e = threadIdx.x; e < kBridgeTokens * kBridgeRows; e += kBridgeThreads) {
+  for (int e = threadIdx.x; e < TOK * kBridgeRows; e += kBridgeThreads) {
     const int t = e / kBridgeRows, r = e % kBridgeRows;
     sh_h[t][r] = t < nb ? __bfloat162float(p.h[(int64_t)(b0 + t) * p.d_model + r0 + r]) : 0.f;
   }
   __syncthreads();
 
-  float acc[kBridgeTokens][4];
+  float acc[TOK][4];
 #pragma unroll
-  for (int t = 0; t < kBridgeTokens; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+  for (int t = 0; t < TOK; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
 #pragma unroll
   for (int j = 0; j < kRowsPerWarp; ++j) {
     const int r = warp + j * kBridgeWarps;
     const float2 w01 = bf16x2_to_float2(wr[j].x), w23 = bf16x2_to_float2(wr[j].y);
 #pragma unroll
-    for (int t = 0; t < kBridgeTokens; ++t) {
+    for (int t = 0; t < TOK; ++t) {
       const float hv = sh_h[t][r];
       acc[t][0] = fmaf(hv, w01.x, acc[t][0]);
       acc[t][1] = fmaf(hv, w01.y, acc[t][1]);
@@ -93,17 +97,18 @@ __global__ void __launch_bounds__(kBridgeThreads) bridge_kernel(const BridgePara
     }
   }
 #pragma unroll
-  for (int t = 0; t < kBridgeTokens; ++t)
+  for (int t = 0; t < TOK; ++t)
     *reinterpret_cast<float4 *>(&sh_red[warp][t][4 * lane]) = make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
   __syncthreads();
 
   // this split's tile: warp `tok` sums the 8 warps' rows of token tok in warp order
   const int tok = warp;
-  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (tok < nb && active) {
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int w8 = 0; w8 < kBridgeWarps; ++w8) s = add4(s, *reinterpret_cast<const float4 *>(&sh_red[w8][tok][4 * lane]));
-  if (tok < nb && active)
+    for (int w8 = 0; w8 < kBridgeWarps; ++w8) s = add4(s, *reinterpret_cast<const float4 *>(&sh_red[w8][tok][4 * lane]));
     __stcg(reinterpret_cast<float4 *>(p.partial + (((int64_t)kv * p.nsplit + split) * p.B + b0 + tok) * p.N + col), s);
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
     // one gpu-scope fence after the barrier orders every thread's partial
@@ -197,7 +202,11 @@ cudaError_t launch_bridge(const BridgeParams &p0, void *workspace, cudaStream_t 
   p.tickets = static_cast<int32_t *>(workspace);
   p.partial = reinterpret_cast<float *>(static_cast<char *>(workspace) + align256_((size_t)ticket_words(p.B, p.N) * 4));
   const dim3 grid(p.ntiles, p.nsplit, 2 * p.ngroups);
-  return launch_ex(bridge_kernel, grid, dim3(kBridgeThreads), 0, s, 0, p);
+  const dim3 block(kBridgeThreads);
+  if (p.B == 1) return launch_ex(bridge_kernel<1>, grid, block, 0, s, 0, p);
+  if (p.B == 2) return launch_ex(bridge_kernel<2>, grid, block, 0, s, 0, p);
+  if (p.B <= 4) return launch_ex(bridge_kernel<4>, grid, block, 0, s, 0, p);
+  return launch_ex(bridge_kernel<kBridgeTokens>, grid, block, 0, s, 0, p);
 }
 
 }  // namespace hs2
