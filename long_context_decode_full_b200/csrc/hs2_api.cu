@@ -749,7 +749,25 @@ struct SmemAttr {
 std::mutex g_attr_mu;
 SmemAttr g_attr[512];
 int g_nattr = 0;
+struct WideAttr {
+  const void *kern;
+  int dev;
+};
+WideAttr g_wide[128];
+int g_nwide = 0;
 }  // namespace
+
+cudaError_t allow_wide_clusters_once(const void *kern) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  for (int i = 0; i < g_nwide; ++i)
+    if (g_wide[i].kern == kern && g_wide[i].dev == dev) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess && g_nwide < 128) g_wide[g_nwide++] = WideAttr{kern, dev};
+  return e;
+}
 
 cudaError_t set_smem_once(const void *kern, int bytes) {
   int dev = 0;

@@ -82,6 +82,9 @@ size_t full_tc_smem_bytes(int B, bool fp8);
 // device (again only to raise it): the attribute call costs host time on
 // every launch otherwise.
 cudaError_t set_smem_once(const void *kern, int bytes);
+// cudaFuncSetAttribute(NonPortableClusterSizeAllowed) once per kernel and
+// device, for clusters of more than 8 CTAs.
+cudaError_t allow_wide_clusters_once(const void *kern);
 
 // Launch with programmatic stream serialization (unless HS2_PDL=0) and an
 // optional 1-D cluster.

@@ -362,11 +362,9 @@ cudaError_t launch_f32_t(const SparseParams &p, int64_t num_slots, cudaStream_t 
   auto kern = sparse_f32_kernel<D>;
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), (int)smem);
   if (e != cudaSuccess) return e;
-  static bool wide_ok = false;  // clusters above 8 CTAs need the non-portable size allowed (once)
-  if (p.splits > 8 && !wide_ok) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (p.splits > 8) {
+    e = allow_wide_clusters_once(reinterpret_cast<const void *>(kern));
     if (e != cudaSuccess) return e;
-    wide_ok = true;
   }
   return launch_ex(kern, dim3(p.splits, p.Hkv, p.B), dim3(32 * kSpF32Warps), smem, s, p.splits, p, num_slots);
 }
@@ -379,7 +377,7 @@ cudaError_t launch_mma_t(const SparseParams &p, int64_t num_slots, cudaStream_t 
   cudaError_t e = set_smem_once(reinterpret_cast<const void *>(kern), (int)smem);
   if (e != cudaSuccess) return e;
   if (p.splits > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = allow_wide_clusters_once(reinterpret_cast<const void *>(kern));
     if (e != cudaSuccess) return e;
   }
   return launch_ex(kern, dim3(p.splits, p.Hkv * ((p.G + 7) / 8), p.B), dim3(32 * NW), smem, s, p.splits, p, num_slots);
